@@ -1,0 +1,207 @@
+"""The compact KV store as a set definition, and decode over it.
+
+TEST INFRASTRUCTURE (see ``oracle/__init__.py``).
+
+Source: the FastDMS announcement (aiwitness.kr/community/1t3vlrx). DMS decides
+per head which tokens' KV slots are dropped; FastDMS keeps the survivors in a
+compact store that physically reclaims the dropped slots, next to a staging
+area ("KV/stage memory is the cache or cache plus staging", sentence under the
+KV-memory table). The pages give no algorithm for either; the readings below
+are the plainest ones the rest supports.
+
+State of one (layer, seq): n tokens appended (positions 0..n-1) and r positions
+resolved. Per kv head h, every token j carries keep[j] in {0, 1}.
+
+* Window reading. The benchmark configs keep "the last N tokens always"; that
+  is read as a standing recent window W: token j is visible while j >= n - W
+  whatever its keep bit, and afterwards only if keep[j] = 1. Visible set:
+      S = { j < n : j >= n - W  or  keep[j] = 1 }.
+  (W = 0 is immediate eviction.)
+* Resolution. A token's keep bit is applied when it is resolved, i.e. moved out
+  of the staging ring: survivors are appended to the store, the others dropped.
+  Resolution happens in passes: after an append that brings n to n',
+      r' = n' - W   if n' - W - r >= P,   else r' = r,
+  so with period P = 1 every token is resolved as it leaves the window, and with
+  P = 64 the out-of-window tokens are resolved 64 at a time ("a full compaction
+  pass every 64 steps"). Pending tokens (r <= j < n - W) stay visible iff kept,
+  so P changes where a token lives, never what decode sees.
+* Store of (layer, seq, h): the positions { j < r : keep[j] = 1 } in ascending
+  order (stable, order-preserving compaction), with their payload rows.
+  store_len = popcount(keep[0:r]).
+* Ring (staging) of (layer, seq, h): positions r..n-1 with payload and keep bit.
+* Payload: the bf16 input bits (BF16 cache) or E4M3 codes (FP8 cache).
+* FP8 scale (configs give "one fp32 scale per (layer, kv head, 64-token
+  block)"; how it is chosen is not on the pages). Reading: each (layer, seq, kv
+  head) gets one scale for K and one for V when its sequence first receives
+  tokens: max(amax over that call's K (resp. V) values, 2^-126) / 448, or the
+  caller's values. Every store block and the ring use that scale, so a
+  per-block scale field holds the same number in every block of a head.
+* Stored value of a slot: the bf16 value, or E4M3 value * scale (exact in fp64).
+* Decode happens after the token of the step is appended, so it attends to
+  itself.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import numerics as nm
+from .attention import attend_gather, attend_dense_masked
+from .memory import dense_kv_bytes
+
+
+def resolved_after(n_new: int, r_old: int, window: int, period: int) -> int:
+    """Resolved count after an append brings the sequence to n_new tokens."""
+    if n_new - window - r_old >= period:
+        return n_new - window
+    return r_old
+
+
+class OracleCache:
+    """Plain model of the compact cache, one numpy array per tensor.
+
+    Rows are kept in the input layout [L][B][pos][Hkv][D] (bf16 bits as uint16);
+    FP8 caches also keep the E4M3 codes of every row.
+    """
+
+    def __init__(self, layers, batch, q_heads, kv_heads, head_dim, window, period,
+                 kv_dtype="bf16", capacity=1024, softmax_scale=None):
+        assert q_heads % kv_heads == 0
+        assert kv_dtype in ("bf16", "fp8_e4m3")
+        self.L, self.B, self.Hq, self.Hkv, self.D = layers, batch, q_heads, kv_heads, head_dim
+        self.W, self.P = window, period
+        self.kv_dtype = kv_dtype
+        self.elt = 2 if kv_dtype == "bf16" else 1
+        self.cap = capacity
+        self.scale = (1.0 / np.sqrt(head_dim)) if softmax_scale is None else float(softmax_scale)
+        shape = (layers, batch, capacity, kv_heads, head_dim)
+        self.k = np.zeros(shape, np.uint16)
+        self.v = np.zeros(shape, np.uint16)
+        self.keep = np.zeros(shape[:4], np.uint8)
+        if kv_dtype == "fp8_e4m3":
+            self.kq = np.zeros(shape, np.uint8)
+            self.vq = np.zeros(shape, np.uint8)
+        self.kv_scale = np.zeros((layers, batch, kv_heads, 2), np.float32)
+        self.n = np.zeros((layers, batch), np.int64)
+        self.r = np.zeros((layers, batch), np.int64)
+        self.saturations = 0
+
+    # ---------------------------------------------------------------- append
+    def append(self, layer, n_new, k_bits, v_bits, keep, kv_scale=None):
+        """Append n_new[b] tokens to every sequence b of one layer.
+
+        k_bits / v_bits: uint16 [B][max_new][Hkv][D]; keep uint8 [B][max_new][Hkv];
+        kv_scale: optional float32 [B][Hkv][2] used at a sequence's first append.
+        """
+        k_bits = np.asarray(k_bits, np.uint16)
+        v_bits = np.asarray(v_bits, np.uint16)
+        keep = np.asarray(keep, np.uint8)
+        for b in range(self.B):
+            m = int(n_new[b])
+            if m == 0:
+                continue
+            n0 = int(self.n[layer, b])
+            n1 = n0 + m
+            if n1 > self.cap:
+                raise ValueError("oracle capacity exceeded")
+            self.k[layer, b, n0:n1] = k_bits[b, :m]
+            self.v[layer, b, n0:n1] = v_bits[b, :m]
+            self.keep[layer, b, n0:n1] = keep[b, :m]
+            if self.kv_dtype == "fp8_e4m3":
+                if n0 == 0:
+                    for h in range(self.Hkv):
+                        if kv_scale is not None:
+                            sk, sv = np.float32(kv_scale[b][h][0]), np.float32(kv_scale[b][h][1])
+                        else:
+                            ak = np.max(np.abs(nm.bf16_to_f32(k_bits[b, :m, h])))
+                            av = np.max(np.abs(nm.bf16_to_f32(v_bits[b, :m, h])))
+                            sk, sv = nm.calibration_scale(ak), nm.calibration_scale(av)
+                        self.kv_scale[layer, b, h] = (sk, sv)
+                for h in range(self.Hkv):
+                    kc, s1 = nm.quantise_e4m3(k_bits[b, :m, h], self.kv_scale[layer, b, h, 0])
+                    vc, s2 = nm.quantise_e4m3(v_bits[b, :m, h], self.kv_scale[layer, b, h, 1])
+                    self.kq[layer, b, n0:n1, h] = kc
+                    self.vq[layer, b, n0:n1, h] = vc
+                    self.saturations += s1 + s2
+            self.n[layer, b] = n1
+            self.r[layer, b] = resolved_after(n1, int(self.r[layer, b]), self.W, self.P)
+
+    # ----------------------------------------------------------------- views
+    def _payload(self, layer, b, h, pos):
+        if self.kv_dtype == "bf16":
+            return self.k[layer, b, pos, h], self.v[layer, b, pos, h]
+        return self.kq[layer, b, pos, h], self.vq[layer, b, pos, h]
+
+    def store(self, layer, b, h):
+        """(positions int32[len], K payload [len][D], V payload [len][D])."""
+        r = int(self.r[layer, b])
+        pos = np.flatnonzero(self.keep[layer, b, :r, h]).astype(np.int32)
+        kp, vp = self._payload(layer, b, h, pos)
+        return pos, kp, vp
+
+    def ring(self, layer, b, h):
+        """(positions r..n-1, K payload, V payload, keep bits)."""
+        r, n = int(self.r[layer, b]), int(self.n[layer, b])
+        pos = np.arange(r, n, dtype=np.int32)
+        kp, vp = self._payload(layer, b, h, pos)
+        return pos, kp, vp, self.keep[layer, b, r:n, h].copy()
+
+    def visible(self, layer, b, h):
+        """Bool mask over positions 0..n-1: recent window or kept."""
+        n = int(self.n[layer, b])
+        j = np.arange(n)
+        return (j >= n - self.W) | (self.keep[layer, b, :n, h] == 1)
+
+    def values(self, layer, b, h, pos, mode="stored"):
+        """fp64 (K, V) rows at positions ``pos``.
+
+        mode "stored": what the cache holds (bf16 value, or E4M3 value * scale).
+        mode "true": the bf16 inputs, before any FP8 quantisation.
+        """
+        if self.kv_dtype == "bf16" or mode == "true":
+            return (nm.bf16_to_f64(self.k[layer, b, pos, h]),
+                    nm.bf16_to_f64(self.v[layer, b, pos, h]))
+        sk, sv = self.kv_scale[layer, b, h]
+        return (nm.e4m3_to_f64(self.kq[layer, b, pos, h]) * np.float64(sk),
+                nm.e4m3_to_f64(self.vq[layer, b, pos, h]) * np.float64(sv))
+
+    # ---------------------------------------------------------------- decode
+    def attention(self, layer, b, q_bits, mode="stored", routine="gather"):
+        """Decode output of every query head of sequence b: fp64 [Hq][D].
+
+        q_bits: bf16 bits [Hq][D]. routine "gather" (survivors only) or "dense"
+        (all tokens, evicted scores at -inf).
+        """
+        q = nm.bf16_to_f64(q_bits)
+        G = self.Hq // self.Hkv
+        out = np.zeros((self.Hq, self.D))
+        n = int(self.n[layer, b])
+        for h in range(self.Hkv):
+            qg = q[h * G:(h + 1) * G]
+            vis = self.visible(layer, b, h)
+            if routine == "gather":
+                pos = np.flatnonzero(vis)
+                kk, vv = self.values(layer, b, h, pos, mode)
+                out[h * G:(h + 1) * G] = attend_gather(qg, kk, vv, self.scale)
+            else:
+                kk, vv = self.values(layer, b, h, np.arange(n), mode)
+                out[h * G:(h + 1) * G] = attend_dense_masked(qg, kk, vv, vis, self.scale)[0]
+        return out
+
+    # ----------------------------------------------------------------- stats
+    def stats(self):
+        slots_store = 0
+        for layer in range(self.L):
+            for b in range(self.B):
+                r = int(self.r[layer, b])
+                slots_store += int(np.count_nonzero(self.keep[layer, b, :r]))
+        slots_ring = int(np.sum(self.n - self.r)) * self.Hkv
+        tokens = int(np.sum(self.n))
+        row = 2 * self.D * self.elt
+        return {
+            "tokens_appended": tokens,
+            "slots_store": slots_store,
+            "slots_ring": slots_ring,
+            "bytes_compact": (slots_store + slots_ring) * row,
+            "bytes_dense_equiv": dense_kv_bytes(tokens, 1, self.Hkv, self.D, self.elt),
+            "fp8_saturations": int(self.saturations),
+        }
