@@ -39,6 +39,9 @@ resolved. Per kv head h, every token j carries keep[j] in {0, 1}.
 * Stored value of a slot: the bf16 value, or E4M3 value * scale (exact in fp64).
 * Decode happens after the token of the step is appended, so it attends to
   itself.
+* FP8 saturation counter: the number of elements written into the cache (store
+  or ring) whose quotient |fp32(x) / scale| exceeded 448. A token dropped by
+  the very append that brought it is never written and is not counted.
 """
 from __future__ import annotations
 
@@ -116,14 +119,22 @@ class OracleCache:
                             av = np.max(np.abs(nm.bf16_to_f32(v_bits[b, :m, h])))
                             sk, sv = nm.calibration_scale(ak), nm.calibration_scale(av)
                         self.kv_scale[layer, b, h] = (sk, sv)
+            r1 = resolved_after(n1, int(self.r[layer, b]), self.W, self.P)
+            if self.kv_dtype == "fp8_e4m3":
+                # rows dropped by the call that brought them are never written,
+                # so they cannot count as clipped
+                pos = np.arange(n0, n1)
                 for h in range(self.Hkv):
-                    kc, s1 = nm.quantise_e4m3(k_bits[b, :m, h], self.kv_scale[layer, b, h, 0])
-                    vc, s2 = nm.quantise_e4m3(v_bits[b, :m, h], self.kv_scale[layer, b, h, 1])
+                    written = (pos >= r1) | (keep[b, :m, h] == 1)
+                    kc, s1 = nm.quantise_e4m3(k_bits[b, :m, h], self.kv_scale[layer, b, h, 0],
+                                              written)
+                    vc, s2 = nm.quantise_e4m3(v_bits[b, :m, h], self.kv_scale[layer, b, h, 1],
+                                              written)
                     self.kq[layer, b, n0:n1, h] = kc
                     self.vq[layer, b, n0:n1, h] = vc
                     self.saturations += s1 + s2
             self.n[layer, b] = n1
-            self.r[layer, b] = resolved_after(n1, int(self.r[layer, b]), self.W, self.P)
+            self.r[layer, b] = r1
 
     # ----------------------------------------------------------------- views
     def _payload(self, layer, b, h, pos):

@@ -86,15 +86,19 @@ def e4m3_from_f32(x) -> np.ndarray:
     return (code | np.where(sign, 0x80, 0).astype(np.uint8)).astype(np.uint8)
 
 
-def quantise_e4m3(x_bf16_bits, scale_f32) -> tuple:
+def quantise_e4m3(x_bf16_bits, scale_f32, counted=None) -> tuple:
     """Quantise bf16 values with an fp32 scale: (codes uint8, saturated count).
 
     A value counts as saturated when |fp32(x) / scale| > 448 (it was clipped).
+    ``counted``, if given, is a boolean mask over the leading axis: only those
+    rows enter the count.
     """
     xf = bf16_to_f32(x_bf16_bits)
     qf = (xf / np.float32(scale_f32)).astype(np.float32)   # IEEE fp32 quotient
-    sat = int(np.count_nonzero(np.abs(qf) > np.float32(E4M3_MAX)))
-    return e4m3_from_f32(qf), sat
+    clipped = np.abs(qf) > np.float32(E4M3_MAX)
+    if counted is not None:
+        clipped = clipped[np.asarray(counted, bool)]
+    return e4m3_from_f32(qf), int(np.count_nonzero(clipped))
 
 
 def calibration_scale(amax_f32) -> np.float32:
