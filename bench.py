@@ -1,0 +1,457 @@
+#!/usr/bin/env python
+"""Decode-step benchmark: compact-KV decode attention on B200.
+
+One step = for every layer: append one token per sequence with its keep bits
+(fdms_append_evict: ring write, eviction, compaction) and run decode attention
+for all query heads (fdms_decode_attn: split kernel + combine kernel). Inputs
+are the seeded synthetic workloads of ``workloads`` (shapes of the FastDMS
+announcement's benchmark: ctx 8192, Llama-3.2-1B / Qwen3-8B shapes, c = 1 or 8).
+
+Metric: compact KV bytes read by decode per second over whole steps (GB/s),
+with µs per step beside it. Bytes are exact: the cache counts the slots every
+decode call reads (a K row and a V row each).
+
+Timing: the W warm-up steps run eagerly; the K timed steps are one CUDA graph,
+captured once and replayed once between a barrier + synchronize on both sides,
+timed with CUDA events on the launching stream (max over ranks). Events inside
+the graph bracket every decode call, which gives the per-launch duration used
+for the roofline. Every step reads more compact KV than the 126 MB L2 holds, so
+no step finds the previous step's data in L2.
+
+N > 1 (torchrun): every rank runs its own sequences (the path shards by
+sequence with no exchange); value = bytes of all ranks / max time.
+
+--impl reference: the fp64 CPU oracle timed on this host's cores on a bounded
+sample of the same workload (one layer, all sequences), same metric and unit.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as wk  # noqa: E402
+
+METRIC = "decode-attn µs/step and achieved HBM GB/s on compact KV (% of B200 peak)"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="llama1b_c8", choices=sorted(wk.WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="budget of the oracle's timed sample")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-ctas", type=int, default=0)
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "MEASURED_PEAKS.json hbm_gbs (measured)"
+    return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (no MEASURED_PEAKS.json)"
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def config_dict(wl):
+    return {
+        "workload": wl.name, "batch": wl.batch, "layers": wl.layers, "q_heads": wl.q_heads,
+        "kv_heads": wl.kv_heads, "head_dim": wl.head_dim, "kv_dtype": wl.kv_dtype,
+        "ctx": list(wl.ctx_range) if wl.ctx_range else wl.ctx, "window": wl.window,
+        "period": wl.period, "keep_rate": wl.rate if wl.rate is not None else list(wl.rate_range),
+    }
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device: int, period_s=0.002):
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = int(vis.split(",")[device]) if vis else device
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception as e:  # no NVML: report that, keep going
+            self.error = str(e)
+        self.period = period_s
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self._ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
+                    "note": "NVML unavailable: " + getattr(self, "error", "")}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples),
+                "source": "NVML polled every 2 ms during the timed region"}
+
+
+# ----------------------------------------------------------------- oracle leg
+def to_bits(t: torch.Tensor) -> np.ndarray:
+    """bf16 CPU tensor -> uint16 bit patterns (what the oracle reads)."""
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def oracle_sample(wl, budget_s: float, min_steps=1, max_steps=None, warmup=0):
+    """Time the fp64 oracle on one layer of the workload, all sequences.
+
+    Returns (bytes per second, per-step seconds list, description). Bytes are the
+    compact slots the oracle's decode reads (store + ring, K and V rows).
+    """
+    from threadpoolctl import threadpool_limits
+    from oracle.cache import OracleCache
+
+    layer = 0
+    ctx = wk.context_lengths(wl)
+    n_steps = max_steps if max_steps is not None else wl.steps
+    oc = OracleCache(1, wl.batch, wl.q_heads, wl.kv_heads, wl.head_dim, wl.window, wl.period,
+                     wl.kv_dtype, capacity=int(ctx.max()) + n_steps + warmup + 1)
+    pre = wk.prefill_inputs(wl, layer)
+    elt = 1 if wl.kv_dtype == "fp8_e4m3" else 2
+    row = 2 * wl.head_dim * elt
+    times, bytes_ = [], 0
+    with threadpool_limits(limits=1):
+        oc.append(0, pre["n_new"].numpy(), to_bits(pre["k"]), to_bits(pre["v"]),
+                  pre["keep"].numpy())
+        total_t = 0.0
+        for step in range(warmup + n_steps):
+            inp = wk.decode_inputs(wl, layer, step)
+            q = to_bits(wk.decode_query(wl, layer, step))
+            kb, vb, keep = to_bits(inp["k"]), to_bits(inp["v"]), inp["keep"].numpy()
+            t0 = time.perf_counter()
+            oc.append(0, inp["n_new"].numpy(), kb, vb, keep)
+            for b in range(wl.batch):
+                oc.attention(0, b, q[b])
+            dt = time.perf_counter() - t0
+            if step < warmup:
+                continue
+            units = int(np.sum((oc.n - oc.r)) * wl.kv_heads)
+            for b in range(wl.batch):
+                r = int(oc.r[0, b])
+                units += int(np.count_nonzero(oc.keep[0, b, :r]))
+            bytes_ += units * row
+            times.append(dt)
+            total_t += dt
+            if len(times) >= min_steps and total_t >= budget_s:
+                break
+    desc = (f"fp64 numpy oracle, layer 0 of {wl.layers}, all {wl.batch} sequences x "
+            f"{wl.kv_heads} kv heads, {len(times)} decode steps (append + attention) "
+            f"after a {int(ctx.max())}-token prefill; 1 thread")
+    return bytes_ / sum(times), times, desc
+
+
+def run_reference(args, wl):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    bps, times, desc = oracle_sample(wl, budget_s=1e9, min_steps=args.steps,
+                                     max_steps=args.steps, warmup=args.warmup)
+    gbs = bps / 1e9
+    ms = 1e3 * sum(times) / len(times)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": len(times), "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {**config_dict(wl), "step": "one layer, all sequences"},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- native leg
+def pool_blocks(wl, steps_total):
+    """Blocks for the pool: worst case when it fits in 40 GB, else a bound
+    from the keep rates with a 6-sigma margin per head."""
+    ctx = wk.context_lengths(wl)
+    elt = 1 if wl.kv_dtype == "fp8_e4m3" else 2
+    block_bytes = 2 * 64 * wl.head_dim * elt
+    n = ctx[None, :, None] + steps_total
+    worst = int(np.sum(np.ceil(np.broadcast_to(n, (wl.layers, wl.batch, wl.kv_heads)) / 64)))
+    if worst * block_bytes <= 40e9:
+        return 0
+    p = wk.keep_rates(wl)
+    mean = n * p
+    sd = np.sqrt(n * p * (1 - p))
+    return int(np.sum(np.ceil(np.minimum(n, mean + 6 * sd + 64) / 64) + 1))
+
+
+def run_native(args, wl):
+    import compressed_decode_attention_fdms_b200 as fd
+
+    world, rank, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        wl = wk.scaled(wl, seed=wl.seed + 7919 * rank)   # each rank: its own sequences
+
+    W, K = args.warmup, args.steps
+    KE = 0 if args.no_e2e else args.e2e_steps
+    WE = 0 if args.no_e2e else 3
+    steps_total = W + K + WE + KE
+    cfg = fd.make_config(wl.layers, wl.batch, wl.q_heads, wl.kv_heads, wl.head_dim, wl.window,
+                         wl.period, wl.max_ctx + steps_total, pool_blocks(wl, steps_total),
+                         wl.kv_dtype, 0.0, args.decode_ctas)
+    stream = torch.cuda.Stream(dev)
+    cache = fd.fdms_cache_create(cfg, local, stream)
+    L, B = wl.layers, wl.batch
+    elt = 1 if wl.kv_dtype == "fp8_e4m3" else 2
+    row = 2 * wl.head_dim * elt
+    qo_bytes = 2 * B * wl.q_heads * wl.head_dim * 2      # q read + out written, bf16
+
+    with torch.cuda.stream(stream):
+        for layer in range(L):                            # prefill (not timed)
+            inp = wk.prefill_inputs(wl, layer, device=dev)
+            fd.fdms_append_evict(cache, layer, B, inp["n_new"], inp["max_new"], inp["k"],
+                                 inp["v"], inp["keep"], stream=stream)
+            del inp
+        # decode inputs of the device-timed steps, resident in HBM before timing
+        steps_in = [[wk.decode_inputs(wl, l, s, device=dev) for l in range(L)]
+                    for s in range(W + K)]
+        qs = [[wk.decode_query(wl, l, s, device=dev) for l in range(L)] for s in range(W + K)]
+        outs = [torch.empty((B, wl.q_heads, wl.head_dim), dtype=torch.bfloat16, device=dev)
+                for _ in range(L)]
+    stream.synchronize()
+
+    def step(s, ev=None):
+        for layer in range(L):
+            inp = steps_in[s][layer]
+            fd.fdms_append_evict(cache, layer, B, inp["n_new"], 1, inp["k"], inp["v"],
+                                 inp["keep"], stream=stream)
+            if ev is not None:
+                ev[layer][0].record(stream)
+            fd.fdms_decode_attn(cache, layer, B, qs[s][layer], outs[layer], stream=stream)
+            if ev is not None:
+                ev[layer][1].record(stream)
+
+    with torch.cuda.stream(stream):
+        for s in range(W):
+            step(s)
+    stream.synchronize()
+
+    # capture the K timed steps as one graph, with external events per decode call
+    evs = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+            for _ in range(L)] for _ in range(K)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream, capture_error_mode="thread_local"):
+        for s in range(K):
+            step(W + s, evs[s])
+    st0 = fd.fdms_cache_stats(cache, stream)
+
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        graph.replay()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    elapsed_ms = t0.elapsed_time(t1)
+    st1 = fd.fdms_cache_stats(cache, stream)
+    if st1["error"]:
+        raise RuntimeError(f"device error latched: {fd.status_string(st1['error'])}")
+    slots = st1["slots_decoded"] - st0["slots_decoded"]
+    calls = st1["decode_calls"] - st0["decode_calls"]
+    assert calls == K * L, (calls, K * L)
+    kv_bytes = slots * row
+    dec_ms = [evs[s][l][0].elapsed_time(evs[s][l][1]) for s in range(K) for l in range(L)]
+    dec_avg_ms = sum(dec_ms) / len(dec_ms)
+    per_launch_bytes = kv_bytes / calls + qo_bytes
+
+    # whole-job numbers: max time over ranks, bytes summed over ranks
+    t_max, bytes_all = elapsed_ms, float(kv_bytes)
+    if world > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        bb = torch.tensor([float(kv_bytes)], dtype=torch.float64, device=dev)
+        dist.all_reduce(bb, op=dist.ReduceOp.SUM)
+        t_max, bytes_all = float(tt.item()), float(bb.item())
+    value = bytes_all / (t_max * 1e-3) / 1e9
+
+    # ---- end to end through the public API with pinned host buffers
+    e2e = None
+    if KE > 0:
+        e2e = run_e2e(fd, cache, wl, stream, dev, W + K, WE, KE, row)
+        if world > 1:
+            import torch.distributed as dist
+            tt = torch.tensor([e2e["ms"], e2e["bytes"]], dtype=torch.float64, device=dev)
+            dist.all_reduce(tt[0:1], op=dist.ReduceOp.MAX)
+            dist.all_reduce(tt[1:2], op=dist.ReduceOp.SUM)
+            e2e["ms"], e2e["bytes"] = float(tt[0]), float(tt[1])
+
+    peak, peak_src = load_peaks()
+    achieved = per_launch_bytes / (dec_avg_ms * 1e-3) / 1e9
+    result = None
+    if rank == 0:
+        clocks = clk.summary()
+        result = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": t_max / K, "us_per_step": 1e3 * t_max / K,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {**config_dict(wl), "parallelism": f"replicas{world}" if world > 1 else "1gpu",
+                       "l2": "inputs larger than L2: every step reads "
+                             f"{kv_bytes / K / 1e6:.0f} MB of compact KV (L2 126 MB)",
+                       "timing": "K steps in one CUDA graph; events around each decode call"},
+            "roofline": {
+                "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": None,
+                "kernel": "fdms_decode_attn (k_decode_split + k_decode_combine)",
+                "per_launch_bytes": per_launch_bytes, "launch_us": dec_avg_ms * 1e3,
+                "peak_source": peak_src,
+            },
+            "clocks": clocks,
+            "gpu_launches": K * L * 3,
+            "kv_gb_per_step": kv_bytes / K / 1e9,
+            "decode_share_of_step": sum(dec_ms) / elapsed_ms,
+        }
+        if e2e:
+            result["e2e"] = {"value": e2e["bytes"] / (e2e["ms"] * 1e-3) / 1e9, "unit": "GB/s",
+                             "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                             "us_per_step": 1e3 * e2e["ms"] / KE, "steps": KE,
+                             "path": "Python binding -> C ABI, eager calls per layer"}
+        if not args.no_cpu_baseline and world == 1:
+            bps, times, desc = oracle_sample(wl, args.cpu_seconds)
+            result["cpu_baseline"] = {"value": bps / 1e9, "unit": "GB/s", "cores": 1,
+                                      "kind": "oracle", "sample": desc}
+    del graph
+    fd.fdms_cache_destroy(cache)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if result is not None:
+        print(json.dumps(result), flush=True)
+    return 0
+
+
+def run_e2e(fd, cache, wl, stream, dev, s0, warm, steps, row):
+    """Steps through the public API with host buffers: H2D of the step's inputs
+    from pinned memory, every layer's append + decode, D2H of every output."""
+    L, B = wl.layers, wl.batch
+    host = []
+    for s in range(s0, s0 + warm + steps):
+        per = []
+        for layer in range(L):
+            inp = wk.decode_inputs(wl, layer, s)
+            q = wk.decode_query(wl, layer, s)
+            per.append({k: v.pin_memory() for k, v in
+                        (("n_new", inp["n_new"]), ("k", inp["k"]), ("v", inp["v"]),
+                         ("keep", inp["keep"]), ("q", q))})
+        host.append(per)
+    dbuf = [{k: torch.empty_like(v, device=dev) for k, v in host[0][l].items()} for l in range(L)]
+    dout = [torch.empty((B, wl.q_heads, wl.head_dim), dtype=torch.bfloat16, device=dev)
+            for _ in range(L)]
+    hout = [torch.empty_like(dout[0], device="cpu").pin_memory() for _ in range(L)]
+    h2d = sum(v.numel() * v.element_size() for v in host[0][0].values()) * L
+    d2h = sum(o.numel() * o.element_size() for o in dout)
+
+    def one(s):
+        for layer in range(L):
+            for k, v in host[s][layer].items():
+                dbuf[layer][k].copy_(v, non_blocking=True)
+            d = dbuf[layer]
+            fd.fdms_append_evict(cache, layer, B, d["n_new"], 1, d["k"], d["v"], d["keep"],
+                                 stream=stream)
+            fd.fdms_decode_attn(cache, layer, B, d["q"], dout[layer], stream=stream)
+            hout[layer].copy_(dout[layer], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for s in range(warm):
+            one(s)
+    stream.synchronize()
+    st0 = fd.fdms_cache_stats(cache, stream)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for s in range(warm, warm + steps):
+            one(s)
+        t1.record(stream)
+    torch.cuda.synchronize()
+    st1 = fd.fdms_cache_stats(cache, stream)
+    return {"ms": t0.elapsed_time(t1), "bytes": (st1["slots_decoded"] - st0["slots_decoded"]) * row,
+            "h2d": h2d, "d2h": d2h}
+
+
+def main():
+    args = parse_args()
+    wl = wk.get(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_native(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

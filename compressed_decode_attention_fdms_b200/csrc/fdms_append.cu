@@ -1,0 +1,283 @@
+// Append + evict + compact: one CTA per (seq, kv head) of the call.
+//
+// What it applies (FastDMS announcement, aiwitness.kr/community/1t3vlrx, the
+// paragraphs on DMS per-head token eviction and on the compact store that
+// physically reclaims evicted slots, with its staging area):
+//   1. new tokens of the call take positions n0 .. n1-1;
+//   2. if at least P out-of-window tokens are unresolved, all positions
+//      r0 .. n1-W-1 are resolved now: in position order, those with keep = 1
+//      are appended to the head's compact store, the rest are dropped;
+//   3. the still-unresolved new tokens are written to the ring (staging).
+// Resolution is a stable stream compaction: each 256-position chunk takes a
+// warp ballot of the keep bits, a popcount prefix inside each warp, and an
+// exclusive scan of the 8 warp totals, so survivors keep their order.
+// Store blocks for all survivors of the call are taken from the pool with one
+// atomic bump before any row is written; if the pool cannot cover them the
+// head is left unchanged and FDMS_ERR_OUT_OF_BLOCKS is latched.
+//
+// FP8 cache: a sequence's first append fixes each head's K and V scales
+// (max(amax, 2^-126) / 448 of the call's values, or the caller's); every new
+// row is stored as e4m3_rne_satfinite(fp32(x) / scale) with the division in
+// IEEE fp32 and the rounding by the hardware conversion.
+#include "fdms_internal.cuh"
+
+namespace fdms {
+namespace {
+
+constexpr int kAppendThreads = 256;
+constexpr int kWarps = kAppendThreads / 32;
+
+__device__ __forceinline__ float block_max(float x, float* red) {
+  for (int off = 16; off > 0; off >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
+  const int w = threadIdx.x / 32, l = threadIdx.x % 32;
+  __syncthreads();
+  if (l == 0) red[w] = x;
+  __syncthreads();
+  float m = red[0];
+  for (int i = 1; i < kWarps; ++i) m = fmaxf(m, red[i]);
+  return m;
+}
+
+// Absolute maximum over m rows of D bf16 values (row stride `stride` elements).
+__device__ float rows_amax(const uint16_t* base, int m, int D, long long stride, float* red) {
+  float a = 0.0f;
+  const int vpr = D / 8;   // 16-byte vectors per row
+  for (long long i = threadIdx.x; i < (long long)m * vpr; i += kAppendThreads) {
+    const long long row = i / vpr;
+    const int vec = (int)(i % vpr);
+    const uint4 x = *reinterpret_cast<const uint4*>(base + row * stride + vec * 8);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      a = fmaxf(a, fabsf(bf16lo_to_f32(w[j])));
+      a = fmaxf(a, fabsf(bf16hi_to_f32(w[j])));
+    }
+  }
+  return block_max(a, red);
+}
+
+// 8 bf16 (one 16-byte vector) / scale -> 8 E4M3 codes; counts clipped values.
+__device__ __forceinline__ uint2 quantise8(uint4 x, float scale, unsigned& sat) {
+  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+  uint32_t out[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    float f[4];
+    f[0] = __fdiv_rn(bf16lo_to_f32(w[2 * j]), scale);
+    f[1] = __fdiv_rn(bf16hi_to_f32(w[2 * j]), scale);
+    f[2] = __fdiv_rn(bf16lo_to_f32(w[2 * j + 1]), scale);
+    f[3] = __fdiv_rn(bf16hi_to_f32(w[2 * j + 1]), scale);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) sat += fabsf(f[t]) > 448.0f ? 1u : 0u;
+    out[j] = (uint32_t)f32x2_to_e4m3x2(f[0], f[1]) | ((uint32_t)f32x2_to_e4m3x2(f[2], f[3]) << 16);
+  }
+  return make_uint2(out[0], out[1]);
+}
+
+// Copy one 16-byte vector `vec` of an input row into a cache row (quantising in
+// FP8 mode, where the cache row has half the bytes and a vector is 8 bytes of
+// output per 16 bytes of input).
+template <bool FP8>
+__device__ __forceinline__ void put_input_vec(uint8_t* dst_row, const uint16_t* src_row, int vec,
+                                              float scale, unsigned& sat) {
+  const uint4 x = *reinterpret_cast<const uint4*>(src_row + vec * 8);
+  if constexpr (FP8) {
+    *reinterpret_cast<uint2*>(dst_row + vec * 8) = quantise8(x, scale, sat);
+  } else {
+    *reinterpret_cast<uint4*>(dst_row + vec * 16) = x;
+  }
+}
+
+template <bool FP8>
+__global__ void __launch_bounds__(kAppendThreads)
+k_append_evict(CacheView c, int layer, const int32_t* __restrict__ n_new, int max_new,
+               const uint16_t* __restrict__ k_in, const uint16_t* __restrict__ v_in,
+               const uint8_t* __restrict__ keep_in, const float* __restrict__ kv_scale) {
+  __shared__ float s_red[kWarps];
+  __shared__ int s_warp[kWarps];
+  __shared__ int s_src[kAppendThreads];   // survivors of the current chunk: positions
+  __shared__ int s_fail;
+  __shared__ long long s_base_blk;
+  __shared__ float s_scale[2];
+
+  const int b = blockIdx.x / c.Hkv, h = blockIdx.x % c.Hkv;
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const long long hi = head_index(c, layer, b, h);
+  const int m = n_new[b];
+  if (m < 0 || m > max_new) {
+    if (tid == 0) latch_error(c.ctr, FDMS_ERR_DEVICE);
+    return;
+  }
+  if (m == 0) return;
+  const int n0 = c.tok_n[hi], r0 = c.tok_r[hi], len0 = c.store_len[hi];
+  if ((long long)n0 + m > c.max_seq_len) {
+    if (tid == 0) latch_error(c.ctr, FDMS_ERR_DEVICE);
+    return;
+  }
+  const int n1 = n0 + m;
+  const int r1 = (n1 - c.W - r0 >= c.P) ? n1 - c.W : r0;
+  const long long in_stride = (long long)c.Hkv * c.D;          // elements between tokens
+  const uint16_t* k_rows = k_in + ((long long)b * max_new * c.Hkv + h) * c.D;
+  const uint16_t* v_rows = v_in + ((long long)b * max_new * c.Hkv + h) * c.D;
+  const uint8_t* keep_rows = keep_in + (long long)b * max_new * c.Hkv + h;
+  uint8_t* rkeep = c.ring_keep + hi * c.Rpad;
+
+  // ---- FP8 scales
+  float sk = 1.0f, sv = 1.0f;
+  if constexpr (FP8) {
+    if (n0 == 0) {
+      if (kv_scale) {
+        sk = kv_scale[((long long)b * c.Hkv + h) * 2];
+        sv = kv_scale[((long long)b * c.Hkv + h) * 2 + 1];
+      } else {
+        const float ak = rows_amax(k_rows, m, c.D, in_stride, s_red);
+        const float av = rows_amax(v_rows, m, c.D, in_stride, s_red);
+        sk = __fdiv_rn(fmaxf(ak, 1.17549435e-38f), 448.0f);
+        sv = __fdiv_rn(fmaxf(av, 1.17549435e-38f), 448.0f);
+      }
+      if (tid == 0) {
+        c.head_scale[hi * 2] = sk;
+        c.head_scale[hi * 2 + 1] = sv;
+      }
+    } else {
+      if (tid == 0) {
+        s_scale[0] = c.head_scale[hi * 2];
+        s_scale[1] = c.head_scale[hi * 2 + 1];
+      }
+      __syncthreads();
+      sk = s_scale[0];
+      sv = s_scale[1];
+    }
+  }
+
+  auto keep_of = [&](int p) -> int {
+    return p < n0 ? (rkeep[p % c.R] != 0) : (keep_rows[(long long)(p - n0) * c.Hkv] != 0);
+  };
+
+  // ---- pass 1: how many survivors, and their blocks
+  int total = 0;
+  for (int base = r0; base < r1; base += kAppendThreads) {
+    const int p = base + tid;
+    total += __syncthreads_count(p < r1 && keep_of(p));
+  }
+  const int len1 = len0 + total;
+  const int nb0 = (len0 + kBlockSlots - 1) / kBlockSlots;
+  const int nb1 = (len1 + kBlockSlots - 1) / kBlockSlots;
+  if (tid == 0) {
+    s_fail = 0;
+    s_base_blk = 0;
+    if (nb1 > nb0) {
+      const unsigned long long need = (unsigned long long)(nb1 - nb0);
+      const unsigned long long base = atomicAdd(&c.ctr->blocks_next, need);
+      if (base + need > (unsigned long long)c.num_blocks) {
+        latch_error(c.ctr, FDMS_ERR_OUT_OF_BLOCKS);
+        s_fail = 1;
+      } else {
+        s_base_blk = (long long)base;
+      }
+    }
+  }
+  __syncthreads();
+  if (s_fail) return;
+  int32_t* bt = c.block_table + hi * c.max_blocks;
+  float* bts = c.bt_scale + hi * c.max_blocks * 2;
+  for (int j = nb0 + tid; j < nb1; j += kAppendThreads) {
+    bt[j] = (int32_t)(s_base_blk + (j - nb0));
+    bts[2 * j] = sk;
+    bts[2 * j + 1] = sv;
+  }
+  __syncthreads();
+
+  const int VPR = c.D / 8;      // 16-byte input vectors per row (8 bf16 each)
+  unsigned sat = 0;
+
+  // ---- pass 2: stable compaction of positions r0 .. r1-1 into the store
+  int written = 0;
+  for (int base = r0; base < r1; base += kAppendThreads) {
+    const int p = base + tid;
+    const int bit = (p < r1) ? keep_of(p) : 0;
+    const unsigned ball = __ballot_sync(0xffffffffu, bit);
+    const int in_warp = __popc(ball & ((1u << lane) - 1u));
+    if (lane == 0) s_warp[warp] = __popc(ball);
+    __syncthreads();
+    int warp_off = 0, chunk = 0;
+    for (int i = 0; i < kWarps; ++i) {
+      warp_off += (i < warp) ? s_warp[i] : 0;
+      chunk += s_warp[i];
+    }
+    if (bit) s_src[warp_off + in_warp] = p;
+    __syncthreads();
+    // copy the chunk's survivors: (survivor, vector) pairs over the CTA
+    for (int i = tid; i < chunk * VPR; i += kAppendThreads) {
+      const int sidx = i / VPR, vec = i % VPR;
+      const int src = s_src[sidx];
+      const int d = len0 + written + sidx;
+      const long long blk = bt[d / kBlockSlots];
+      const int row = d % kBlockSlots;
+      uint8_t* kd = block_k(c, blk) + (long long)row * c.RB;
+      uint8_t* vd = block_v(c, blk) + (long long)row * c.RB;
+      if (src < n0) {   // from the ring: already in cache format
+        const int slot = src % c.R;
+        const int vb = FP8 ? 8 : 16;   // cache bytes per vector
+        const uint8_t* ks = ring_k(c, hi) + (long long)slot * c.RB + vec * vb;
+        const uint8_t* vs = ring_v(c, hi) + (long long)slot * c.RB + vec * vb;
+        if constexpr (FP8) {
+          *reinterpret_cast<uint2*>(kd + vec * 8) = *reinterpret_cast<const uint2*>(ks);
+          *reinterpret_cast<uint2*>(vd + vec * 8) = *reinterpret_cast<const uint2*>(vs);
+        } else {
+          *reinterpret_cast<uint4*>(kd + vec * 16) = *reinterpret_cast<const uint4*>(ks);
+          *reinterpret_cast<uint4*>(vd + vec * 16) = *reinterpret_cast<const uint4*>(vs);
+        }
+      } else {          // straight from this call's input
+        const long long t = src - n0;
+        put_input_vec<FP8>(kd, k_rows + t * in_stride, vec, sk, sat);
+        put_input_vec<FP8>(vd, v_rows + t * in_stride, vec, sv, sat);
+      }
+      if (vec == 0) c.blk_pos[blk * kBlockSlots + row] = src;
+    }
+    written += chunk;
+    __syncthreads();
+  }
+
+  // ---- ring: unresolved new tokens (after all ring reads above)
+  const int w0 = r1 > n0 ? r1 : n0;
+  for (long long i = tid; i < (long long)(n1 - w0) * VPR; i += kAppendThreads) {
+    const int p = w0 + (int)(i / VPR), vec = (int)(i % VPR);
+    const long long t = p - n0;
+    const int slot = p % c.R;
+    put_input_vec<FP8>(ring_k(c, hi) + (long long)slot * c.RB, k_rows + t * in_stride, vec, sk, sat);
+    put_input_vec<FP8>(ring_v(c, hi) + (long long)slot * c.RB, v_rows + t * in_stride, vec, sv, sat);
+    if (vec == 0) rkeep[slot] = keep_rows[t * c.Hkv] ? 1 : 0;
+  }
+
+  if constexpr (FP8) {
+    for (int off = 16; off > 0; off >>= 1) sat += __shfl_xor_sync(0xffffffffu, sat, off);
+    if (lane == 0 && sat) atomicAdd(&c.ctr->saturations, (unsigned long long)sat);
+  }
+  if (tid == 0) {
+    c.store_len[hi] = len1;
+    c.tok_n[hi] = n1;
+    c.tok_r[hi] = r1;
+  }
+}
+
+}  // namespace
+}  // namespace fdms
+
+using namespace fdms;
+
+fdms_status fdms_launch_append(fdms_cache* cache, int layer, int batch, const int32_t* n_new,
+                               int max_new, const void* k, const void* v, const uint8_t* keep,
+                               const float* kv_scale, cudaStream_t s) {
+  const CacheView& c = cache->view;
+  const dim3 grid((unsigned)(batch * c.Hkv));
+  const uint16_t* kk = static_cast<const uint16_t*>(k);
+  const uint16_t* vv = static_cast<const uint16_t*>(v);
+  if (c.fp8)
+    k_append_evict<true><<<grid, kAppendThreads, 0, s>>>(c, layer, n_new, max_new, kk, vv, keep,
+                                                         kv_scale);
+  else
+    k_append_evict<false><<<grid, kAppendThreads, 0, s>>>(c, layer, n_new, max_new, kk, vv, keep,
+                                                          nullptr);
+  return cudaGetLastError() == cudaSuccess ? FDMS_OK : FDMS_ERR_CUDA;
+}

@@ -1,0 +1,194 @@
+// Internal layout of the compact KV cache and device helpers shared by the
+// kernels. Not part of the ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/fdms.h"
+
+namespace fdms {
+
+constexpr int kBlockSlots = 64;        // slots per pool block (= FP8 scale granularity)
+constexpr int kMaxGroup = 8;
+
+// Device-side counters and the sticky error word.
+struct DevCounters {
+  unsigned long long blocks_next;      // bump allocator over the pool
+  unsigned long long saturations;      // FP8 elements clipped on write
+  int error;                           // first error code latched (fdms_status)
+  int pad;
+  unsigned long long slots_decoded;    // cumulative units scanned by decode calls
+  unsigned long long decode_calls;
+  // stats scratch (filled by the stats kernel)
+  unsigned long long tokens, slots_store, slots_ring;
+};
+
+// Everything a kernel needs to find a head's data. Passed by value.
+//
+// Head index hi = (layer * Bmax + seq) * Hkv + kv_head.
+//   block_table[hi * max_blocks + j]   physical block of the head's j-th store block
+//   bt_scale[(hi * max_blocks + j) * 2 + {0,1}]  K / V scale of that block
+//   store_len[hi], tok_n[hi], tok_r[hi]
+//   ring:      hi * 2 * R * RB bytes; K rows [R][RB] then V rows [R][RB]
+//              (position p lives in slot p % R)
+//   ring_keep: hi * Rpad bytes
+//   head_scale[hi * 2 + {0,1}]         FP8 scale of K / V
+// Pool block b: K rows [64][RB] at pool + b * 2 * 64 * RB, V rows right after;
+//   blk_pos[b * 64 + row] is the token position of each slot.
+struct CacheView {
+  uint8_t* pool;
+  int32_t* blk_pos;
+  float* bt_scale;
+  int32_t* block_table;
+  int32_t* store_len;
+  int32_t* tok_n;
+  int32_t* tok_r;
+  uint8_t* ring;
+  uint8_t* ring_keep;
+  float* head_scale;
+  DevCounters* ctr;
+  long long num_blocks;
+  int L, Bmax, Hq, Hkv, G, D, RB, W, P, R, Rpad, max_blocks, max_seq_len;
+  int fp8;
+  float softmax_scale;
+};
+
+__host__ __device__ inline long long head_index(const CacheView& c, int layer, int seq, int h) {
+  return ((long long)layer * c.Bmax + seq) * c.Hkv + h;
+}
+__host__ __device__ inline uint8_t* block_k(const CacheView& c, long long blk) {
+  return c.pool + blk * 2LL * kBlockSlots * c.RB;
+}
+__host__ __device__ inline uint8_t* block_v(const CacheView& c, long long blk) {
+  return block_k(c, blk) + (long long)kBlockSlots * c.RB;
+}
+__host__ __device__ inline uint8_t* ring_k(const CacheView& c, long long hi) {
+  return c.ring + hi * 2LL * c.R * c.RB;
+}
+__host__ __device__ inline uint8_t* ring_v(const CacheView& c, long long hi) {
+  return ring_k(c, hi) + (long long)c.R * c.RB;
+}
+
+// Decode workspace (split partials and the plan the combine reads back).
+struct DecodeWork {
+  float* part_o;          // [max_parts][G][D], unnormalised sum of p * v
+  float* part_ml;         // [max_parts][G][2]: running max (log2 domain) and sum
+  long long* head_off;    // [heads + 1]: prefix of units over the call's heads
+  int* n_eff;             // split CTAs actually used
+  int max_parts;
+  int max_ctas;
+};
+
+__device__ inline void latch_error(DevCounters* ctr, int code) {
+  atomicCAS(&ctr->error, 0, code);
+}
+
+// ---------------------------------------------------------------- numerics
+__device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// f32 -> bf16 bits, round to nearest even
+__device__ __forceinline__ uint16_t f32_to_bf16_rn(float x) {
+  uint16_t r;
+  asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(x));
+  return r;
+}
+
+// two E4M3 codes (low byte first) -> two f32, exact (via f16x2)
+__device__ __forceinline__ float2 e4m3x2_to_f32x2(uint16_t two) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(two));
+  float lo, hi;
+  asm("{.reg .f16 a, b;\n mov.b32 {a, b}, %2;\n cvt.f32.f16 %0, a;\n cvt.f32.f16 %1, b;}"
+      : "=f"(lo), "=f"(hi) : "r"(h));
+  return make_float2(lo, hi);
+}
+
+// two f32 -> two E4M3 codes (x0 in the low byte), round to nearest even, satfinite
+__device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float x0, float x1) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(x1), "f"(x0));
+  return r;
+}
+
+// packed fp32 fused multiply-add (sm_100): d = a * b + c on both lanes
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{.reg .b64 ra, rb, rc, rd;\n"
+      " mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n mov.b64 rc, {%6, %7};\n"
+      " fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0, %1}, rd;}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// ------------------------------------------------- bulk copy + mbarrier (PTX)
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count));
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+               ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
+}
+// returns true once the phase with the given parity has completed
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p;\n"
+      "  mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      "  selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+// global -> shared bulk copy (no multicast), completion counted on `bar`
+__device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src, uint32_t bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_addr(dst_smem)), "l"(src), "r"(bytes), "r"(smem_addr(bar)) : "memory");
+}
+
+// Programmatic dependent launch: wait for the preceding grid's memory, and let
+// the next grid start its prologue.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;");
+}
+
+}  // namespace fdms
+
+// Host-side cache object.
+struct fdms_cache {
+  fdms_config cfg;
+  int device;
+  int num_sms;
+  fdms::CacheView view;
+  fdms::DecodeWork work;
+  size_t bytes_reserved;
+  // allocations (freed at destroy)
+  void* allocs[32];
+  int nallocs;
+  int decode_ctas;        // split grid used
+  int ctas_per_sm;
+};
+
+// launchers (defined in their .cu files)
+fdms_status fdms_launch_append(fdms_cache* c, int layer, int batch, const int32_t* n_new,
+                               int max_new, const void* k, const void* v, const uint8_t* keep,
+                               const float* kv_scale, cudaStream_t s);
+fdms_status fdms_launch_decode(fdms_cache* c, int layer, int batch, const void* q, void* out,
+                               int out_f32, float* lse, cudaStream_t s);
+fdms_status fdms_decode_setup(fdms_cache* c);

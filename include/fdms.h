@@ -1,0 +1,193 @@
+/*
+ * fdms.h - C ABI of the compact-KV decode-attention library (sm_100a).
+ *
+ * The method: DMS learns, per attention head, which tokens' KV slots to drop;
+ * FastDMS keeps only the survivors, in a compact store that physically
+ * reclaims the dropped slots, next to a staging area, and decodes over that
+ * store in BF16 or FP8 ("FastDMS: 6.4X KV-cache compression running faster
+ * than vLLM BF16/FP8", aiwitness.kr/community/1t3vlrx: the paragraphs on DMS
+ * per-head eviction and on the compact store, and the KV-memory table with its
+ * BF16 / FP8 columns and "KV/stage memory = cache, or cache + staging").
+ *
+ * This library holds that cache on one GPU and runs the three steps of a decode
+ * layer on it:
+ *   fdms_append_evict  - append new tokens, apply the keep decision of tokens
+ *                        that leave the recent window, compact survivors;
+ *   fdms_decode_attn   - single-token attention of every query head over the
+ *                        survivors of its kv head (split over the GPU, then
+ *                        merged);
+ *   fdms_cache_stats   - counters, including compact vs dense-equivalent bytes
+ *                        (the quantity of the pages' KV-memory table).
+ *
+ * Semantics (the pages give none in detail; these are the readings used):
+ *   - Per (layer, seq, kv head) the tokens have positions 0..n-1. Token j is
+ *     visible to decode iff j >= n - W (recent window) or keep[j] = 1.
+ *   - A token's keep bit is applied when it is resolved: resolution runs after
+ *     an append that leaves at least P out-of-window tokens unresolved, and then
+ *     resolves all of them (P = 1: each token as it leaves the window). Kept
+ *     tokens are appended, in position order, to the head's compact store;
+ *     the others are dropped and their memory is never used.
+ *   - Unresolved tokens (at most W + P - 1 per head) live in a per-head ring:
+ *     the staging area.
+ *   - Query head i reads kv head floor(i / G), G = num_q_heads / num_kv_heads.
+ *   - Decode runs after the step's token is appended (it attends to itself).
+ *   - FP8 E4M3 cache: each (layer, seq, kv head) gets one fp32 scale for K and
+ *     one for V at its first append (max(amax, 2^-126) / 448 over that call's
+ *     values, or the caller's); a value is stored as
+ *     e4m3_rne_satfinite(fp32(x) / scale). Each 64-slot store block carries its
+ *     own scale pair, which decode applies per block.
+ *
+ * Memory and ownership: the cache owns all device memory it allocates at
+ * fdms_cache_create (pool, tables, ring, decode workspace) and frees it at
+ * fdms_cache_destroy. The caller owns every buffer passed in (inputs, outputs,
+ * streams) and keeps them alive until the work queued on the stream is done.
+ * No call allocates device memory after creation.
+ *
+ * Errors: every call validates its arguments on the host and returns a status
+ * before queuing any work. Calls that queue kernels are asynchronous; errors
+ * found by the device (pool exhausted, sequence too long) are latched into a
+ * sticky word with the first error code and the affected head is left
+ * unchanged; fdms_cache_stats reports the word. Device code never traps or
+ * waits without a bound.
+ *
+ * Layouts: all tensors are dense, row-major, in the order written; "bf16" is
+ * the IEEE binary32 upper half. Device pointers must be 16-byte aligned.
+ * A stream argument is a cudaStream_t (NULL = the legacy default stream).
+ */
+#ifndef FDMS_H
+#define FDMS_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct fdms_cache fdms_cache;              /* opaque, owned by the library */
+
+typedef enum {
+  FDMS_OK = 0,
+  FDMS_ERR_INVALID_ARG = 1,   /* bad argument, found on the host; nothing queued */
+  FDMS_ERR_OUT_OF_BLOCKS = 2, /* the shared block pool ran out (device-latched) */
+  FDMS_ERR_CUDA = 3,          /* a CUDA runtime call failed */
+  FDMS_ERR_UNSUPPORTED = 4,   /* configuration this build has no kernel for */
+  FDMS_ERR_DEVICE = 5,        /* other device-detected error (sequence longer than
+                                 max_seq_len, a bounded wait that ran out) */
+} fdms_status;
+
+typedef enum { FDMS_KV_BF16 = 0, FDMS_KV_FP8_E4M3 = 1 } fdms_kv_dtype;
+
+typedef struct {
+  int num_layers;        /* L >= 1 */
+  int max_batch;         /* sequence slots per layer, >= 1 */
+  int num_q_heads;       /* Hq, a multiple of num_kv_heads */
+  int num_kv_heads;      /* Hkv >= 1; G = Hq / Hkv in {1, 2, 4, 8} */
+  int head_dim;          /* D in {64, 128} */
+  int window;            /* W >= 0: always-visible recent tokens */
+  int compact_period;    /* P >= 1: resolve out-of-window tokens P at a time */
+  int max_seq_len;       /* tokens one (layer, seq) may hold, >= 1 */
+  long long num_blocks;  /* 64-slot blocks in the shared pool; 0 = enough for
+                            max_seq_len tokens in every (layer, seq, kv head) */
+  fdms_kv_dtype kv_dtype;
+  float softmax_scale;   /* 0 -> 1 / sqrt(head_dim) */
+  int decode_ctas;       /* split-kernel grid; 0 -> SM count x CTAs per SM */
+} fdms_config;
+
+typedef struct {
+  long long tokens_appended;   /* sum over (layer, seq) of tokens appended */
+  long long slots_store;       /* survivors in compact stores, all heads */
+  long long slots_ring;        /* unresolved tokens in rings, all heads */
+  long long blocks_used;       /* pool blocks handed out */
+  long long blocks_free;       /* pool blocks left */
+  long long bytes_compact;     /* (slots_store + slots_ring) * 2 * D * element bytes */
+  long long bytes_dense_equiv; /* tokens_appended * num_kv_heads * 2 * D * element
+                                  bytes: what a dense cache of the same dtype holds */
+  long long bytes_reserved;    /* device bytes the cache allocated */
+  long long fp8_saturations;   /* FP8: stored elements clipped to +-448 */
+  long long slots_decoded;     /* cumulative slots (K row + V row each) read by
+                                  decode calls: store slots plus ring slots */
+  long long decode_calls;      /* decode calls so far */
+  int error;                   /* sticky device error (an fdms_status), 0 if none */
+} fdms_stats;
+
+typedef struct {
+  int num_tokens;  /* n: tokens appended to this (layer, seq, kv head) */
+  int resolved;    /* r: positions resolved (store or dropped) */
+  int store_len;   /* survivors in the compact store */
+  int ring_len;    /* n - r: tokens in the ring */
+} fdms_head_info;
+
+/* Short English name of a status. Never NULL. */
+const char* fdms_status_string(fdms_status s);
+
+/* Create a cache on `device` and zero its state on `stream` (the call waits for
+ * that work). *out receives the handle. Returns INVALID_ARG for a bad config,
+ * UNSUPPORTED for a head_dim / group size without a kernel, CUDA when device
+ * memory cannot be had (nothing is left allocated). */
+fdms_status fdms_cache_create(const fdms_config* cfg, int device, void* stream,
+                              fdms_cache** out);
+
+/* Free everything the cache allocated. Synchronises the device first. NULL is OK. */
+fdms_status fdms_cache_destroy(fdms_cache* cache);
+
+/* Append tokens to sequences 0..batch-1 of `layer` and run eviction/compaction.
+ *   n_new_dev     int32 [batch], device: tokens appended to each sequence,
+ *                 0..max_new (values outside that range latch DEVICE).
+ *   k_dev, v_dev  bf16 [batch][max_new][Hkv][D], device; row t of sequence b is
+ *                 its position n_b + t.
+ *   keep_dev      uint8 [batch][max_new][Hkv], device; nonzero = keep the slot
+ *                 when it is resolved (the DMS decision).
+ *   kv_scale_dev  FP8 only, optional: float [batch][Hkv][2] (K, V scales) used
+ *                 for sequences that receive their first tokens in this call;
+ *                 NULL = max(amax, 2^-126) / 448 of this call's values per head.
+ *                 Must be NULL for a BF16 cache.
+ * A sequence that would exceed max_seq_len is left unchanged and latches DEVICE.
+ * A head whose survivors do not fit in the pool is left unchanged and latches
+ * OUT_OF_BLOCKS. */
+fdms_status fdms_append_evict(fdms_cache* cache, int layer, int batch,
+                              const int32_t* n_new_dev, int max_new,
+                              const void* k_dev, const void* v_dev,
+                              const uint8_t* keep_dev, const float* kv_scale_dev,
+                              void* stream);
+
+/* Decode attention of sequences 0..batch-1 of `layer`:
+ *   q_dev    bf16 [batch][Hq][D], device.
+ *   out_dev  bf16 [batch][Hq][D], device: softmax(scale * q K_S^T) V_S over the
+ *            visible set S of the query head's kv head, rounded to nearest even.
+ *            A head with no visible token gets zeros.
+ * The split partials live in the cache's workspace, so two decode calls on one
+ * cache must not overlap (queue them on one stream). */
+fdms_status fdms_decode_attn(fdms_cache* cache, int layer, int batch,
+                             const void* q_dev, void* out_dev, void* stream);
+
+/* fdms_decode_attn with fp32 output and, if lse_dev is not NULL, the natural
+ * log of the softmax denominator per query head (float [batch][Hq], -inf for an
+ * empty head): log sum_{j in S} exp(scale * q.k_j). */
+fdms_status fdms_decode_attn_f32(fdms_cache* cache, int layer, int batch,
+                                 const void* q_dev, float* out_dev, float* lse_dev,
+                                 void* stream);
+
+/* Gather the counters on `stream` and wait for them. */
+fdms_status fdms_cache_stats(fdms_cache* cache, fdms_stats* host_out, void* stream);
+
+/* Copy one head's contents to host memory, in position order: entries
+ * [0, store_len) are the compact store, [store_len, store_len + ring_len) the
+ * ring. Waits for `stream` first.
+ *   capacity     entries the host buffers hold (INVALID_ARG if too few).
+ *   pos_host     int32 [capacity]: token positions.
+ *   keep_host    uint8 [capacity]: keep bits (1 for store entries).
+ *   k_host/v_host  [capacity][D * element bytes]: stored payload (bf16 or E4M3).
+ *   scale_host   float [capacity][2]: (K, V) scale applied to each entry
+ *                (1.0 for BF16).
+ *   info_host    counts, always filled.
+ * Any pointer but info_host may be NULL to skip it. */
+fdms_status fdms_cache_read_head(fdms_cache* cache, int layer, int seq, int kv_head,
+                                 int capacity, int32_t* pos_host, uint8_t* keep_host,
+                                 void* k_host, void* v_host, float* scale_host,
+                                 fdms_head_info* info_host, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FDMS_H */

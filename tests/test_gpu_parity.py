@@ -1,0 +1,266 @@
+"""GPU path against the fp64 oracle, through the C ABI (needs a B200).
+
+Bars (max-abs on the decode output):
+  * BF16 cache: 3e-3 against the oracle (the stated tolerance).
+  * FP8 cache: 3e-2 against the oracle on the unquantised inputs (the stated
+    tolerance), and 3e-3 against the oracle on its own E4M3 encoding ("mirror":
+    the GPU and the oracle then differ only by fp32 vs fp64 arithmetic and the
+    final bf16 rounding).
+  * fp32 output: 2e-5 + 2e-5 * |o| against the mirror oracle. Derivation: scores
+    and sums are fp32 (unit roundoff 6e-8) over at most a few thousand terms,
+    and 2^x uses the hardware approximation (relative error below 2^-21), so
+    the relative error of o stays below ~1e-5.
+  * Compaction (positions, keep bits, lengths, payload bytes, scales) and the
+    integer counters: bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads as wk
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+from _pair import Pair, bits  # noqa: E402
+
+TOL_BF16 = 3e-3
+TOL_FP8_TRUE = 3e-2
+TOL_FP8_MIRROR = 3e-3
+
+
+def _max_err(gpu_out, ref: dict):
+    g = gpu_out.float().cpu().numpy()
+    return max(float(np.max(np.abs(g[b] - ref[b]))) for b in ref)
+
+
+def _f32_ok(gpu_f32, ref: dict):
+    g = gpu_f32.cpu().numpy().astype(np.float64)
+    for b in ref:
+        err = np.abs(g[b] - ref[b])
+        assert np.all(err <= 2e-5 + 2e-5 * np.abs(ref[b])), float(err.max())
+
+
+def run_workload(wl, steps=None, check_every=1, num_blocks=0, decode_ctas=0, prefill_seqs=None):
+    p = Pair(wl, num_blocks=num_blocks, decode_ctas=decode_ctas)
+    try:
+        for layer in range(wl.layers):
+            p.append(layer, wk.prefill_inputs(wl, layer, seqs=prefill_seqs))
+            p.check_heads(layer)
+        for step in range(wl.steps if steps is None else steps):
+            for layer in range(wl.layers):
+                p.append(layer, wk.decode_inputs(wl, layer, step))
+                q = wk.decode_query(wl, layer, step)
+                out = p.decode(layer, q)
+                ref = p.oracle_out(layer, q)
+                tol = TOL_BF16 if wl.kv_dtype == "bf16" else TOL_FP8_MIRROR
+                assert _max_err(out, ref) <= tol, (layer, step)
+                if wl.kv_dtype == "fp8_e4m3":
+                    ref_t = p.oracle_out(layer, q, mode="true")
+                    assert _max_err(out, ref_t) <= TOL_FP8_TRUE
+                if step % check_every == 0:
+                    of, lse = p.decode(layer, q, f32=True)
+                    _f32_ok(of, ref)
+                    p.check_heads(layer)
+        p.check_stats()
+    finally:
+        p.close()
+
+
+def test_tiny_workload_all_steps():
+    run_workload(wk.get("tiny"))
+
+
+# Scaled-down shapes of the larger workloads: several 64-slot pages, ragged tails,
+# all group sizes and head dims the configs use.
+SMALL = {
+    "llama_shape_c1": wk.scaled(wk.get("llama1b_c1"), layers=2, ctx=1000, steps=5),
+    "llama_shape_c3_ragged": wk.scaled(wk.get("llama1b_c8"), layers=2, batch=3, ctx=777, steps=4),
+    "qwen_shape_fp8": wk.scaled(wk.get("qwen8b_c8_fp8"), layers=2, batch=2, ctx=901, steps=4),
+    "long_fp8_p64": wk.scaled(wk.get("qwen8b_long_fp8"), layers=1, batch=4,
+                              ctx_range=(60, 1500), steps=70),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_scaled_workloads(name):
+    wl = SMALL[name]
+    run_workload(wl, check_every=max(1, wl.steps // 3))
+
+
+# Edge cases: window / period / group / head dim / dtype sweeps on tiny shapes.
+EDGE = [
+    dict(window=0, period=1), dict(window=1, period=1), dict(window=16, period=64),
+    dict(window=0, period=64), dict(window=256, period=1, ctx=100),
+    dict(q_heads=2, kv_heads=2), dict(q_heads=8, kv_heads=1), dict(q_heads=16, kv_heads=2),
+    dict(head_dim=128), dict(kv_dtype="fp8_e4m3"), dict(kv_dtype="fp8_e4m3", head_dim=64),
+    dict(kv_dtype="fp8_e4m3", q_heads=2, kv_heads=1, head_dim=128, period=5, window=3),
+]
+
+
+@pytest.mark.parametrize("i", range(len(EDGE)))
+def test_edge_shapes(i):
+    base = wk.scaled(wk.get("tiny"), ctx=200, steps=6, batch=2, rate=0.3)
+    run_workload(wk.scaled(base, **EDGE[i]))
+
+
+@pytest.mark.parametrize("ctx", [0, 1, 63, 64, 65, 127, 128, 129])
+def test_store_lengths_around_page_boundaries(ctx):
+    # W = 0, keep-all: the store length is exactly ctx + steps
+    wl = wk.scaled(wk.get("tiny"), ctx=max(ctx, 1), steps=3, window=0, rate=1.0)
+    p = Pair(wl)
+    try:
+        if ctx > 0:
+            p.append(0, wk.prefill_inputs(wl, 0))
+            p.check_heads(0)
+        for step in range(3):
+            p.append(0, wk.decode_inputs(wl, 0, step))
+            q = wk.decode_query(wl, 0, step)
+            assert _max_err(p.decode(0, q), p.oracle_out(0, q)) <= TOL_BF16
+            p.check_heads(0)
+    finally:
+        p.close()
+
+
+def test_all_evicted_outside_window_and_keep_all():
+    for rate in (0.0, 1.0):
+        run_workload(wk.scaled(wk.get("tiny"), ctx=300, steps=4, rate=rate))
+
+
+def test_empty_sequences_in_a_ragged_batch():
+    wl = wk.scaled(wk.get("llama1b_c8"), layers=1, batch=4, ctx=300, steps=3)
+    run_workload(wl, prefill_seqs=[0, 2])
+
+
+def test_single_visible_token_is_returned_exactly():
+    # W = 1, nothing kept: after each decode step only the newest token is visible
+    wl = wk.scaled(wk.get("tiny"), ctx=50, steps=3, window=1, rate=0.0)
+    p = Pair(wl)
+    try:
+        p.append(0, wk.prefill_inputs(wl, 0))
+        for step in range(3):
+            inp = wk.decode_inputs(wl, 0, step)
+            p.append(0, inp)
+            q = wk.decode_query(wl, 0, step)
+            out = p.decode(0, q)
+            G = wl.group
+            for qh in range(wl.q_heads):
+                assert torch.equal(out[0, qh].cpu(), inp["v"][0, 0, qh // G])
+    finally:
+        p.close()
+
+
+def test_decode_is_deterministic_and_split_invariant():
+    wl = wk.scaled(wk.get("llama1b_c8"), layers=1, batch=3, ctx=2000, steps=1)
+    outs = []
+    for ctas in (0, 7, 300):
+        p = Pair(wl, decode_ctas=ctas)
+        try:
+            p.append(0, wk.prefill_inputs(wl, 0))
+            p.append(0, wk.decode_inputs(wl, 0, 0))
+            q = wk.decode_query(wl, 0, 0)
+            a, _ = p.decode(0, q, f32=True)
+            b, _ = p.decode(0, q, f32=True)
+            assert torch.equal(a, b)
+            outs.append(a.cpu())
+        finally:
+            p.close()
+    for o in outs[1:]:
+        assert torch.allclose(o, outs[0], atol=1e-5, rtol=1e-5)
+
+
+def test_lse_matches_oracle():
+    wl = wk.scaled(wk.get("tiny"), ctx=300, steps=1)
+    p = Pair(wl)
+    try:
+        p.append(0, wk.prefill_inputs(wl, 0))
+        p.append(0, wk.decode_inputs(wl, 0, 0))
+        q = wk.decode_query(wl, 0, 0)
+        _, lse = p.decode(0, q, f32=True)
+        from oracle.numerics import bf16_to_f64
+        qf = bf16_to_f64(bits(q))[0]
+        G = wl.group
+        for qh in range(wl.q_heads):
+            h = qh // G
+            S = np.flatnonzero(p.oc.visible(0, 0, h))
+            k, _ = p.oc.values(0, 0, h, S)
+            s = (k @ qf[qh]) / np.sqrt(wl.head_dim)
+            ref = np.log(np.sum(np.exp(s - s.max()))) + s.max()
+            assert abs(float(lse[0, qh]) - ref) <= 1e-4 * max(1.0, abs(ref))
+    finally:
+        p.close()
+
+
+def test_caller_fp8_scales():
+    wl = wk.scaled(wk.get("tiny"), ctx=120, steps=2, kv_dtype="fp8_e4m3")
+    p = Pair(wl)
+    try:
+        sc = torch.tensor([[[0.01, 0.02], [0.005, 0.04]]], dtype=torch.float32)
+        p.append(0, wk.prefill_inputs(wl, 0), kv_scale=sc)
+        for step in range(2):
+            p.append(0, wk.decode_inputs(wl, 0, step))
+            q = wk.decode_query(wl, 0, step)
+            assert _max_err(p.decode(0, q), p.oracle_out(0, q)) <= TOL_FP8_MIRROR
+        p.check_heads(0)
+        st = p.check_stats()
+        assert st["fp8_saturations"] > 0     # 0.005 * 448 = 2.24 < max |N(0,1)|
+    finally:
+        p.close()
+
+
+def test_pool_exhaustion_latches_error_and_leaves_head_unchanged():
+    import compressed_decode_attention_fdms_b200 as fd
+    wl = wk.scaled(wk.get("tiny"), ctx=500, steps=0, window=0, rate=1.0)
+    p = Pair(wl, num_blocks=9)      # 2 heads x 8 blocks needed
+    try:
+        p.append(0, wk.prefill_inputs(wl, 0))
+        st = fd.fdms_cache_stats(p.cache)
+        assert st["error"] == fd.FDMS_ERR_OUT_OF_BLOCKS
+        infos = [fd.fdms_cache_read_head(p.cache, 0, 0, h) for h in range(2)]
+        done = [i for i in infos if i["num_tokens"] == 500]
+        untouched = [i for i in infos if i["num_tokens"] == 0]
+        assert len(done) == 1 and len(untouched) == 1
+        assert untouched[0]["store_len"] == 0
+    finally:
+        p.close()
+
+
+def test_sequence_longer_than_max_latches_device_error():
+    import compressed_decode_attention_fdms_b200 as fd
+    wl = wk.scaled(wk.get("tiny"), ctx=100, steps=0)
+    p = Pair(wl, max_seq_len=128, oracle_capacity=256)
+    try:
+        dev = "cuda:0"
+        p.append(0, wk.prefill_inputs(wl, 0))
+        more = wk.prefill_inputs(wk.scaled(wl, ctx=40), 0)     # 100 + 40 > 128
+        fd.fdms_append_evict(p.cache, 0, 1, more["n_new"].to(dev), more["max_new"],
+                             more["k"].to(dev), more["v"].to(dev), more["keep"].to(dev))
+        st = fd.fdms_cache_stats(p.cache)
+        assert st["error"] == fd.FDMS_ERR_DEVICE
+        assert fd.fdms_cache_read_head(p.cache, 0, 0, 0)["num_tokens"] == 100
+    finally:
+        p.close()
+
+
+def test_host_side_argument_errors():
+    import compressed_decode_attention_fdms_b200 as fd
+    wl = wk.get("tiny")
+    p = Pair(wl)
+    try:
+        lib = fd.load_library()
+        import ctypes
+        h = ctypes.c_void_p(p.cache.handle)
+        assert lib.fdms_append_evict(h, 5, 1, None, 1, None, None, None, None, None) == \
+            fd.FDMS_ERR_INVALID_ARG
+        assert lib.fdms_decode_attn(h, 0, 2, None, None, None) == fd.FDMS_ERR_INVALID_ARG
+        x = torch.zeros(64, dtype=torch.bfloat16, device="cuda")
+        # bf16 cache must not receive FP8 scales
+        assert lib.fdms_append_evict(h, 0, 1, ctypes.c_void_p(x.data_ptr()), 1,
+                                     ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(x.data_ptr()),
+                                     ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(x.data_ptr()),
+                                     None) == fd.FDMS_ERR_INVALID_ARG
+        assert fd.fdms_cache_stats(p.cache)["error"] == 0
+    finally:
+        p.close()
