@@ -110,6 +110,19 @@ __device__ __forceinline__ void consumer_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(128) : "memory");
 }
 
+// Barrier over the 128 consumer threads that also ORs a flag across them, so
+// that a failed wait makes every consumer leave the loop together.
+__device__ __forceinline__ bool consumer_sync_any(bool x) {
+  uint32_t r;
+  asm volatile(
+      "{ .reg .pred p, q;\n"
+      "  setp.ne.u32 p, %1, 0;\n"
+      "  bar.red.or.pred q, 1, 128, p;\n"
+      "  selp.u32 %0, 1, 0, q; }"
+      : "=r"(r) : "r"((uint32_t)x) : "memory");
+  return r != 0;
+}
+
 template <class T>
 __device__ __forceinline__ int upper_bound(const T* a, int n, T x) {
   int lo = 0, hi = n;   // first index with a[i] > x
@@ -343,11 +356,12 @@ k_decode_split(CacheView c, DecodeWork w, int layer, int batch, const uint16_t* 
 
   for (int i = 0; i < ntiles; ++i) {
     const int s = i % NSTAGE;
-    if (!mbar_wait(&full[s], (i / NSTAGE) & 1)) {
-      latch_error(c.ctr, FDMS_ERR_DEVICE);
-      break;
+    const bool ok = mbar_wait(&full[s], (i / NSTAGE) & 1);
+    TileMeta mt = meta[s];
+    if (!ok) {            // stage never filled: touch nothing of it
+      mt.nrows = 0;
+      mt.flags = 0;
     }
-    const TileMeta mt = meta[s];
     const uint8_t* Ks = smem + s * T::STAGE_BYTES;
     const uint8_t* Vs = Ks + T::KV_BYTES;
     const uint16_t* Qs = reinterpret_cast<const uint16_t*>(Vs + T::KV_BYTES);
@@ -401,7 +415,10 @@ k_decode_split(CacheView c, DecodeWork w, int layer, int batch, const uint16_t* 
         for (int g = 0; g < G; ++g) s_scores[g * kTile + row] = vis ? sc[g] * mt.ks : -INFINITY;
       }
     }
-    consumer_sync();
+    if (consumer_sync_any(!ok)) {
+      if (tid == 0) latch_error(c.ctr, FDMS_ERR_DEVICE);
+      break;
+    }
 
     // ---- online softmax, one warp per head (two heads per warp when G = 8)
 #pragma unroll
