@@ -13,10 +13,11 @@ decode call reads (a K row and a V row each).
 
 Timing: the W warm-up steps run eagerly; the K timed steps are one CUDA graph,
 captured once and replayed once between a barrier + synchronize on both sides,
-timed with CUDA events on the launching stream (max over ranks). Events inside
-the graph bracket every decode call, which gives the per-launch duration used
-for the roofline. Every step reads more compact KV than the 126 MB L2 holds, so
-no step finds the previous step's data in L2.
+timed with CUDA events on the launching stream (max over ranks). A second graph
+holds K rounds of the decode calls of every layer alone (decode changes nothing
+in the cache); its event-timed duration over the number of calls is the
+per-launch duration of the roofline. Every step (and every round) reads more
+compact KV than the 126 MB L2 holds, so nothing is found in L2 from before.
 
 N > 1 (torchrun): every rank runs its own sequences (the path shards by
 sequence with no exchange); value = bytes of all ranks / max time.
@@ -278,54 +279,59 @@ def run_native(args, wl):
                 for _ in range(L)]
     stream.synchronize()
 
-    def step(s, ev=None):
+    def step(s):
         for layer in range(L):
             inp = steps_in[s][layer]
             fd.fdms_append_evict(cache, layer, B, inp["n_new"], 1, inp["k"], inp["v"],
                                  inp["keep"], stream=stream)
-            if ev is not None:
-                ev[layer][0].record(stream)
             fd.fdms_decode_attn(cache, layer, B, qs[s][layer], outs[layer], stream=stream)
-            if ev is not None:
-                ev[layer][1].record(stream)
 
     with torch.cuda.stream(stream):
         for s in range(W):
             step(s)
     stream.synchronize()
 
-    # capture the K timed steps as one graph, with external events per decode call
-    evs = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
-            for _ in range(L)] for _ in range(K)]
+    # (1) the K timed steps as one graph
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream, capture_error_mode="thread_local"):
         for s in range(K):
-            step(W + s, evs[s])
-    st0 = fd.fdms_cache_stats(cache, stream)
+            step(W + s)
+    # (2) decode launches alone (decode reads the cache and changes nothing in
+    # it), K rounds over all layers: the per-launch duration of the roofline
+    graph_dec = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_dec, stream=stream, capture_error_mode="thread_local"):
+        for s in range(K):
+            for layer in range(L):
+                fd.fdms_decode_attn(cache, layer, B, qs[W + s][layer], outs[layer], stream=stream)
 
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        t0.record(stream)
-        graph.replay()
-        t1.record(stream)
+    def timed(g):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            torch.distributed.barrier()
         torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    elapsed_ms = t0.elapsed_time(t1)
-    st1 = fd.fdms_cache_stats(cache, stream)
-    if st1["error"]:
-        raise RuntimeError(f"device error latched: {fd.status_string(st1['error'])}")
-    slots = st1["slots_decoded"] - st0["slots_decoded"]
-    calls = st1["decode_calls"] - st0["decode_calls"]
+        st_a = fd.fdms_cache_stats(cache, stream)
+        with torch.cuda.stream(stream):       # replay on the stream the events see
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        st_b = fd.fdms_cache_stats(cache, stream)
+        if st_b["error"]:
+            raise RuntimeError(f"device error latched: {fd.status_string(st_b['error'])}")
+        return (a.elapsed_time(b), st_b["slots_decoded"] - st_a["slots_decoded"],
+                st_b["decode_calls"] - st_a["decode_calls"])
+
+    with ClockSampler(local) as clk:
+        elapsed_ms, slots, calls = timed(graph)
     assert calls == K * L, (calls, K * L)
     kv_bytes = slots * row
-    dec_ms = [evs[s][l][0].elapsed_time(evs[s][l][1]) for s in range(K) for l in range(L)]
-    dec_avg_ms = sum(dec_ms) / len(dec_ms)
-    per_launch_bytes = kv_bytes / calls + qo_bytes
+    dec_ms_total, dec_slots, dec_calls = timed(graph_dec)
+    assert dec_calls == K * L
+    dec_avg_ms = dec_ms_total / dec_calls
+    per_launch_bytes = dec_slots * row / dec_calls + qo_bytes
 
     # whole-job numbers: max time over ranks, bytes summed over ranks
     t_max, bytes_all = elapsed_ms, float(kv_bytes)
@@ -368,12 +374,14 @@ def run_native(args, wl):
                 "frac": achieved / peak, "traffic": None,
                 "kernel": "fdms_decode_attn (k_decode_split + k_decode_combine)",
                 "per_launch_bytes": per_launch_bytes, "launch_us": dec_avg_ms * 1e3,
+                "launch_timing": f"CUDA events around one graph of {K * L} back-to-back "
+                                 "decode calls (all layers, K rounds); duration / calls",
                 "peak_source": peak_src,
             },
             "clocks": clocks,
             "gpu_launches": K * L * 3,
             "kv_gb_per_step": kv_bytes / K / 1e9,
-            "decode_share_of_step": sum(dec_ms) / elapsed_ms,
+            "decode_share_of_step": dec_avg_ms * L * K / elapsed_ms,
         }
         if e2e:
             result["e2e"] = {"value": e2e["bytes"] / (e2e["ms"] * 1e-3) / 1e9, "unit": "GB/s",
@@ -384,7 +392,7 @@ def run_native(args, wl):
             bps, times, desc = oracle_sample(wl, args.cpu_seconds)
             result["cpu_baseline"] = {"value": bps / 1e9, "unit": "GB/s", "cores": 1,
                                       "kind": "oracle", "sample": desc}
-    del graph
+    del graph, graph_dec
     fd.fdms_cache_destroy(cache)
     if world > 1:
         import torch.distributed as dist
