@@ -74,17 +74,32 @@ __device__ __forceinline__ uint2 quantise8(uint4 x, float scale, unsigned& sat) 
   return make_uint2(out[0], out[1]);
 }
 
-// Copy one 16-byte vector `vec` of an input row into a cache row (quantising in
-// FP8 mode, where the cache row has half the bytes and a vector is 8 bytes of
-// output per 16 bytes of input).
+// Copy one 16-byte vector `vec` (8 bf16 values) of an input row into row `row`
+// of a cache page (quantising in FP8 mode, where it becomes 8 bytes), at its
+// place in the page's chunk permutation.
 template <bool FP8>
 __device__ __forceinline__ void put_input_vec(uint8_t* dst_row, const uint16_t* src_row, int vec,
-                                              float scale, unsigned& sat) {
+                                              float scale, unsigned& sat, int RB, bool is_v,
+                                              int row) {
   const uint4 x = *reinterpret_cast<const uint4*>(src_row + vec * 8);
   if constexpr (FP8) {
-    *reinterpret_cast<uint2*>(dst_row + vec * 8) = quantise8(x, scale, sat);
+    *reinterpret_cast<uint2*>(dst_row + swz_byte(RB, is_v, row, vec * 8)) =
+        quantise8(x, scale, sat);
   } else {
-    *reinterpret_cast<uint4*>(dst_row + vec * 16) = x;
+    *reinterpret_cast<uint4*>(dst_row + swz_byte(RB, is_v, row, vec * 16)) = x;
+  }
+}
+
+// Move one vector of a cached row between pages (ring slot -> store row).
+template <bool FP8>
+__device__ __forceinline__ void move_vec(uint8_t* dst_row, int dst_r, const uint8_t* src_row,
+                                         int src_r, int vec, int RB, bool is_v) {
+  if constexpr (FP8) {
+    *reinterpret_cast<uint2*>(dst_row + swz_byte(RB, is_v, dst_r, vec * 8)) =
+        *reinterpret_cast<const uint2*>(src_row + swz_byte(RB, is_v, src_r, vec * 8));
+  } else {
+    *reinterpret_cast<uint4*>(dst_row + swz_byte(RB, is_v, dst_r, vec * 16)) =
+        *reinterpret_cast<const uint4*>(src_row + swz_byte(RB, is_v, src_r, vec * 16));
   }
 }
 
@@ -218,20 +233,12 @@ k_append_evict(CacheView c, int layer, const int32_t* __restrict__ n_new, int ma
       uint8_t* vd = block_v(c, blk) + (long long)row * c.RB;
       if (src < n0) {   // from the ring: already in cache format
         const int slot = src % c.R;
-        const int vb = FP8 ? 8 : 16;   // cache bytes per vector
-        const uint8_t* ks = ring_k(c, hi) + (long long)slot * c.RB + vec * vb;
-        const uint8_t* vs = ring_v(c, hi) + (long long)slot * c.RB + vec * vb;
-        if constexpr (FP8) {
-          *reinterpret_cast<uint2*>(kd + vec * 8) = *reinterpret_cast<const uint2*>(ks);
-          *reinterpret_cast<uint2*>(vd + vec * 8) = *reinterpret_cast<const uint2*>(vs);
-        } else {
-          *reinterpret_cast<uint4*>(kd + vec * 16) = *reinterpret_cast<const uint4*>(ks);
-          *reinterpret_cast<uint4*>(vd + vec * 16) = *reinterpret_cast<const uint4*>(vs);
-        }
+        move_vec<FP8>(kd, row, ring_k(c, hi) + (long long)slot * c.RB, slot, vec, c.RB, false);
+        move_vec<FP8>(vd, row, ring_v(c, hi) + (long long)slot * c.RB, slot, vec, c.RB, true);
       } else {          // straight from this call's input
         const long long t = src - n0;
-        put_input_vec<FP8>(kd, k_rows + t * in_stride, vec, sk, sat);
-        put_input_vec<FP8>(vd, v_rows + t * in_stride, vec, sv, sat);
+        put_input_vec<FP8>(kd, k_rows + t * in_stride, vec, sk, sat, c.RB, false, row);
+        put_input_vec<FP8>(vd, v_rows + t * in_stride, vec, sv, sat, c.RB, true, row);
       }
       if (vec == 0) c.blk_pos[blk * kBlockSlots + row] = src;
     }
@@ -245,8 +252,10 @@ k_append_evict(CacheView c, int layer, const int32_t* __restrict__ n_new, int ma
     const int p = w0 + (int)(i / VPR), vec = (int)(i % VPR);
     const long long t = p - n0;
     const int slot = p % c.R;
-    put_input_vec<FP8>(ring_k(c, hi) + (long long)slot * c.RB, k_rows + t * in_stride, vec, sk, sat);
-    put_input_vec<FP8>(ring_v(c, hi) + (long long)slot * c.RB, v_rows + t * in_stride, vec, sv, sat);
+    put_input_vec<FP8>(ring_k(c, hi) + (long long)slot * c.RB, k_rows + t * in_stride, vec, sk, sat,
+                       c.RB, false, slot);
+    put_input_vec<FP8>(ring_v(c, hi) + (long long)slot * c.RB, v_rows + t * in_stride, vec, sv, sat,
+                       c.RB, true, slot);
     if (vec == 0) rkeep[slot] = keep_rows[t * c.Hkv] ? 1 : 0;
   }
 

@@ -145,8 +145,10 @@ fdms_status fdms_cache_create(const fdms_config* cfg, int device, void* stream,
   v.RB = v.D * (v.fp8 ? 1 : 2);
   v.W = cfg->window;
   v.P = cfg->compact_period;
-  v.R = v.W + v.P - 1;
-  v.Rpad = (v.R + 15) / 16 * 16;
+  // ring capacity: W + P - 1 unresolved tokens at most, rounded up to whole
+  // 64-slot pages so that ring pages line up with the store's page rows
+  v.R = (v.W + v.P - 1 + kBlockSlots - 1) / kBlockSlots * kBlockSlots;
+  v.Rpad = v.R;
   v.max_seq_len = cfg->max_seq_len;
   v.max_blocks = (cfg->max_seq_len + kBlockSlots - 1) / kBlockSlots;
   v.softmax_scale = cfg->softmax_scale > 0.0f ? cfg->softmax_scale
@@ -320,15 +322,24 @@ fdms_status fdms_cache_read_head(fdms_cache* c, int layer, int seq, int kv_head,
                      cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return FDMS_ERR_CUDA;
   }
+  std::vector<uint8_t> tmp((size_t)kBlockSlots * RB);
+  auto unswizzle = [&](uint8_t* dst, const uint8_t* src, int row, bool is_v) {
+    for (int b = 0; b < RB; b += 16) std::memcpy(dst + b, src + swz_byte(RB, is_v, row, b), 16);
+  };
   for (int j = 0; j < nblk && e == cudaSuccess; ++j) {
     const int rows = (len - j * kBlockSlots) < kBlockSlots ? (len - j * kBlockSlots) : kBlockSlots;
     const int base = j * kBlockSlots;
     const long long blk = bt[j];
-    if (kh) e = cudaMemcpy(kh + (size_t)base * RB, block_k(v, blk), (size_t)rows * RB,
-                           cudaMemcpyDeviceToHost);
-    if (vh && e == cudaSuccess)
-      e = cudaMemcpy(vh + (size_t)base * RB, block_v(v, blk), (size_t)rows * RB,
-                     cudaMemcpyDeviceToHost);
+    if (kh) {
+      e = cudaMemcpy(tmp.data(), block_k(v, blk), (size_t)rows * RB, cudaMemcpyDeviceToHost);
+      for (int i = 0; i < rows; ++i)
+        unswizzle(kh + (size_t)(base + i) * RB, tmp.data() + (size_t)i * RB, i, false);
+    }
+    if (vh && e == cudaSuccess) {
+      e = cudaMemcpy(tmp.data(), block_v(v, blk), (size_t)rows * RB, cudaMemcpyDeviceToHost);
+      for (int i = 0; i < rows; ++i)
+        unswizzle(vh + (size_t)(base + i) * RB, tmp.data() + (size_t)i * RB, i, true);
+    }
     if (pos_host && e == cudaSuccess)
       e = cudaMemcpy(pos_host + base, v.blk_pos + blk * kBlockSlots, (size_t)rows * 4,
                      cudaMemcpyDeviceToHost);
@@ -356,8 +367,8 @@ fdms_status fdms_cache_read_head(fdms_cache* c, int layer, int seq, int kv_head,
       const int slot = p % v.R, i = len + (p - r);
       if (pos_host) pos_host[i] = p;
       if (keep_host) keep_host[i] = rkeep[slot];
-      if (kh) std::memcpy(kh + (size_t)i * RB, rk.data() + (size_t)slot * RB, RB);
-      if (vh) std::memcpy(vh + (size_t)i * RB, rv.data() + (size_t)slot * RB, RB);
+      if (kh) unswizzle(kh + (size_t)i * RB, rk.data() + (size_t)slot * RB, slot, false);
+      if (vh) unswizzle(vh + (size_t)i * RB, rv.data() + (size_t)slot * RB, slot, true);
       if (scale_host) {
         scale_host[2 * i] = hs[0];
         scale_host[2 * i + 1] = hs[1];

@@ -8,22 +8,29 @@
 // S_h = the head's compact store plus its visible ring slots.
 //
 // Split kernel (memory bound: every byte of a visible K and V row is read once):
-//   - Work is balanced over the whole GPU by slots, not by heads: the visible
-//     slot lists of all heads of the call are laid end to end (units = store
-//     slots + ring slots) and CTA c takes units [c*T/N, (c+1)*T/N). A CTA
-//     therefore reads the same number of bytes whatever the mix of lengths;
-//     it emits one partial (m, l, o) per head it touches.
-//   - A producer warp walks the CTA's 64-slot pages (a store block, or 64 ring
-//     slots) and stages each page's K rows and V rows into shared memory with
-//     1-D bulk copies (cp.async.bulk, completion on an mbarrier), NSTAGE pages
-//     ahead. Each lane of the producer owns one stage, so the block-table load
-//     for the next page overlaps the wait for its stage to drain.
-//   - Four consumer warps compute the G x 64 scores (fp32, packed f32x2 FMA),
-//     an online softmax in the log2 domain, and accumulate p * v, all in fp32.
-//     FP8 codes are converted exactly; the block's scales multiply the scores
-//     and the probabilities, never the elements.
-// Combine kernel: per (seq, kv head) the partials of the CTAs that covered it
-// are merged: o = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c.
+//   - Work is balanced over the GPU by slots, not by heads. The slot lists of
+//     all heads of the call are laid end to end (units = store slots + ring
+//     slots) and cut into equal ranges, one per consumer warp of the grid; a
+//     warp therefore reads the same number of bytes whatever the mix of head
+//     lengths, and emits one partial (m, l, o) per head its range touches.
+//   - A producer warp walks each consumer warp's pages (64 rows of a store
+//     block, or 64 ring slots; 32 rows when a row is 256 bytes) and stages a
+//     page's K rows, V rows and the head's q into shared memory with 1-D bulk
+//     copies (cp.async.bulk, completion on an mbarrier). Rows keep their page
+//     row in shared memory, so the chunk permutation they are stored with
+//     makes the fragment loads below free of bank conflicts. Every consumer
+//     warp owns two stages (double buffering) and never waits for another.
+//   - A consumer warp computes the G x 64 scores of a page on the tensor cores
+//     (mma.sync m16n8k16, fp32 accumulate; the G query heads sharing the kv
+//     head are rows 0..G-1 of the 16-row tile), an online softmax in fp32 in
+//     the log2 domain, and p.v on the tensor cores again. p is split into a
+//     16-bit head and a 16-bit remainder so its rounding stays below 2^-16.
+//     BF16 pages feed the bf16 MMA directly. FP8 pages are converted exactly
+//     to f16 (cvt e4m3x2 -> f16x2) and q is brought into f16 range by a power
+//     of two that the score scale undoes; the page's K scale multiplies the
+//     scores and its V scale the probabilities, never the elements.
+// Combine kernel: per (seq, kv head) the partials of the warps that covered it
+// are merged: o = sum_w 2^(m_w - M) o_w / sum_w 2^(m_w - M) l_w.
 #include <cfloat>
 #include <cstdio>
 
@@ -32,8 +39,7 @@
 namespace fdms {
 namespace {
 
-constexpr int kTile = 64;              // rows per page (= pool block)
-constexpr int kMinUnitsPerCta = 64;    // a CTA gets at least one page of work
+constexpr int kMinUnitsPerRange = 64;  // a consumer warp gets at least one page of work
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
 
@@ -41,12 +47,15 @@ enum : int { kFirst = 1, kLast = 2, kRing = 4, kPending = 8 };
 
 struct TileMeta {
   int hidx;      // head of the call (b * Hkv + h)
-  int nrows;     // rows staged (<= 64)
+  int row0;      // rows [row0, row1) of the page frame hold this tile's slots
+  int row1;
   int flags;
-  int p0;        // ring tiles: position of row 0
+  int p0;        // ring tiles: position of row row0
   int thresh;    // ring tiles: positions below n - W need their keep bit
   int R;         // ring capacity (slot = p % R)
-  float ks, vs;  // K / V scale of the page
+  float ks;      // K scale of the page
+  float vrel;    // V scale of the page / the head's V scale
+  float vhead;   // the head's V scale (1 for BF16)
   long long keep_base;   // ring tiles: index of the head's ring_keep
 };
 
@@ -55,32 +64,45 @@ struct Dec {
   static constexpr int D = D_, G = G_;
   static constexpr bool FP8 = FP8_;
   static constexpr int ELT = FP8 ? 1 : 2;
-  static constexpr int RB = D * ELT;          // bytes per row
-  static constexpr int CPR = RB / 16;         // 16-byte chunks per row
-  static constexpr int EPC = 16 / ELT;        // elements per chunk
-  static constexpr int NCW = 4;               // consumer warps
+  static constexpr int RB = D * ELT;           // bytes per row
+  static constexpr int TR = RB <= 128 ? 64 : 32;   // rows per tile (a page or half a page)
+  static constexpr int NCW = 4;                // consumer warps
   static constexpr int NC = NCW * 32;
-  static constexpr int NT = NC + 32;          // + one producer warp
-  static constexpr int RPP = NC / CPR;        // rows per consumer pass
-  static constexpr int NSTAGE = RB <= 128 ? 4 : 3;
-  static constexpr int KV_BYTES = kTile * RB;
+  static constexpr int NT = NC + 32;           // + one producer warp
+  static constexpr int SPW = 2;                // stages per consumer warp
+  static constexpr int NSTAGE = NCW * SPW;
+  static constexpr int KV_BYTES = TR * RB;
   static constexpr int Q_BYTES = G * D * 2;
   static constexpr int STAGE_BYTES = 2 * KV_BYTES + ((Q_BYTES + 127) / 128) * 128;
+  static constexpr int NJ = TR / 8;            // score n-tiles (8 keys each)
+  static constexpr int NU = TR / 16;           // p.v k-steps (16 keys each)
+  static constexpr int KS = D / 16;            // q.k k-steps (16 dims each)
+  static constexpr int ND = D / 8;             // p.v n-tiles (8 dims each)
+  static constexpr int EC = 16 / ELT;          // elements per 16-byte chunk
+  static constexpr int KCPT = (RB / 16) / 4;   // K chunks per thread (1, 2 or 4)
   static_assert(NSTAGE <= 32, "one producer lane per stage");
-  static_assert(CPR <= 32 && 32 % CPR == 0, "a row's chunks stay inside one warp");
 
-  // fixed part of shared memory (the per-head arrays follow)
   static constexpr int OFF_META = NSTAGE * STAGE_BYTES;
   static constexpr int OFF_BAR = OFF_META + NSTAGE * (int)sizeof(TileMeta);
-  static constexpr int OFF_SCORES = OFF_BAR + 2 * NSTAGE * 8;
-  static constexpr int OFF_P = OFF_SCORES + G * kTile * 4;
-  static constexpr int OFF_ALPHA = OFF_P + kTile * G * 4;
-  static constexpr int OFF_RED = OFF_ALPHA + ((G * 4 + 15) / 16) * 16;
-  static constexpr int OFF_HEADS = OFF_RED + NCW * G * D * 4;
+  static constexpr int OFF_HEADS = OFF_BAR + 2 * NSTAGE * 8;
   static size_t smem_bytes(int nh) {
-    // head_off (i64), page_off (i32), len, n, r (i32), scales (2 x f32), per head
-    return 128 + OFF_HEADS + (size_t)(nh + 1) * 8 + (size_t)(nh + 1) * 4 + (size_t)nh * 4 * 3 +
-           (size_t)nh * 8 + 64;
+    // head_off (i64), page_off (i32), len, n, r (i32), head scales (2 x f32)
+    return 128 + OFF_HEADS + (size_t)(nh + 1) * 8 + (size_t)(nh + 1) * 4 +
+           (size_t)nh * 4 * 3 + (size_t)nh * 8 + 64;
+  }
+
+  // unpermuted 16-byte K chunk i (0 .. KCPT-1) of lane column t
+  __device__ static int kchunk(int t, int i) { return RB == 256 ? t + 4 * i : KCPT * t + i; }
+  // element (dim) of the row behind k-step s, slot e (0..3) of lane column t:
+  // e = 0, 1 are the fragment's k = 2t, 2t+1; e = 2, 3 are k = 2t+8, 2t+9
+  __device__ static int kdim(int t, int s, int e) {
+    const int se = 4 * s + e;
+    return kchunk(t, se / EC) * EC + se % EC;
+  }
+  // dim held by p.v n-tile d in the B columns of lane group g
+  __device__ static int vdim(int g, int d) {
+    if (RB == 256) return d < 8 ? 8 * g + d : 64 + 8 * g + (d - 8);
+    return ND * g + d;   // RB 128: 8 (bf16) or 16 (fp8) dims per lane group; RB 64: 8
   }
 };
 
@@ -106,23 +128,6 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
-__device__ __forceinline__ void consumer_sync() {
-  asm volatile("bar.sync 1, %0;" ::"n"(128) : "memory");
-}
-
-// Barrier over the 128 consumer threads that also ORs a flag across them, so
-// that a failed wait makes every consumer leave the loop together.
-__device__ __forceinline__ bool consumer_sync_any(bool x) {
-  uint32_t r;
-  asm volatile(
-      "{ .reg .pred p, q;\n"
-      "  setp.ne.u32 p, %1, 0;\n"
-      "  bar.red.or.pred q, 1, 128, p;\n"
-      "  selp.u32 %0, 1, 0, q; }"
-      : "=r"(r) : "r"((uint32_t)x) : "memory");
-  return r != 0;
-}
-
 template <class T>
 __device__ __forceinline__ int upper_bound(const T* a, int n, T x) {
   int lo = 0, hi = n;   // first index with a[i] > x
@@ -133,37 +138,70 @@ __device__ __forceinline__ int upper_bound(const T* a, int n, T x) {
   return lo;
 }
 
-// 16 bytes of K or V -> EPC floats as float2 pairs
-template <bool FP8>
-__device__ __forceinline__ void unpack16(const uint4 x, float2* f) {
-  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-  if constexpr (FP8) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      f[2 * j] = e4m3x2_to_f32x2((uint16_t)(w[j] & 0xFFFF));
-      f[2 * j + 1] = e4m3x2_to_f32x2((uint16_t)(w[j] >> 16));
-    }
+// ------------------------------------------------------------- MMA helpers
+template <bool F16>
+__device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a2, uint32_t b0,
+                                         uint32_t b1) {
+  // A rows 8..15 are padding (zero): a1 = a3 = 0
+  if constexpr (F16) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
   } else {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) f[j] = make_float2(bf16lo_to_f32(w[j]), bf16hi_to_f32(w[j]));
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
   }
 }
 
+// two f32 -> packed 16-bit pair (x0 in the low half), round to nearest even
+template <bool F16>
+__device__ __forceinline__ uint32_t pack2(float x0, float x1) {
+  uint32_t r;
+  if constexpr (F16)
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(x1), "f"(x0));
+  else
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(x1), "f"(x0));
+  return r;
+}
+template <bool F16>
+__device__ __forceinline__ float2 unpack2(uint32_t w) {
+  if constexpr (F16) {
+    float lo, hi;
+    asm("{.reg .f16 a, b;\n mov.b32 {a, b}, %2;\n cvt.f32.f16 %0, a;\n cvt.f32.f16 %1, b;}"
+        : "=f"(lo), "=f"(hi) : "r"(w));
+    return make_float2(lo, hi);
+  } else {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+  }
+}
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"((uint16_t)two));
+  return h;
+}
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
 template <class T>
-__global__ void __launch_bounds__(T::NT)
+__global__ void __launch_bounds__(T::NT, 1)
 k_decode_split(CacheView c, DecodeWork w, int layer, int batch, const uint16_t* __restrict__ q,
-               int n_launch) {
-  constexpr int D = T::D, G = T::G, RB = T::RB, CPR = T::CPR, EPC = T::EPC, NC = T::NC,
-                RPP = T::RPP, NSTAGE = T::NSTAGE, NCW = T::NCW;
+               int n_launch_ranges) {
+  constexpr int D = T::D, G = T::G, RB = T::RB, TR = T::TR, NSTAGE = T::NSTAGE,
+                NCW = T::NCW, SPW = T::SPW, NJ = T::NJ, NU = T::NU, KS = T::KS, ND = T::ND;
+  constexpr bool FP8 = T::FP8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 127) & ~(uintptr_t)127);
   TileMeta* meta = reinterpret_cast<TileMeta*>(smem + T::OFF_META);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + T::OFF_BAR);
   uint64_t* empty = full + NSTAGE;
-  float* s_scores = reinterpret_cast<float*>(smem + T::OFF_SCORES);   // [G][64]
-  float* s_p = reinterpret_cast<float*>(smem + T::OFF_P);             // [64][G]
-  float* s_alpha = reinterpret_cast<float*>(smem + T::OFF_ALPHA);     // [G]
-  float* s_red = reinterpret_cast<float*>(smem + T::OFF_RED);         // [NCW][G][D]
   const int NH = batch * c.Hkv;
   long long* head_off = reinterpret_cast<long long*>(smem + T::OFF_HEADS);   // [NH + 1]
   int* page_off = reinterpret_cast<int*>(head_off + NH + 1);                 // [NH + 1]
@@ -175,25 +213,30 @@ k_decode_split(CacheView c, DecodeWork w, int layer, int batch, const uint16_t* 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const long long hi0 = (long long)layer * c.Bmax * c.Hkv;   // first head of this layer
 
+  // stale rows of a stage are multiplied by p = 0: start from zeros, not from
+  // whatever bits shared memory held
+  for (int i = tid; i < NSTAGE * T::STAGE_BYTES / 16; i += T::NT)
+    reinterpret_cast<uint4*>(smem)[i] = make_uint4(0u, 0u, 0u, 0u);
+
   // ---- 1. units and pages of every head of the call; exclusive prefix
   {
     const int per = (NH + T::NT - 1) / T::NT;
     const int h0 = tid * per, h1 = min(NH, h0 + per);
     long long su = 0;
     int sp = 0;
+    auto pages = [](int len, int live, int r) {
+      return (len + TR - 1) / TR + (live > 0 ? (live + (r % TR) + TR - 1) / TR : 0);
+    };
     for (int h = h0; h < h1; ++h) {
       const int len = c.store_len[hi0 + h], n = c.tok_n[hi0 + h], r = c.tok_r[hi0 + h];
       s_len[h] = len;
       s_n[h] = n;
       s_r[h] = r;
-      if (T::FP8) {
-        s_hscale[2 * h] = c.head_scale[(hi0 + h) * 2];
-        s_hscale[2 * h + 1] = c.head_scale[(hi0 + h) * 2 + 1];
-      }
+      s_hscale[2 * h] = FP8 ? c.head_scale[(hi0 + h) * 2] : 1.0f;
+      s_hscale[2 * h + 1] = FP8 ? c.head_scale[(hi0 + h) * 2 + 1] : 1.0f;
       su += len + (n - r);
-      sp += (len + kTile - 1) / kTile + (n - r + kTile - 1) / kTile;
+      sp += pages(len, n - r, r);
     }
-    // block exclusive scan of (su, sp)
     long long iu = su;
     int ip = sp;
 #pragma unroll
@@ -206,17 +249,14 @@ k_decode_split(CacheView c, DecodeWork w, int layer, int batch, const uint16_t* 
     __shared__ int s_wp[T::NT / 32];
     if (lane == 31) { s_wu[warp] = iu; s_wp[warp] = ip; }
     __syncthreads();
-    long long bu = 0;
-    int bp = 0;
-    for (int i = 0; i < warp; ++i) { bu += s_wu[i]; bp += s_wp[i]; }
-    long long eu = bu + iu - su;
-    int ep = bp + ip - sp;
+    long long eu = iu - su;
+    int ep = ip - sp;
+    for (int i = 0; i < warp; ++i) { eu += s_wu[i]; ep += s_wp[i]; }
     for (int h = h0; h < h1; ++h) {
       head_off[h] = eu;
       page_off[h] = ep;
-      const int len = s_len[h], live = s_n[h] - s_r[h];
-      eu += len + live;
-      ep += (len + kTile - 1) / kTile + (live + kTile - 1) / kTile;
+      eu += s_len[h] + (s_n[h] - s_r[h]);
+      ep += pages(s_len[h], s_n[h] - s_r[h], s_r[h]);
     }
     if (tid == T::NT - 1) {
       head_off[NH] = eu;
@@ -225,8 +265,8 @@ k_decode_split(CacheView c, DecodeWork w, int layer, int batch, const uint16_t* 
     __syncthreads();
   }
   const long long total = head_off[NH];
-  const long long want = (total + kMinUnitsPerCta - 1) / kMinUnitsPerCta;
-  const int n_eff = (int)(want < n_launch ? (want > 0 ? want : 1) : n_launch);
+  const long long want = (total + kMinUnitsPerRange - 1) / kMinUnitsPerRange;
+  const int n_eff = (int)(want < n_launch_ranges ? (want > 0 ? want : 1) : n_launch_ranges);
   if (blockIdx.x == 0) {
     for (int h = tid; h <= NH; h += T::NT) w.head_off[h] = head_off[h];
     if (tid == 0) {
@@ -235,285 +275,375 @@ k_decode_split(CacheView c, DecodeWork w, int layer, int batch, const uint16_t* 
       c.ctr->decode_calls += 1ull;
     }
   }
-  if ((int)blockIdx.x >= n_eff || total == 0) return;
-  const long long gs = (long long)blockIdx.x * total / n_eff;
-  const long long ge = (long long)(blockIdx.x + 1) * total / n_eff;
-  if (gs >= ge) return;
+  if ((int)blockIdx.x * NCW >= n_eff || total == 0) return;
 
-  // global page holding global unit x
+  // page (in the call's page numbering) holding global unit x
   auto gpage = [&](long long x) -> int {
     const int h = upper_bound(head_off, NH + 1, x) - 1;
     const long long u = x - head_off[h];
     const int len = s_len[h];
-    const int lp = u < len ? (int)(u / kTile) : (len + kTile - 1) / kTile + (int)((u - len) / kTile);
+    const int lp = u < len ? (int)(u / TR)
+                           : (len + TR - 1) / TR + (int)((u - len + s_r[h] % TR) / TR);
     return page_off[h] + lp;
   };
-  const int gp_first = gpage(gs);
-  const int ntiles = gpage(ge - 1) - gp_first + 1;
+  // unit range of consumer warp cw of this CTA, and its first page / page count
+  auto range_of = [&](int cw, long long& gs, long long& ge, int& gp0, int& nt) {
+    const long long v = (long long)blockIdx.x * NCW + cw;
+    nt = 0;
+    gs = ge = 0;
+    gp0 = 0;
+    if (v >= n_eff) return;
+    gs = v * total / n_eff;
+    ge = (v + 1) * total / n_eff;
+    if (gs >= ge) return;
+    gp0 = gpage(gs);
+    nt = gpage(ge - 1) - gp0 + 1;
+  };
 
   if (tid == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], NC);
+      mbar_init(&empty[s], 1);
     }
     fence_mbar_init();
   }
   __syncthreads();
 
   if (warp == NCW) {
-    // ================= producer: lane s owns stage s, tiles s, s + NSTAGE, ...
+    // ================= producer: lane l owns stage l, i.e. consumer warp l / SPW
+    // and that warp's tiles l % SPW, l % SPW + SPW, ...
     if (lane < NSTAGE) {
-      for (int i = lane; i < ntiles; i += NSTAGE) {
-        const int gp = gp_first + i;
+      const int cw = lane / SPW;
+      long long gs, ge;
+      int gp0, nt;
+      range_of(cw, gs, ge, gp0, nt);
+      for (int k = lane % SPW; k < nt; k += SPW) {
+        const int gp = gp0 + k;
         const int hidx = upper_bound(page_off, NH + 1, gp) - 1;
         const int lp = gp - page_off[hidx];
         const int len = s_len[hidx], n = s_n[hidx], r = s_r[hidx];
-        const int sp = (len + kTile - 1) / kTile;
+        const int sp = (len + TR - 1) / TR;
         const long long hoff = head_off[hidx];
-        const long long lo = gs > hoff ? gs - hoff : 0;
-        const long long hi_u = ge - hoff;   // exclusive bound in head units
+        const long long lo = gs > hoff ? gs - hoff : 0;   // head units of this range
+        const long long hi_u = ge - hoff;
         const long long hi = hi0 + hidx;
         TileMeta mt;
         mt.hidx = hidx;
-        mt.flags = (i == 0 || lp == 0 ? kFirst : 0) |
-                   (i == ntiles - 1 || gp + 1 == page_off[hidx + 1] ? kLast : 0);
-        const uint8_t *ksrc0, *vsrc0, *ksrc1 = nullptr, *vsrc1 = nullptr;
-        int n0rows, n1rows = 0;
-        if (lp < sp) {   // store page lp
-          const long long u0 = max((long long)lp * kTile, lo);
-          const long long u1 = min((long long)min((lp + 1) * kTile, len), hi_u);
-          const int row0 = (int)(u0 - (long long)lp * kTile);
-          mt.nrows = (int)(u1 - u0);
-          const long long blk = c.block_table[hi * c.max_blocks + lp];
-          if (T::FP8) {
-            mt.ks = c.bt_scale[(hi * c.max_blocks + lp) * 2];
-            mt.vs = c.bt_scale[(hi * c.max_blocks + lp) * 2 + 1];
+        mt.flags = (k == 0 || lp == 0 ? kFirst : 0) |
+                   (k == nt - 1 || gp + 1 == page_off[hidx + 1] ? kLast : 0);
+        mt.vhead = s_hscale[2 * hidx + 1];
+        mt.p0 = mt.thresh = mt.R = 0;
+        mt.keep_base = 0;
+        const uint8_t *ksrc, *vsrc;
+        if (lp < sp) {   // store page lp: block lp * TR / 64, rows from (lp * TR) % 64
+          const long long u0 = max((long long)lp * TR, lo);
+          const long long u1 = min((long long)min((lp + 1) * TR, len), hi_u);
+          const int j = lp * TR / kBlockSlots;
+          const int rb = (lp * TR) % kBlockSlots;          // block row of frame row 0
+          mt.row0 = (int)(u0 - (long long)lp * TR);
+          mt.row1 = (int)(u1 - (long long)lp * TR);
+          const long long blk = c.block_table[hi * c.max_blocks + j];
+          if (FP8) {
+            mt.ks = c.bt_scale[(hi * c.max_blocks + j) * 2];
+            mt.vrel = c.bt_scale[(hi * c.max_blocks + j) * 2 + 1] / mt.vhead;
           } else {
-            mt.ks = mt.vs = 1.0f;
+            mt.ks = mt.vrel = 1.0f;
           }
-          ksrc0 = block_k(c, blk) + (long long)row0 * RB;
-          vsrc0 = block_v(c, blk) + (long long)row0 * RB;
-          n0rows = mt.nrows;
-        } else {         // ring page lp - sp: units len + 64 * (lp - sp) ...
-          const int rp = lp - sp;
-          const long long u0 = max((long long)len + (long long)rp * kTile, lo);
-          const long long u1 = min((long long)len + min((rp + 1) * kTile, n - r), hi_u);
-          mt.nrows = (int)(u1 - u0);
-          mt.p0 = r + (int)(u0 - len);
+          ksrc = block_k(c, blk) + (long long)(rb + mt.row0) * RB;
+          vsrc = block_v(c, blk) + (long long)(rb + mt.row0) * RB;
+        } else {         // ring page: live units [TR*rp - off, TR*(rp+1) - off)
+          const int rp = lp - sp, off = r % TR, live = n - r;
+          const long long a = max((long long)len + max(TR * rp - off, 0), lo);
+          const long long b = min((long long)len + min(TR * (rp + 1) - off, live), hi_u);
+          const int p0 = r + (int)(a - len);
+          const int slot0 = p0 % c.R;
+          mt.row0 = slot0 % TR;
+          mt.row1 = mt.row0 + (int)(b - a);
+          mt.p0 = p0;
           mt.thresh = n - c.W;
           mt.R = c.R;
           mt.keep_base = hi * c.Rpad;
-          mt.flags |= kRing | (mt.p0 < mt.thresh ? kPending : 0);
-          mt.ks = T::FP8 ? s_hscale[2 * hidx] : 1.0f;
-          mt.vs = T::FP8 ? s_hscale[2 * hidx + 1] : 1.0f;
-          const int slot0 = mt.p0 % c.R;
-          n0rows = min(mt.nrows, c.R - slot0);
-          n1rows = mt.nrows - n0rows;
-          ksrc0 = ring_k(c, hi) + (long long)slot0 * RB;
-          vsrc0 = ring_v(c, hi) + (long long)slot0 * RB;
-          ksrc1 = ring_k(c, hi);
-          vsrc1 = ring_v(c, hi);
+          mt.flags |= kRing | (p0 < mt.thresh ? kPending : 0);
+          mt.ks = s_hscale[2 * hidx];
+          mt.vrel = 1.0f;
+          ksrc = ring_k(c, hi) + (long long)slot0 * RB;
+          vsrc = ring_v(c, hi) + (long long)slot0 * RB;
         }
         const int s = lane;
-        const int k = i / NSTAGE;
-        if (k > 0 && !mbar_wait(&empty[s], (k - 1) & 1)) {
+        const int use = k / SPW;
+        if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1)) {
           latch_error(c.ctr, FDMS_ERR_DEVICE);
           break;
         }
         meta[s] = mt;
         uint8_t* kdst = smem + s * T::STAGE_BYTES;
         uint8_t* vdst = kdst + T::KV_BYTES;
-        const bool first = (mt.flags & kFirst) != 0;
-        const uint32_t bytes = 2u * mt.nrows * RB + (first ? (uint32_t)T::Q_BYTES : 0u);
-        mbar_arrive_expect_tx(&full[s], bytes);
-        bulk_g2s(kdst, ksrc0, n0rows * RB, &full[s]);
-        bulk_g2s(vdst, vsrc0, n0rows * RB, &full[s]);
-        if (n1rows > 0) {
-          bulk_g2s(kdst + n0rows * RB, ksrc1, n1rows * RB, &full[s]);
-          bulk_g2s(vdst + n0rows * RB, vsrc1, n1rows * RB, &full[s]);
-        }
-        if (first) {
-          const int b = hidx / c.Hkv, h = hidx % c.Hkv;
-          const uint16_t* qsrc = q + ((long long)b * c.Hq + (long long)h * G) * D;
-          bulk_g2s(vdst + T::KV_BYTES, qsrc, T::Q_BYTES, &full[s]);
-        }
+        const uint32_t rows = (uint32_t)(mt.row1 - mt.row0);
+        mbar_arrive_expect_tx(&full[s], 2u * rows * RB + (uint32_t)T::Q_BYTES);
+        bulk_g2s(kdst + mt.row0 * RB, ksrc, rows * RB, &full[s]);
+        bulk_g2s(vdst + mt.row0 * RB, vsrc, rows * RB, &full[s]);
+        const int b = hidx / c.Hkv, h = hidx % c.Hkv;
+        bulk_g2s(vdst + T::KV_BYTES, q + ((long long)b * c.Hq + (long long)h * G) * D, T::Q_BYTES,
+                 &full[s]);
       }
     }
     return;
   }
 
-  // ================= consumers
-  const int ch = tid % CPR;   // chunk of a row this thread owns
-  const int rs = tid / CPR;   // row subset
+  // ================= consumer warp `warp`
+  const int g = lane >> 2, t = lane & 3;
+  long long gs, ge;
+  int gp0, nt;
+  range_of(warp, gs, ge, gp0, nt);
+  const long long range_id = (long long)blockIdx.x * NCW + warp;
   const float qscale = c.softmax_scale * kLog2e;
-  float2 qf[G][EPC / 2];
-  float2 acc[G][EPC / 2];
-  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};   // softmax warps
-#pragma unroll
-  for (int g = 0; g < G; ++g)
-#pragma unroll
-    for (int e = 0; e < EPC / 2; ++e) acc[g][e] = make_float2(0.f, 0.f);
 
-  for (int i = 0; i < ntiles; ++i) {
-    const int s = i % NSTAGE;
-    const bool ok = mbar_wait(&full[s], (i / NSTAGE) & 1);
-    TileMeta mt = meta[s];
-    if (!ok) {            // stage never filled: touch nothing of it
-      mt.nrows = 0;
-      mt.flags = 0;
+  uint32_t qa[KS][2];          // q A-fragments (row g, k-steps)
+  float qmul = 0.f;            // score multiplier of row g (scale, log2 e, q's power of two)
+  int cur_hidx = -1;
+  float m_run = -INFINITY, l_run = 0.f;
+  float oacc[ND][4];
+#pragma unroll
+  for (int d = 0; d < ND; ++d) oacc[d][0] = oacc[d][1] = oacc[d][2] = oacc[d][3] = 0.f;
+
+  for (int k = 0; k < nt; ++k) {
+    const int s = warp * SPW + (k % SPW);
+    const bool ok = mbar_wait(&full[s], (k / SPW) & 1);
+    if (!__all_sync(0xffffffffu, ok)) {
+      if (lane == 0) latch_error(c.ctr, FDMS_ERR_DEVICE);
+      break;
     }
+    const TileMeta mt = meta[s];
     const uint8_t* Ks = smem + s * T::STAGE_BYTES;
     const uint8_t* Vs = Ks + T::KV_BYTES;
     const uint16_t* Qs = reinterpret_cast<const uint16_t*>(Vs + T::KV_BYTES);
-    const int nrows = mt.nrows;
+    const int row0 = mt.row0, row1 = mt.row1;
 
-    if (mt.flags & kFirst) {
+    // ---- q fragments of the head (only when the head changes)
+    if (mt.hidx != cur_hidx) {
+      cur_hidx = mt.hidx;
+      if constexpr (FP8) {
+        // f16 q scaled by 2^a so that max |q| of the row is in [2^14, 2^15)
+        float amax = 0.f;
+        if (g < G) {
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
+          for (int s2 = 0; s2 < KS; ++s2)
 #pragma unroll
-        for (int v8 = 0; v8 < EPC / 8; ++v8) {   // q is bf16: 8 elements per 16 bytes
-          const uint4 x = *reinterpret_cast<const uint4*>(Qs + g * D + ch * EPC + v8 * 8);
-          float2 f[4];
-          unpack16<false>(x, f);
+            for (int e = 0; e < 4; ++e)
+              amax = fmaxf(amax,
+                           fabsf(__uint_as_float((uint32_t)Qs[g * D + T::kdim(t, s2, e)] << 16)));
+        }
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        int ex = 0;
+        if (amax > 0.f) ex = 141 - (int)((__float_as_uint(amax) >> 23) & 0xFF);
+        ex = max(-126, min(126, ex));
+        const float up = __uint_as_float((uint32_t)(ex + 127) << 23);
+        const float down = __uint_as_float((uint32_t)(127 - ex) << 23);
+        qmul = qscale * down;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            qf[g][v8 * 4 + j] = make_float2(f[j].x * qscale, f[j].y * qscale);
-            acc[g][v8 * 4 + j] = make_float2(0.f, 0.f);
-          }
+        for (int s2 = 0; s2 < KS; ++s2) {
+          float v4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            v4[e] = g < G ? __uint_as_float((uint32_t)Qs[g * D + T::kdim(t, s2, e)] << 16) * up
+                          : 0.f;
+          qa[s2][0] = pack2<true>(v4[0], v4[1]);
+          qa[s2][1] = pack2<true>(v4[2], v4[3]);
+        }
+      } else {
+        qmul = qscale;
+#pragma unroll
+        for (int s2 = 0; s2 < KS; ++s2) {
+          const int d0 = T::kdim(t, s2, 0), d2 = T::kdim(t, s2, 2);
+          qa[s2][0] = g < G ? *reinterpret_cast<const uint32_t*>(Qs + g * D + d0) : 0u;
+          qa[s2][1] = g < G ? *reinterpret_cast<const uint32_t*>(Qs + g * D + d2) : 0u;
         }
       }
-      m_run[0] = m_run[1] = -INFINITY;
-      l_run[0] = l_run[1] = 0.0f;
+    }
+    if (mt.flags & kFirst) {
+      m_run = -INFINITY;
+      l_run = 0.f;
+#pragma unroll
+      for (int d = 0; d < ND; ++d) oacc[d][0] = oacc[d][1] = oacc[d][2] = oacc[d][3] = 0.f;
     }
 
-    // ---- scores: rows rs, rs + RPP, ... of this page
+    // ---- scores of rows 8j + (0..7): S[head g][keys 8j + 2t, 8j + 2t + 1]
+    float sc[NJ][2];
+    const float mul = qmul * mt.ks;
     const bool pend = (mt.flags & kPending) != 0;
-    for (int k0 = 0; k0 < nrows; k0 += RPP) {
-      const int row = k0 + rs;
-      const uint4 x = *reinterpret_cast<const uint4*>(Ks + row * RB + ch * 16);
-      float2 kf[EPC / 2];
-      unpack16<T::FP8>(x, kf);
-      float sc[G];
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float2 a = make_float2(0.f, 0.f);
+    for (int j = 0; j < NJ; ++j) {
+      sc[j][0] = sc[j][1] = -INFINITY;
+      if (8 * j + 8 <= row0 || 8 * j >= row1) continue;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      const int r = 8 * j + g;   // key row this lane loads for the B fragment
+      uint32_t kw[T::KCPT][4];
 #pragma unroll
-        for (int e = 0; e < EPC / 2; ++e) a = ffma2(qf[g][e], kf[e], a);
-        sc[g] = a.x + a.y;
+      for (int i = 0; i < T::KCPT; ++i) {
+        const uint4 x = *reinterpret_cast<const uint4*>(
+            Ks + r * RB + 16 * swz_chunk(RB, false, r, T::kchunk(t, i)));
+        kw[i][0] = x.x; kw[i][1] = x.y; kw[i][2] = x.z; kw[i][3] = x.w;
       }
 #pragma unroll
-      for (int off = CPR / 2; off > 0; off >>= 1)
+      for (int s2 = 0; s2 < KS; ++s2) {
+        uint32_t b0, b1;
+        if constexpr (FP8) {
+          const uint32_t wv = kw[(4 * s2) / 16][((4 * s2) % 16) / 4];   // 4 codes
+          b0 = e4m3x2_to_f16x2(wv & 0xFFFF);
+          b1 = e4m3x2_to_f16x2(wv >> 16);
+        } else {
+          const int se = 4 * s2;                      // span elements 4 s2 .. 4 s2 + 3
+          b0 = kw[se / 8][(se % 8) / 2];
+          b1 = kw[se / 8][(se % 8) / 2 + 1];
+        }
+        mma16816<FP8>(acc, qa[s2][0], qa[s2][1], b0, b1);
+      }
+      const int ra = 8 * j + 2 * t;
 #pragma unroll
-        for (int g = 0; g < G; ++g) sc[g] += __shfl_xor_sync(0xffffffffu, sc[g], off);
-      if (ch == 0 && row < nrows) {
-        bool vis = true;
-        if (pend) {
-          const int p = mt.p0 + row;
+      for (int e = 0; e < 2; ++e) {
+        const int row = ra + e;
+        bool vis = row >= row0 && row < row1;
+        if (vis && pend) {
+          const int p = mt.p0 + (row - row0);
           if (p < mt.thresh) vis = c.ring_keep[mt.keep_base + p % mt.R] != 0;
         }
-#pragma unroll
-        for (int g = 0; g < G; ++g) s_scores[g * kTile + row] = vis ? sc[g] * mt.ks : -INFINITY;
+        sc[j][e] = vis ? acc[e] * mul : -INFINITY;
       }
     }
-    if (consumer_sync_any(!ok)) {
-      if (tid == 0) latch_error(c.ctr, FDMS_ERR_DEVICE);
-      break;
-    }
 
-    // ---- online softmax, one warp per head (two heads per warp when G = 8)
+    // ---- online softmax for row g (the 4 lanes of a quad share it)
+    float mx = -INFINITY;
 #pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      const int g = warp + t * NCW;
-      if (g < G) {
-        const float s0 = lane < nrows ? s_scores[g * kTile + lane] : -INFINITY;
-        const float s1 = lane + 32 < nrows ? s_scores[g * kTile + lane + 32] : -INFINITY;
-        float mt_ = fmaxf(s0, s1);
+    for (int j = 0; j < NJ; ++j) mx = fmaxf(mx, fmaxf(sc[j][0], sc[j][1]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float mn = fmaxf(m_run, mx);
+    float alpha = 1.f;
+    float pr[NJ][2];
+    if (mn == -INFINITY) {
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mt_ = fmaxf(mt_, __shfl_xor_sync(0xffffffffu, mt_, off));
-        const float mn = fmaxf(m_run[t], mt_);
-        float p0 = 0.f, p1 = 0.f, al = 1.f;
-        if (mn != -INFINITY) {
-          p0 = fast_exp2(s0 - mn);
-          p1 = fast_exp2(s1 - mn);
-          al = fast_exp2(m_run[t] - mn);
-        }
-        float ls = p0 + p1;
+      for (int j = 0; j < NJ; ++j) pr[j][0] = pr[j][1] = 0.f;
+    } else {
+      alpha = fast_exp2(m_run - mn);
+      float ls = 0.f;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, off);
-        l_run[t] = l_run[t] * al + ls;
-        m_run[t] = mn;
-        s_p[lane * G + g] = p0 * mt.vs;
-        s_p[(lane + 32) * G + g] = p1 * mt.vs;
-        if (lane == 0) s_alpha[g] = al;
+      for (int j = 0; j < NJ; ++j) {
+        pr[j][0] = fast_exp2(sc[j][0] - mn);
+        pr[j][1] = fast_exp2(sc[j][1] - mn);
+        ls += pr[j][0] + pr[j][1];
       }
+      l_run = l_run * alpha + ls;
+      m_run = mn;
     }
-    consumer_sync();
+#pragma unroll
+    for (int d = 0; d < ND; ++d) {
+      oacc[d][0] *= alpha;
+      oacc[d][1] *= alpha;
+    }
 
-    // ---- o += p * v over the page's rows
+    // ---- o += p v, keys 16u .. 16u + 15 per k-step
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float a = s_alpha[g];
+    for (int u = 0; u < NU; ++u) {
+      if (16 * u + 16 <= row0 || 16 * u >= row1) continue;
+      const float v0 = pr[2 * u][0] * mt.vrel, v1 = pr[2 * u][1] * mt.vrel;
+      const float v2 = pr[2 * u + 1][0] * mt.vrel, v3 = pr[2 * u + 1][1] * mt.vrel;
+      const uint32_t ah0 = pack2<FP8>(v0, v1), ah2 = pack2<FP8>(v2, v3);
+      const float2 f0 = unpack2<FP8>(ah0), f2 = unpack2<FP8>(ah2);
+      const uint32_t al0 = pack2<FP8>(v0 - f0.x, v1 - f0.y);
+      const uint32_t al2 = pack2<FP8>(v2 - f2.x, v3 - f2.y);
+      // V rows 16u + 2t + {0, 1, 8, 9}: the dims of lane group g
+      const int rr[4] = {16 * u + 2 * t, 16 * u + 2 * t + 1, 16 * u + 2 * t + 8,
+                         16 * u + 2 * t + 9};
+      if constexpr (RB == 64) {     // FP8, D = 64: 8 bytes (8 dims) per row
+        uint2 x[4];
 #pragma unroll
-      for (int e = 0; e < EPC / 2; ++e) acc[g][e] = make_float2(acc[g][e].x * a, acc[g][e].y * a);
-    }
-    for (int k0 = 0; k0 < nrows; k0 += RPP) {
-      const int row = k0 + rs;
-      if (row < nrows) {
-        const uint4 x = *reinterpret_cast<const uint4*>(Vs + row * RB + ch * 16);
-        float2 vf[EPC / 2];
-        unpack16<T::FP8>(x, vf);
-        float p[G];
+        for (int i = 0; i < 4; ++i)
+          x[i] = *reinterpret_cast<const uint2*>(Vs + rr[i] * RB + 8 * g);
 #pragma unroll
-        for (int g = 0; g < G; ++g) p[g] = s_p[row * G + g];
+        for (int e = 0; e < 2; ++e) {            // words: dims 4e .. 4e + 3
+          const uint32_t a0w = e ? x[0].y : x[0].x, a1w = e ? x[1].y : x[1].x;
+          const uint32_t a8w = e ? x[2].y : x[2].x, a9w = e ? x[3].y : x[3].x;
+          const uint32_t lo01 = prmt(a0w, a1w, 0x5140), hi01 = prmt(a0w, a1w, 0x7362);
+          const uint32_t lo89 = prmt(a8w, a9w, 0x5140), hi89 = prmt(a8w, a9w, 0x7362);
+          const uint32_t b0s[4] = {e4m3x2_to_f16x2(lo01 & 0xFFFF), e4m3x2_to_f16x2(lo01 >> 16),
+                                   e4m3x2_to_f16x2(hi01 & 0xFFFF), e4m3x2_to_f16x2(hi01 >> 16)};
+          const uint32_t b1s[4] = {e4m3x2_to_f16x2(lo89 & 0xFFFF), e4m3x2_to_f16x2(lo89 >> 16),
+                                   e4m3x2_to_f16x2(hi89 & 0xFFFF), e4m3x2_to_f16x2(hi89 >> 16)};
 #pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-          for (int e = 0; e < EPC / 2; ++e) acc[g][e] = ffma2(make_float2(p[g], p[g]), vf[e], acc[g][e]);
-      }
-    }
-    mbar_arrive(&empty[s]);
-
-    if (mt.flags & kLast) {
-      // sum the row subsets: first inside the warp, then across the warps
-#pragma unroll
-      for (int off = CPR; off < 32; off <<= 1)
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-          for (int e = 0; e < EPC / 2; ++e) {
-            acc[g][e].x += __shfl_xor_sync(0xffffffffu, acc[g][e].x, off);
-            acc[g][e].y += __shfl_xor_sync(0xffffffffu, acc[g][e].y, off);
+          for (int q4 = 0; q4 < 4; ++q4) {
+            mma16816<true>(oacc[4 * e + q4], ah0, ah2, b0s[q4], b1s[q4]);
+            mma16816<true>(oacc[4 * e + q4], al0, al2, b0s[q4], b1s[q4]);
           }
-      if (lane < CPR) {
+        }
+      } else {
+        constexpr int VCH = RB == 256 ? 2 : 1;   // 16-byte chunks of a lane group per row
 #pragma unroll
-        for (int g = 0; g < G; ++g)
+        for (int ci = 0; ci < VCH; ++ci) {
+          const int chunk = RB == 256 ? g + 8 * ci : g;
+          uint4 x[4];
 #pragma unroll
-          for (int e = 0; e < EPC / 2; ++e)
-            *reinterpret_cast<float2*>(&s_red[(warp * G + g) * D + ch * EPC + 2 * e]) = acc[g][e];
-      }
-      consumer_sync();
-      const long long part = (long long)blockIdx.x + mt.hidx;
-      for (int idx = tid; idx < G * D; idx += NC) {
-        float sum = 0.f;
+          for (int i = 0; i < 4; ++i)
+            x[i] = *reinterpret_cast<const uint4*>(Vs + rr[i] * RB +
+                                                  16 * swz_chunk(RB, true, rr[i], chunk));
+          const uint32_t w0[4] = {x[0].x, x[0].y, x[0].z, x[0].w};
+          const uint32_t w1[4] = {x[1].x, x[1].y, x[1].z, x[1].w};
+          const uint32_t w8[4] = {x[2].x, x[2].y, x[2].z, x[2].w};
+          const uint32_t w9[4] = {x[3].x, x[3].y, x[3].z, x[3].w};
 #pragma unroll
-        for (int wv = 0; wv < NCW; ++wv) sum += s_red[wv * G * D + idx];
-        w.part_o[part * G * D + idx] = sum;
-      }
+          for (int e = 0; e < 4; ++e) {
+            if constexpr (FP8) {                 // 4 dims per word: n-tiles 4e .. 4e + 3
+              const uint32_t lo01 = prmt(w0[e], w1[e], 0x5140), hi01 = prmt(w0[e], w1[e], 0x7362);
+              const uint32_t lo89 = prmt(w8[e], w9[e], 0x5140), hi89 = prmt(w8[e], w9[e], 0x7362);
+              const uint32_t b0s[4] = {e4m3x2_to_f16x2(lo01 & 0xFFFF), e4m3x2_to_f16x2(lo01 >> 16),
+                                       e4m3x2_to_f16x2(hi01 & 0xFFFF), e4m3x2_to_f16x2(hi01 >> 16)};
+              const uint32_t b1s[4] = {e4m3x2_to_f16x2(lo89 & 0xFFFF), e4m3x2_to_f16x2(lo89 >> 16),
+                                       e4m3x2_to_f16x2(hi89 & 0xFFFF), e4m3x2_to_f16x2(hi89 >> 16)};
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const int g = warp + t * NCW;
-        if (g < G && lane == 0) {
-          w.part_ml[(part * G + g) * 2] = m_run[t];
-          w.part_ml[(part * G + g) * 2 + 1] = l_run[t];
+              for (int q4 = 0; q4 < 4; ++q4) {
+                mma16816<true>(oacc[4 * e + q4], ah0, ah2, b0s[q4], b1s[q4]);
+                mma16816<true>(oacc[4 * e + q4], al0, al2, b0s[q4], b1s[q4]);
+              }
+            } else {                              // 2 dims per word: n-tiles 2e, 2e + 1
+              const int d0 = 8 * ci + 2 * e;
+              const uint32_t b0a = prmt(w0[e], w1[e], 0x5410), b1a = prmt(w8[e], w9[e], 0x5410);
+              const uint32_t b0b = prmt(w0[e], w1[e], 0x7632), b1b = prmt(w8[e], w9[e], 0x7632);
+              mma16816<false>(oacc[d0], ah0, ah2, b0a, b1a);
+              mma16816<false>(oacc[d0], al0, al2, b0a, b1a);
+              mma16816<false>(oacc[d0 + 1], ah0, ah2, b0b, b1b);
+              mma16816<false>(oacc[d0 + 1], al0, al2, b0b, b1b);
+            }
+          }
         }
       }
-      consumer_sync();
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+
+    // ---- end of this head inside the range: write the partial
+    if (mt.flags & kLast) {
+      float l = l_run;
+      l += __shfl_xor_sync(0xffffffffu, l, 1);
+      l += __shfl_xor_sync(0xffffffffu, l, 2);
+      const long long part = range_id + mt.hidx;
+      if (g < G) {
+        float* po = w.part_o + (part * G + g) * D;
+#pragma unroll
+        for (int d = 0; d < ND; ++d) {
+          po[T::vdim(2 * t, d)] = oacc[d][0] * mt.vhead;
+          po[T::vdim(2 * t + 1, d)] = oacc[d][1] * mt.vhead;
+        }
+        if (t == 0) {
+          w.part_ml[(part * G + g) * 2] = m_run;
+          w.part_ml[(part * G + g) * 2 + 1] = l;
+        }
+      }
     }
   }
 }
 
-// CTA of unit x under the split: the largest c with floor(c * T / N) <= x.
-__device__ __forceinline__ int cta_of(long long x, long long total, int n) {
+// range of unit x under the split: the largest v with floor(v * T / N) <= x.
+__device__ __forceinline__ int range_of_unit(long long x, long long total, int n) {
   return (int)(((x + 1) * n - 1) / total);
 }
 
@@ -529,7 +659,7 @@ k_decode_combine(DecodeWork w, int Hkv, int Hq, int batch, void* out, float* lse
   const int n = *w.n_eff;
   float o = 0.f, M = -INFINITY, L = 0.f;
   if (e > s) {
-    const int c0 = cta_of(s, total, n), c1 = cta_of(e - 1, total, n);
+    const int c0 = range_of_unit(s, total, n), c1 = range_of_unit(e - 1, total, n);
     for (int cc = c0; cc <= c1; ++cc) {
       const long long part = (long long)cc + hidx;
       M = fmaxf(M, w.part_ml[(part * G + g) * 2]);
@@ -538,6 +668,7 @@ k_decode_combine(DecodeWork w, int Hkv, int Hq, int batch, void* out, float* lse
       for (int cc = c0; cc <= c1; ++cc) {
         const long long part = (long long)cc + hidx;
         const float m = w.part_ml[(part * G + g) * 2];
+        if (m == -INFINITY) continue;
         const float sc = exp2f(m - M);
         L += w.part_ml[(part * G + g) * 2 + 1] * sc;
         o += w.part_o[(part * G + g) * D + d] * sc;
@@ -549,7 +680,8 @@ k_decode_combine(DecodeWork w, int Hkv, int Hq, int batch, void* out, float* lse
   if constexpr (F32) {
     static_cast<float*>(out)[oi] = o;
     if (lse && d == 0)
-      lse[(long long)b * Hq + qh] = (M == -INFINITY) ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
+      lse[(long long)b * Hq + qh] =
+          (M == -INFINITY) ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
   } else {
     static_cast<uint16_t*>(out)[oi] = f32_to_bf16_rn(o);
   }
@@ -562,7 +694,8 @@ fdms_status launch_split_t(fdms_cache* cache, int layer, int batch, const void* 
   const int nh = batch * cache->view.Hkv;
   const size_t smem = T::smem_bytes(nh);
   k_decode_split<T><<<cache->decode_ctas, T::NT, smem, s>>>(
-      cache->view, cache->work, layer, batch, static_cast<const uint16_t*>(q), cache->decode_ctas);
+      cache->view, cache->work, layer, batch, static_cast<const uint16_t*>(q),
+      cache->decode_ctas * T::NCW);
   return cudaGetLastError() == cudaSuccess ? FDMS_OK : FDMS_ERR_CUDA;
 }
 
@@ -570,6 +703,7 @@ template <class T>
 fdms_status setup_t(fdms_cache* cache) {
   const int nh = cache->view.Bmax * cache->view.Hkv;
   const size_t smem = T::smem_bytes(nh);
+  if (smem > 227 * 1024) return FDMS_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(k_decode_split<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return FDMS_ERR_UNSUPPORTED;
@@ -578,6 +712,7 @@ fdms_status setup_t(fdms_cache* cache) {
           cudaSuccess || per_sm < 1)
     return FDMS_ERR_UNSUPPORTED;
   cache->ctas_per_sm = per_sm;
+  cache->ranges_per_cta = T::NCW;
   return FDMS_OK;
 }
 
@@ -622,7 +757,7 @@ fdms_status fdms_decode_setup(fdms_cache* cache) {
   const CacheView& c = cache->view;
   DecodeWork& w = cache->work;
   w.max_ctas = ctas;
-  w.max_parts = ctas + c.Bmax * c.Hkv;
+  w.max_parts = ctas * cache->ranges_per_cta + c.Bmax * c.Hkv;
   void* p = nullptr;
   auto take = [&](size_t bytes) -> void* {
     if (cudaMalloc(&p, bytes) != cudaSuccess) return nullptr;

@@ -31,7 +31,7 @@ struct DevCounters {
 //   bt_scale[(hi * max_blocks + j) * 2 + {0,1}]  K / V scale of that block
 //   store_len[hi], tok_n[hi], tok_r[hi]
 //   ring:      hi * 2 * R * RB bytes; K rows [R][RB] then V rows [R][RB]
-//              (position p lives in slot p % R)
+//              (position p lives in slot p % R; R is a multiple of 64)
 //   ring_keep: hi * Rpad bytes
 //   head_scale[hi * 2 + {0,1}]         FP8 scale of K / V
 // Pool block b: K rows [64][RB] at pool + b * 2 * 64 * RB, V rows right after;
@@ -53,6 +53,23 @@ struct CacheView {
   int fp8;
   float softmax_scale;
 };
+
+// Row layout inside a 64-row page (a store block, or 64 ring slots): the 16-byte
+// chunks of row r are stored XOR-permuted by r, so that the decode kernel's
+// tensor-core fragment loads from shared memory touch every bank once. Rows
+// keep their page-row index r in shared memory, so the permutation survives a
+// straight bulk copy. K and V rows use different permutations when rows are 256
+// bytes, the same one when they are 128 bytes, none when they are 64 bytes.
+__host__ __device__ inline int swz_chunk(int RB, bool is_v, int row, int chunk) {
+  if (RB == 128) return chunk ^ (row & 7);
+  if (RB == 256) return is_v ? (chunk ^ (row & 6)) : (chunk ^ ((row & 1) << 2));
+  return chunk;
+}
+// Byte offset inside a row of the logical byte b (the chunk permutation keeps
+// the byte's place inside its chunk).
+__host__ __device__ inline int swz_byte(int RB, bool is_v, int row, int b) {
+  return swz_chunk(RB, is_v, row, b >> 4) * 16 + (b & 15);
+}
 
 __host__ __device__ inline long long head_index(const CacheView& c, int layer, int seq, int h) {
   return ((long long)layer * c.Bmax + seq) * c.Hkv + h;
@@ -183,6 +200,7 @@ struct fdms_cache {
   int nallocs;
   int decode_ctas;        // split grid used
   int ctas_per_sm;
+  int ranges_per_cta;     // consumer warps per split CTA (one unit range each)
 };
 
 // launchers (defined in their .cu files)
