@@ -29,6 +29,7 @@ FDMS_KV_BF16, FDMS_KV_FP8_E4M3 = 0, 1
 EXPORTED = (
     "fdms_status_string", "fdms_cache_create", "fdms_cache_destroy", "fdms_append_evict",
     "fdms_decode_attn", "fdms_decode_attn_f32", "fdms_cache_stats", "fdms_cache_read_head",
+    "fdms_decode_attn_noalloc",
 )
 
 
@@ -93,6 +94,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fdms_decode_attn.argtypes = [P, I, I, P, P, P]
     lib.fdms_decode_attn_f32.restype = I
     lib.fdms_decode_attn_f32.argtypes = [P, I, I, P, P, P, P]
+    lib.fdms_decode_attn_noalloc.restype = I
+    lib.fdms_decode_attn_noalloc.argtypes = [P, I, I, P, P, P]
     lib.fdms_cache_stats.restype = I
     lib.fdms_cache_stats.argtypes = [P, ctypes.POINTER(fdms_stats), P]
     lib.fdms_cache_read_head.restype = I
@@ -225,6 +228,18 @@ def fdms_decode_attn_f32(cache: Cache, layer: int, batch: int, q: torch.Tensor,
         ctypes.c_void_p(cache.handle), layer, batch, ctypes.c_void_p(qp), ctypes.c_void_p(op),
         ctypes.c_void_p(lp), ctypes.c_void_p(_stream_ptr(stream, cache.device))),
         "fdms_decode_attn_f32")
+
+
+def fdms_decode_attn_noalloc(cache: Cache, layer: int, batch: int, q: torch.Tensor,
+                             out: torch.Tensor, stream=None):
+    """fdms_decode_attn with its scratch in the library's fixed array (no allocation)."""
+    c = cache.config
+    shape = (batch, c.num_q_heads, c.head_dim)
+    qp = _dev_tensor(q, torch.bfloat16, shape, "q", cache.device)
+    op = _dev_tensor(out, torch.bfloat16, shape, "out", cache.device)
+    _check(load_library().fdms_decode_attn_noalloc(
+        ctypes.c_void_p(cache.handle), layer, batch, ctypes.c_void_p(qp), ctypes.c_void_p(op),
+        ctypes.c_void_p(_stream_ptr(stream, cache.device))), "fdms_decode_attn_noalloc")
 
 
 def fdms_cache_stats(cache: Cache, stream=None) -> dict:

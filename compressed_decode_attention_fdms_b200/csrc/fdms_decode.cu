@@ -33,6 +33,7 @@
 // are merged: o = sum_w 2^(m_w - M) o_w / sum_w 2^(m_w - M) l_w.
 #include <cfloat>
 #include <cstdio>
+#include <mutex>
 
 #include "fdms_internal.cuh"
 
@@ -789,4 +790,90 @@ fdms_status fdms_launch_decode(fdms_cache* cache, int layer, int batch, const vo
     return cudaGetLastError() == cudaSuccess ? FDMS_OK : FDMS_ERR_CUDA;
   };
   return by_config(c, comb);
+}
+
+// ------------------------------------------------- decode without allocation
+// A fixed scratch array for fdms_decode_attn_noalloc: the split partials and the
+// plan that the combine kernel reads. Host code only learns its device address
+// through cudaGetSymbolAddress (the host-side name is a stand-in, not a device
+// pointer); device code never names it, it receives the address as arguments.
+static __device__ __align__(256) unsigned char fdms_noalloc_scratch[FDMS_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up once).
+cudaError_t scratch_address(int device, void** out) {
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_addr[device]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, fdms_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[device] = p;
+  }
+  *out = g_scratch_addr[device];
+  return cudaSuccess;
+}
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+template <class T>
+fdms_status launch_noalloc_t(fdms_cache* cache, const DecodeWork& w, int layer, int batch,
+                             const void* q, void* out, cudaStream_t s) {
+  const CacheView& c = cache->view;
+  const size_t smem = T::smem_bytes(batch * c.Hkv);
+  k_decode_split<T><<<cache->decode_ctas, T::NT, smem, s>>>(
+      c, w, layer, batch, static_cast<const uint16_t*>(q), cache->decode_ctas * T::NCW);
+  if (cudaGetLastError() != cudaSuccess) return FDMS_ERR_CUDA;
+  k_decode_combine<T::D, T::G, false><<<batch * c.Hkv, T::G * T::D, 0, s>>>(w, c.Hkv, c.Hq,
+                                                                           batch, out, nullptr);
+  return cudaGetLastError() == cudaSuccess ? FDMS_OK : FDMS_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" fdms_status fdms_decode_attn_noalloc(fdms_cache* cache, int layer, int batch,
+                                                const void* q_dev, void* out_dev, void* stream) {
+  if (!cache) return FDMS_ERR_INVALID_ARG;
+  const CacheView& c = cache->view;
+  if (layer < 0 || layer >= c.L || batch < 0 || batch > c.Bmax) return FDMS_ERR_INVALID_ARG;
+  if (batch == 0) return FDMS_OK;
+  if (!q_dev || !out_dev || (((uintptr_t)q_dev | (uintptr_t)out_dev) & 15))
+    return FDMS_ERR_INVALID_ARG;
+  if (cache->device < 0 || cache->device >= kMaxDevices) return FDMS_ERR_UNSUPPORTED;
+  // layout of the scratch for this call
+  const long long parts = (long long)cache->decode_ctas * cache->ranges_per_cta +
+                          (long long)batch * c.Hkv;
+  const size_t o_bytes = align256((size_t)parts * c.G * c.D * sizeof(float));
+  const size_t ml_bytes = align256((size_t)parts * c.G * 2 * sizeof(float));
+  const size_t off_bytes = align256((size_t)(batch * c.Hkv + 1) * sizeof(long long));
+  const size_t need = o_bytes + ml_bytes + off_bytes + 256;
+  if (need > FDMS_STATIC_SCRATCH_BYTES) return FDMS_ERR_INVALID_ARG;
+
+  int prev = -1;
+  if (cudaGetDevice(&prev) != cudaSuccess) return FDMS_ERR_CUDA;
+  if (prev != cache->device && cudaSetDevice(cache->device) != cudaSuccess) return FDMS_ERR_CUDA;
+  void* base = nullptr;
+  fdms_status st = FDMS_OK;
+  if (scratch_address(cache->device, &base) != cudaSuccess) {
+    st = FDMS_ERR_CUDA;
+  } else {
+    unsigned char* b = static_cast<unsigned char*>(base);
+    DecodeWork w;
+    w.part_o = reinterpret_cast<float*>(b);
+    w.part_ml = reinterpret_cast<float*>(b + o_bytes);
+    w.head_off = reinterpret_cast<long long*>(b + o_bytes + ml_bytes);
+    w.n_eff = reinterpret_cast<int*>(b + o_bytes + ml_bytes + off_bytes);
+    w.max_parts = (int)parts;
+    w.max_ctas = cache->decode_ctas;
+    st = by_config(c, [&](auto t) {
+      return launch_noalloc_t<decltype(t)>(cache, w, layer, batch, q_dev, out_dev,
+                                           static_cast<cudaStream_t>(stream));
+    });
+  }
+  if (prev != cache->device) cudaSetDevice(prev);
+  return st;
 }

@@ -167,6 +167,31 @@ fdms_status fdms_decode_attn_f32(fdms_cache* cache, int layer, int batch,
                                  const void* q_dev, float* out_dev, float* lse_dev,
                                  void* stream);
 
+/* Bytes of the library's fixed decode scratch array (one per device). */
+#define FDMS_STATIC_SCRATCH_BYTES (4u << 20)
+
+/* fdms_decode_attn for callers that cannot allocate device memory. The pages
+ * describe nothing like it: it exists for code that must not call cudaMalloc
+ * (or anything that allocates, torch's allocator included) on its decode path,
+ * for example a runtime whose device memory is all handed out up front by
+ * another owner, or a loop that may not allocate once it is running.
+ * Same arguments, layouts and result as fdms_decode_attn. The split partials,
+ * which fdms_decode_attn keeps in workspace the cache allocated, go instead
+ * into one static array of FDMS_STATIC_SCRATCH_BYTES compiled into the library;
+ * every device that loads the library holds that array until the process exits.
+ *   - Needs (decode CTAs x 4 + batch x Hkv) x G x (4 D + 8) bytes plus the
+ *     per-head plan; a call that needs more than the array returns
+ *     FDMS_ERR_INVALID_ARG and queues nothing.
+ *   - The first call on a device looks up the array's device address (a
+ *     runtime query, no allocation); make that first call before any stream
+ *     capture.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     behind: calls whose work overlaps on the GPU (different streams, or
+ *     different caches at once) race. Queue them on one stream.
+ * Allocates nothing and calls no allocating routine. */
+fdms_status fdms_decode_attn_noalloc(fdms_cache* cache, int layer, int batch,
+                                     const void* q_dev, void* out_dev, void* stream);
+
 /* Gather the counters on `stream` and wait for them. */
 fdms_status fdms_cache_stats(fdms_cache* cache, fdms_stats* host_out, void* stream);
 
