@@ -118,6 +118,8 @@ k_append_evict(CacheView c, int layer, const int32_t* __restrict__ n_new, int ma
   const int b = blockIdx.x / c.Hkv, h = blockIdx.x % c.Hkv;
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const long long hi = head_index(c, layer, b, h);
+  pdl_wait();                 // the previous kernel's writes are visible from here on
+  pdl_launch_dependents();
   const int m = n_new[b];
   if (m < 0 || m > max_new) {
     if (tid == 0) latch_error(c.ctr, FDMS_ERR_DEVICE);
@@ -270,6 +272,175 @@ k_append_evict(CacheView c, int layer, const int32_t* __restrict__ n_new, int ma
   }
 }
 
+
+// Decode-step path: one warp per (seq, kv head), for calls that bring at most
+// kSmallMax tokens per sequence. Same semantics as k_append_evict; the loads
+// whose addresses are known are issued together, so a decode step costs about
+// two dependent memory round trips.
+constexpr int kSmallMax = 16;
+constexpr int kSmallWarps = 8;
+
+template <bool FP8>
+__global__ void __launch_bounds__(kSmallWarps * 32)
+k_append_small(CacheView c, int layer, int batch, const int32_t* __restrict__ n_new, int max_new,
+               const uint16_t* __restrict__ k_in, const uint16_t* __restrict__ v_in,
+               const uint8_t* __restrict__ keep_in, const float* __restrict__ kv_scale) {
+  pdl_wait();                 // the previous kernel's writes are visible from here on
+  pdl_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int hid = blockIdx.x * kSmallWarps + (threadIdx.x >> 5);
+  if (hid >= batch * c.Hkv) return;
+  const int b = hid / c.Hkv, h = hid % c.Hkv;
+  const long long hi = head_index(c, layer, b, h);
+  const long long in_stride = (long long)c.Hkv * c.D;   // elements between tokens
+  const uint16_t* k_rows = k_in + ((long long)b * max_new * c.Hkv + h) * c.D;
+  const uint16_t* v_rows = v_in + ((long long)b * max_new * c.Hkv + h) * c.D;
+  const uint8_t* keep_rows = keep_in + (long long)b * max_new * c.Hkv + h;
+  uint8_t* rkeep = c.ring_keep + hi * c.Rpad;
+  const int VPR = c.D / 8;    // 16-byte input vectors per row
+
+  const int m = n_new[b];
+  const int n0 = c.tok_n[hi], r0 = c.tok_r[hi], len0 = c.store_len[hi];
+  if (m < 0 || m > max_new) {
+    if (lane == 0) latch_error(c.ctr, FDMS_ERR_DEVICE);
+    return;
+  }
+  if (m == 0) return;
+  if ((long long)n0 + m > c.max_seq_len) {
+    if (lane == 0) latch_error(c.ctr, FDMS_ERR_DEVICE);
+    return;
+  }
+  const int n1 = n0 + m;
+  const int r1 = (n1 - c.W - r0 >= c.P) ? n1 - c.W : r0;
+
+  float sk = 1.0f, sv = 1.0f;
+  if constexpr (FP8) {
+    if (n0 == 0) {
+      if (kv_scale) {
+        sk = kv_scale[((long long)b * c.Hkv + h) * 2];
+        sv = kv_scale[((long long)b * c.Hkv + h) * 2 + 1];
+      } else {
+        float ak = 0.f, av = 0.f;
+        for (int i = lane; i < m * VPR; i += 32) {
+          const long long row = i / VPR;
+          const int vec = i % VPR;
+          const uint4 xk = *reinterpret_cast<const uint4*>(k_rows + row * in_stride + vec * 8);
+          const uint4 xv = *reinterpret_cast<const uint4*>(v_rows + row * in_stride + vec * 8);
+          const uint32_t wk[4] = {xk.x, xk.y, xk.z, xk.w}, wv[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            ak = fmaxf(ak, fmaxf(fabsf(bf16lo_to_f32(wk[j])), fabsf(bf16hi_to_f32(wk[j]))));
+            av = fmaxf(av, fmaxf(fabsf(bf16lo_to_f32(wv[j])), fabsf(bf16hi_to_f32(wv[j]))));
+          }
+        }
+        for (int off = 16; off > 0; off >>= 1) {
+          ak = fmaxf(ak, __shfl_xor_sync(0xffffffffu, ak, off));
+          av = fmaxf(av, __shfl_xor_sync(0xffffffffu, av, off));
+        }
+        sk = __fdiv_rn(fmaxf(ak, 1.17549435e-38f), 448.0f);
+        sv = __fdiv_rn(fmaxf(av, 1.17549435e-38f), 448.0f);
+      }
+      if (lane == 0) {
+        c.head_scale[hi * 2] = sk;
+        c.head_scale[hi * 2 + 1] = sv;
+      }
+    } else {
+      sk = c.head_scale[hi * 2];
+      sv = c.head_scale[hi * 2 + 1];
+    }
+  }
+
+  auto keep_of = [&](int p) -> int {
+    return p < n0 ? (rkeep[p % c.R] != 0) : (keep_rows[(long long)(p - n0) * c.Hkv] != 0);
+  };
+  // survivors of positions r0 .. r1-1, and their blocks
+  int total = 0;
+  for (int base = r0; base < r1; base += 32) {
+    const int p = base + lane;
+    total += __popc(__ballot_sync(0xffffffffu, p < r1 && keep_of(p)));
+  }
+  const int len1 = len0 + total;
+  const int nb0 = (len0 + kBlockSlots - 1) / kBlockSlots;
+  const int nb1 = (len1 + kBlockSlots - 1) / kBlockSlots;
+  long long base_blk = 0;
+  if (nb1 > nb0) {
+    int fail = 0;
+    if (lane == 0) {
+      const unsigned long long need = (unsigned long long)(nb1 - nb0);
+      const unsigned long long base = atomicAdd(&c.ctr->blocks_next, need);
+      if (base + need > (unsigned long long)c.num_blocks) {
+        latch_error(c.ctr, FDMS_ERR_OUT_OF_BLOCKS);
+        fail = 1;
+      } else {
+        base_blk = (long long)base;
+      }
+    }
+    if (__shfl_sync(0xffffffffu, fail, 0)) return;
+    base_blk = __shfl_sync(0xffffffffu, base_blk, 0);
+  }
+  int32_t* bt = c.block_table + hi * c.max_blocks;
+  float* bts = c.bt_scale + hi * c.max_blocks * 2;
+  for (int j = nb0 + lane; j < nb1; j += 32) {
+    bt[j] = (int32_t)(base_blk + (j - nb0));
+    bts[2 * j] = sk;
+    bts[2 * j + 1] = sv;
+  }
+  const long long tail_blk = (len0 % kBlockSlots) ? bt[nb0 - 1] : 0;   // partly filled block
+  __syncwarp();
+
+  unsigned sat = 0;
+  int written = 0;
+  for (int base = r0; base < r1; base += 32) {
+    const int p = base + lane;
+    const unsigned ball = __ballot_sync(0xffffffffu, p < r1 && keep_of(p));
+    const int cnt = __popc(ball);
+    for (int i = lane; i < cnt * VPR; i += 32) {
+      const int sidx = i / VPR, vec = i % VPR;
+      const int src = base + (int)__fns(ball, 0, sidx + 1);
+      const int d = len0 + written + sidx;
+      const int j = d / kBlockSlots;
+      const long long blk = j < nb0 ? tail_blk : base_blk + (j - nb0);
+      const int row = d % kBlockSlots;
+      uint8_t* kd = block_k(c, blk) + (long long)row * c.RB;
+      uint8_t* vd = block_v(c, blk) + (long long)row * c.RB;
+      if (src < n0) {
+        const int slot = src % c.R;
+        move_vec<FP8>(kd, row, ring_k(c, hi) + (long long)slot * c.RB, slot, vec, c.RB, false);
+        move_vec<FP8>(vd, row, ring_v(c, hi) + (long long)slot * c.RB, slot, vec, c.RB, true);
+      } else {
+        const long long t = src - n0;
+        put_input_vec<FP8>(kd, k_rows + t * in_stride, vec, sk, sat, c.RB, false, row);
+        put_input_vec<FP8>(vd, v_rows + t * in_stride, vec, sv, sat, c.RB, true, row);
+      }
+      if (vec == 0) c.blk_pos[blk * kBlockSlots + row] = src;
+    }
+    written += cnt;
+  }
+  __syncwarp();   // ring slots read above may be overwritten below
+
+  const int w0 = r1 > n0 ? r1 : n0;
+  for (int i = lane; i < (n1 - w0) * VPR; i += 32) {
+    const int p = w0 + i / VPR, vec = i % VPR;
+    const long long t = p - n0;
+    const int slot = p % c.R;
+    put_input_vec<FP8>(ring_k(c, hi) + (long long)slot * c.RB, k_rows + t * in_stride, vec, sk,
+                       sat, c.RB, false, slot);
+    put_input_vec<FP8>(ring_v(c, hi) + (long long)slot * c.RB, v_rows + t * in_stride, vec, sv,
+                       sat, c.RB, true, slot);
+    if (vec == 0) rkeep[slot] = keep_rows[t * c.Hkv] ? 1 : 0;
+  }
+  if constexpr (FP8) {
+    for (int off = 16; off > 0; off >>= 1) sat += __shfl_xor_sync(0xffffffffu, sat, off);
+    if (lane == 0 && sat) atomicAdd(&c.ctr->saturations, (unsigned long long)sat);
+  }
+  __syncwarp();
+  if (lane == 0) {
+    c.store_len[hi] = len1;
+    c.tok_n[hi] = n1;
+    c.tok_r[hi] = r1;
+  }
+}
+
 }  // namespace
 }  // namespace fdms
 
@@ -279,14 +450,31 @@ fdms_status fdms_launch_append(fdms_cache* cache, int layer, int batch, const in
                                int max_new, const void* k, const void* v, const uint8_t* keep,
                                const float* kv_scale, cudaStream_t s) {
   const CacheView& c = cache->view;
-  const dim3 grid((unsigned)(batch * c.Hkv));
   const uint16_t* kk = static_cast<const uint16_t*>(k);
   const uint16_t* vv = static_cast<const uint16_t*>(v);
-  if (c.fp8)
-    k_append_evict<true><<<grid, kAppendThreads, 0, s>>>(c, layer, n_new, max_new, kk, vv, keep,
-                                                         kv_scale);
-  else
-    k_append_evict<false><<<grid, kAppendThreads, 0, s>>>(c, layer, n_new, max_new, kk, vv, keep,
-                                                          nullptr);
-  return cudaGetLastError() == cudaSuccess ? FDMS_OK : FDMS_ERR_CUDA;
+  const float* sc = c.fp8 ? kv_scale : nullptr;
+  cudaLaunchConfig_t cfg = {};
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
+  if (max_new <= kSmallMax) {
+    cfg.gridDim = dim3((unsigned)((batch * c.Hkv + kSmallWarps - 1) / kSmallWarps));
+    cfg.blockDim = dim3(kSmallWarps * 32);
+    e = c.fp8 ? cudaLaunchKernelEx(&cfg, k_append_small<true>, c, layer, batch, n_new, max_new,
+                                   kk, vv, keep, sc)
+              : cudaLaunchKernelEx(&cfg, k_append_small<false>, c, layer, batch, n_new, max_new,
+                                   kk, vv, keep, sc);
+  } else {
+    cfg.gridDim = dim3((unsigned)(batch * c.Hkv));
+    cfg.blockDim = dim3(kAppendThreads);
+    e = c.fp8 ? cudaLaunchKernelEx(&cfg, k_append_evict<true>, c, layer, n_new, max_new, kk, vv,
+                                   keep, sc)
+              : cudaLaunchKernelEx(&cfg, k_append_evict<false>, c, layer, n_new, max_new, kk, vv,
+                                   keep, sc);
+  }
+  return e == cudaSuccess ? FDMS_OK : FDMS_ERR_CUDA;
 }

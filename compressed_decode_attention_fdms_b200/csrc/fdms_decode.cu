@@ -1,4 +1,4 @@
-// Decode attention over the compact store: split kernel + combine kernel.
+// Decode attention over the compact store: one kernel, split and merge.
 //
 // FastDMS decodes over the survivors of per-head eviction only, reading 5-8x
 // less KV than a dense cache ("FastDMS: 6.4X KV-cache compression running
@@ -7,30 +7,35 @@
 //     o_g = sum_{j in S_h} softmax_j(scale * q_g . k_j) v_j,
 // S_h = the head's compact store plus its visible ring slots.
 //
-// Split kernel (memory bound: every byte of a visible K and V row is read once):
+// The kernel is memory bound: every byte of a visible K and V row is read once.
 //   - Work is balanced over the GPU by slots, not by heads. The slot lists of
 //     all heads of the call are laid end to end (units = store slots + ring
 //     slots) and cut into equal ranges, one per consumer warp of the grid; a
 //     warp therefore reads the same number of bytes whatever the mix of head
 //     lengths, and emits one partial (m, l, o) per head its range touches.
-//   - A producer warp walks each consumer warp's pages (64 rows of a store
-//     block, or 64 ring slots; 32 rows when a row is 256 bytes) and stages a
-//     page's K rows, V rows and the head's q into shared memory with 1-D bulk
-//     copies (cp.async.bulk, completion on an mbarrier). Rows keep their page
-//     row in shared memory, so the chunk permutation they are stored with
-//     makes the fragment loads below free of bank conflicts. Every consumer
-//     warp owns two stages (double buffering) and never waits for another.
-//   - A consumer warp computes the G x 64 scores of a page on the tensor cores
-//     (mma.sync m16n8k16, fp32 accumulate; the G query heads sharing the kv
-//     head are rows 0..G-1 of the 16-row tile), an online softmax in fp32 in
-//     the log2 domain, and p.v on the tensor cores again. p is split into a
-//     16-bit head and a 16-bit remainder so its rounding stays below 2^-16.
-//     BF16 pages feed the bf16 MMA directly. FP8 pages are converted exactly
-//     to f16 (cvt e4m3x2 -> f16x2) and q is brought into f16 range by a power
-//     of two that the score scale undoes; the page's K scale multiplies the
-//     scores and its V scale the probabilities, never the elements.
-// Combine kernel: per (seq, kv head) the partials of the warps that covered it
-// are merged: o = sum_w 2^(m_w - M) o_w / sum_w 2^(m_w - M) l_w.
+//   - A producer warp walks every consumer warp's tiles (32 rows of a 64-slot
+//     page for 128-byte rows) and stages a tile's K rows, V rows and the head's
+//     q into shared memory with 1-D bulk copies (cp.async.bulk, completion on an
+//     mbarrier). Rows keep their page row in shared memory, so the chunk
+//     permutation they are stored with makes the fragment loads below free of
+//     bank conflicts. Each of the 8 consumer warps owns two stages.
+//   - A consumer warp computes the scores of a tile on the tensor cores
+//     (mma.sync m16n8k16, fp32 accumulate; the G query heads of the kv head
+//     are rows 0..G-1 of the 16-row A tile, keys are the columns), an online
+//     softmax in fp32 in the log2 domain, and o^T += V^T p^T on the tensor
+//     cores again (head dims are the rows, heads the columns, keys the
+//     reduction): the score accumulators already have the layout of p^T's B
+//     fragments. p is split into a 16-bit head and a 16-bit remainder so its
+//     rounding stays below 2^-16 relative. FP8 pages are converted exactly to f16
+//     (cvt e4m3x2 -> f16x2) and q is brought into f16 range by a power of two
+//     that the score scale undoes; the page's K scale multiplies the scores
+//     and its V scale the probabilities, never the elements.
+//   - Merge: when a warp has written its partial for a head it counts it on
+//     the head's counter; the warp that completes the count merges all of the
+//     head's partials, o = sum_w 2^(m_w - M) o_w / sum_w 2^(m_w - M) l_w, and
+//     writes the output. Heads with no slot get zeros.
+//   - The launch allows programmatic dependent launch: set-up that reads no
+//     global memory runs while the previous kernel in the stream finishes.
 #include <cfloat>
 #include <cstdio>
 #include <mutex>
@@ -40,7 +45,7 @@
 namespace fdms {
 namespace {
 
-constexpr int kMinUnitsPerRange = 64;  // a consumer warp gets at least one page of work
+constexpr int kMinUnitsPerRange = 64;  // a consumer warp gets at least 64 slots of work
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
 
@@ -48,7 +53,7 @@ enum : int { kFirst = 1, kLast = 2, kRing = 4, kPending = 8 };
 
 struct TileMeta {
   int hidx;      // head of the call (b * Hkv + h)
-  int row0;      // rows [row0, row1) of the page frame hold this tile's slots
+  int row0;      // rows [row0, row1) of the tile frame hold this tile's slots
   int row1;
   int flags;
   int p0;        // ring tiles: position of row row0
@@ -60,14 +65,21 @@ struct TileMeta {
   long long keep_base;   // ring tiles: index of the head's ring_keep
 };
 
+// where the merged output goes
+struct OutArgs {
+  void* out;     // bf16 or fp32 [batch][Hq][D]
+  float* lse;    // fp32 [batch][Hq] or null
+  int f32;
+};
+
 template <int D_, bool FP8_, int G_>
 struct Dec {
   static constexpr int D = D_, G = G_;
   static constexpr bool FP8 = FP8_;
   static constexpr int ELT = FP8 ? 1 : 2;
   static constexpr int RB = D * ELT;           // bytes per row
-  static constexpr int TR = RB <= 128 ? 64 : 32;   // rows per tile (a page or half a page)
-  static constexpr int NCW = 4;                // consumer warps
+  static constexpr int TR = 4096 / RB;         // rows per tile: 4 KB of K, 4 KB of V
+  static constexpr int NCW = G * D >= 1024 ? 4 : 8;   // consumer warps
   static constexpr int NC = NCW * 32;
   static constexpr int NT = NC + 32;           // + one producer warp
   static constexpr int SPW = 2;                // stages per consumer warp
@@ -78,14 +90,22 @@ struct Dec {
   static constexpr int NJ = TR / 8;            // score n-tiles (8 keys each)
   static constexpr int NU = TR / 16;           // p.v k-steps (16 keys each)
   static constexpr int KS = D / 16;            // q.k k-steps (16 dims each)
-  static constexpr int ND = D / 8;             // p.v n-tiles (8 dims each)
+  static constexpr int MT = D / 16;            // p.v m-tiles (16 dims each)
   static constexpr int EC = 16 / ELT;          // elements per 16-byte chunk
-  static constexpr int KCPT = (RB / 16) / 4;   // K chunks per thread (1, 2 or 4)
+  static constexpr int KCPT = RB / 64;         // K chunks per lane column (1, 2 or 4)
+  static constexpr bool SPLIT = true;          // p = 16-bit head + 16-bit remainder
   static_assert(NSTAGE <= 32, "one producer lane per stage");
+  static_assert(TR >= 16 && TR <= 64 && 64 % TR == 0, "tiles tile a page");
+
+  // a consumer warp's unmerged partial of a head it shares with other warps:
+  // [hidx, pad x3][m x G][l x G][pad][o x G*D] floats
+  static constexpr int SLOT_O = (4 + 2 * G + 3) / 4 * 4;
+  static constexpr int SLOT_F = SLOT_O + G * D;
 
   static constexpr int OFF_META = NSTAGE * STAGE_BYTES;
   static constexpr int OFF_BAR = OFF_META + NSTAGE * (int)sizeof(TileMeta);
-  static constexpr int OFF_HEADS = OFF_BAR + 2 * NSTAGE * 8;
+  static constexpr int OFF_SLOTS = OFF_BAR + 2 * NSTAGE * 8 + 16;   // + the merge flag
+  static constexpr int OFF_HEADS = OFF_SLOTS + 2 * NCW * SLOT_F * 4;
   static size_t smem_bytes(int nh) {
     // head_off (i64), page_off (i32), len, n, r (i32), head scales (2 x f32)
     return 128 + OFF_HEADS + (size_t)(nh + 1) * 8 + (size_t)(nh + 1) * 4 +
@@ -94,16 +114,16 @@ struct Dec {
 
   // unpermuted 16-byte K chunk i (0 .. KCPT-1) of lane column t
   __device__ static int kchunk(int t, int i) { return RB == 256 ? t + 4 * i : KCPT * t + i; }
-  // element (dim) of the row behind k-step s, slot e (0..3) of lane column t:
+  // element (dim) behind q.k k-step s, slot e (0..3) of lane column t:
   // e = 0, 1 are the fragment's k = 2t, 2t+1; e = 2, 3 are k = 2t+8, 2t+9
   __device__ static int kdim(int t, int s, int e) {
     const int se = 4 * s + e;
     return kchunk(t, se / EC) * EC + se % EC;
   }
-  // dim held by p.v n-tile d in the B columns of lane group g
-  __device__ static int vdim(int g, int d) {
-    if (RB == 256) return d < 8 ? 8 * g + d : 64 + 8 * g + (d - 8);
-    return ND * g + d;   // RB 128: 8 (bf16) or 16 (fp8) dims per lane group; RB 64: 8
+  // dim of row g (hi = 0) or row g + 8 (hi = 1) of p.v m-tile i
+  __device__ static int vdim(int g, int i, int hi) {
+    if (RB == 256) return (i < 4 ? 8 * g + 2 * i : 64 + 8 * g + 2 * (i - 4)) + hi;
+    return (D / 8) * g + 2 * i + hi;
   }
 };
 
@@ -125,6 +145,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// named barrier 1 over the consumer warps (the producer warp has left)
+template <int NC>
+__device__ __forceinline__ void consumer_sync_n() {
+  asm volatile("bar.sync 1, %0;" ::"n"(NC) : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
@@ -139,23 +165,27 @@ __device__ __forceinline__ int upper_bound(const T* a, int n, T x) {
   return lo;
 }
 
+// range of unit x under the split: the largest v with floor(v * T / N) <= x.
+__device__ __forceinline__ int range_of_unit(long long x, long long total, int n) {
+  return (int)(((x + 1) * n - 1) / total);
+}
+
 // ------------------------------------------------------------- MMA helpers
 template <bool F16>
-__device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a2, uint32_t b0,
-                                         uint32_t b1) {
-  // A rows 8..15 are padding (zero): a1 = a3 = 0
+__device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
   if constexpr (F16) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%0,%1,%2,%3};"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
   } else {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%0,%1,%2,%3};"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
   }
 }
 
@@ -193,10 +223,10 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 
 template <class T>
 __global__ void __launch_bounds__(T::NT, 1)
-k_decode_split(CacheView c, DecodeWork w, int layer, int batch, const uint16_t* __restrict__ q,
-               int n_launch_ranges) {
+k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
+               const uint16_t* __restrict__ q, int n_launch_ranges) {
   constexpr int D = T::D, G = T::G, RB = T::RB, TR = T::TR, NSTAGE = T::NSTAGE,
-                NCW = T::NCW, SPW = T::SPW, NJ = T::NJ, NU = T::NU, KS = T::KS, ND = T::ND;
+                NCW = T::NCW, SPW = T::SPW, NJ = T::NJ, NU = T::NU, KS = T::KS, MT = T::MT;
   constexpr bool FP8 = T::FP8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 127) & ~(uintptr_t)127);
@@ -214,12 +244,44 @@ k_decode_split(CacheView c, DecodeWork w, int layer, int batch, const uint16_t* 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const long long hi0 = (long long)layer * c.Bmax * c.Hkv;   // first head of this layer
 
-  // stale rows of a stage are multiplied by p = 0: start from zeros, not from
-  // whatever bits shared memory held
-  for (int i = tid; i < NSTAGE * T::STAGE_BYTES / 16; i += T::NT)
-    reinterpret_cast<uint4*>(smem)[i] = make_uint4(0u, 0u, 0u, 0u);
+  // ---- set-up that reads no data the previous kernel writes: it overlaps
+  // that kernel. Stale V rows of a stage are multiplied by p = 0, so they must
+  // hold numbers: start from zeros, not from whatever bits shared memory held
+  // (stale K rows only produce scores that are then masked).
+  for (int i = tid; i < NSTAGE * (T::KV_BYTES / 16); i += T::NT) {
+    const int st = i / (T::KV_BYTES / 16), off = i % (T::KV_BYTES / 16);
+    reinterpret_cast<uint4*>(smem + st * T::STAGE_BYTES + T::KV_BYTES)[off] =
+        make_uint4(0u, 0u, 0u, 0u);
+  }
+  // warm L2 with this layer's lengths and block tables (read after the wait)
+  {
+    const int NHL = batch * c.Hkv;
+    const long long bt_lines = ((long long)NHL * c.max_blocks * 4 + 127) / 128;
+    const char* btp = reinterpret_cast<const char*>(c.block_table + hi0 * c.max_blocks);
+    for (long long i = (long long)blockIdx.x * T::NT + tid; i < bt_lines;
+         i += (long long)gridDim.x * T::NT)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(btp + i * 128));
+    if (tid < 4 && blockIdx.x < 8) {
+      const char* arr = tid == 0   ? reinterpret_cast<const char*>(c.store_len + hi0)
+                        : tid == 1 ? reinterpret_cast<const char*>(c.tok_n + hi0)
+                        : tid == 2 ? reinterpret_cast<const char*>(c.tok_r + hi0)
+                                   : reinterpret_cast<const char*>(c.head_scale + hi0 * 2);
+      const int bytes = tid == 3 ? NHL * 8 : NHL * 4;   // this layer's slice only
+      for (int j = blockIdx.x; j * 128 < bytes; j += 8)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(arr + j * 128));
+    }
+  }
+  if (tid == 0) {
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    fence_mbar_init();
+  }
+  pdl_wait();                 // the previous kernel's writes are visible from here on
+  pdl_launch_dependents();
 
-  // ---- 1. units and pages of every head of the call; exclusive prefix
+  // ---- units and pages of every head of the call; exclusive prefix
   {
     const int per = (NH + T::NT - 1) / T::NT;
     const int h0 = tid * per, h1 = min(NH, h0 + per);
@@ -268,12 +330,19 @@ k_decode_split(CacheView c, DecodeWork w, int layer, int batch, const uint16_t* 
   const long long total = head_off[NH];
   const long long want = (total + kMinUnitsPerRange - 1) / kMinUnitsPerRange;
   const int n_eff = (int)(want < n_launch_ranges ? (want > 0 ? want : 1) : n_launch_ranges);
-  if (blockIdx.x == 0) {
-    for (int h = tid; h <= NH; h += T::NT) w.head_off[h] = head_off[h];
-    if (tid == 0) {
-      *w.n_eff = n_eff;
-      c.ctr->slots_decoded += (unsigned long long)total;   // one CTA, launches are ordered
-      c.ctr->decode_calls += 1ull;
+  if (blockIdx.x == 0 && tid == 0) {
+    c.ctr->slots_decoded += (unsigned long long)total;   // one thread, launches are ordered
+    c.ctr->decode_calls += 1ull;
+  }
+  // heads without a single slot get zeros (nobody else writes them)
+  for (int h = blockIdx.x; h < NH; h += gridDim.x) {
+    if (head_off[h + 1] != head_off[h]) continue;
+    const int b = h / c.Hkv, kh = h % c.Hkv;
+    for (int i = tid; i < G * D; i += T::NT) {
+      const long long oi = ((long long)b * c.Hq + (long long)kh * G) * D + i;
+      if (oa.f32) static_cast<float*>(oa.out)[oi] = 0.f;
+      else static_cast<uint16_t*>(oa.out)[oi] = 0;
+      if (oa.lse && i % D == 0) oa.lse[(long long)b * c.Hq + kh * G + i / D] = -INFINITY;
     }
   }
   if ((int)blockIdx.x * NCW >= n_eff || total == 0) return;
@@ -301,15 +370,6 @@ k_decode_split(CacheView c, DecodeWork w, int layer, int batch, const uint16_t* 
     nt = gpage(ge - 1) - gp0 + 1;
   };
 
-  if (tid == 0) {
-    for (int s = 0; s < NSTAGE; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    fence_mbar_init();
-  }
-  __syncthreads();
-
   if (warp == NCW) {
     // ================= producer: lane l owns stage l, i.e. consumer warp l / SPW
     // and that warp's tiles l % SPW, l % SPW + SPW, ...
@@ -336,7 +396,7 @@ k_decode_split(CacheView c, DecodeWork w, int layer, int batch, const uint16_t* 
         mt.p0 = mt.thresh = mt.R = 0;
         mt.keep_base = 0;
         const uint8_t *ksrc, *vsrc;
-        if (lp < sp) {   // store page lp: block lp * TR / 64, rows from (lp * TR) % 64
+        if (lp < sp) {   // store tile lp: block lp * TR / 64, rows from (lp * TR) % 64
           const long long u0 = max((long long)lp * TR, lo);
           const long long u1 = min((long long)min((lp + 1) * TR, len), hi_u);
           const int j = lp * TR / kBlockSlots;
@@ -352,7 +412,7 @@ k_decode_split(CacheView c, DecodeWork w, int layer, int batch, const uint16_t* 
           }
           ksrc = block_k(c, blk) + (long long)(rb + mt.row0) * RB;
           vsrc = block_v(c, blk) + (long long)(rb + mt.row0) * RB;
-        } else {         // ring page: live units [TR*rp - off, TR*(rp+1) - off)
+        } else {         // ring tile: live units [TR*rp - off, TR*(rp+1) - off)
           const int rp = lp - sp, off = r % TR, live = n - r;
           const long long a = max((long long)len + max(TR * rp - off, 0), lo);
           const long long b = min((long long)len + min(TR * (rp + 1) - off, live), hi_u);
@@ -396,16 +456,17 @@ k_decode_split(CacheView c, DecodeWork w, int layer, int batch, const uint16_t* 
   long long gs, ge;
   int gp0, nt;
   range_of(warp, gs, ge, gp0, nt);
-  const long long range_id = (long long)blockIdx.x * NCW + warp;
   const float qscale = c.softmax_scale * kLog2e;
+  float* slots = reinterpret_cast<float*>(smem + T::OFF_SLOTS);
+  if (lane < 2) slots[(warp * 2 + lane) * T::SLOT_F] = __int_as_float(-1);   // empty
 
   uint32_t qa[KS][2];          // q A-fragments (row g, k-steps)
   float qmul = 0.f;            // score multiplier of row g (scale, log2 e, q's power of two)
   int cur_hidx = -1;
-  float m_run = -INFINITY, l_run = 0.f;
-  float oacc[ND][4];
+  float m_run = -INFINITY, l_run = 0.f;    // softmax state of head g (shared by its quad)
+  float oacc[MT][4];           // o^T: [dims g, g+8 of m-tile i] x [heads 2t, 2t+1]
 #pragma unroll
-  for (int d = 0; d < ND; ++d) oacc[d][0] = oacc[d][1] = oacc[d][2] = oacc[d][3] = 0.f;
+  for (int i = 0; i < MT; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
 
   for (int k = 0; k < nt; ++k) {
     const int s = warp * SPW + (k % SPW);
@@ -466,13 +527,14 @@ k_decode_split(CacheView c, DecodeWork w, int layer, int batch, const uint16_t* 
       m_run = -INFINITY;
       l_run = 0.f;
 #pragma unroll
-      for (int d = 0; d < ND; ++d) oacc[d][0] = oacc[d][1] = oacc[d][2] = oacc[d][3] = 0.f;
+      for (int i = 0; i < MT; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
     }
 
     // ---- scores of rows 8j + (0..7): S[head g][keys 8j + 2t, 8j + 2t + 1]
     float sc[NJ][2];
     const float mul = qmul * mt.ks;
     const bool pend = (mt.flags & kPending) != 0;
+    const bool full_tile = row0 == 0 && row1 == TR && !pend;
 #pragma unroll
     for (int j = 0; j < NJ; ++j) {
       sc[j][0] = sc[j][1] = -INFINITY;
@@ -498,22 +560,27 @@ k_decode_split(CacheView c, DecodeWork w, int layer, int batch, const uint16_t* 
           b0 = kw[se / 8][(se % 8) / 2];
           b1 = kw[se / 8][(se % 8) / 2 + 1];
         }
-        mma16816<FP8>(acc, qa[s2][0], qa[s2][1], b0, b1);
+        mma16816<FP8>(acc, qa[s2][0], 0u, qa[s2][1], 0u, b0, b1);
       }
       const int ra = 8 * j + 2 * t;
+      if (full_tile) {
+        sc[j][0] = acc[0] * mul;
+        sc[j][1] = acc[1] * mul;
+      } else {
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int row = ra + e;
-        bool vis = row >= row0 && row < row1;
-        if (vis && pend) {
-          const int p = mt.p0 + (row - row0);
-          if (p < mt.thresh) vis = c.ring_keep[mt.keep_base + p % mt.R] != 0;
+        for (int e = 0; e < 2; ++e) {
+          const int row = ra + e;
+          bool vis = row >= row0 && row < row1;
+          if (vis && pend) {
+            const int p = mt.p0 + (row - row0);
+            if (p < mt.thresh) vis = c.ring_keep[mt.keep_base + p % mt.R] != 0;
+          }
+          sc[j][e] = vis ? acc[e] * mul : -INFINITY;
         }
-        sc[j][e] = vis ? acc[e] * mul : -INFINITY;
       }
     }
 
-    // ---- online softmax for row g (the 4 lanes of a quad share it)
+    // ---- online softmax for row (head) g; the 4 lanes of a quad share it
     float mx = -INFINITY;
 #pragma unroll
     for (int j = 0; j < NJ; ++j) mx = fmaxf(mx, fmaxf(sc[j][0], sc[j][1]));
@@ -537,45 +604,52 @@ k_decode_split(CacheView c, DecodeWork w, int layer, int batch, const uint16_t* 
       l_run = l_run * alpha + ls;
       m_run = mn;
     }
+    // o^T columns are heads 2t, 2t+1: their rescale factors live in quads 2t, 2t+1
+    const float al_e = __shfl_sync(0xffffffffu, alpha, 8 * t);
+    const float al_o = __shfl_sync(0xffffffffu, alpha, 8 * t + 4);
 #pragma unroll
-    for (int d = 0; d < ND; ++d) {
-      oacc[d][0] *= alpha;
-      oacc[d][1] *= alpha;
+    for (int i = 0; i < MT; ++i) {
+      oacc[i][0] *= al_e;
+      oacc[i][1] *= al_o;
+      oacc[i][2] *= al_e;
+      oacc[i][3] *= al_o;
     }
 
-    // ---- o += p v, keys 16u .. 16u + 15 per k-step
+    // ---- o^T += V^T p^T, keys 16u .. 16u + 15 per k-step
 #pragma unroll
     for (int u = 0; u < NU; ++u) {
       if (16 * u + 16 <= row0 || 16 * u >= row1) continue;
-      const float v0 = pr[2 * u][0] * mt.vrel, v1 = pr[2 * u][1] * mt.vrel;
-      const float v2 = pr[2 * u + 1][0] * mt.vrel, v3 = pr[2 * u + 1][1] * mt.vrel;
-      const uint32_t ah0 = pack2<FP8>(v0, v1), ah2 = pack2<FP8>(v2, v3);
-      const float2 f0 = unpack2<FP8>(ah0), f2 = unpack2<FP8>(ah2);
-      const uint32_t al0 = pack2<FP8>(v0 - f0.x, v1 - f0.y);
-      const uint32_t al2 = pack2<FP8>(v2 - f2.x, v3 - f2.y);
+      // p^T B fragment: (keys 16u + 2t, +1) and (16u + 8 + 2t, +1) of head g
+      const float p0 = pr[2 * u][0] * mt.vrel, p1 = pr[2 * u][1] * mt.vrel;
+      const float p2 = pr[2 * u + 1][0] * mt.vrel, p3 = pr[2 * u + 1][1] * mt.vrel;
+      const uint32_t bh0 = pack2<FP8>(p0, p1), bh1 = pack2<FP8>(p2, p3);
+      uint32_t bl0 = 0u, bl1 = 0u;
+      if constexpr (T::SPLIT) {
+        const float2 f0 = unpack2<FP8>(bh0), f1 = unpack2<FP8>(bh1);
+        bl0 = pack2<FP8>(p0 - f0.x, p1 - f0.y);
+        bl1 = pack2<FP8>(p2 - f1.x, p3 - f1.y);
+      }
       // V rows 16u + 2t + {0, 1, 8, 9}: the dims of lane group g
       const int rr[4] = {16 * u + 2 * t, 16 * u + 2 * t + 1, 16 * u + 2 * t + 8,
                          16 * u + 2 * t + 9};
-      if constexpr (RB == 64) {     // FP8, D = 64: 8 bytes (8 dims) per row
+      if constexpr (RB == 64) {     // FP8, D = 64: 8 bytes (8 dims) of lane group g per row
         uint2 x[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          x[i] = *reinterpret_cast<const uint2*>(Vs + rr[i] * RB + 8 * g);
+        for (int i = 0; i < 4; ++i) x[i] = *reinterpret_cast<const uint2*>(Vs + rr[i] * RB + 8 * g);
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {            // words: dims 4e .. 4e + 3
-          const uint32_t a0w = e ? x[0].y : x[0].x, a1w = e ? x[1].y : x[1].x;
-          const uint32_t a8w = e ? x[2].y : x[2].x, a9w = e ? x[3].y : x[3].x;
-          const uint32_t lo01 = prmt(a0w, a1w, 0x5140), hi01 = prmt(a0w, a1w, 0x7362);
-          const uint32_t lo89 = prmt(a8w, a9w, 0x5140), hi89 = prmt(a8w, a9w, 0x7362);
-          const uint32_t b0s[4] = {e4m3x2_to_f16x2(lo01 & 0xFFFF), e4m3x2_to_f16x2(lo01 >> 16),
-                                   e4m3x2_to_f16x2(hi01 & 0xFFFF), e4m3x2_to_f16x2(hi01 >> 16)};
-          const uint32_t b1s[4] = {e4m3x2_to_f16x2(lo89 & 0xFFFF), e4m3x2_to_f16x2(lo89 >> 16),
-                                   e4m3x2_to_f16x2(hi89 & 0xFFFF), e4m3x2_to_f16x2(hi89 >> 16)};
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            mma16816<true>(oacc[4 * e + q4], ah0, ah2, b0s[q4], b1s[q4]);
-            mma16816<true>(oacc[4 * e + q4], al0, al2, b0s[q4], b1s[q4]);
-          }
+        for (int e = 0; e < 2; ++e) {            // word e: dims 8g + 4e .. +3 = m-tiles 2e, 2e+1
+          const uint32_t w0 = e ? x[0].y : x[0].x, w1 = e ? x[1].y : x[1].x;
+          const uint32_t w8 = e ? x[2].y : x[2].x, w9 = e ? x[3].y : x[3].x;
+          const uint32_t lo01 = prmt(w0, w1, 0x5140), hi01 = prmt(w0, w1, 0x7362);
+          const uint32_t lo89 = prmt(w8, w9, 0x5140), hi89 = prmt(w8, w9, 0x7362);
+          const uint32_t A0 = e4m3x2_to_f16x2(lo01 & 0xFFFF), A1 = e4m3x2_to_f16x2(lo01 >> 16);
+          const uint32_t A2 = e4m3x2_to_f16x2(lo89 & 0xFFFF), A3 = e4m3x2_to_f16x2(lo89 >> 16);
+          const uint32_t B0 = e4m3x2_to_f16x2(hi01 & 0xFFFF), B1 = e4m3x2_to_f16x2(hi01 >> 16);
+          const uint32_t B2 = e4m3x2_to_f16x2(hi89 & 0xFFFF), B3 = e4m3x2_to_f16x2(hi89 >> 16);
+          mma16816<true>(oacc[2 * e], A0, A1, A2, A3, bh0, bh1);
+          mma16816<true>(oacc[2 * e], A0, A1, A2, A3, bl0, bl1);
+          mma16816<true>(oacc[2 * e + 1], B0, B1, B2, B3, bh0, bh1);
+          mma16816<true>(oacc[2 * e + 1], B0, B1, B2, B3, bl0, bl1);
         }
       } else {
         constexpr int VCH = RB == 256 ? 2 : 1;   // 16-byte chunks of a lane group per row
@@ -593,26 +667,27 @@ k_decode_split(CacheView c, DecodeWork w, int layer, int batch, const uint16_t* 
           const uint32_t w9[4] = {x[3].x, x[3].y, x[3].z, x[3].w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            if constexpr (FP8) {                 // 4 dims per word: n-tiles 4e .. 4e + 3
+            if constexpr (FP8) {     // word e: 4 dims = m-tiles 2e, 2e + 1
               const uint32_t lo01 = prmt(w0[e], w1[e], 0x5140), hi01 = prmt(w0[e], w1[e], 0x7362);
               const uint32_t lo89 = prmt(w8[e], w9[e], 0x5140), hi89 = prmt(w8[e], w9[e], 0x7362);
-              const uint32_t b0s[4] = {e4m3x2_to_f16x2(lo01 & 0xFFFF), e4m3x2_to_f16x2(lo01 >> 16),
-                                       e4m3x2_to_f16x2(hi01 & 0xFFFF), e4m3x2_to_f16x2(hi01 >> 16)};
-              const uint32_t b1s[4] = {e4m3x2_to_f16x2(lo89 & 0xFFFF), e4m3x2_to_f16x2(lo89 >> 16),
-                                       e4m3x2_to_f16x2(hi89 & 0xFFFF), e4m3x2_to_f16x2(hi89 >> 16)};
-#pragma unroll
-              for (int q4 = 0; q4 < 4; ++q4) {
-                mma16816<true>(oacc[4 * e + q4], ah0, ah2, b0s[q4], b1s[q4]);
-                mma16816<true>(oacc[4 * e + q4], al0, al2, b0s[q4], b1s[q4]);
-              }
-            } else {                              // 2 dims per word: n-tiles 2e, 2e + 1
-              const int d0 = 8 * ci + 2 * e;
-              const uint32_t b0a = prmt(w0[e], w1[e], 0x5410), b1a = prmt(w8[e], w9[e], 0x5410);
-              const uint32_t b0b = prmt(w0[e], w1[e], 0x7632), b1b = prmt(w8[e], w9[e], 0x7632);
-              mma16816<false>(oacc[d0], ah0, ah2, b0a, b1a);
-              mma16816<false>(oacc[d0], al0, al2, b0a, b1a);
-              mma16816<false>(oacc[d0 + 1], ah0, ah2, b0b, b1b);
-              mma16816<false>(oacc[d0 + 1], al0, al2, b0b, b1b);
+              const uint32_t A0 = e4m3x2_to_f16x2(lo01 & 0xFFFF),
+                             A1 = e4m3x2_to_f16x2(lo01 >> 16);
+              const uint32_t A2 = e4m3x2_to_f16x2(lo89 & 0xFFFF),
+                             A3 = e4m3x2_to_f16x2(lo89 >> 16);
+              const uint32_t B0 = e4m3x2_to_f16x2(hi01 & 0xFFFF),
+                             B1 = e4m3x2_to_f16x2(hi01 >> 16);
+              const uint32_t B2 = e4m3x2_to_f16x2(hi89 & 0xFFFF),
+                             B3 = e4m3x2_to_f16x2(hi89 >> 16);
+              mma16816<true>(oacc[2 * e], A0, A1, A2, A3, bh0, bh1);
+              mma16816<true>(oacc[2 * e], A0, A1, A2, A3, bl0, bl1);
+              mma16816<true>(oacc[2 * e + 1], B0, B1, B2, B3, bh0, bh1);
+              mma16816<true>(oacc[2 * e + 1], B0, B1, B2, B3, bl0, bl1);
+            } else {                 // word e: 2 dims = m-tile 4 ci + e (rows g, g + 8)
+              const int i = 4 * ci + e;
+              const uint32_t a0 = prmt(w0[e], w1[e], 0x5410), a1 = prmt(w0[e], w1[e], 0x7632);
+              const uint32_t a2 = prmt(w8[e], w9[e], 0x5410), a3 = prmt(w8[e], w9[e], 0x7632);
+              mma16816<false>(oacc[i], a0, a1, a2, a3, bh0, bh1);
+              mma16816<false>(oacc[i], a0, a1, a2, a3, bl0, bl1);
             }
           }
         }
@@ -621,83 +696,209 @@ k_decode_split(CacheView c, DecodeWork w, int layer, int batch, const uint16_t* 
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
 
-    // ---- end of this head inside the range: write the partial
+    // ---- end of this head inside the range
     if (mt.flags & kLast) {
       float l = l_run;
       l += __shfl_xor_sync(0xffffffffu, l, 1);
       l += __shfl_xor_sync(0xffffffffu, l, 2);
-      const long long part = range_id + mt.hidx;
-      if (g < G) {
-        float* po = w.part_o + (part * G + g) * D;
+      const int hidx = mt.hidx;
+      const long long hs = head_off[hidx], he = head_off[hidx + 1];
+      const int kb = hidx / c.Hkv, kh = hidx % c.Hkv;
+      if (hs >= gs && he <= ge) {
+        // the whole head lies in this warp's range: write the output now
 #pragma unroll
-        for (int d = 0; d < ND; ++d) {
-          po[T::vdim(2 * t, d)] = oacc[d][0] * mt.vhead;
-          po[T::vdim(2 * t + 1, d)] = oacc[d][1] * mt.vhead;
+        for (int e = 0; e < 2; ++e) {
+          const int h = 2 * t + e;
+          const float lh = __shfl_sync(0xffffffffu, l, 4 * (h & 7));
+          const float mh = __shfl_sync(0xffffffffu, m_run, 4 * (h & 7));
+          if (h < G) {
+            const float inv = mh == -INFINITY ? 0.f : mt.vhead / lh;
+            const long long ob = ((long long)kb * c.Hq + (long long)kh * G + h) * D;
+#pragma unroll
+            for (int i = 0; i < MT; ++i)
+#pragma unroll
+              for (int hi = 0; hi < 2; ++hi) {
+                const float o = oacc[i][2 * hi + e] * inv;
+                const long long oi = ob + T::vdim(g, i, hi);
+                if (oa.f32) static_cast<float*>(oa.out)[oi] = o;
+                else static_cast<uint16_t*>(oa.out)[oi] = f32_to_bf16_rn(o);
+              }
+            if (oa.lse && g == 0)
+              oa.lse[(long long)kb * c.Hq + kh * G + h] =
+                  mh == -INFINITY ? -INFINITY : (mh + log2f(lh)) * 0.6931471805599453f;
+          }
         }
-        if (t == 0) {
-          w.part_ml[(part * G + g) * 2] = m_run;
-          w.part_ml[(part * G + g) * 2 + 1] = l;
+      } else {
+        // shared with other warps: leave the unmerged partial in this warp's slot
+        // 0 (the head began before the range) or 1 (it goes on after it)
+        float* sl = slots + (warp * 2 + (hs < gs ? 0 : 1)) * T::SLOT_F;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int h = 2 * t + e;
+          if (h < G) {
+#pragma unroll
+            for (int i = 0; i < MT; ++i) {
+              sl[T::SLOT_O + h * D + T::vdim(g, i, 0)] = oacc[i][e] * mt.vhead;
+              sl[T::SLOT_O + h * D + T::vdim(g, i, 1)] = oacc[i][2 + e] * mt.vhead;
+            }
+          }
         }
+        if (t == 0 && g < G) {
+          sl[4 + g] = m_run;
+          sl[4 + G + g] = l;
+        }
+        __syncwarp();
+        if (lane == 0) sl[0] = __int_as_float(hidx);
       }
     }
   }
-}
 
-// range of unit x under the split: the largest v with floor(v * T / N) <= x.
-__device__ __forceinline__ int range_of_unit(long long x, long long total, int n) {
-  return (int)(((x + 1) * n - 1) / total);
-}
-
-template <int D, int G, bool F32>
-__global__ void __launch_bounds__(G * D)
-k_decode_combine(DecodeWork w, int Hkv, int Hq, int batch, void* out, float* lse) {
-  const int hidx = blockIdx.x;
-  const int g = threadIdx.x / D, d = threadIdx.x % D;
-  const int b = hidx / Hkv, h = hidx % Hkv;
-  const int qh = h * G + g;
-  const long long s = w.head_off[hidx], e = w.head_off[hidx + 1];
-  const long long total = w.head_off[batch * Hkv];
-  const int n = *w.n_eff;
-  float o = 0.f, M = -INFINITY, L = 0.f;
-  if (e > s) {
-    const int c0 = range_of_unit(s, total, n), c1 = range_of_unit(e - 1, total, n);
-    for (int cc = c0; cc <= c1; ++cc) {
-      const long long part = (long long)cc + hidx;
-      M = fmaxf(M, w.part_ml[(part * G + g) * 2]);
+  // ================= merge of the heads this CTA shares between warps / CTAs
+  // Valid slots carry non-decreasing heads in slot order (ranges follow the
+  // unit order), so each head is one run of slots, empty slots aside.
+  // Phase 1 merges the slots of every such head (shared memory) and writes the
+  // output of heads that lie inside this CTA's range, or a CTA partial of the
+  // others; phase 2 counts the CTA partials; phase 3 lets the CTA that
+  // completes a head's count merge its (few) CTA partials.
+  consumer_sync_n<T::NC>();
+  {
+    constexpr int kMaxRuns = 2 * NCW;
+    __shared__ int s_run_head[kMaxRuns], s_run_lo[kMaxRuns], s_run_hi[kMaxRuns];
+    __shared__ int s_run_flag[kMaxRuns];
+    __shared__ int s_nruns;
+    const long long v0 = (long long)blockIdx.x * NCW;
+    const long long v1 = min((long long)n_eff, v0 + NCW);
+    const long long cgs = v0 * total / n_eff, cge = v1 * total / n_eff;
+    if (tid == 0) {
+      int nr = 0, si = 0;
+      auto slot_head = [&](int k) { return __float_as_int(slots[k * T::SLOT_F]); };
+      while (si < 2 * NCW) {
+        const int hd = slot_head(si);
+        if (hd < 0) { ++si; continue; }
+        int sj = si + 1;
+        while (sj < 2 * NCW && (slot_head(sj) < 0 || slot_head(sj) == hd)) ++sj;
+        s_run_head[nr] = hd;
+        s_run_lo[nr] = si;
+        s_run_hi[nr] = sj;
+        s_run_flag[nr] = 0;
+        ++nr;
+        si = sj;
+      }
+      s_nruns = nr;
     }
-    if (M != -INFINITY) {
-      for (int cc = c0; cc <= c1; ++cc) {
-        const long long part = (long long)cc + hidx;
-        const float m = w.part_ml[(part * G + g) * 2];
+    consumer_sync_n<T::NC>();
+    const int nr = s_nruns;
+    // phase 1
+    for (int it = tid; it < nr * G * D; it += T::NC) {
+      const int run = it / (G * D), idx = it % (G * D);
+      const int hd = s_run_head[run], h = idx / D, d = idx % D;
+      float M = -INFINITY, L = 0.f, O = 0.f;
+      for (int sk = s_run_lo[run]; sk < s_run_hi[run]; ++sk) {
+        const float* sl = slots + sk * T::SLOT_F;
+        if (__float_as_int(sl[0]) != hd) continue;
+        const float m = sl[4 + h];
         if (m == -INFINITY) continue;
-        const float sc = exp2f(m - M);
-        L += w.part_ml[(part * G + g) * 2 + 1] * sc;
-        o += w.part_o[(part * G + g) * D + d] * sc;
+        const float mn2 = fmaxf(M, m);
+        const float a = fast_exp2(M - mn2), bb = fast_exp2(m - mn2);
+        L = L * a + sl[4 + G + h] * bb;
+        O = O * a + sl[T::SLOT_O + h * D + d] * bb;
+        M = mn2;
       }
-      o = o / L;
+      const long long hs = head_off[hd], he = head_off[hd + 1];
+      const int kb = hd / c.Hkv, kh = hd % c.Hkv;
+      if (hs >= cgs && he <= cge) {
+        const float o = M == -INFINITY ? 0.f : O / L;
+        const long long oi = ((long long)kb * c.Hq + (long long)kh * G + h) * D + d;
+        if (oa.f32) static_cast<float*>(oa.out)[oi] = o;
+        else static_cast<uint16_t*>(oa.out)[oi] = f32_to_bf16_rn(o);
+        if (oa.lse && d == 0)
+          oa.lse[(long long)kb * c.Hq + kh * G + h] =
+              M == -INFINITY ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
+      } else {
+        const long long part = (long long)blockIdx.x + hd;
+        w.part_o[(part * G + h) * D + d] = O;
+        if (d == 0) {
+          w.part_ml[(part * G + h) * 2] = M;
+          w.part_ml[(part * G + h) * 2 + 1] = L;
+        }
+      }
     }
-  }
-  const long long oi = ((long long)b * Hq + qh) * D + d;
-  if constexpr (F32) {
-    static_cast<float*>(out)[oi] = o;
-    if (lse && d == 0)
-      lse[(long long)b * Hq + qh] =
-          (M == -INFINITY) ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
-  } else {
-    static_cast<uint16_t*>(out)[oi] = f32_to_bf16_rn(o);
+    // phase 2
+    __threadfence();
+    consumer_sync_n<T::NC>();
+    if (tid < nr) {
+      const int hd = s_run_head[tid];
+      const long long hs = head_off[hd], he = head_off[hd + 1];
+      if (!(hs >= cgs && he <= cge)) {
+        const int first = range_of_unit(hs, total, n_eff) / NCW;
+        const int last = range_of_unit(he - 1, total, n_eff) / NCW;
+        s_run_flag[tid] = atomicAdd(&w.head_cnt[hd], 1) == last - first;
+      }
+    }
+    consumer_sync_n<T::NC>();
+    // phase 3
+    constexpr int kBatch = 8;
+    for (int it = tid; it < nr * G * D; it += T::NC) {
+      const int run = it / (G * D), idx = it % (G * D);
+      if (!s_run_flag[run]) continue;
+      __threadfence();
+      const int hd = s_run_head[run], h = idx / D, d = idx % D;
+      const long long hs = head_off[hd], he = head_off[hd + 1];
+      const int first = range_of_unit(hs, total, n_eff) / NCW;
+      const int last = range_of_unit(he - 1, total, n_eff) / NCW;
+      float M = -INFINITY, L = 0.f, O = 0.f;
+      for (int c0 = first; c0 <= last; c0 += kBatch) {
+        float mb[kBatch], lb[kBatch], ob[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {   // loads first, all independent
+          const long long pp = (long long)(c0 + u) + hd;
+          const bool live = c0 + u <= last;
+          mb[u] = live ? __ldcg(&w.part_ml[(pp * G + h) * 2]) : -INFINITY;
+          lb[u] = live ? __ldcg(&w.part_ml[(pp * G + h) * 2 + 1]) : 0.f;
+          ob[u] = live ? __ldcg(&w.part_o[(pp * G + h) * D + d]) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+          if (mb[u] == -INFINITY) continue;
+          const float mn2 = fmaxf(M, mb[u]);
+          const float a = fast_exp2(M - mn2), bb = fast_exp2(mb[u] - mn2);
+          L = L * a + lb[u] * bb;
+          O = O * a + ob[u] * bb;
+          M = mn2;
+        }
+      }
+      const int kb = hd / c.Hkv, kh = hd % c.Hkv;
+      const float o = M == -INFINITY ? 0.f : O / L;
+      const long long oi = ((long long)kb * c.Hq + (long long)kh * G + h) * D + d;
+      if (oa.f32) static_cast<float*>(oa.out)[oi] = o;
+      else static_cast<uint16_t*>(oa.out)[oi] = f32_to_bf16_rn(o);
+      if (oa.lse && d == 0)
+        oa.lse[(long long)kb * c.Hq + kh * G + h] =
+            M == -INFINITY ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
+      if (idx == 0) w.head_cnt[hd] = 0;   // ready for the next call
+    }
   }
 }
 
 // ------------------------------------------------------------------ dispatch
 template <class T>
-fdms_status launch_split_t(fdms_cache* cache, int layer, int batch, const void* q,
-                           cudaStream_t s) {
+fdms_status launch_split_t(fdms_cache* cache, const DecodeWork& w, OutArgs oa, int layer,
+                           int batch, const void* q, cudaStream_t s) {
   const int nh = batch * cache->view.Hkv;
-  const size_t smem = T::smem_bytes(nh);
-  k_decode_split<T><<<cache->decode_ctas, T::NT, smem, s>>>(
-      cache->view, cache->work, layer, batch, static_cast<const uint16_t*>(q),
-      cache->decode_ctas * T::NCW);
-  return cudaGetLastError() == cudaSuccess ? FDMS_OK : FDMS_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)cache->decode_ctas);
+  cfg.blockDim = dim3(T::NT);
+  cfg.dynamicSmemBytes = T::smem_bytes(nh);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_decode_split<T>, cache->view, w, oa, layer,
+                                           batch, static_cast<const uint16_t*>(q),
+                                           cache->decode_ctas * T::NCW);
+  return e == cudaSuccess ? FDMS_OK : FDMS_ERR_CUDA;
 }
 
 template <class T>
@@ -715,13 +916,6 @@ fdms_status setup_t(fdms_cache* cache) {
   cache->ctas_per_sm = per_sm;
   cache->ranges_per_cta = T::NCW;
   return FDMS_OK;
-}
-
-template <int D, int G, bool F32>
-void launch_combine_t(fdms_cache* cache, int batch, void* out, float* lse, cudaStream_t s) {
-  const CacheView& c = cache->view;
-  k_decode_combine<D, G, F32><<<batch * c.Hkv, G * D, 0, s>>>(cache->work, c.Hkv, c.Hq, batch,
-                                                              out, lse);
 }
 
 template <int D, bool FP8, class F>
@@ -766,36 +960,29 @@ fdms_status fdms_decode_setup(fdms_cache* cache) {
     cache->bytes_reserved += bytes;
     return p;
   };
+  w.head_cnt = static_cast<int*>(take((size_t)c.Bmax * c.Hkv * sizeof(int)));
   w.part_o = static_cast<float*>(take((size_t)w.max_parts * c.G * c.D * sizeof(float)));
   w.part_ml = static_cast<float*>(take((size_t)w.max_parts * c.G * 2 * sizeof(float)));
-  w.head_off = static_cast<long long*>(take((size_t)(c.Bmax * c.Hkv + 1) * sizeof(long long)));
-  w.n_eff = static_cast<int*>(take(sizeof(int)));
-  if (!w.part_o || !w.part_ml || !w.head_off || !w.n_eff) return FDMS_ERR_CUDA;
+  w.head_off = nullptr;   // the plan lives in shared memory only
+  w.n_eff = nullptr;
+  if (!w.head_cnt || !w.part_o || !w.part_ml) return FDMS_ERR_CUDA;
+  if (cudaMemset(w.head_cnt, 0, (size_t)c.Bmax * c.Hkv * sizeof(int)) != cudaSuccess)
+    return FDMS_ERR_CUDA;
   return FDMS_OK;
 }
 
 fdms_status fdms_launch_decode(fdms_cache* cache, int layer, int batch, const void* q, void* out,
                                int out_f32, float* lse, cudaStream_t s) {
-  const CacheView& c = cache->view;
-  fdms_status st = by_config(c, [&](auto t) {
-    return launch_split_t<decltype(t)>(cache, layer, batch, q, s);
+  OutArgs oa{out, lse, out_f32};
+  return by_config(cache->view, [&](auto t) {
+    return launch_split_t<decltype(t)>(cache, cache->work, oa, layer, batch, q, s);
   });
-  if (st != FDMS_OK) return st;
-  auto comb = [&](auto t) -> fdms_status {
-    using T = decltype(t);
-    if (out_f32)
-      launch_combine_t<T::D, T::G, true>(cache, batch, out, lse, s);
-    else
-      launch_combine_t<T::D, T::G, false>(cache, batch, out, nullptr, s);
-    return cudaGetLastError() == cudaSuccess ? FDMS_OK : FDMS_ERR_CUDA;
-  };
-  return by_config(c, comb);
 }
 
 // ------------------------------------------------- decode without allocation
-// A fixed scratch array for fdms_decode_attn_noalloc: the split partials and the
-// plan that the combine kernel reads. Host code only learns its device address
-// through cudaGetSymbolAddress (the host-side name is a stand-in, not a device
+// A fixed scratch array for fdms_decode_attn_noalloc: the per-head counters and
+// the split partials. Host code only learns its device address through
+// cudaGetSymbolAddress (the host-side name is a stand-in, not a device
 // pointer); device code never names it, it receives the address as arguments.
 static __device__ __align__(256) unsigned char fdms_noalloc_scratch[FDMS_STATIC_SCRATCH_BYTES];
 
@@ -820,19 +1007,6 @@ cudaError_t scratch_address(int device, void** out) {
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-template <class T>
-fdms_status launch_noalloc_t(fdms_cache* cache, const DecodeWork& w, int layer, int batch,
-                             const void* q, void* out, cudaStream_t s) {
-  const CacheView& c = cache->view;
-  const size_t smem = T::smem_bytes(batch * c.Hkv);
-  k_decode_split<T><<<cache->decode_ctas, T::NT, smem, s>>>(
-      c, w, layer, batch, static_cast<const uint16_t*>(q), cache->decode_ctas * T::NCW);
-  if (cudaGetLastError() != cudaSuccess) return FDMS_ERR_CUDA;
-  k_decode_combine<T::D, T::G, false><<<batch * c.Hkv, T::G * T::D, 0, s>>>(w, c.Hkv, c.Hq,
-                                                                           batch, out, nullptr);
-  return cudaGetLastError() == cudaSuccess ? FDMS_OK : FDMS_ERR_CUDA;
-}
-
 }  // namespace
 
 extern "C" fdms_status fdms_decode_attn_noalloc(fdms_cache* cache, int layer, int batch,
@@ -844,13 +1018,13 @@ extern "C" fdms_status fdms_decode_attn_noalloc(fdms_cache* cache, int layer, in
   if (!q_dev || !out_dev || (((uintptr_t)q_dev | (uintptr_t)out_dev) & 15))
     return FDMS_ERR_INVALID_ARG;
   if (cache->device < 0 || cache->device >= kMaxDevices) return FDMS_ERR_UNSUPPORTED;
-  // layout of the scratch for this call
+  // layout of the scratch for this call: counters, partials (o), partials (m, l)
   const long long parts = (long long)cache->decode_ctas * cache->ranges_per_cta +
                           (long long)batch * c.Hkv;
+  const size_t cnt_bytes = align256((size_t)batch * c.Hkv * sizeof(int));
   const size_t o_bytes = align256((size_t)parts * c.G * c.D * sizeof(float));
   const size_t ml_bytes = align256((size_t)parts * c.G * 2 * sizeof(float));
-  const size_t off_bytes = align256((size_t)(batch * c.Hkv + 1) * sizeof(long long));
-  const size_t need = o_bytes + ml_bytes + off_bytes + 256;
+  const size_t need = cnt_bytes + o_bytes + ml_bytes;
   if (need > FDMS_STATIC_SCRATCH_BYTES) return FDMS_ERR_INVALID_ARG;
 
   int prev = -1;
@@ -858,21 +1032,28 @@ extern "C" fdms_status fdms_decode_attn_noalloc(fdms_cache* cache, int layer, in
   if (prev != cache->device && cudaSetDevice(cache->device) != cudaSuccess) return FDMS_ERR_CUDA;
   void* base = nullptr;
   fdms_status st = FDMS_OK;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (scratch_address(cache->device, &base) != cudaSuccess) {
     st = FDMS_ERR_CUDA;
   } else {
     unsigned char* b = static_cast<unsigned char*>(base);
     DecodeWork w;
-    w.part_o = reinterpret_cast<float*>(b);
-    w.part_ml = reinterpret_cast<float*>(b + o_bytes);
-    w.head_off = reinterpret_cast<long long*>(b + o_bytes + ml_bytes);
-    w.n_eff = reinterpret_cast<int*>(b + o_bytes + ml_bytes + off_bytes);
+    w.head_cnt = reinterpret_cast<int*>(b);
+    w.part_o = reinterpret_cast<float*>(b + cnt_bytes);
+    w.part_ml = reinterpret_cast<float*>(b + cnt_bytes + o_bytes);
+    w.head_off = nullptr;
+    w.n_eff = nullptr;
     w.max_parts = (int)parts;
     w.max_ctas = cache->decode_ctas;
-    st = by_config(c, [&](auto t) {
-      return launch_noalloc_t<decltype(t)>(cache, w, layer, batch, q_dev, out_dev,
-                                           static_cast<cudaStream_t>(stream));
-    });
+    // the array keeps the previous call's contents: the counters must start at 0
+    if (cudaMemsetAsync(w.head_cnt, 0, cnt_bytes, s) != cudaSuccess) {
+      st = FDMS_ERR_CUDA;
+    } else {
+      OutArgs oa{out_dev, nullptr, 0};
+      st = by_config(c, [&](auto t) {
+        return launch_split_t<decltype(t)>(cache, w, oa, layer, batch, q_dev, s);
+      });
+    }
   }
   if (prev != cache->device) cudaSetDevice(prev);
   return st;

@@ -282,3 +282,30 @@ def test_host_side_argument_errors():
         assert fd.fdms_cache_stats(p.cache)["error"] == 0
     finally:
         p.close()
+
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "fp8_e4m3"])
+@pytest.mark.parametrize("window,period", [(16, 1), (0, 1), (5, 7), (16, 64)])
+def test_mixed_append_sizes(kv_dtype, window, period):
+    """Appends of 1..16 tokens (warp path) mixed with larger ones (CTA path)."""
+    rng = np.random.default_rng(window * 100 + period)
+    wl = wk.scaled(wk.get("tiny"), batch=3, ctx=40, steps=0, window=window, period=period,
+                   kv_dtype=kv_dtype, rate=0.4)
+    p = Pair(wl, max_seq_len=1200, oracle_capacity=1200)
+    try:
+        step = 0
+        for it in range(24):
+            m = int(rng.choice([1, 1, 2, 5, 16, 17, 40, 0]))
+            big = wk.scaled(wl, ctx=max(m, 1))
+            inp = wk.prefill_inputs(big, 0)
+            inp = {**inp, "n_new": torch.tensor([m, max(m - 1, 0), m // 2], dtype=torch.int32)}
+            p.append(0, inp)
+            q = wk.decode_query(wl, 0, step)
+            step += 1
+            out = p.decode(0, q)
+            assert _max_err(out, p.oracle_out(0, q)) <= (TOL_BF16 if kv_dtype == "bf16" else
+                                                          TOL_FP8_MIRROR)
+            p.check_heads(0)
+        p.check_stats()
+    finally:
+        p.close()
