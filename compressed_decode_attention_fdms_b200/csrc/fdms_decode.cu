@@ -1,4 +1,4 @@
-// Decode attention over the compact store: one kernel, split and merge.
+// Decode attention over the compact store: split kernel + combine kernel.
 //
 // FastDMS decodes over the survivors of per-head eviction only, reading 5-8x
 // less KV than a dense cache ("FastDMS: 6.4X KV-cache compression running
@@ -30,12 +30,14 @@
 //     (cvt e4m3x2 -> f16x2) and q is brought into f16 range by a power of two
 //     that the score scale undoes; the page's K scale multiplies the scores
 //     and its V scale the probabilities, never the elements.
-//   - Merge: when a warp has written its partial for a head it counts it on
-//     the head's counter; the warp that completes the count merges all of the
-//     head's partials, o = sum_w 2^(m_w - M) o_w / sum_w 2^(m_w - M) l_w, and
-//     writes the output. Heads with no slot get zeros.
-//   - The launch allows programmatic dependent launch: set-up that reads no
-//     global memory runs while the previous kernel in the stream finishes.
+//   - A head that lies whole inside one warp's range is written by that warp;
+//     heads with no slot get zeros. Warps that share a head leave their
+//     partials in shared memory; the CTA merges them and writes the heads that
+//     lie inside its range, and leaves one CTA partial of the others; a small
+//     combine kernel merges those (2-4 per head at 8K context),
+//     o = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c.
+//   - Both kernels allow programmatic dependent launch: set-up that reads no
+//     data of the previous kernel runs while that kernel finishes.
 #include <cfloat>
 #include <cstdio>
 #include <mutex>
@@ -104,7 +106,7 @@ struct Dec {
 
   static constexpr int OFF_META = NSTAGE * STAGE_BYTES;
   static constexpr int OFF_BAR = OFF_META + NSTAGE * (int)sizeof(TileMeta);
-  static constexpr int OFF_SLOTS = OFF_BAR + 2 * NSTAGE * 8 + 16;   // + the merge flag
+  static constexpr int OFF_SLOTS = OFF_BAR + 2 * NSTAGE * 8;
   static constexpr int OFF_HEADS = OFF_SLOTS + 2 * NCW * SLOT_F * 4;
   static size_t smem_bytes(int nh) {
     // head_off (i64), page_off (i32), len, n, r (i32), head scales (2 x f32)
@@ -165,9 +167,23 @@ __device__ __forceinline__ int upper_bound(const T* a, int n, T x) {
   return lo;
 }
 
+// floor(a / b) for 0 <= a < 2^53, 0 < b: exact through fp64 when the quotient
+// is below 2^20 and b below 2^32 (a non-integer quotient then keeps a
+// fractional part of at least 1/b > 2^-32, larger than the rounding error of
+// the fp64 division); the 64-bit integer division, a long software sequence
+// on the GPU, is kept for the rest.
+__device__ __forceinline__ long long floor_div(long long a, long long b) {
+  if (a < (1LL << 52) && b < (1LL << 32) && a < (b << 20))
+    return (long long)floor(__ddiv_rn((double)a, (double)b));
+  return a / b;
+}
+// first unit of range v when T units are cut into n ranges: floor(v * T / n)
+__device__ __forceinline__ long long range_start(long long v, long long total, int n) {
+  return floor_div(v * total, n);
+}
 // range of unit x under the split: the largest v with floor(v * T / N) <= x.
 __device__ __forceinline__ int range_of_unit(long long x, long long total, int n) {
-  return (int)(((x + 1) * n - 1) / total);
+  return (int)floor_div((x + 1) * n - 1, total);
 }
 
 // ------------------------------------------------------------- MMA helpers
@@ -330,9 +346,13 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   const long long total = head_off[NH];
   const long long want = (total + kMinUnitsPerRange - 1) / kMinUnitsPerRange;
   const int n_eff = (int)(want < n_launch_ranges ? (want > 0 ? want : 1) : n_launch_ranges);
-  if (blockIdx.x == 0 && tid == 0) {
-    c.ctr->slots_decoded += (unsigned long long)total;   // one thread, launches are ordered
-    c.ctr->decode_calls += 1ull;
+  if (blockIdx.x == 0) {   // the plan the combine kernel reads back
+    for (int h = tid; h <= NH; h += T::NT) w.head_off[h] = head_off[h];
+    if (tid == 0) {
+      *w.n_eff = n_eff;
+      c.ctr->slots_decoded += (unsigned long long)total;   // one thread, launches are ordered
+      c.ctr->decode_calls += 1ull;
+    }
   }
   // heads without a single slot get zeros (nobody else writes them)
   for (int h = blockIdx.x; h < NH; h += gridDim.x) {
@@ -356,18 +376,39 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
                            : (len + TR - 1) / TR + (int)((u - len + s_r[h] % TR) / TR);
     return page_off[h] + lp;
   };
-  // unit range of consumer warp cw of this CTA, and its first page / page count
+  // unit range of every consumer warp of this CTA, and its first page / page
+  // count: one thread per warp, once
+  __shared__ long long s_gs[NCW], s_ge[NCW];
+  __shared__ int s_gp0[NCW], s_nt[NCW];
+  __shared__ long long s_cgs, s_cge;   // the CTA's unit range
+  if (tid == NCW) {
+    const int v0 = blockIdx.x * NCW;
+    s_cgs = v0 < n_eff ? range_start(v0, total, n_eff) : total;
+    s_cge = range_start(min(n_eff, v0 + NCW), total, n_eff);
+  }
+  if (tid < NCW) {
+    const long long v = (long long)blockIdx.x * NCW + tid;
+    long long a = 0, b = 0;
+    int p0 = 0, n = 0;
+    if (v < n_eff) {
+      a = range_start(v, total, n_eff);
+      b = range_start(v + 1, total, n_eff);
+      if (a < b) {
+        p0 = gpage(a);
+        n = gpage(b - 1) - p0 + 1;
+      }
+    }
+    s_gs[tid] = a;
+    s_ge[tid] = b;
+    s_gp0[tid] = p0;
+    s_nt[tid] = n;
+  }
+  __syncthreads();
   auto range_of = [&](int cw, long long& gs, long long& ge, int& gp0, int& nt) {
-    const long long v = (long long)blockIdx.x * NCW + cw;
-    nt = 0;
-    gs = ge = 0;
-    gp0 = 0;
-    if (v >= n_eff) return;
-    gs = v * total / n_eff;
-    ge = (v + 1) * total / n_eff;
-    if (gs >= ge) return;
-    gp0 = gpage(gs);
-    nt = gpage(ge - 1) - gp0 + 1;
+    gs = s_gs[cw];
+    ge = s_ge[cw];
+    gp0 = s_gp0[cw];
+    nt = s_nt[cw];
   };
 
   if (warp == NCW) {
@@ -460,6 +501,24 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   float* slots = reinterpret_cast<float*>(smem + T::OFF_SLOTS);
   if (lane < 2) slots[(warp * 2 + lane) * T::SLOT_F] = __int_as_float(-1);   // empty
 
+  // shared-memory byte offsets of this lane's fragment loads inside a tile:
+  // K rows 8j + g (the row permutation bits are g for every j), V rows
+  // 16u + 2t + {0, 1, 8, 9} (permutation bits 2t + {0, 1})
+  int koff[T::KCPT];
+#pragma unroll
+  for (int i = 0; i < T::KCPT; ++i)
+    koff[i] = g * RB + 16 * swz_chunk(RB, false, g, T::kchunk(t, i));
+  constexpr int VCHK = RB == 256 ? 2 : 1;
+  int voff[4][VCHK];
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    const int rr = 2 * t + (q4 & 1) + 8 * (q4 >> 1);
+#pragma unroll
+    for (int ci = 0; ci < VCHK; ++ci)
+      voff[q4][ci] = rr * RB + (RB == 64 ? 8 * g
+                                          : 16 * swz_chunk(RB, true, rr, RB == 256 ? g + 8 * ci : g));
+  }
+
   uint32_t qa[KS][2];          // q A-fragments (row g, k-steps)
   float qmul = 0.f;            // score multiplier of row g (scale, log2 e, q's power of two)
   int cur_hidx = -1;
@@ -540,12 +599,10 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
       sc[j][0] = sc[j][1] = -INFINITY;
       if (8 * j + 8 <= row0 || 8 * j >= row1) continue;
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      const int r = 8 * j + g;   // key row this lane loads for the B fragment
-      uint32_t kw[T::KCPT][4];
+      uint32_t kw[T::KCPT][4];   // key row 8j + g, this lane's chunks
 #pragma unroll
       for (int i = 0; i < T::KCPT; ++i) {
-        const uint4 x = *reinterpret_cast<const uint4*>(
-            Ks + r * RB + 16 * swz_chunk(RB, false, r, T::kchunk(t, i)));
+        const uint4 x = *reinterpret_cast<const uint4*>(Ks + 8 * j * RB + koff[i]);
         kw[i][0] = x.x; kw[i][1] = x.y; kw[i][2] = x.z; kw[i][3] = x.w;
       }
 #pragma unroll
@@ -630,12 +687,11 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
         bl1 = pack2<FP8>(p2 - f1.x, p3 - f1.y);
       }
       // V rows 16u + 2t + {0, 1, 8, 9}: the dims of lane group g
-      const int rr[4] = {16 * u + 2 * t, 16 * u + 2 * t + 1, 16 * u + 2 * t + 8,
-                         16 * u + 2 * t + 9};
+      const uint8_t* Vu = Vs + 16 * u * RB;
       if constexpr (RB == 64) {     // FP8, D = 64: 8 bytes (8 dims) of lane group g per row
         uint2 x[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) x[i] = *reinterpret_cast<const uint2*>(Vs + rr[i] * RB + 8 * g);
+        for (int i = 0; i < 4; ++i) x[i] = *reinterpret_cast<const uint2*>(Vu + voff[i][0]);
 #pragma unroll
         for (int e = 0; e < 2; ++e) {            // word e: dims 8g + 4e .. +3 = m-tiles 2e, 2e+1
           const uint32_t w0 = e ? x[0].y : x[0].x, w1 = e ? x[1].y : x[1].x;
@@ -655,12 +711,9 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
         constexpr int VCH = RB == 256 ? 2 : 1;   // 16-byte chunks of a lane group per row
 #pragma unroll
         for (int ci = 0; ci < VCH; ++ci) {
-          const int chunk = RB == 256 ? g + 8 * ci : g;
           uint4 x[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            x[i] = *reinterpret_cast<const uint4*>(Vs + rr[i] * RB +
-                                                  16 * swz_chunk(RB, true, rr[i], chunk));
+          for (int i = 0; i < 4; ++i) x[i] = *reinterpret_cast<const uint4*>(Vu + voff[i][ci]);
           const uint32_t w0[4] = {x[0].x, x[0].y, x[0].z, x[0].w};
           const uint32_t w1[4] = {x[1].x, x[1].y, x[1].z, x[1].w};
           const uint32_t w8[4] = {x[2].x, x[2].y, x[2].z, x[2].w};
@@ -753,60 +806,59 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
     }
   }
 
-  // ================= merge of the heads this CTA shares between warps / CTAs
-  // Valid slots carry non-decreasing heads in slot order (ranges follow the
-  // unit order), so each head is one run of slots, empty slots aside.
-  // Phase 1 merges the slots of every such head (shared memory) and writes the
-  // output of heads that lie inside this CTA's range, or a CTA partial of the
-  // others; phase 2 counts the CTA partials; phase 3 lets the CTA that
-  // completes a head's count merge its (few) CTA partials.
+  // ================= heads shared between warps: merge their slots (shared
+  // memory); write heads inside this CTA's range, leave one CTA partial of the
+  // others for the combine kernel. Valid slots carry non-decreasing heads in
+  // slot order, so each head is one run of slots, empty slots aside.
   consumer_sync_n<T::NC>();
   {
     constexpr int kMaxRuns = 2 * NCW;
-    __shared__ int s_run_head[kMaxRuns], s_run_lo[kMaxRuns], s_run_hi[kMaxRuns];
-    __shared__ int s_run_flag[kMaxRuns];
+    __shared__ int s_run_head[kMaxRuns];
     __shared__ int s_nruns;
-    const long long v0 = (long long)blockIdx.x * NCW;
-    const long long v1 = min((long long)n_eff, v0 + NCW);
-    const long long cgs = v0 * total / n_eff, cge = v1 * total / n_eff;
-    if (tid == 0) {
-      int nr = 0, si = 0;
-      auto slot_head = [&](int k) { return __float_as_int(slots[k * T::SLOT_F]); };
-      while (si < 2 * NCW) {
-        const int hd = slot_head(si);
-        if (hd < 0) { ++si; continue; }
-        int sj = si + 1;
-        while (sj < 2 * NCW && (slot_head(sj) < 0 || slot_head(sj) == hd)) ++sj;
-        s_run_head[nr] = hd;
-        s_run_lo[nr] = si;
-        s_run_hi[nr] = sj;
-        s_run_flag[nr] = 0;
-        ++nr;
-        si = sj;
+    if (warp == 0) {
+      const int hk = lane < 2 * NCW ? __float_as_int(slots[lane * T::SLOT_F]) : -1;
+      int pm = hk;   // inclusive prefix max of the heads (heads only grow)
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, pm, off);
+        if (lane >= off) pm = max(pm, o);
       }
-      s_nruns = nr;
+      int prev = __shfl_up_sync(0xffffffffu, pm, 1);
+      if (lane == 0) prev = -1;
+      const bool start = hk >= 0 && hk > prev;
+      const unsigned ball = __ballot_sync(0xffffffffu, start);
+      if (start) s_run_head[__popc(ball & ((1u << lane) - 1u))] = hk;
+      if (lane == 0) s_nruns = __popc(ball);
     }
     consumer_sync_n<T::NC>();
     const int nr = s_nruns;
-    // phase 1
+    const long long cgs = s_cgs, cge = s_cge;
     for (int it = tid; it < nr * G * D; it += T::NC) {
       const int run = it / (G * D), idx = it % (G * D);
       const int hd = s_run_head[run], h = idx / D, d = idx % D;
-      float M = -INFINITY, L = 0.f, O = 0.f;
-      for (int sk = s_run_lo[run]; sk < s_run_hi[run]; ++sk) {
+      float mk[2 * NCW], lk[2 * NCW], ok[2 * NCW];
+      float M = -INFINITY;
+#pragma unroll
+      for (int sk = 0; sk < 2 * NCW; ++sk) {   // independent loads, then the merge
         const float* sl = slots + sk * T::SLOT_F;
-        if (__float_as_int(sl[0]) != hd) continue;
-        const float m = sl[4 + h];
-        if (m == -INFINITY) continue;
-        const float mn2 = fmaxf(M, m);
-        const float a = fast_exp2(M - mn2), bb = fast_exp2(m - mn2);
-        L = L * a + sl[4 + G + h] * bb;
-        O = O * a + sl[T::SLOT_O + h * D + d] * bb;
-        M = mn2;
+        const bool mine = __float_as_int(sl[0]) == hd;
+        mk[sk] = mine ? sl[4 + h] : -INFINITY;
+        lk[sk] = sl[4 + G + h];
+        ok[sk] = sl[T::SLOT_O + h * D + d];
+        M = fmaxf(M, mk[sk]);
       }
-      const long long hs = head_off[hd], he = head_off[hd + 1];
+      float L = 0.f, O = 0.f;
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int sk = 0; sk < 2 * NCW; ++sk) {
+          if (mk[sk] == -INFINITY) continue;
+          const float bb = fast_exp2(mk[sk] - M);
+          L += lk[sk] * bb;
+          O += ok[sk] * bb;
+        }
+      }
       const int kb = hd / c.Hkv, kh = hd % c.Hkv;
-      if (hs >= cgs && he <= cge) {
+      if (head_off[hd] >= cgs && head_off[hd + 1] <= cge) {
         const float o = M == -INFINITY ? 0.f : O / L;
         const long long oi = ((long long)kb * c.Hq + (long long)kh * G + h) * D + d;
         if (oa.f32) static_cast<float*>(oa.out)[oi] = o;
@@ -823,60 +875,63 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
         }
       }
     }
-    // phase 2
-    __threadfence();
-    consumer_sync_n<T::NC>();
-    if (tid < nr) {
-      const int hd = s_run_head[tid];
-      const long long hs = head_off[hd], he = head_off[hd + 1];
-      if (!(hs >= cgs && he <= cge)) {
-        const int first = range_of_unit(hs, total, n_eff) / NCW;
-        const int last = range_of_unit(he - 1, total, n_eff) / NCW;
-        s_run_flag[tid] = atomicAdd(&w.head_cnt[hd], 1) == last - first;
-      }
-    }
-    consumer_sync_n<T::NC>();
-    // phase 3
-    constexpr int kBatch = 8;
-    for (int it = tid; it < nr * G * D; it += T::NC) {
-      const int run = it / (G * D), idx = it % (G * D);
-      if (!s_run_flag[run]) continue;
-      __threadfence();
-      const int hd = s_run_head[run], h = idx / D, d = idx % D;
-      const long long hs = head_off[hd], he = head_off[hd + 1];
-      const int first = range_of_unit(hs, total, n_eff) / NCW;
-      const int last = range_of_unit(he - 1, total, n_eff) / NCW;
-      float M = -INFINITY, L = 0.f, O = 0.f;
-      for (int c0 = first; c0 <= last; c0 += kBatch) {
-        float mb[kBatch], lb[kBatch], ob[kBatch];
+  }
+}
+
+// Merge of the CTA partials of one (seq, kv head) that several split CTAs
+// covered: o = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c. Heads inside one
+// CTA's range, or with no slot, were written by the split kernel. The (m, l, o)
+// of all partials are loaded together, in rounds of 8 partials.
+template <int D, int G, int NCW>
+__global__ void __launch_bounds__(256)
+k_decode_combine(DecodeWork w, int Hkv, int Hq, int batch, OutArgs oa) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int hidx = blockIdx.x, tid = threadIdx.x;
+  const long long hs = w.head_off[hidx], he = w.head_off[hidx + 1];
+  const long long total = w.head_off[batch * Hkv];
+  const int n = *w.n_eff;
+  if (he == hs) return;
+  const int c0 = range_of_unit(hs, total, n) / NCW, c1 = range_of_unit(he - 1, total, n) / NCW;
+  if (c0 == c1) return;
+  const int kb = hidx / Hkv, kh = hidx % Hkv;
+  for (int idx = tid; idx < G * D; idx += 256) {
+    const int h = idx / D, d = idx % D;
+    float M = -INFINITY, L = 0.f, O = 0.f;
+    constexpr int B = 8;
+    for (int p0 = c0; p0 <= c1; p0 += B) {
+      float mb[B], lb[B], ob[B];
 #pragma unroll
-        for (int u = 0; u < kBatch; ++u) {   // loads first, all independent
-          const long long pp = (long long)(c0 + u) + hd;
-          const bool live = c0 + u <= last;
-          mb[u] = live ? __ldcg(&w.part_ml[(pp * G + h) * 2]) : -INFINITY;
-          lb[u] = live ? __ldcg(&w.part_ml[(pp * G + h) * 2 + 1]) : 0.f;
-          ob[u] = live ? __ldcg(&w.part_o[(pp * G + h) * D + d]) : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-          if (mb[u] == -INFINITY) continue;
-          const float mn2 = fmaxf(M, mb[u]);
-          const float a = fast_exp2(M - mn2), bb = fast_exp2(mb[u] - mn2);
-          L = L * a + lb[u] * bb;
-          O = O * a + ob[u] * bb;
-          M = mn2;
-        }
+      for (int u = 0; u < B; ++u) {   // loads first, all independent
+        const long long pp = (long long)(p0 + u) + hidx;
+        const bool live = p0 + u <= c1;
+        mb[u] = live ? __ldcg(&w.part_ml[(pp * G + h) * 2]) : -INFINITY;
+        lb[u] = live ? __ldcg(&w.part_ml[(pp * G + h) * 2 + 1]) : 0.f;
+        ob[u] = live ? __ldcg(&w.part_o[(pp * G + h) * D + d]) : 0.f;
       }
-      const int kb = hd / c.Hkv, kh = hd % c.Hkv;
-      const float o = M == -INFINITY ? 0.f : O / L;
-      const long long oi = ((long long)kb * c.Hq + (long long)kh * G + h) * D + d;
-      if (oa.f32) static_cast<float*>(oa.out)[oi] = o;
-      else static_cast<uint16_t*>(oa.out)[oi] = f32_to_bf16_rn(o);
-      if (oa.lse && d == 0)
-        oa.lse[(long long)kb * c.Hq + kh * G + h] =
-            M == -INFINITY ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
-      if (idx == 0) w.head_cnt[hd] = 0;   // ready for the next call
+      float mx = M;
+#pragma unroll
+      for (int u = 0; u < B; ++u) mx = fmaxf(mx, mb[u]);
+      if (mx == -INFINITY) continue;
+      const float a = M == -INFINITY ? 0.f : exp2f(M - mx);
+      L *= a;
+      O *= a;
+#pragma unroll
+      for (int u = 0; u < B; ++u) {
+        if (mb[u] == -INFINITY) continue;
+        const float bb = exp2f(mb[u] - mx);
+        L += lb[u] * bb;
+        O += ob[u] * bb;
+      }
+      M = mx;
     }
+    const float o = M == -INFINITY ? 0.f : O / L;
+    const long long oi = ((long long)kb * Hq + (long long)kh * G + h) * D + d;
+    if (oa.f32) static_cast<float*>(oa.out)[oi] = o;
+    else static_cast<uint16_t*>(oa.out)[oi] = f32_to_bf16_rn(o);
+    if (oa.lse && d == 0)
+      oa.lse[(long long)kb * Hq + kh * G + h] =
+          M == -INFINITY ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
   }
 }
 
@@ -895,9 +950,15 @@ fdms_status launch_split_t(fdms_cache* cache, const DecodeWork& w, OutArgs oa, i
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_decode_split<T>, cache->view, w, oa, layer,
-                                           batch, static_cast<const uint16_t*>(q),
-                                           cache->decode_ctas * T::NCW);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, k_decode_split<T>, cache->view, w, oa, layer, batch,
+                                     static_cast<const uint16_t*>(q),
+                                     cache->decode_ctas * T::NCW);
+  if (e != cudaSuccess) return FDMS_ERR_CUDA;
+  cfg.gridDim = dim3((unsigned)nh);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  e = cudaLaunchKernelEx(&cfg, k_decode_combine<T::D, T::G, T::NCW>, w, cache->view.Hkv, cache->view.Hq,
+                         batch, oa);
   return e == cudaSuccess ? FDMS_OK : FDMS_ERR_CUDA;
 }
 
@@ -952,7 +1013,7 @@ fdms_status fdms_decode_setup(fdms_cache* cache) {
   const CacheView& c = cache->view;
   DecodeWork& w = cache->work;
   w.max_ctas = ctas;
-  w.max_parts = ctas * cache->ranges_per_cta + c.Bmax * c.Hkv;
+  w.max_parts = ctas + c.Bmax * c.Hkv;   // CTA c's partial of head h sits at c + h
   void* p = nullptr;
   auto take = [&](size_t bytes) -> void* {
     if (cudaMalloc(&p, bytes) != cudaSuccess) return nullptr;
@@ -960,14 +1021,11 @@ fdms_status fdms_decode_setup(fdms_cache* cache) {
     cache->bytes_reserved += bytes;
     return p;
   };
-  w.head_cnt = static_cast<int*>(take((size_t)c.Bmax * c.Hkv * sizeof(int)));
   w.part_o = static_cast<float*>(take((size_t)w.max_parts * c.G * c.D * sizeof(float)));
   w.part_ml = static_cast<float*>(take((size_t)w.max_parts * c.G * 2 * sizeof(float)));
-  w.head_off = nullptr;   // the plan lives in shared memory only
-  w.n_eff = nullptr;
-  if (!w.head_cnt || !w.part_o || !w.part_ml) return FDMS_ERR_CUDA;
-  if (cudaMemset(w.head_cnt, 0, (size_t)c.Bmax * c.Hkv * sizeof(int)) != cudaSuccess)
-    return FDMS_ERR_CUDA;
+  w.head_off = static_cast<long long*>(take((size_t)(c.Bmax * c.Hkv + 1) * sizeof(long long)));
+  w.n_eff = static_cast<int*>(take(sizeof(int)));
+  if (!w.part_o || !w.part_ml || !w.head_off || !w.n_eff) return FDMS_ERR_CUDA;
   return FDMS_OK;
 }
 
@@ -980,8 +1038,8 @@ fdms_status fdms_launch_decode(fdms_cache* cache, int layer, int batch, const vo
 }
 
 // ------------------------------------------------- decode without allocation
-// A fixed scratch array for fdms_decode_attn_noalloc: the per-head counters and
-// the split partials. Host code only learns its device address through
+// A fixed scratch array for fdms_decode_attn_noalloc: the split plan and the
+// split partials. Host code only learns its device address through
 // cudaGetSymbolAddress (the host-side name is a stand-in, not a device
 // pointer); device code never names it, it receives the address as arguments.
 static __device__ __align__(256) unsigned char fdms_noalloc_scratch[FDMS_STATIC_SCRATCH_BYTES];
@@ -1018,13 +1076,13 @@ extern "C" fdms_status fdms_decode_attn_noalloc(fdms_cache* cache, int layer, in
   if (!q_dev || !out_dev || (((uintptr_t)q_dev | (uintptr_t)out_dev) & 15))
     return FDMS_ERR_INVALID_ARG;
   if (cache->device < 0 || cache->device >= kMaxDevices) return FDMS_ERR_UNSUPPORTED;
-  // layout of the scratch for this call: counters, partials (o), partials (m, l)
-  const long long parts = (long long)cache->decode_ctas * cache->ranges_per_cta +
-                          (long long)batch * c.Hkv;
-  const size_t cnt_bytes = align256((size_t)batch * c.Hkv * sizeof(int));
+  // layout of the scratch for this call: the plan (head prefix, ranges used),
+  // partials (o), partials (m, l); everything is written before it is read
+  const long long parts = (long long)cache->decode_ctas + (long long)batch * c.Hkv;
+  const size_t plan_bytes = align256((size_t)(batch * c.Hkv + 1) * sizeof(long long) + 16);
   const size_t o_bytes = align256((size_t)parts * c.G * c.D * sizeof(float));
   const size_t ml_bytes = align256((size_t)parts * c.G * 2 * sizeof(float));
-  const size_t need = cnt_bytes + o_bytes + ml_bytes;
+  const size_t need = plan_bytes + o_bytes + ml_bytes;
   if (need > FDMS_STATIC_SCRATCH_BYTES) return FDMS_ERR_INVALID_ARG;
 
   int prev = -1;
@@ -1038,22 +1096,18 @@ extern "C" fdms_status fdms_decode_attn_noalloc(fdms_cache* cache, int layer, in
   } else {
     unsigned char* b = static_cast<unsigned char*>(base);
     DecodeWork w;
-    w.head_cnt = reinterpret_cast<int*>(b);
-    w.part_o = reinterpret_cast<float*>(b + cnt_bytes);
-    w.part_ml = reinterpret_cast<float*>(b + cnt_bytes + o_bytes);
-    w.head_off = nullptr;
-    w.n_eff = nullptr;
+    w.head_off = reinterpret_cast<long long*>(b);
+    w.n_eff = reinterpret_cast<int*>(b + plan_bytes - 16);
+    w.part_o = reinterpret_cast<float*>(b + plan_bytes);
+    w.part_ml = reinterpret_cast<float*>(b + plan_bytes + o_bytes);
     w.max_parts = (int)parts;
     w.max_ctas = cache->decode_ctas;
-    // the array keeps the previous call's contents: the counters must start at 0
-    if (cudaMemsetAsync(w.head_cnt, 0, cnt_bytes, s) != cudaSuccess) {
-      st = FDMS_ERR_CUDA;
-    } else {
-      OutArgs oa{out_dev, nullptr, 0};
-      st = by_config(c, [&](auto t) {
-        return launch_split_t<decltype(t)>(cache, w, oa, layer, batch, q_dev, s);
-      });
-    }
+    // the array keeps the previous call's contents; nothing in it needs to
+    // start at zero (every value is written by this call before it is read)
+    OutArgs oa{out_dev, nullptr, 0};
+    st = by_config(c, [&](auto t) {
+      return launch_split_t<decltype(t)>(cache, w, oa, layer, batch, q_dev, s);
+    });
   }
   if (prev != cache->device) cudaSetDevice(prev);
   return st;

@@ -89,7 +89,6 @@ __host__ __device__ inline uint8_t* ring_v(const CacheView& c, long long hi) {
 
 // Decode workspace (split partials and the plan the combine reads back).
 struct DecodeWork {
-  int* head_cnt;          // [heads]: partials written so far this call (0 between calls)
   float* part_o;          // [max_parts][G][D], unnormalised sum of p * v
   float* part_ml;         // [max_parts][G][2]: running max (log2 domain) and sum
   long long* head_off;    // [heads + 1]: prefix of units over the call's heads
