@@ -10,16 +10,19 @@
 // The kernel is memory bound: every byte of a visible K and V row is read once.
 //   - Work is balanced over the GPU by slots, not by heads. The slot lists of
 //     all heads of the call are laid end to end (units = store slots + ring
-//     slots) and cut into equal ranges, one per consumer warp of the grid; a
+//     slots) and cut into equal ranges, one per warp of the grid; a
 //     warp therefore reads the same number of bytes whatever the mix of head
 //     lengths, and emits one partial (m, l, o) per head its range touches.
-//   - A producer warp walks every consumer warp's tiles (32 rows of a 64-slot
-//     page for 128-byte rows) and stages a tile's K rows, V rows and the head's
-//     q into shared memory with 1-D bulk copies (cp.async.bulk, completion on an
-//     mbarrier). Rows keep their page row in shared memory, so the chunk
+//   - Each warp stages its own tiles (32 rows of a 64-slot page for 128-byte
+//     rows): the K rows, V rows and the head's q go to shared memory by 1-D
+//     bulk copies (cp.async.bulk, completion on an mbarrier) into one of the
+//     warp's two stages, and the warp refills a stage as soon as it has read
+//     it. The tile descriptors (head, rows, source address) are worked out 32
+//     at a time, one lane per tile, so the block-table reads of a warp's first
+//     tiles overlap. Rows keep their page row in shared memory, so the chunk
 //     permutation they are stored with makes the fragment loads below free of
-//     bank conflicts. Each of the 8 consumer warps owns two stages.
-//   - A consumer warp computes the scores of a tile on the tensor cores
+//     bank conflicts.
+//   - A warp computes the scores of a tile on the tensor cores
 //     (mma.sync m16n8k16, fp32 accumulate; the G query heads of the kv head
 //     are rows 0..G-1 of the 16-row A tile, keys are the columns), an online
 //     softmax in fp32 in the log2 domain, and o^T += V^T p^T on the tensor
@@ -47,24 +50,21 @@
 namespace fdms {
 namespace {
 
-constexpr int kMinUnitsPerRange = 64;  // a consumer warp gets at least 64 slots of work
+constexpr int kMinUnitsPerRange = 64;  // a warp gets at least 64 slots of work
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
 
 enum : int { kFirst = 1, kLast = 2, kRing = 4, kPending = 8 };
 
 struct TileMeta {
-  int hidx;      // head of the call (b * Hkv + h)
-  int row0;      // rows [row0, row1) of the tile frame hold this tile's slots
-  int row1;
-  int flags;
-  int p0;        // ring tiles: position of row row0
-  int thresh;    // ring tiles: positions below n - W need their keep bit
-  int R;         // ring capacity (slot = p % R)
-  float ks;      // K scale of the page
-  float vrel;    // V scale of the page / the head's V scale
-  float vhead;   // the head's V scale (1 for BF16)
-  long long keep_base;   // ring tiles: index of the head's ring_keep
+  const uint8_t* ksrc;   // first K row of the tile; its V rows follow the block's
+                         // (or the ring's) K rows
+  int hidx;              // head of the call (b * Hkv + h)
+  int rows;              // row0 | row1 << 8 | flags << 16: frame rows [row0, row1)
+  int p0;                // ring tiles: position of row row0
+  float ks;              // K scale of the page
+  float vrel;            // V scale of the page / the head's V scale
+  int pad;
 };
 
 // where the merged output goes
@@ -81,11 +81,11 @@ struct Dec {
   static constexpr int ELT = FP8 ? 1 : 2;
   static constexpr int RB = D * ELT;           // bytes per row
   static constexpr int TR = 4096 / RB;         // rows per tile: 4 KB of K, 4 KB of V
-  static constexpr int NCW = G * D >= 1024 ? 4 : 8;   // consumer warps
-  static constexpr int NC = NCW * 32;
-  static constexpr int NT = NC + 32;           // + one producer warp
-  static constexpr int SPW = 2;                // stages per consumer warp
+  static constexpr int NCW = G * D >= 1024 ? 4 : 8;   // warps (one unit range each)
+  static constexpr int NT = NCW * 32;
+  static constexpr int SPW = 2;                // stages per warp
   static constexpr int NSTAGE = NCW * SPW;
+  static constexpr int NMR = 64;               // tile descriptors held per warp
   static constexpr int KV_BYTES = TR * RB;
   static constexpr int Q_BYTES = G * D * 2;
   static constexpr int STAGE_BYTES = 2 * KV_BYTES + ((Q_BYTES + 127) / 128) * 128;
@@ -96,17 +96,16 @@ struct Dec {
   static constexpr int EC = 16 / ELT;          // elements per 16-byte chunk
   static constexpr int KCPT = RB / 64;         // K chunks per lane column (1, 2 or 4)
   static constexpr bool SPLIT = true;          // p = 16-bit head + 16-bit remainder
-  static_assert(NSTAGE <= 32, "one producer lane per stage");
   static_assert(TR >= 16 && TR <= 64 && 64 % TR == 0, "tiles tile a page");
 
-  // a consumer warp's unmerged partial of a head it shares with other warps:
+  // a warp's unmerged partial of a head it shares with other warps:
   // [hidx, pad x3][m x G][l x G][pad][o x G*D] floats
   static constexpr int SLOT_O = (4 + 2 * G + 3) / 4 * 4;
   static constexpr int SLOT_F = SLOT_O + G * D;
 
   static constexpr int OFF_META = NSTAGE * STAGE_BYTES;
-  static constexpr int OFF_BAR = OFF_META + NSTAGE * (int)sizeof(TileMeta);
-  static constexpr int OFF_SLOTS = OFF_BAR + 2 * NSTAGE * 8;
+  static constexpr int OFF_BAR = OFF_META + NCW * NMR * (int)sizeof(TileMeta);
+  static constexpr int OFF_SLOTS = OFF_BAR + NSTAGE * 8;
   static constexpr int OFF_HEADS = OFF_SLOTS + 2 * NCW * SLOT_F * 4;
   static size_t smem_bytes(int nh) {
     // head_off (i64), page_off (i32), len, n, r (i32), head scales (2 x f32)
@@ -147,15 +146,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// named barrier 1 over the consumer warps (the producer warp has left)
-template <int NC>
-__device__ __forceinline__ void consumer_sync_n() {
-  asm volatile("bar.sync 1, %0;" ::"n"(NC) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
-}
 
 template <class T>
 __device__ __forceinline__ int upper_bound(const T* a, int n, T x) {
@@ -242,13 +232,12 @@ __global__ void __launch_bounds__(T::NT, 1)
 k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
                const uint16_t* __restrict__ q, int n_launch_ranges) {
   constexpr int D = T::D, G = T::G, RB = T::RB, TR = T::TR, NSTAGE = T::NSTAGE,
-                NCW = T::NCW, SPW = T::SPW, NJ = T::NJ, NU = T::NU, KS = T::KS, MT = T::MT;
+                NCW = T::NCW, SPW = T::SPW, NJ = T::NJ, NU = T::NU, KS = T::KS, MT = T::MT,
+                NMR = T::NMR;
   constexpr bool FP8 = T::FP8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 127) & ~(uintptr_t)127);
-  TileMeta* meta = reinterpret_cast<TileMeta*>(smem + T::OFF_META);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + T::OFF_BAR);
-  uint64_t* empty = full + NSTAGE;
   const int NH = batch * c.Hkv;
   long long* head_off = reinterpret_cast<long long*>(smem + T::OFF_HEADS);   // [NH + 1]
   int* page_off = reinterpret_cast<int*>(head_off + NH + 1);                 // [NH + 1]
@@ -259,6 +248,7 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const long long hi0 = (long long)layer * c.Bmax * c.Hkv;   // first head of this layer
+  TileMeta* ring = reinterpret_cast<TileMeta*>(smem + T::OFF_META) + warp * NMR;
 
   // ---- set-up that reads no data the previous kernel writes: it overlaps
   // that kernel. Stale V rows of a stage are multiplied by p = 0, so they must
@@ -287,13 +277,10 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
         asm volatile("prefetch.global.L2 [%0];" ::"l"(arr + j * 128));
     }
   }
-  if (tid == 0) {
-    for (int s = 0; s < NSTAGE; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    fence_mbar_init();
-  }
+  if (lane < SPW) mbar_init(&full[warp * SPW + lane], 1);
+  fence_mbar_init();
+  float* slots = reinterpret_cast<float*>(smem + T::OFF_SLOTS);
+  if (lane < 2) slots[(warp * 2 + lane) * T::SLOT_F] = __int_as_float(-1);   // empty
   pdl_wait();                 // the previous kernel's writes are visible from here on
   pdl_launch_dependents();
 
@@ -376,130 +363,109 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
                            : (len + TR - 1) / TR + (int)((u - len + s_r[h] % TR) / TR);
     return page_off[h] + lp;
   };
-  // unit range of every consumer warp of this CTA, and its first page / page
-  // count: one thread per warp, once
-  __shared__ long long s_gs[NCW], s_ge[NCW];
-  __shared__ int s_gp0[NCW], s_nt[NCW];
-  __shared__ long long s_cgs, s_cge;   // the CTA's unit range
-  if (tid == NCW) {
-    const int v0 = blockIdx.x * NCW;
-    s_cgs = v0 < n_eff ? range_start(v0, total, n_eff) : total;
-    s_cge = range_start(min(n_eff, v0 + NCW), total, n_eff);
-  }
-  if (tid < NCW) {
-    const long long v = (long long)blockIdx.x * NCW + tid;
-    long long a = 0, b = 0;
-    int p0 = 0, n = 0;
-    if (v < n_eff) {
-      a = range_start(v, total, n_eff);
-      b = range_start(v + 1, total, n_eff);
-      if (a < b) {
-        p0 = gpage(a);
-        n = gpage(b - 1) - p0 + 1;
-      }
-    }
-    s_gs[tid] = a;
-    s_ge[tid] = b;
-    s_gp0[tid] = p0;
-    s_nt[tid] = n;
-  }
-  __syncthreads();
-  auto range_of = [&](int cw, long long& gs, long long& ge, int& gp0, int& nt) {
-    gs = s_gs[cw];
-    ge = s_ge[cw];
-    gp0 = s_gp0[cw];
-    nt = s_nt[cw];
-  };
-
-  if (warp == NCW) {
-    // ================= producer: lane l owns stage l, i.e. consumer warp l / SPW
-    // and that warp's tiles l % SPW, l % SPW + SPW, ...
-    if (lane < NSTAGE) {
-      const int cw = lane / SPW;
-      long long gs, ge;
-      int gp0, nt;
-      range_of(cw, gs, ge, gp0, nt);
-      for (int k = lane % SPW; k < nt; k += SPW) {
-        const int gp = gp0 + k;
-        const int hidx = upper_bound(page_off, NH + 1, gp) - 1;
-        const int lp = gp - page_off[hidx];
-        const int len = s_len[hidx], n = s_n[hidx], r = s_r[hidx];
-        const int sp = (len + TR - 1) / TR;
-        const long long hoff = head_off[hidx];
-        const long long lo = gs > hoff ? gs - hoff : 0;   // head units of this range
-        const long long hi_u = ge - hoff;
-        const long long hi = hi0 + hidx;
-        TileMeta mt;
-        mt.hidx = hidx;
-        mt.flags = (k == 0 || lp == 0 ? kFirst : 0) |
-                   (k == nt - 1 || gp + 1 == page_off[hidx + 1] ? kLast : 0);
-        mt.vhead = s_hscale[2 * hidx + 1];
-        mt.p0 = mt.thresh = mt.R = 0;
-        mt.keep_base = 0;
-        const uint8_t *ksrc, *vsrc;
-        if (lp < sp) {   // store tile lp: block lp * TR / 64, rows from (lp * TR) % 64
-          const long long u0 = max((long long)lp * TR, lo);
-          const long long u1 = min((long long)min((lp + 1) * TR, len), hi_u);
-          const int j = lp * TR / kBlockSlots;
-          const int rb = (lp * TR) % kBlockSlots;          // block row of frame row 0
-          mt.row0 = (int)(u0 - (long long)lp * TR);
-          mt.row1 = (int)(u1 - (long long)lp * TR);
-          const long long blk = c.block_table[hi * c.max_blocks + j];
-          if (FP8) {
-            mt.ks = c.bt_scale[(hi * c.max_blocks + j) * 2];
-            mt.vrel = c.bt_scale[(hi * c.max_blocks + j) * 2 + 1] / mt.vhead;
-          } else {
-            mt.ks = mt.vrel = 1.0f;
-          }
-          ksrc = block_k(c, blk) + (long long)(rb + mt.row0) * RB;
-          vsrc = block_v(c, blk) + (long long)(rb + mt.row0) * RB;
-        } else {         // ring tile: live units [TR*rp - off, TR*(rp+1) - off)
-          const int rp = lp - sp, off = r % TR, live = n - r;
-          const long long a = max((long long)len + max(TR * rp - off, 0), lo);
-          const long long b = min((long long)len + min(TR * (rp + 1) - off, live), hi_u);
-          const int p0 = r + (int)(a - len);
-          const int slot0 = p0 % c.R;
-          mt.row0 = slot0 % TR;
-          mt.row1 = mt.row0 + (int)(b - a);
-          mt.p0 = p0;
-          mt.thresh = n - c.W;
-          mt.R = c.R;
-          mt.keep_base = hi * c.Rpad;
-          mt.flags |= kRing | (p0 < mt.thresh ? kPending : 0);
-          mt.ks = s_hscale[2 * hidx];
-          mt.vrel = 1.0f;
-          ksrc = ring_k(c, hi) + (long long)slot0 * RB;
-          vsrc = ring_v(c, hi) + (long long)slot0 * RB;
-        }
-        const int s = lane;
-        const int use = k / SPW;
-        if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1)) {
-          latch_error(c.ctr, FDMS_ERR_DEVICE);
-          break;
-        }
-        meta[s] = mt;
-        uint8_t* kdst = smem + s * T::STAGE_BYTES;
-        uint8_t* vdst = kdst + T::KV_BYTES;
-        const uint32_t rows = (uint32_t)(mt.row1 - mt.row0);
-        mbar_arrive_expect_tx(&full[s], 2u * rows * RB + (uint32_t)T::Q_BYTES);
-        bulk_g2s(kdst + mt.row0 * RB, ksrc, rows * RB, &full[s]);
-        bulk_g2s(vdst + mt.row0 * RB, vsrc, rows * RB, &full[s]);
-        const int b = hidx / c.Hkv, h = hidx % c.Hkv;
-        bulk_g2s(vdst + T::KV_BYTES, q + ((long long)b * c.Hq + (long long)h * G) * D, T::Q_BYTES,
-                 &full[s]);
-      }
-    }
-    return;
-  }
-
-  // ================= consumer warp `warp`
-  const int g = lane >> 2, t = lane & 3;
-  long long gs, ge;
+  // ---- this warp's unit range [gs, ge), its pages [gp0, gp0 + nt), and the
+  // CTA's unit range [cgs, cge): one bound per lane
+  long long gs, ge, cgs, cge;
   int gp0, nt;
-  range_of(warp, gs, ge, gp0, nt);
+  {
+    const int v = (int)blockIdx.x * NCW + warp, v0 = (int)blockIdx.x * NCW;
+    const int vv = lane == 0 ? v : lane == 1 ? v + 1 : lane == 2 ? v0 : min(n_eff, v0 + NCW);
+    const long long x = lane < 4 && vv < n_eff ? range_start(vv, total, n_eff) : total;
+    gs = __shfl_sync(0xffffffffu, x, 0);
+    ge = __shfl_sync(0xffffffffu, x, 1);
+    cgs = __shfl_sync(0xffffffffu, x, 2);
+    cge = __shfl_sync(0xffffffffu, x, 3);
+    const int pg = lane < 2 && gs < ge ? gpage(lane == 0 ? gs : ge - 1) : 0;
+    gp0 = __shfl_sync(0xffffffffu, pg, 0);
+    nt = gs < ge ? __shfl_sync(0xffffffffu, pg, 1) - gp0 + 1 : 0;
+  }
+
+  // descriptor of this warp's tile k (one lane per tile)
+  auto make_meta = [&](int k) -> TileMeta {
+    TileMeta mt;
+    const int gp = gp0 + k;
+    const int hidx = upper_bound(page_off, NH + 1, gp) - 1;
+    const int lp = gp - page_off[hidx];
+    const int len = s_len[hidx], n = s_n[hidx], r = s_r[hidx];
+    const int sp = (len + TR - 1) / TR;
+    const long long hoff = head_off[hidx];
+    const long long lo = gs > hoff ? gs - hoff : 0;   // head units of this range
+    const long long hi_u = ge - hoff;
+    const long long hi = hi0 + hidx;
+    int flags = (k == 0 || lp == 0 ? kFirst : 0) |
+                (k == nt - 1 || gp + 1 == page_off[hidx + 1] ? kLast : 0);
+    int row0, row1;
+    mt.hidx = hidx;
+    mt.p0 = 0;
+    mt.pad = 0;
+    if (lp < sp) {   // store tile lp: block lp * TR / 64, rows from (lp * TR) % 64
+      const long long u0 = max((long long)lp * TR, lo);
+      const long long u1 = min((long long)min((lp + 1) * TR, len), hi_u);
+      const int j = lp * TR / kBlockSlots;
+      const int rb = (lp * TR) % kBlockSlots;          // block row of frame row 0
+      row0 = (int)(u0 - (long long)lp * TR);
+      row1 = (int)(u1 - (long long)lp * TR);
+      const long long blk = c.block_table[hi * c.max_blocks + j];
+      if (FP8) {
+        mt.ks = c.bt_scale[(hi * c.max_blocks + j) * 2];
+        mt.vrel = c.bt_scale[(hi * c.max_blocks + j) * 2 + 1] / s_hscale[2 * hidx + 1];
+      } else {
+        mt.ks = mt.vrel = 1.0f;
+      }
+      mt.ksrc = block_k(c, blk) + (long long)(rb + row0) * RB;
+    } else {         // ring tile: live units [TR*rp - off, TR*(rp+1) - off)
+      const int rp = lp - sp, off = r % TR, live = n - r;
+      const long long a = max((long long)len + max(TR * rp - off, 0), lo);
+      const long long b = min((long long)len + min(TR * (rp + 1) - off, live), hi_u);
+      const int p0 = r + (int)(a - len);
+      const int slot0 = p0 % c.R;
+      row0 = slot0 % TR;
+      row1 = row0 + (int)(b - a);
+      mt.p0 = p0;
+      flags |= kRing | (p0 < n - c.W ? kPending : 0);
+      mt.ks = s_hscale[2 * hidx];
+      mt.vrel = 1.0f;
+      mt.ksrc = ring_k(c, hi) + (long long)slot0 * RB;
+    }
+    mt.rows = row0 | row1 << 8 | flags << 16;
+    return mt;
+  };
+  // stage the K rows, V rows and q of tile k (one lane)
+  auto issue = [&](const TileMeta& mt, int k) {
+    const int s = warp * SPW + k % SPW;
+    uint8_t* kdst = smem + s * T::STAGE_BYTES;
+    uint8_t* vdst = kdst + T::KV_BYTES;
+    const int row0 = mt.rows & 0xFF, row1 = (mt.rows >> 8) & 0xFF;
+    const uint32_t nb = (uint32_t)(row1 - row0) * RB;
+    const long long voff =
+        (long long)((mt.rows >> 16) & kRing ? c.R : kBlockSlots) * RB;
+    mbar_arrive_expect_tx(&full[s], 2u * nb + (uint32_t)T::Q_BYTES);
+    bulk_g2s(kdst + row0 * RB, mt.ksrc, nb, &full[s]);
+    bulk_g2s(vdst + row0 * RB, mt.ksrc + voff, nb, &full[s]);
+    const int b = mt.hidx / c.Hkv, h = mt.hidx % c.Hkv;
+    bulk_g2s(vdst + T::KV_BYTES, q + ((long long)b * c.Hq + (long long)h * G) * D, T::Q_BYTES,
+             &full[s]);
+  };
+  // descriptors of tiles [k0, k0 + 32) into the warp's ring
+  auto fill = [&](int k0) {
+    const int k = k0 + lane;
+    if (k < nt) ring[k % NMR] = make_meta(k);
+  };
+  // first descriptors; lanes 0 .. SPW-1 stage their tiles at once
+  {
+    const int k = lane;
+    if (k < nt) {
+      const TileMeta mt = make_meta(k);
+      ring[k] = mt;
+      if (k < SPW) issue(mt, k);
+    }
+    fill(32);
+    __syncwarp();
+  }
+
+  // ================= tiles of this warp
+  const int g = lane >> 2, t = lane & 3;
   const float qscale = c.softmax_scale * kLog2e;
-  float* slots = reinterpret_cast<float*>(smem + T::OFF_SLOTS);
-  if (lane < 2) slots[(warp * 2 + lane) * T::SLOT_F] = __int_as_float(-1);   // empty
 
   // shared-memory byte offsets of this lane's fragment loads inside a tile:
   // K rows 8j + g (the row permutation bits are g for every j), V rows
@@ -534,7 +500,23 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
       if (lane == 0) latch_error(c.ctr, FDMS_ERR_DEVICE);
       break;
     }
-    const TileMeta mt = meta[s];
+    const TileMeta tm = ring[k % NMR];
+    struct {
+      int hidx, row0, row1, flags, p0, thresh, R;
+      float ks, vrel, vhead;
+      long long keep_base;
+    } mt;
+    mt.hidx = tm.hidx;
+    mt.row0 = tm.rows & 0xFF;
+    mt.row1 = (tm.rows >> 8) & 0xFF;
+    mt.flags = tm.rows >> 16;
+    mt.p0 = tm.p0;
+    mt.thresh = s_n[tm.hidx] - c.W;
+    mt.R = c.R;
+    mt.ks = tm.ks;
+    mt.vrel = tm.vrel;
+    mt.vhead = s_hscale[2 * tm.hidx + 1];
+    mt.keep_base = (hi0 + tm.hidx) * c.Rpad;
     const uint8_t* Ks = smem + s * T::STAGE_BYTES;
     const uint8_t* Vs = Ks + T::KV_BYTES;
     const uint16_t* Qs = reinterpret_cast<const uint16_t*>(Vs + T::KV_BYTES);
@@ -747,7 +729,13 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
       }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
+    // the stage is free: refill it with tile k + SPW (descriptors come 32 at a
+    // time, those of tiles k + 33 .. k + 64 once tile k + 1 starts a new 32)
+    if ((k + 1) % 32 == 0 && k + 33 < nt) {
+      fill(k + 33);
+      __syncwarp();
+    }
+    if (lane == 0 && k + SPW < nt) issue(ring[(k + SPW) % NMR], k + SPW);
 
     // ---- end of this head inside the range
     if (mt.flags & kLast) {
@@ -810,7 +798,7 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   // memory); write heads inside this CTA's range, leave one CTA partial of the
   // others for the combine kernel. Valid slots carry non-decreasing heads in
   // slot order, so each head is one run of slots, empty slots aside.
-  consumer_sync_n<T::NC>();
+  __syncthreads();
   {
     constexpr int kMaxRuns = 2 * NCW;
     __shared__ int s_run_head[kMaxRuns];
@@ -830,10 +818,9 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
       if (start) s_run_head[__popc(ball & ((1u << lane) - 1u))] = hk;
       if (lane == 0) s_nruns = __popc(ball);
     }
-    consumer_sync_n<T::NC>();
+    __syncthreads();
     const int nr = s_nruns;
-    const long long cgs = s_cgs, cge = s_cge;
-    for (int it = tid; it < nr * G * D; it += T::NC) {
+    for (int it = tid; it < nr * G * D; it += T::NT) {
       const int run = it / (G * D), idx = it % (G * D);
       const int hd = s_run_head[run], h = idx / D, d = idx % D;
       float mk[2 * NCW], lk[2 * NCW], ok[2 * NCW];

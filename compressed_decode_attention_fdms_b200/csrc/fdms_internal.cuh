@@ -200,7 +200,7 @@ struct fdms_cache {
   int nallocs;
   int decode_ctas;        // split grid used
   int ctas_per_sm;
-  int ranges_per_cta;     // consumer warps per split CTA (one unit range each)
+  int ranges_per_cta;     // warps per split CTA (one unit range each)
 };
 
 // launchers (defined in their .cu files)
