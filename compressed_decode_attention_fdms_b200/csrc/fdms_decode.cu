@@ -34,11 +34,10 @@
 //     that the score scale undoes; the page's K scale multiplies the scores
 //     and its V scale the probabilities, never the elements.
 //   - A head that lies whole inside one warp's range is written by that warp;
-//     heads with no slot get zeros. Warps that share a head leave their
-//     partials in shared memory; the CTA merges them and writes the heads that
-//     lie inside its range, and leaves one CTA partial of the others; a small
-//     combine kernel merges those (2-4 per head at 8K context),
-//     o = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c.
+//     heads with no slot get zeros. Every other head has one partial
+//     (m, l, o) per warp that covered part of it, written to a workspace; a
+//     combine kernel merges them, one output element per thread, loading the
+//     partials together: o = sum_w 2^(m_w - M) o_w / sum_w 2^(m_w - M) l_w.
 //   - Both kernels allow programmatic dependent launch: set-up that reads no
 //     data of the previous kernel runs while that kernel finishes.
 #include <cfloat>
@@ -98,15 +97,9 @@ struct Dec {
   static constexpr bool SPLIT = true;          // p = 16-bit head + 16-bit remainder
   static_assert(TR >= 16 && TR <= 64 && 64 % TR == 0, "tiles tile a page");
 
-  // a warp's unmerged partial of a head it shares with other warps:
-  // [hidx, pad x3][m x G][l x G][pad][o x G*D] floats
-  static constexpr int SLOT_O = (4 + 2 * G + 3) / 4 * 4;
-  static constexpr int SLOT_F = SLOT_O + G * D;
-
   static constexpr int OFF_META = NSTAGE * STAGE_BYTES;
   static constexpr int OFF_BAR = OFF_META + NCW * NMR * (int)sizeof(TileMeta);
-  static constexpr int OFF_SLOTS = OFF_BAR + NSTAGE * 8;
-  static constexpr int OFF_HEADS = OFF_SLOTS + 2 * NCW * SLOT_F * 4;
+  static constexpr int OFF_HEADS = OFF_BAR + NSTAGE * 8;
   static size_t smem_bytes(int nh) {
     // head_off (i64), page_off (i32), len, n, r (i32), head scales (2 x f32)
     return 128 + OFF_HEADS + (size_t)(nh + 1) * 8 + (size_t)(nh + 1) * 4 +
@@ -147,33 +140,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 }
 
 
-template <class T>
-__device__ __forceinline__ int upper_bound(const T* a, int n, T x) {
-  int lo = 0, hi = n;   // first index with a[i] > x
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (a[mid] <= x) lo = mid + 1; else hi = mid;
-  }
-  return lo;
-}
-
-// floor(a / b) for 0 <= a < 2^53, 0 < b: exact through fp64 when the quotient
-// is below 2^20 and b below 2^32 (a non-integer quotient then keeps a
-// fractional part of at least 1/b > 2^-32, larger than the rounding error of
-// the fp64 division); the 64-bit integer division, a long software sequence
-// on the GPU, is kept for the rest.
-__device__ __forceinline__ long long floor_div(long long a, long long b) {
-  if (a < (1LL << 52) && b < (1LL << 32) && a < (b << 20))
-    return (long long)floor(__ddiv_rn((double)a, (double)b));
+// a / b for 0 <= a, 0 < b: 32-bit division when both fit (a short sequence),
+// the 64-bit one (a long software sequence) otherwise.
+__device__ __forceinline__ long long udiv(long long a, long long b) {
+  if (a < (1LL << 32) && b < (1LL << 32)) return (long long)((unsigned)a / (unsigned)b);
   return a / b;
-}
-// first unit of range v when T units are cut into n ranges: floor(v * T / n)
-__device__ __forceinline__ long long range_start(long long v, long long total, int n) {
-  return floor_div(v * total, n);
-}
-// range of unit x under the split: the largest v with floor(v * T / N) <= x.
-__device__ __forceinline__ int range_of_unit(long long x, long long total, int n) {
-  return (int)floor_div((x + 1) * n - 1, total);
 }
 
 // ------------------------------------------------------------- MMA helpers
@@ -230,7 +201,7 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 template <class T>
 __global__ void __launch_bounds__(T::NT, 1)
 k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
-               const uint16_t* __restrict__ q, int n_launch_ranges) {
+               const uint16_t* __restrict__ q, int n_ranges, double inv_ranges) {
   constexpr int D = T::D, G = T::G, RB = T::RB, TR = T::TR, NSTAGE = T::NSTAGE,
                 NCW = T::NCW, SPW = T::SPW, NJ = T::NJ, NU = T::NU, KS = T::KS, MT = T::MT,
                 NMR = T::NMR;
@@ -279,8 +250,6 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   }
   if (lane < SPW) mbar_init(&full[warp * SPW + lane], 1);
   fence_mbar_init();
-  float* slots = reinterpret_cast<float*>(smem + T::OFF_SLOTS);
-  if (lane < 2) slots[(warp * 2 + lane) * T::SLOT_F] = __int_as_float(-1);   // empty
   pdl_wait();                 // the previous kernel's writes are visible from here on
   pdl_launch_dependents();
 
@@ -331,12 +300,21 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
     __syncthreads();
   }
   const long long total = head_off[NH];
-  const long long want = (total + kMinUnitsPerRange - 1) / kMinUnitsPerRange;
-  const int n_eff = (int)(want < n_launch_ranges ? (want > 0 ? want : 1) : n_launch_ranges);
+  // Warp v reads units [v S, (v + 1) S) of the call's units, S = ceil(total /
+  // ranges) (at least kMinUnitsPerRange): an fp64 estimate of the quotient made
+  // exact by integer correction.
+  long long S;
+  {
+    long long qq = (long long)((double)total * inv_ranges);
+    while (qq * n_ranges > total) --qq;
+    while ((qq + 1) * n_ranges <= total) ++qq;
+    S = qq + (qq * n_ranges < total ? 1 : 0);
+    S = S > kMinUnitsPerRange ? S : kMinUnitsPerRange;
+  }
   if (blockIdx.x == 0) {   // the plan the combine kernel reads back
     for (int h = tid; h <= NH; h += T::NT) w.head_off[h] = head_off[h];
     if (tid == 0) {
-      *w.n_eff = n_eff;
+      *w.span = S;
       c.ctr->slots_decoded += (unsigned long long)total;   // one thread, launches are ordered
       c.ctr->decode_calls += 1ull;
     }
@@ -352,39 +330,47 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
       if (oa.lse && i % D == 0) oa.lse[(long long)b * c.Hq + kh * G + i / D] = -INFINITY;
     }
   }
-  if ((int)blockIdx.x * NCW >= n_eff || total == 0) return;
+  const long long v_range = (long long)blockIdx.x * NCW + warp;
+  if ((long long)blockIdx.x * NCW * S >= total) return;
 
-  // page (in the call's page numbering) holding global unit x
-  auto gpage = [&](long long x) -> int {
-    const int h = upper_bound(head_off, NH + 1, x) - 1;
-    const long long u = x - head_off[h];
-    const int len = s_len[h];
-    const int lp = u < len ? (int)(u / TR)
-                           : (len + TR - 1) / TR + (int)((u - len + s_r[h] % TR) / TR);
-    return page_off[h] + lp;
-  };
-  // ---- this warp's unit range [gs, ge), its pages [gp0, gp0 + nt), and the
-  // CTA's unit range [cgs, cge): one bound per lane
-  long long gs, ge, cgs, cge;
-  int gp0, nt;
-  {
-    const int v = (int)blockIdx.x * NCW + warp, v0 = (int)blockIdx.x * NCW;
-    const int vv = lane == 0 ? v : lane == 1 ? v + 1 : lane == 2 ? v0 : min(n_eff, v0 + NCW);
-    const long long x = lane < 4 && vv < n_eff ? range_start(vv, total, n_eff) : total;
-    gs = __shfl_sync(0xffffffffu, x, 0);
-    ge = __shfl_sync(0xffffffffu, x, 1);
-    cgs = __shfl_sync(0xffffffffu, x, 2);
-    cge = __shfl_sync(0xffffffffu, x, 3);
-    const int pg = lane < 2 && gs < ge ? gpage(lane == 0 ? gs : ge - 1) : 0;
-    gp0 = __shfl_sync(0xffffffffu, pg, 0);
-    nt = gs < ge ? __shfl_sync(0xffffffffu, pg, 1) - gp0 + 1 : 0;
+  // ---- this warp's unit range [gs, ge), the heads h_gs .. h_ge it touches,
+  // its pages [gp0, gp0 + nt)
+  const long long gs = min(v_range * S, total), ge = min(gs + S, total);
+  int h_gs = 0, h_ge = 0, gp0 = 0, nt = 0;
+  if (gs < ge) {
+    // head of unit x: the number of heads h >= 1 with head_off[h] <= x
+    int c0 = 0, c1 = 0;
+    for (int base = 1; base < NH; base += 32) {
+      const int h = base + lane;
+      const long long ho = h < NH ? head_off[h] : total;
+      c0 += __popc(__ballot_sync(0xffffffffu, ho <= gs));
+      c1 += __popc(__ballot_sync(0xffffffffu, ho <= ge - 1));
+    }
+    h_gs = c0;
+    h_ge = c1;
+    // page (in the call's page numbering) holding unit x of head h
+    auto gpage = [&](int h, long long x) -> int {
+      const long long u = x - head_off[h];
+      const int len = s_len[h];
+      const int lp = u < len ? (int)(u / TR)
+                             : (len + TR - 1) / TR + (int)((u - len + s_r[h] % TR) / TR);
+      return page_off[h] + lp;
+    };
+    gp0 = gpage(h_gs, gs);
+    nt = gpage(h_ge, ge - 1) - gp0 + 1;
   }
 
   // descriptor of this warp's tile k (one lane per tile)
   auto make_meta = [&](int k) -> TileMeta {
     TileMeta mt;
     const int gp = gp0 + k;
-    const int hidx = upper_bound(page_off, NH + 1, gp) - 1;
+    // head of page gp: the last h in [h_gs, h_ge] with page_off[h] <= gp
+    int h_lo = h_gs, h_hi = h_ge;
+    while (h_lo < h_hi) {
+      const int mid = (h_lo + h_hi + 1) >> 1;
+      if (page_off[mid] <= gp) h_lo = mid; else h_hi = mid - 1;
+    }
+    const int hidx = h_lo;
     const int lp = gp - page_off[hidx];
     const int len = s_len[hidx], n = s_n[hidx], r = s_r[hidx];
     const int sp = (len + TR - 1) / TR;
@@ -571,15 +557,34 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
       for (int i = 0; i < MT; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
     }
 
+    // ---- visible rows of the tile frame: [row0, row1), less the pending ring
+    // rows whose keep bit is 0 (one ring_keep byte per row, read only then)
+    const bool pend = (mt.flags & kPending) != 0;
+    const bool full_tile = row0 == 0 && row1 == TR && !pend;
+    unsigned long long vmask = ~0ull;
+    if (!full_tile) {
+      vmask = (row1 >= 64 ? ~0ull : (1ull << row1) - 1ull) & ~((1ull << row0) - 1ull);
+      if (pend) {
+#pragma unroll
+        for (int h2 = 0; h2 < (TR + 31) / 32; ++h2) {
+          const int row = 32 * h2 + lane;
+          bool drop = false;
+          if (row < TR && row >= row0 && row < row1) {
+            const int p = mt.p0 + (row - row0);
+            drop = p < mt.thresh && c.ring_keep[mt.keep_base + p % mt.R] == 0;
+          }
+          const unsigned bd = __ballot_sync(0xffffffffu, drop);
+          vmask &= ~((unsigned long long)bd << (32 * h2));
+        }
+      }
+      vmask >>= 2 * t;   // bit 8j + e: row 8j + 2t + e of this lane
+    }
+
     // ---- scores of rows 8j + (0..7): S[head g][keys 8j + 2t, 8j + 2t + 1]
     float sc[NJ][2];
     const float mul = qmul * mt.ks;
-    const bool pend = (mt.flags & kPending) != 0;
-    const bool full_tile = row0 == 0 && row1 == TR && !pend;
 #pragma unroll
     for (int j = 0; j < NJ; ++j) {
-      sc[j][0] = sc[j][1] = -INFINITY;
-      if (8 * j + 8 <= row0 || 8 * j >= row1) continue;
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t kw[T::KCPT][4];   // key row 8j + g, this lane's chunks
 #pragma unroll
@@ -601,48 +606,38 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
         }
         mma16816<FP8>(acc, qa[s2][0], 0u, qa[s2][1], 0u, b0, b1);
       }
-      const int ra = 8 * j + 2 * t;
-      if (full_tile) {
-        sc[j][0] = acc[0] * mul;
-        sc[j][1] = acc[1] * mul;
-      } else {
+      sc[j][0] = acc[0] * mul;
+      sc[j][1] = acc[1] * mul;
+    }
+    if (!full_tile) {
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int row = ra + e;
-          bool vis = row >= row0 && row < row1;
-          if (vis && pend) {
-            const int p = mt.p0 + (row - row0);
-            if (p < mt.thresh) vis = c.ring_keep[mt.keep_base + p % mt.R] != 0;
-          }
-          sc[j][e] = vis ? acc[e] * mul : -INFINITY;
-        }
-      }
+      for (int j = 0; j < NJ; ++j)
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+          if (!((vmask >> (8 * j + e)) & 1ull)) sc[j][e] = -INFINITY;
     }
 
-    // ---- online softmax for row (head) g; the 4 lanes of a quad share it
+    // ---- online softmax for row (head) g; the 4 lanes of a quad share it.
+    // With no visible key so far the reference point is 0: every p is then
+    // 2^-inf = 0 and so is the rescale of the (empty) accumulators.
     float mx = -INFINITY;
 #pragma unroll
     for (int j = 0; j < NJ; ++j) mx = fmaxf(mx, fmaxf(sc[j][0], sc[j][1]));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
     const float mn = fmaxf(m_run, mx);
-    float alpha = 1.f;
+    const float mref = mn == -INFINITY ? 0.f : mn;
+    const float alpha = fast_exp2(m_run - mref);
     float pr[NJ][2];
-    if (mn == -INFINITY) {
+    float ls = 0.f;
 #pragma unroll
-      for (int j = 0; j < NJ; ++j) pr[j][0] = pr[j][1] = 0.f;
-    } else {
-      alpha = fast_exp2(m_run - mn);
-      float ls = 0.f;
-#pragma unroll
-      for (int j = 0; j < NJ; ++j) {
-        pr[j][0] = fast_exp2(sc[j][0] - mn);
-        pr[j][1] = fast_exp2(sc[j][1] - mn);
-        ls += pr[j][0] + pr[j][1];
-      }
-      l_run = l_run * alpha + ls;
-      m_run = mn;
+    for (int j = 0; j < NJ; ++j) {
+      pr[j][0] = fast_exp2(sc[j][0] - mref);
+      pr[j][1] = fast_exp2(sc[j][1] - mref);
+      ls += pr[j][0] + pr[j][1];
     }
+    l_run = l_run * alpha + ls;
+    m_run = mn;
     // o^T columns are heads 2t, 2t+1: their rescale factors live in quads 2t, 2t+1
     const float al_e = __shfl_sync(0xffffffffu, alpha, 8 * t);
     const float al_o = __shfl_sync(0xffffffffu, alpha, 8 * t + 4);
@@ -657,7 +652,6 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
     // ---- o^T += V^T p^T, keys 16u .. 16u + 15 per k-step
 #pragma unroll
     for (int u = 0; u < NU; ++u) {
-      if (16 * u + 16 <= row0 || 16 * u >= row1) continue;
       // p^T B fragment: (keys 16u + 2t, +1) and (16u + 8 + 2t, +1) of head g
       const float p0 = pr[2 * u][0] * mt.vrel, p1 = pr[2 * u][1] * mt.vrel;
       const float p2 = pr[2 * u + 1][0] * mt.vrel, p3 = pr[2 * u + 1][1] * mt.vrel;
@@ -770,143 +764,71 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
           }
         }
       } else {
-        // shared with other warps: leave the unmerged partial in this warp's slot
-        // 0 (the head began before the range) or 1 (it goes on after it)
-        float* sl = slots + (warp * 2 + (hs < gs ? 0 : 1)) * T::SLOT_F;
+        // shared with other warps: this warp's partial goes to the workspace,
+        // at v + hidx (unique: a warp's heads are consecutive, and later
+        // warps never go back to earlier heads)
+        const long long part = v_range + hidx;
+        float* po = w.part_o + part * G * D;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int h = 2 * t + e;
           if (h < G) {
 #pragma unroll
             for (int i = 0; i < MT; ++i) {
-              sl[T::SLOT_O + h * D + T::vdim(g, i, 0)] = oacc[i][e] * mt.vhead;
-              sl[T::SLOT_O + h * D + T::vdim(g, i, 1)] = oacc[i][2 + e] * mt.vhead;
+              po[h * D + T::vdim(g, i, 0)] = oacc[i][e] * mt.vhead;
+              po[h * D + T::vdim(g, i, 1)] = oacc[i][2 + e] * mt.vhead;
             }
           }
         }
         if (t == 0 && g < G) {
-          sl[4 + g] = m_run;
-          sl[4 + G + g] = l;
-        }
-        __syncwarp();
-        if (lane == 0) sl[0] = __int_as_float(hidx);
-      }
-    }
-  }
-
-  // ================= heads shared between warps: merge their slots (shared
-  // memory); write heads inside this CTA's range, leave one CTA partial of the
-  // others for the combine kernel. Valid slots carry non-decreasing heads in
-  // slot order, so each head is one run of slots, empty slots aside.
-  __syncthreads();
-  {
-    constexpr int kMaxRuns = 2 * NCW;
-    __shared__ int s_run_head[kMaxRuns];
-    __shared__ int s_nruns;
-    if (warp == 0) {
-      const int hk = lane < 2 * NCW ? __float_as_int(slots[lane * T::SLOT_F]) : -1;
-      int pm = hk;   // inclusive prefix max of the heads (heads only grow)
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int o = __shfl_up_sync(0xffffffffu, pm, off);
-        if (lane >= off) pm = max(pm, o);
-      }
-      int prev = __shfl_up_sync(0xffffffffu, pm, 1);
-      if (lane == 0) prev = -1;
-      const bool start = hk >= 0 && hk > prev;
-      const unsigned ball = __ballot_sync(0xffffffffu, start);
-      if (start) s_run_head[__popc(ball & ((1u << lane) - 1u))] = hk;
-      if (lane == 0) s_nruns = __popc(ball);
-    }
-    __syncthreads();
-    const int nr = s_nruns;
-    for (int it = tid; it < nr * G * D; it += T::NT) {
-      const int run = it / (G * D), idx = it % (G * D);
-      const int hd = s_run_head[run], h = idx / D, d = idx % D;
-      float mk[2 * NCW], lk[2 * NCW], ok[2 * NCW];
-      float M = -INFINITY;
-#pragma unroll
-      for (int sk = 0; sk < 2 * NCW; ++sk) {   // independent loads, then the merge
-        const float* sl = slots + sk * T::SLOT_F;
-        const bool mine = __float_as_int(sl[0]) == hd;
-        mk[sk] = mine ? sl[4 + h] : -INFINITY;
-        lk[sk] = sl[4 + G + h];
-        ok[sk] = sl[T::SLOT_O + h * D + d];
-        M = fmaxf(M, mk[sk]);
-      }
-      float L = 0.f, O = 0.f;
-      if (M != -INFINITY) {
-#pragma unroll
-        for (int sk = 0; sk < 2 * NCW; ++sk) {
-          if (mk[sk] == -INFINITY) continue;
-          const float bb = fast_exp2(mk[sk] - M);
-          L += lk[sk] * bb;
-          O += ok[sk] * bb;
-        }
-      }
-      const int kb = hd / c.Hkv, kh = hd % c.Hkv;
-      if (head_off[hd] >= cgs && head_off[hd + 1] <= cge) {
-        const float o = M == -INFINITY ? 0.f : O / L;
-        const long long oi = ((long long)kb * c.Hq + (long long)kh * G + h) * D + d;
-        if (oa.f32) static_cast<float*>(oa.out)[oi] = o;
-        else static_cast<uint16_t*>(oa.out)[oi] = f32_to_bf16_rn(o);
-        if (oa.lse && d == 0)
-          oa.lse[(long long)kb * c.Hq + kh * G + h] =
-              M == -INFINITY ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
-      } else {
-        const long long part = (long long)blockIdx.x + hd;
-        w.part_o[(part * G + h) * D + d] = O;
-        if (d == 0) {
-          w.part_ml[(part * G + h) * 2] = M;
-          w.part_ml[(part * G + h) * 2 + 1] = L;
+          w.part_ml[(part * G + g) * 2] = m_run;
+          w.part_ml[(part * G + g) * 2 + 1] = l;
         }
       }
     }
   }
 }
 
-// Merge of the CTA partials of one (seq, kv head) that several split CTAs
-// covered: o = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c. Heads inside one
-// CTA's range, or with no slot, were written by the split kernel. The (m, l, o)
-// of all partials are loaded together, in rounds of 8 partials.
-template <int D, int G, int NCW>
+// Merge of the warp partials of one (seq, kv head) that several warps covered:
+// o = sum_w 2^(m_w - M) o_w / sum_w 2^(m_w - M) l_w. Heads inside one warp's
+// range, or with no slot, were written by the split kernel. A thread merges one
+// output element; the (m, l, o) of up to kChunk partials are loaded together,
+// then merged, so a head with up to kChunk partials costs one round trip.
+template <int D, int G>
 __global__ void __launch_bounds__(256)
 k_decode_combine(DecodeWork w, int Hkv, int Hq, int batch, OutArgs oa) {
+  constexpr int kChunk = 16;
   pdl_wait();
   pdl_launch_dependents();
   const int hidx = blockIdx.x, tid = threadIdx.x;
-  const long long hs = w.head_off[hidx], he = w.head_off[hidx + 1];
-  const long long total = w.head_off[batch * Hkv];
-  const int n = *w.n_eff;
+  const long long hs = w.head_off[hidx], he = w.head_off[hidx + 1], S = *w.span;
   if (he == hs) return;
-  const int c0 = range_of_unit(hs, total, n) / NCW, c1 = range_of_unit(he - 1, total, n) / NCW;
-  if (c0 == c1) return;
+  const long long r0 = udiv(hs, S), r1 = udiv(he - 1, S);
+  if (r0 == r1) return;
   const int kb = hidx / Hkv, kh = hidx % Hkv;
   for (int idx = tid; idx < G * D; idx += 256) {
     const int h = idx / D, d = idx % D;
     float M = -INFINITY, L = 0.f, O = 0.f;
-    constexpr int B = 8;
-    for (int p0 = c0; p0 <= c1; p0 += B) {
-      float mb[B], lb[B], ob[B];
+    for (long long p0 = r0; p0 <= r1; p0 += kChunk) {
+      float mb[kChunk], lb[kChunk], ob[kChunk];
 #pragma unroll
-      for (int u = 0; u < B; ++u) {   // loads first, all independent
-        const long long pp = (long long)(p0 + u) + hidx;
-        const bool live = p0 + u <= c1;
+      for (int u = 0; u < kChunk; ++u) {   // loads first, all independent
+        const long long pp = p0 + u + hidx;
+        const bool live = p0 + u <= r1;
         mb[u] = live ? __ldcg(&w.part_ml[(pp * G + h) * 2]) : -INFINITY;
         lb[u] = live ? __ldcg(&w.part_ml[(pp * G + h) * 2 + 1]) : 0.f;
         ob[u] = live ? __ldcg(&w.part_o[(pp * G + h) * D + d]) : 0.f;
       }
       float mx = M;
 #pragma unroll
-      for (int u = 0; u < B; ++u) mx = fmaxf(mx, mb[u]);
+      for (int u = 0; u < kChunk; ++u) mx = fmaxf(mx, mb[u]);
       if (mx == -INFINITY) continue;
-      const float a = M == -INFINITY ? 0.f : exp2f(M - mx);
+      const float a = fast_exp2(M - mx);   // 0 while M is -inf
       L *= a;
       O *= a;
 #pragma unroll
-      for (int u = 0; u < B; ++u) {
-        if (mb[u] == -INFINITY) continue;
-        const float bb = exp2f(mb[u] - mx);
+      for (int u = 0; u < kChunk; ++u) {
+        const float bb = fast_exp2(mb[u] - mx);   // 0 for empty partials
         L += lb[u] * bb;
         O += ob[u] * bb;
       }
@@ -937,14 +859,15 @@ fdms_status launch_split_t(fdms_cache* cache, const DecodeWork& w, OutArgs oa, i
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  const int n_ranges = cache->decode_ctas * T::NCW;
   cudaError_t e = cudaLaunchKernelEx(&cfg, k_decode_split<T>, cache->view, w, oa, layer, batch,
-                                     static_cast<const uint16_t*>(q),
-                                     cache->decode_ctas * T::NCW);
+                                     static_cast<const uint16_t*>(q), n_ranges,
+                                     1.0 / (double)n_ranges);
   if (e != cudaSuccess) return FDMS_ERR_CUDA;
   cfg.gridDim = dim3((unsigned)nh);
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = 0;
-  e = cudaLaunchKernelEx(&cfg, k_decode_combine<T::D, T::G, T::NCW>, w, cache->view.Hkv, cache->view.Hq,
+  e = cudaLaunchKernelEx(&cfg, k_decode_combine<T::D, T::G>, w, cache->view.Hkv, cache->view.Hq,
                          batch, oa);
   return e == cudaSuccess ? FDMS_OK : FDMS_ERR_CUDA;
 }
@@ -1000,7 +923,7 @@ fdms_status fdms_decode_setup(fdms_cache* cache) {
   const CacheView& c = cache->view;
   DecodeWork& w = cache->work;
   w.max_ctas = ctas;
-  w.max_parts = ctas + c.Bmax * c.Hkv;   // CTA c's partial of head h sits at c + h
+  w.max_parts = ctas * cache->ranges_per_cta + c.Bmax * c.Hkv;   // warp v, head h: v + h
   void* p = nullptr;
   auto take = [&](size_t bytes) -> void* {
     if (cudaMalloc(&p, bytes) != cudaSuccess) return nullptr;
@@ -1011,8 +934,8 @@ fdms_status fdms_decode_setup(fdms_cache* cache) {
   w.part_o = static_cast<float*>(take((size_t)w.max_parts * c.G * c.D * sizeof(float)));
   w.part_ml = static_cast<float*>(take((size_t)w.max_parts * c.G * 2 * sizeof(float)));
   w.head_off = static_cast<long long*>(take((size_t)(c.Bmax * c.Hkv + 1) * sizeof(long long)));
-  w.n_eff = static_cast<int*>(take(sizeof(int)));
-  if (!w.part_o || !w.part_ml || !w.head_off || !w.n_eff) return FDMS_ERR_CUDA;
+  w.span = static_cast<long long*>(take(sizeof(long long)));
+  if (!w.part_o || !w.part_ml || !w.head_off || !w.span) return FDMS_ERR_CUDA;
   return FDMS_OK;
 }
 
@@ -1065,7 +988,8 @@ extern "C" fdms_status fdms_decode_attn_noalloc(fdms_cache* cache, int layer, in
   if (cache->device < 0 || cache->device >= kMaxDevices) return FDMS_ERR_UNSUPPORTED;
   // layout of the scratch for this call: the plan (head prefix, ranges used),
   // partials (o), partials (m, l); everything is written before it is read
-  const long long parts = (long long)cache->decode_ctas + (long long)batch * c.Hkv;
+  const long long parts = (long long)cache->decode_ctas * cache->ranges_per_cta +
+                          (long long)batch * c.Hkv;
   const size_t plan_bytes = align256((size_t)(batch * c.Hkv + 1) * sizeof(long long) + 16);
   const size_t o_bytes = align256((size_t)parts * c.G * c.D * sizeof(float));
   const size_t ml_bytes = align256((size_t)parts * c.G * 2 * sizeof(float));
@@ -1084,7 +1008,7 @@ extern "C" fdms_status fdms_decode_attn_noalloc(fdms_cache* cache, int layer, in
     unsigned char* b = static_cast<unsigned char*>(base);
     DecodeWork w;
     w.head_off = reinterpret_cast<long long*>(b);
-    w.n_eff = reinterpret_cast<int*>(b + plan_bytes - 16);
+    w.span = reinterpret_cast<long long*>(b + plan_bytes - 16);
     w.part_o = reinterpret_cast<float*>(b + plan_bytes);
     w.part_ml = reinterpret_cast<float*>(b + plan_bytes + o_bytes);
     w.max_parts = (int)parts;

@@ -92,7 +92,7 @@ struct DecodeWork {
   float* part_o;          // [max_parts][G][D], unnormalised sum of p * v
   float* part_ml;         // [max_parts][G][2]: running max (log2 domain) and sum
   long long* head_off;    // [heads + 1]: prefix of units over the call's heads
-  int* n_eff;             // unit ranges actually used
+  long long* span;        // units per warp range of the last split
   int max_parts;
   int max_ctas;
 };
