@@ -273,83 +273,19 @@ k_append_evict(CacheView c, int layer, const int32_t* __restrict__ n_new, int ma
 }
 
 
-// Decode-step path: one warp per (seq, kv head), for calls that bring at most
-// kSmallMax tokens per sequence. Same semantics as k_append_evict; the loads
-// whose addresses are known are issued together, so a decode step costs about
-// two dependent memory round trips.
 constexpr int kSmallMax = 16;
 constexpr int kSmallWarps = 8;
 
+// Resolution, ring writes and length update of one (seq, kv head) for the
+// warp-per-head paths: positions r0 .. r1-1 are resolved (survivors appended to
+// the store in order), positions max(r1, n0) .. n1-1 go to the ring.
 template <bool FP8>
-__global__ void __launch_bounds__(kSmallWarps * 32)
-k_append_small(CacheView c, int layer, int batch, const int32_t* __restrict__ n_new, int max_new,
-               const uint16_t* __restrict__ k_in, const uint16_t* __restrict__ v_in,
-               const uint8_t* __restrict__ keep_in, const float* __restrict__ kv_scale) {
-  pdl_wait();                 // the previous kernel's writes are visible from here on
-  pdl_launch_dependents();
-  const int lane = threadIdx.x & 31;
-  const int hid = blockIdx.x * kSmallWarps + (threadIdx.x >> 5);
-  if (hid >= batch * c.Hkv) return;
-  const int b = hid / c.Hkv, h = hid % c.Hkv;
-  const long long hi = head_index(c, layer, b, h);
-  const long long in_stride = (long long)c.Hkv * c.D;   // elements between tokens
-  const uint16_t* k_rows = k_in + ((long long)b * max_new * c.Hkv + h) * c.D;
-  const uint16_t* v_rows = v_in + ((long long)b * max_new * c.Hkv + h) * c.D;
-  const uint8_t* keep_rows = keep_in + (long long)b * max_new * c.Hkv + h;
+__device__ void warp_resolve(const CacheView& c, long long hi, int lane, int n0, int r0,
+                             int len0, int n1, int r1, float sk, float sv,
+                             const uint16_t* k_rows, const uint16_t* v_rows,
+                             const uint8_t* keep_rows, long long in_stride) {
   uint8_t* rkeep = c.ring_keep + hi * c.Rpad;
   const int VPR = c.D / 8;    // 16-byte input vectors per row
-
-  const int m = n_new[b];
-  const int n0 = c.tok_n[hi], r0 = c.tok_r[hi], len0 = c.store_len[hi];
-  if (m < 0 || m > max_new) {
-    if (lane == 0) latch_error(c.ctr, FDMS_ERR_DEVICE);
-    return;
-  }
-  if (m == 0) return;
-  if ((long long)n0 + m > c.max_seq_len) {
-    if (lane == 0) latch_error(c.ctr, FDMS_ERR_DEVICE);
-    return;
-  }
-  const int n1 = n0 + m;
-  const int r1 = (n1 - c.W - r0 >= c.P) ? n1 - c.W : r0;
-
-  float sk = 1.0f, sv = 1.0f;
-  if constexpr (FP8) {
-    if (n0 == 0) {
-      if (kv_scale) {
-        sk = kv_scale[((long long)b * c.Hkv + h) * 2];
-        sv = kv_scale[((long long)b * c.Hkv + h) * 2 + 1];
-      } else {
-        float ak = 0.f, av = 0.f;
-        for (int i = lane; i < m * VPR; i += 32) {
-          const long long row = i / VPR;
-          const int vec = i % VPR;
-          const uint4 xk = *reinterpret_cast<const uint4*>(k_rows + row * in_stride + vec * 8);
-          const uint4 xv = *reinterpret_cast<const uint4*>(v_rows + row * in_stride + vec * 8);
-          const uint32_t wk[4] = {xk.x, xk.y, xk.z, xk.w}, wv[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            ak = fmaxf(ak, fmaxf(fabsf(bf16lo_to_f32(wk[j])), fabsf(bf16hi_to_f32(wk[j]))));
-            av = fmaxf(av, fmaxf(fabsf(bf16lo_to_f32(wv[j])), fabsf(bf16hi_to_f32(wv[j]))));
-          }
-        }
-        for (int off = 16; off > 0; off >>= 1) {
-          ak = fmaxf(ak, __shfl_xor_sync(0xffffffffu, ak, off));
-          av = fmaxf(av, __shfl_xor_sync(0xffffffffu, av, off));
-        }
-        sk = __fdiv_rn(fmaxf(ak, 1.17549435e-38f), 448.0f);
-        sv = __fdiv_rn(fmaxf(av, 1.17549435e-38f), 448.0f);
-      }
-      if (lane == 0) {
-        c.head_scale[hi * 2] = sk;
-        c.head_scale[hi * 2 + 1] = sv;
-      }
-    } else {
-      sk = c.head_scale[hi * 2];
-      sv = c.head_scale[hi * 2 + 1];
-    }
-  }
-
   auto keep_of = [&](int p) -> int {
     return p < n0 ? (rkeep[p % c.R] != 0) : (keep_rows[(long long)(p - n0) * c.Hkv] != 0);
   };
@@ -441,6 +377,298 @@ k_append_small(CacheView c, int layer, int batch, const int32_t* __restrict__ n_
   }
 }
 
+// Decode-step path: one warp per (seq, kv head), for calls that bring at most
+// kSmallMax tokens per sequence. Same semantics as k_append_evict; the loads
+// whose addresses are known are issued together, so a decode step costs about
+// two dependent memory round trips.
+
+template <bool FP8>
+__global__ void __launch_bounds__(kSmallWarps * 32)
+k_append_small(CacheView c, int layer, int batch, const int32_t* __restrict__ n_new, int max_new,
+               const uint16_t* __restrict__ k_in, const uint16_t* __restrict__ v_in,
+               const uint8_t* __restrict__ keep_in, const float* __restrict__ kv_scale) {
+  pdl_wait();                 // the previous kernel's writes are visible from here on
+  pdl_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int hid = blockIdx.x * kSmallWarps + (threadIdx.x >> 5);
+  if (hid >= batch * c.Hkv) return;
+  const int b = hid / c.Hkv, h = hid % c.Hkv;
+  const long long hi = head_index(c, layer, b, h);
+  const long long in_stride = (long long)c.Hkv * c.D;   // elements between tokens
+  const uint16_t* k_rows = k_in + ((long long)b * max_new * c.Hkv + h) * c.D;
+  const uint16_t* v_rows = v_in + ((long long)b * max_new * c.Hkv + h) * c.D;
+  const uint8_t* keep_rows = keep_in + (long long)b * max_new * c.Hkv + h;
+  const int VPR = c.D / 8;    // 16-byte input vectors per row
+
+  const int m = n_new[b];
+  const int n0 = c.tok_n[hi], r0 = c.tok_r[hi], len0 = c.store_len[hi];
+  if (m < 0 || m > max_new) {
+    if (lane == 0) latch_error(c.ctr, FDMS_ERR_DEVICE);
+    return;
+  }
+  if (m == 0) return;
+  if ((long long)n0 + m > c.max_seq_len) {
+    if (lane == 0) latch_error(c.ctr, FDMS_ERR_DEVICE);
+    return;
+  }
+  const int n1 = n0 + m;
+  const int r1 = (n1 - c.W - r0 >= c.P) ? n1 - c.W : r0;
+
+  float sk = 1.0f, sv = 1.0f;
+  if constexpr (FP8) {
+    if (n0 == 0) {
+      if (kv_scale) {
+        sk = kv_scale[((long long)b * c.Hkv + h) * 2];
+        sv = kv_scale[((long long)b * c.Hkv + h) * 2 + 1];
+      } else {
+        float ak = 0.f, av = 0.f;
+        for (int i = lane; i < m * VPR; i += 32) {
+          const long long row = i / VPR;
+          const int vec = i % VPR;
+          const uint4 xk = *reinterpret_cast<const uint4*>(k_rows + row * in_stride + vec * 8);
+          const uint4 xv = *reinterpret_cast<const uint4*>(v_rows + row * in_stride + vec * 8);
+          const uint32_t wk[4] = {xk.x, xk.y, xk.z, xk.w}, wv[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            ak = fmaxf(ak, fmaxf(fabsf(bf16lo_to_f32(wk[j])), fabsf(bf16hi_to_f32(wk[j]))));
+            av = fmaxf(av, fmaxf(fabsf(bf16lo_to_f32(wv[j])), fabsf(bf16hi_to_f32(wv[j]))));
+          }
+        }
+        for (int off = 16; off > 0; off >>= 1) {
+          ak = fmaxf(ak, __shfl_xor_sync(0xffffffffu, ak, off));
+          av = fmaxf(av, __shfl_xor_sync(0xffffffffu, av, off));
+        }
+        sk = __fdiv_rn(fmaxf(ak, 1.17549435e-38f), 448.0f);
+        sv = __fdiv_rn(fmaxf(av, 1.17549435e-38f), 448.0f);
+      }
+      if (lane == 0) {
+        c.head_scale[hi * 2] = sk;
+        c.head_scale[hi * 2 + 1] = sv;
+      }
+    } else {
+      sk = c.head_scale[hi * 2];
+      sv = c.head_scale[hi * 2 + 1];
+    }
+  }
+
+  warp_resolve<FP8>(c, hi, lane, n0, r0, len0, n1, r1, sk, sv, k_rows, v_rows, keep_rows,
+                    in_stride);
+}
+
+// Decode steps proper: at most kStepVecs 16-byte input vectors per sequence
+// (max_new * D / 8 <= 32), one warp per (seq, kv head). Same result as
+// k_append_small; ordered for latency: the head's state, the call's rows and
+// keep bits and the head's FP8 scales are loaded together (they do not depend
+// on each other), then the keep bits and ring rows of the positions resolved
+// now and the store's partly filled block, again together; every write comes
+// after. A step costs two round trips to memory (three when the store needs a
+// new block) where the general order takes five. Resolutions larger than two
+// vectors per lane take the general path.
+constexpr int kStepVecs = 32;
+
+template <bool FP8>
+__global__ void __launch_bounds__(kSmallWarps * 32)
+k_append_step(CacheView c, int layer, int batch, const int32_t* __restrict__ n_new, int max_new,
+              const uint16_t* __restrict__ k_in, const uint16_t* __restrict__ v_in,
+              const uint8_t* __restrict__ keep_in, const float* __restrict__ kv_scale) {
+  pdl_wait();                 // the previous kernel's writes are visible from here on
+  pdl_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int hid = blockIdx.x * kSmallWarps + (threadIdx.x >> 5);
+  if (hid >= batch * c.Hkv) return;
+  const int b = hid / c.Hkv, h = hid % c.Hkv;
+  const long long hi = head_index(c, layer, b, h);
+  const long long in_stride = (long long)c.Hkv * c.D;   // elements between tokens
+  const uint16_t* k_rows = k_in + ((long long)b * max_new * c.Hkv + h) * c.D;
+  const uint16_t* v_rows = v_in + ((long long)b * max_new * c.Hkv + h) * c.D;
+  const uint8_t* keep_rows = keep_in + (long long)b * max_new * c.Hkv + h;
+  uint8_t* rkeep = c.ring_keep + hi * c.Rpad;
+  const int VPR = c.D / 8;    // 16-byte input vectors per row
+  constexpr unsigned kAll = 0xffffffffu;
+
+  // ---- round trip 1: state, the call's rows (vector `lane`), keep bits, scales
+  const int m = n_new[b];
+  const int n0 = c.tok_n[hi], r0 = c.tok_r[hi], len0 = c.store_len[hi];
+  uint4 xk = make_uint4(0u, 0u, 0u, 0u), xv = xk;
+  if (lane < max_new * VPR) {
+    const int t = lane / VPR, vec = lane % VPR;
+    xk = *reinterpret_cast<const uint4*>(k_rows + t * in_stride + vec * 8);
+    xv = *reinterpret_cast<const uint4*>(v_rows + t * in_stride + vec * 8);
+  }
+  const int knew = lane < max_new ? (keep_rows[(long long)lane * c.Hkv] != 0) : 0;
+  float sk = 1.0f, sv = 1.0f;
+  if constexpr (FP8) {
+    sk = c.head_scale[hi * 2];
+    sv = c.head_scale[hi * 2 + 1];
+  }
+  if (m < 0 || m > max_new || (long long)n0 + m > c.max_seq_len) {
+    if (lane == 0) latch_error(c.ctr, FDMS_ERR_DEVICE);
+    return;
+  }
+  if (m == 0) return;
+  const int n1 = n0 + m;
+  const int r1 = (n1 - c.W - r0 >= c.P) ? n1 - c.W : r0;
+  if constexpr (FP8) {
+    if (n0 == 0) {   // a sequence's first append fixes its scales
+      if (kv_scale) {
+        sk = kv_scale[((long long)b * c.Hkv + h) * 2];
+        sv = kv_scale[((long long)b * c.Hkv + h) * 2 + 1];
+      } else {
+        float ak = 0.f, av = 0.f;
+        if (lane < m * VPR) {
+          const uint32_t wk[4] = {xk.x, xk.y, xk.z, xk.w}, wv[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            ak = fmaxf(ak, fmaxf(fabsf(bf16lo_to_f32(wk[j])), fabsf(bf16hi_to_f32(wk[j]))));
+            av = fmaxf(av, fmaxf(fabsf(bf16lo_to_f32(wv[j])), fabsf(bf16hi_to_f32(wv[j]))));
+          }
+        }
+        for (int off = 16; off > 0; off >>= 1) {
+          ak = fmaxf(ak, __shfl_xor_sync(kAll, ak, off));
+          av = fmaxf(av, __shfl_xor_sync(kAll, av, off));
+        }
+        sk = __fdiv_rn(fmaxf(ak, 1.17549435e-38f), 448.0f);
+        sv = __fdiv_rn(fmaxf(av, 1.17549435e-38f), 448.0f);
+      }
+      if (lane == 0) {
+        c.head_scale[hi * 2] = sk;
+        c.head_scale[hi * 2 + 1] = sv;
+      }
+    }
+  }
+  const int nres = r1 - r0;
+  if (nres > 32 || nres * VPR > 2 * 32) {
+    warp_resolve<FP8>(c, hi, lane, n0, r0, len0, n1, r1, sk, sv, k_rows, v_rows, keep_rows,
+                      in_stride);
+    return;
+  }
+
+  // ---- round trip 2: keep bits and ring rows of positions r0 .. r1-1, the
+  // store's partly filled block
+  const int p_l = r0 + lane;
+  const int knew_p = __shfl_sync(kAll, knew, (p_l - n0) & 31);
+  int kp = 0;
+  if (lane < nres) kp = p_l < n0 ? (rkeep[p_l % c.R] != 0) : knew_p;
+  constexpr int EV = FP8 ? 8 : 16;   // bytes of one vector in the cache
+  uint4 rk[2], rv[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    rk[j] = rv[j] = make_uint4(0u, 0u, 0u, 0u);
+    const int i = lane + 32 * j;
+    if (i < nres * VPR) {
+      const int p = r0 + i / VPR, vec = i % VPR;
+      if (p < n0) {
+        const int slot = p % c.R;
+        const uint8_t* ks = ring_k(c, hi) + (long long)slot * c.RB;
+        const uint8_t* vs = ring_v(c, hi) + (long long)slot * c.RB;
+        if constexpr (FP8) {
+          const uint2 a = *reinterpret_cast<const uint2*>(ks + swz_byte(c.RB, false, slot, vec * EV));
+          const uint2 bb = *reinterpret_cast<const uint2*>(vs + swz_byte(c.RB, true, slot, vec * EV));
+          rk[j] = make_uint4(a.x, a.y, 0u, 0u);
+          rv[j] = make_uint4(bb.x, bb.y, 0u, 0u);
+        } else {
+          rk[j] = *reinterpret_cast<const uint4*>(ks + swz_byte(c.RB, false, slot, vec * EV));
+          rv[j] = *reinterpret_cast<const uint4*>(vs + swz_byte(c.RB, true, slot, vec * EV));
+        }
+      }
+    }
+  }
+  int32_t* bt = c.block_table + hi * c.max_blocks;
+  const long long tail_blk = (len0 % kBlockSlots) ? bt[(len0 - 1) / kBlockSlots] : 0;
+  const unsigned ball = __ballot_sync(kAll, kp != 0);
+  const int len1 = len0 + __popc(ball);
+  const int nb0 = (len0 + kBlockSlots - 1) / kBlockSlots;
+  const int nb1 = (len1 + kBlockSlots - 1) / kBlockSlots;
+  long long base_blk = 0;
+  if (nb1 > nb0) {   // new store blocks for this call (one atomic bump)
+    int fail = 0;
+    if (lane == 0) {
+      const unsigned long long need = (unsigned long long)(nb1 - nb0);
+      const unsigned long long base = atomicAdd(&c.ctr->blocks_next, need);
+      if (base + need > (unsigned long long)c.num_blocks) {
+        latch_error(c.ctr, FDMS_ERR_OUT_OF_BLOCKS);
+        fail = 1;
+      } else {
+        base_blk = (long long)base;
+      }
+    }
+    if (__shfl_sync(kAll, fail, 0)) return;
+    base_blk = __shfl_sync(kAll, base_blk, 0);
+    float* bts = c.bt_scale + hi * c.max_blocks * 2;
+    for (int j = nb0 + lane; j < nb1; j += 32) {
+      bt[j] = (int32_t)(base_blk + (j - nb0));
+      bts[2 * j] = sk;
+      bts[2 * j + 1] = sv;
+    }
+  }
+
+  // ---- writes: survivors to the store, in position order
+  unsigned sat = 0;
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int i = lane + 32 * j;
+    if (i >= nres * VPR) continue;
+    const int ri = i / VPR, vec = i % VPR;
+    if (!((ball >> ri) & 1u)) continue;
+    const int d = len0 + __popc(ball & ((1u << ri) - 1u));
+    const int jb = d / kBlockSlots, row = d % kBlockSlots;
+    const long long blk = jb < nb0 ? tail_blk : base_blk + (jb - nb0);
+    uint8_t* kd = block_k(c, blk) + (long long)row * c.RB;
+    uint8_t* vd = block_v(c, blk) + (long long)row * c.RB;
+    const int p = r0 + ri;
+    if (p < n0) {
+      if constexpr (FP8) {
+        *reinterpret_cast<uint2*>(kd + swz_byte(c.RB, false, row, vec * EV)) =
+            make_uint2(rk[j].x, rk[j].y);
+        *reinterpret_cast<uint2*>(vd + swz_byte(c.RB, true, row, vec * EV)) =
+            make_uint2(rv[j].x, rv[j].y);
+      } else {
+        *reinterpret_cast<uint4*>(kd + swz_byte(c.RB, false, row, vec * EV)) = rk[j];
+        *reinterpret_cast<uint4*>(vd + swz_byte(c.RB, true, row, vec * EV)) = rv[j];
+      }
+    } else {   // a token of this call resolved at once (window shorter than the call)
+      const long long t = p - n0;
+      put_input_vec<FP8>(kd, k_rows + t * in_stride, vec, sk, sat, c.RB, false, row);
+      put_input_vec<FP8>(vd, v_rows + t * in_stride, vec, sv, sat, c.RB, true, row);
+    }
+    if (vec == 0) c.blk_pos[blk * kBlockSlots + row] = p;
+  }
+
+  // ---- the call's unresolved tokens to the ring; a new token can take the
+  // ring slot of a position resolved above, whose row was read in round trip 2
+  __syncwarp();
+  const int w0 = r1 > n0 ? r1 : n0;
+  {
+    const int t = lane / VPR, vec = lane % VPR, p = n0 + t;
+    const int keep_t = __shfl_sync(kAll, knew, t & 31);
+    if (lane < m * VPR && p >= w0) {
+      const int slot = p % c.R;
+      uint8_t* kd = ring_k(c, hi) + (long long)slot * c.RB;
+      uint8_t* vd = ring_v(c, hi) + (long long)slot * c.RB;
+      if constexpr (FP8) {
+        *reinterpret_cast<uint2*>(kd + swz_byte(c.RB, false, slot, vec * EV)) =
+            quantise8(xk, sk, sat);
+        *reinterpret_cast<uint2*>(vd + swz_byte(c.RB, true, slot, vec * EV)) =
+            quantise8(xv, sv, sat);
+      } else {
+        *reinterpret_cast<uint4*>(kd + swz_byte(c.RB, false, slot, vec * EV)) = xk;
+        *reinterpret_cast<uint4*>(vd + swz_byte(c.RB, true, slot, vec * EV)) = xv;
+      }
+      if (vec == 0) rkeep[slot] = keep_t ? 1 : 0;
+    }
+  }
+  if constexpr (FP8) {
+    for (int off = 16; off > 0; off >>= 1) sat += __shfl_xor_sync(kAll, sat, off);
+    if (lane == 0 && sat) atomicAdd(&c.ctr->saturations, (unsigned long long)sat);
+  }
+  __syncwarp();
+  if (lane == 0) {
+    c.store_len[hi] = len1;
+    c.tok_n[hi] = n1;
+    c.tok_r[hi] = r1;
+  }
+}
+
 }  // namespace
 }  // namespace fdms
 
@@ -461,7 +689,14 @@ fdms_status fdms_launch_append(fdms_cache* cache, int layer, int batch, const in
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e;
-  if (max_new <= kSmallMax) {
+  if (max_new * (c.D / 8) <= kStepVecs) {
+    cfg.gridDim = dim3((unsigned)((batch * c.Hkv + kSmallWarps - 1) / kSmallWarps));
+    cfg.blockDim = dim3(kSmallWarps * 32);
+    e = c.fp8 ? cudaLaunchKernelEx(&cfg, k_append_step<true>, c, layer, batch, n_new, max_new,
+                                   kk, vv, keep, sc)
+              : cudaLaunchKernelEx(&cfg, k_append_step<false>, c, layer, batch, n_new, max_new,
+                                   kk, vv, keep, sc);
+  } else if (max_new <= kSmallMax) {
     cfg.gridDim = dim3((unsigned)((batch * c.Hkv + kSmallWarps - 1) / kSmallWarps));
     cfg.blockDim = dim3(kSmallWarps * 32);
     e = c.fp8 ? cudaLaunchKernelEx(&cfg, k_append_small<true>, c, layer, batch, n_new, max_new,

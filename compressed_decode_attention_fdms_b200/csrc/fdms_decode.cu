@@ -8,11 +8,12 @@
 // S_h = the head's compact store plus its visible ring slots.
 //
 // The kernel is memory bound: every byte of a visible K and V row is read once.
-//   - Work is balanced over the GPU by slots, not by heads. The slot lists of
-//     all heads of the call are laid end to end (units = store slots + ring
-//     slots) and cut into equal ranges, one per warp of the grid; a
-//     warp therefore reads the same number of bytes whatever the mix of head
-//     lengths, and emits one partial (m, l, o) per head its range touches.
+//   - Work is balanced over the GPU by tiles, not by heads. The tiles of all
+//     heads of the call (a tile = up to 32 rows of one 64-slot page for
+//     128-byte rows: the head's store pages, then its ring slots) are laid end
+//     to end and cut into equal ranges, one per warp of the grid; a warp does
+//     the same number of tile steps whatever the mix of head lengths, and
+//     emits one partial (m, l, o) per head its range touches.
 //   - Each warp stages its own tiles (32 rows of a 64-slot page for 128-byte
 //     rows): the K rows, V rows and the head's q go to shared memory by 1-D
 //     bulk copies (cp.async.bulk, completion on an mbarrier) into one of the
@@ -49,7 +50,6 @@
 namespace fdms {
 namespace {
 
-constexpr int kMinUnitsPerRange = 64;  // a warp gets at least 64 slots of work
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
 
@@ -300,19 +300,20 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
     __syncthreads();
   }
   const long long total = head_off[NH];
-  // Warp v reads units [v S, (v + 1) S) of the call's units, S = ceil(total /
-  // ranges) (at least kMinUnitsPerRange): an fp64 estimate of the quotient made
-  // exact by integer correction.
-  long long S;
+  const int P = page_off[NH];   // tiles of the call
+  // Warp v reads tiles [v S, (v + 1) S), S = ceil(P / ranges): a tile costs
+  // the same compute full or not, so whole tiles are what gets balanced. The
+  // quotient is an fp64 estimate made exact by integer correction.
+  int S;
   {
-    long long qq = (long long)((double)total * inv_ranges);
-    while (qq * n_ranges > total) --qq;
-    while ((qq + 1) * n_ranges <= total) ++qq;
-    S = qq + (qq * n_ranges < total ? 1 : 0);
-    S = S > kMinUnitsPerRange ? S : kMinUnitsPerRange;
+    long long qq = (long long)((double)P * inv_ranges);
+    while (qq * n_ranges > P) --qq;
+    while ((qq + 1) * n_ranges <= P) ++qq;
+    S = (int)qq + (qq * n_ranges < P ? 1 : 0);
+    S = S > 1 ? S : 1;
   }
   if (blockIdx.x == 0) {   // the plan the combine kernel reads back
-    for (int h = tid; h <= NH; h += T::NT) w.head_off[h] = head_off[h];
+    for (int h = tid; h <= NH; h += T::NT) w.head_off[h] = page_off[h];
     if (tid == 0) {
       *w.span = S;
       c.ctr->slots_decoded += (unsigned long long)total;   // one thread, launches are ordered
@@ -321,7 +322,7 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   }
   // heads without a single slot get zeros (nobody else writes them)
   for (int h = blockIdx.x; h < NH; h += gridDim.x) {
-    if (head_off[h + 1] != head_off[h]) continue;
+    if (page_off[h + 1] != page_off[h]) continue;
     const int b = h / c.Hkv, kh = h % c.Hkv;
     for (int i = tid; i < G * D; i += T::NT) {
       const long long oi = ((long long)b * c.Hq + (long long)kh * G) * D + i;
@@ -331,33 +332,20 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
     }
   }
   const long long v_range = (long long)blockIdx.x * NCW + warp;
-  if ((long long)blockIdx.x * NCW * S >= total) return;
+  if ((long long)blockIdx.x * NCW * S >= P) return;
 
-  // ---- this warp's unit range [gs, ge), the heads h_gs .. h_ge it touches,
-  // its pages [gp0, gp0 + nt)
-  const long long gs = min(v_range * S, total), ge = min(gs + S, total);
-  int h_gs = 0, h_ge = 0, gp0 = 0, nt = 0;
-  if (gs < ge) {
-    // head of unit x: the number of heads h >= 1 with head_off[h] <= x
-    int c0 = 0, c1 = 0;
+  // ---- this warp's tiles [gp0, gp0 + nt) and the heads h_gs .. h_ge they
+  // belong to (the number of heads h >= 1 with page_off[h] <= page)
+  const int gp0 = (int)min(v_range * S, (long long)P);
+  const int nt = min(gp0 + S, P) - gp0;
+  int h_gs = 0, h_ge = 0;
+  if (nt > 0) {
     for (int base = 1; base < NH; base += 32) {
       const int h = base + lane;
-      const long long ho = h < NH ? head_off[h] : total;
-      c0 += __popc(__ballot_sync(0xffffffffu, ho <= gs));
-      c1 += __popc(__ballot_sync(0xffffffffu, ho <= ge - 1));
+      const int po = h < NH ? page_off[h] : P;
+      h_gs += __popc(__ballot_sync(0xffffffffu, po <= gp0));
+      h_ge += __popc(__ballot_sync(0xffffffffu, po <= gp0 + nt - 1));
     }
-    h_gs = c0;
-    h_ge = c1;
-    // page (in the call's page numbering) holding unit x of head h
-    auto gpage = [&](int h, long long x) -> int {
-      const long long u = x - head_off[h];
-      const int len = s_len[h];
-      const int lp = u < len ? (int)(u / TR)
-                             : (len + TR - 1) / TR + (int)((u - len + s_r[h] % TR) / TR);
-      return page_off[h] + lp;
-    };
-    gp0 = gpage(h_gs, gs);
-    nt = gpage(h_ge, ge - 1) - gp0 + 1;
   }
 
   // descriptor of this warp's tile k (one lane per tile)
@@ -374,9 +362,6 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
     const int lp = gp - page_off[hidx];
     const int len = s_len[hidx], n = s_n[hidx], r = s_r[hidx];
     const int sp = (len + TR - 1) / TR;
-    const long long hoff = head_off[hidx];
-    const long long lo = gs > hoff ? gs - hoff : 0;   // head units of this range
-    const long long hi_u = ge - hoff;
     const long long hi = hi0 + hidx;
     int flags = (k == 0 || lp == 0 ? kFirst : 0) |
                 (k == nt - 1 || gp + 1 == page_off[hidx + 1] ? kLast : 0);
@@ -385,12 +370,10 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
     mt.p0 = 0;
     mt.pad = 0;
     if (lp < sp) {   // store tile lp: block lp * TR / 64, rows from (lp * TR) % 64
-      const long long u0 = max((long long)lp * TR, lo);
-      const long long u1 = min((long long)min((lp + 1) * TR, len), hi_u);
       const int j = lp * TR / kBlockSlots;
       const int rb = (lp * TR) % kBlockSlots;          // block row of frame row 0
-      row0 = (int)(u0 - (long long)lp * TR);
-      row1 = (int)(u1 - (long long)lp * TR);
+      row0 = 0;
+      row1 = min(TR, len - lp * TR);
       const long long blk = c.block_table[hi * c.max_blocks + j];
       if (FP8) {
         mt.ks = c.bt_scale[(hi * c.max_blocks + j) * 2];
@@ -398,15 +381,14 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
       } else {
         mt.ks = mt.vrel = 1.0f;
       }
-      mt.ksrc = block_k(c, blk) + (long long)(rb + row0) * RB;
+      mt.ksrc = block_k(c, blk) + (long long)rb * RB;
     } else {         // ring tile: live units [TR*rp - off, TR*(rp+1) - off)
       const int rp = lp - sp, off = r % TR, live = n - r;
-      const long long a = max((long long)len + max(TR * rp - off, 0), lo);
-      const long long b = min((long long)len + min(TR * (rp + 1) - off, live), hi_u);
-      const int p0 = r + (int)(a - len);
+      const int a = max(TR * rp - off, 0), b = min(TR * (rp + 1) - off, live);
+      const int p0 = r + a;
       const int slot0 = p0 % c.R;
       row0 = slot0 % TR;
-      row1 = row0 + (int)(b - a);
+      row1 = row0 + (b - a);
       mt.p0 = p0;
       flags |= kRing | (p0 < n - c.W ? kPending : 0);
       mt.ks = s_hscale[2 * hidx];
@@ -737,9 +719,8 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
       l += __shfl_xor_sync(0xffffffffu, l, 1);
       l += __shfl_xor_sync(0xffffffffu, l, 2);
       const int hidx = mt.hidx;
-      const long long hs = head_off[hidx], he = head_off[hidx + 1];
       const int kb = hidx / c.Hkv, kh = hidx % c.Hkv;
-      if (hs >= gs && he <= ge) {
+      if (page_off[hidx] >= gp0 && page_off[hidx + 1] <= gp0 + nt) {
         // the whole head lies in this warp's range: write the output now
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
@@ -791,57 +772,87 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
 
 // Merge of the warp partials of one (seq, kv head) that several warps covered:
 // o = sum_w 2^(m_w - M) o_w / sum_w 2^(m_w - M) l_w. Heads inside one warp's
-// range, or with no slot, were written by the split kernel. A thread merges one
-// output element; the (m, l, o) of up to kChunk partials are loaded together,
-// then merged, so a head with up to kChunk partials costs one round trip.
+// range, or with no slot, were written by the split kernel. CPH CTAs share a
+// head, TPE adjacent threads one output element: each loads its share of the
+// partials (up to kChunk at once, all loads before any use), merges them, and
+// the TPE results are merged across the threads by shuffles. Up to
+// TPE * kChunk partials per head cost one round trip to memory.
 template <int D, int G>
-__global__ void __launch_bounds__(256)
+struct Combine {
+  static constexpr int NE = G * D;    // output elements of a head
+  static constexpr int TPE = 4;       // threads per element
+  static constexpr int NT = 256;      // threads per CTA
+  static constexpr int EPC = NT / TPE;                 // elements per CTA
+  static constexpr int CPH = NE / EPC;                 // CTAs per head
+  static_assert(NE % EPC == 0, "whole CTAs per head");
+};
+
+// merge (M2, L2, O2) into (M, L, O), both in the log2 domain
+__device__ __forceinline__ void merge_mlo(float& M, float& L, float& O, float M2, float L2,
+                                          float O2) {
+  const float mx = fmaxf(M, M2);
+  if (mx == -INFINITY) return;
+  const float a = fast_exp2(M - mx), b = fast_exp2(M2 - mx);   // 0 for an empty side
+  L = L * a + L2 * b;
+  O = O * a + O2 * b;
+  M = mx;
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(Combine<D, G>::NT)
 k_decode_combine(DecodeWork w, int Hkv, int Hq, int batch, OutArgs oa) {
-  constexpr int kChunk = 16;
+  using C = Combine<D, G>;
+  constexpr int kChunk = 16, TPE = C::TPE;
   pdl_wait();
   pdl_launch_dependents();
-  const int hidx = blockIdx.x, tid = threadIdx.x;
+  const int hidx = blockIdx.x / C::CPH, tid = threadIdx.x, sub = tid % TPE;
+  // the head's tiles and the tiles per warp of the split
   const long long hs = w.head_off[hidx], he = w.head_off[hidx + 1], S = *w.span;
   if (he == hs) return;
   const long long r0 = udiv(hs, S), r1 = udiv(he - 1, S);
   if (r0 == r1) return;
   const int kb = hidx / Hkv, kh = hidx % Hkv;
-  for (int idx = tid; idx < G * D; idx += 256) {
-    const int h = idx / D, d = idx % D;
-    float M = -INFINITY, L = 0.f, O = 0.f;
-    for (long long p0 = r0; p0 <= r1; p0 += kChunk) {
-      float mb[kChunk], lb[kChunk], ob[kChunk];
+  const int idx = (blockIdx.x % C::CPH) * C::EPC + tid / TPE;
+  const int h = idx / D, d = idx % D;
+  float M = -INFINITY, L = 0.f, O = 0.f;
+  for (long long p0 = r0 + sub; p0 <= r1; p0 += (long long)kChunk * TPE) {
+    float mb[kChunk], lb[kChunk], ob[kChunk];
 #pragma unroll
-      for (int u = 0; u < kChunk; ++u) {   // loads first, all independent
-        const long long pp = p0 + u + hidx;
-        const bool live = p0 + u <= r1;
-        mb[u] = live ? __ldcg(&w.part_ml[(pp * G + h) * 2]) : -INFINITY;
-        lb[u] = live ? __ldcg(&w.part_ml[(pp * G + h) * 2 + 1]) : 0.f;
-        ob[u] = live ? __ldcg(&w.part_o[(pp * G + h) * D + d]) : 0.f;
-      }
-      float mx = M;
-#pragma unroll
-      for (int u = 0; u < kChunk; ++u) mx = fmaxf(mx, mb[u]);
-      if (mx == -INFINITY) continue;
-      const float a = fast_exp2(M - mx);   // 0 while M is -inf
-      L *= a;
-      O *= a;
-#pragma unroll
-      for (int u = 0; u < kChunk; ++u) {
-        const float bb = fast_exp2(mb[u] - mx);   // 0 for empty partials
-        L += lb[u] * bb;
-        O += ob[u] * bb;
-      }
-      M = mx;
+    for (int u = 0; u < kChunk; ++u) {   // loads first, all independent
+      const long long pr = p0 + (long long)u * TPE;
+      const long long pp = pr + hidx;
+      const bool live = pr <= r1;
+      mb[u] = live ? __ldcg(&w.part_ml[(pp * G + h) * 2]) : -INFINITY;
+      lb[u] = live ? __ldcg(&w.part_ml[(pp * G + h) * 2 + 1]) : 0.f;
+      ob[u] = live ? __ldcg(&w.part_o[(pp * G + h) * D + d]) : 0.f;
     }
-    const float o = M == -INFINITY ? 0.f : O / L;
-    const long long oi = ((long long)kb * Hq + (long long)kh * G + h) * D + d;
-    if (oa.f32) static_cast<float*>(oa.out)[oi] = o;
-    else static_cast<uint16_t*>(oa.out)[oi] = f32_to_bf16_rn(o);
-    if (oa.lse && d == 0)
-      oa.lse[(long long)kb * Hq + kh * G + h] =
-          M == -INFINITY ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
+    float mx = M;
+#pragma unroll
+    for (int u = 0; u < kChunk; ++u) mx = fmaxf(mx, mb[u]);
+    if (mx == -INFINITY) continue;
+    const float a = fast_exp2(M - mx);   // 0 while M is -inf
+    L *= a;
+    O *= a;
+#pragma unroll
+    for (int u = 0; u < kChunk; ++u) {
+      const float bb = fast_exp2(mb[u] - mx);   // 0 for empty partials
+      L += lb[u] * bb;
+      O += ob[u] * bb;
+    }
+    M = mx;
   }
+#pragma unroll
+  for (int off = 1; off < TPE; off <<= 1)
+    merge_mlo(M, L, O, __shfl_xor_sync(0xffffffffu, M, off),
+              __shfl_xor_sync(0xffffffffu, L, off), __shfl_xor_sync(0xffffffffu, O, off));
+  if (sub != 0) return;
+  const float o = M == -INFINITY ? 0.f : O / L;
+  const long long oi = ((long long)kb * Hq + (long long)kh * G + h) * D + d;
+  if (oa.f32) static_cast<float*>(oa.out)[oi] = o;
+  else static_cast<uint16_t*>(oa.out)[oi] = f32_to_bf16_rn(o);
+  if (oa.lse && d == 0)
+    oa.lse[(long long)kb * Hq + kh * G + h] =
+        M == -INFINITY ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
 }
 
 // ------------------------------------------------------------------ dispatch
@@ -864,8 +875,8 @@ fdms_status launch_split_t(fdms_cache* cache, const DecodeWork& w, OutArgs oa, i
                                      static_cast<const uint16_t*>(q), n_ranges,
                                      1.0 / (double)n_ranges);
   if (e != cudaSuccess) return FDMS_ERR_CUDA;
-  cfg.gridDim = dim3((unsigned)nh);
-  cfg.blockDim = dim3(256);
+  cfg.gridDim = dim3((unsigned)(nh * Combine<T::D, T::G>::CPH));
+  cfg.blockDim = dim3(Combine<T::D, T::G>::NT);
   cfg.dynamicSmemBytes = 0;
   e = cudaLaunchKernelEx(&cfg, k_decode_combine<T::D, T::G>, w, cache->view.Hkv, cache->view.Hq,
                          batch, oa);

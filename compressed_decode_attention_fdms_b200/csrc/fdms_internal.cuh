@@ -91,8 +91,8 @@ __host__ __device__ inline uint8_t* ring_v(const CacheView& c, long long hi) {
 struct DecodeWork {
   float* part_o;          // [max_parts][G][D], unnormalised sum of p * v
   float* part_ml;         // [max_parts][G][2]: running max (log2 domain) and sum
-  long long* head_off;    // [heads + 1]: prefix of units over the call's heads
-  long long* span;        // units per warp range of the last split
+  long long* head_off;    // [heads + 1]: prefix of tiles over the call's heads
+  long long* span;        // tiles per warp range of the last split
   int max_parts;
   int max_ctas;
 };
