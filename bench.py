@@ -72,6 +72,28 @@ def load_peaks():
     return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (no MEASURED_PEAKS.json)"
 
 
+def load_traffic(workload):
+    """DRAM bytes of one decode call from the committed ncu summary, if it was
+    taken on the decode sources as they are now; else None."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "decode_traffic.txt")
+    if not os.path.exists(p):
+        return None, "no capture"
+    src = os.path.join(ROOT, "compressed_decode_attention_fdms_b200", "csrc")
+    now = [hashlib.sha256(open(os.path.join(src, f), "rb").read()).hexdigest()[:16]
+           for f in ("fdms_decode.cu", "fdms_internal.cuh")]
+    for line in open(p):
+        f = line.split()
+        if not f or f[0].startswith("#") or f[0] != workload:
+            continue
+        if f[2:4] == now:
+            return float(f[1]), "ncu dram__bytes_read.sum + dram__bytes_write.sum of " \
+                                "k_decode_split + k_decode_combine, profiles/decode_step_" + \
+                                workload + ".md"
+        return None, "decode kernels changed since the ncu capture"
+    return None, "no capture for this workload"
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -356,6 +378,7 @@ def run_native(args, wl):
             e2e["ms"], e2e["bytes"] = float(tt[0]), float(tt[1])
 
     peak, peak_src = load_peaks()
+    traffic, traffic_src = load_traffic(wl.name)
     achieved = per_launch_bytes / (dec_avg_ms * 1e-3) / 1e9
     result = None
     if rank == 0:
@@ -371,7 +394,7 @@ def run_native(args, wl):
                        "timing": "K steps in one CUDA graph; events around each decode call"},
             "roofline": {
                 "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": None,
+                "frac": achieved / peak, "traffic": traffic, "traffic_source": traffic_src,
                 "kernel": "fdms_decode_attn (k_decode_split + k_decode_combine)",
                 "per_launch_bytes": per_launch_bytes, "launch_us": dec_avg_ms * 1e3,
                 "launch_timing": f"CUDA events around one graph of {K * L} back-to-back "
