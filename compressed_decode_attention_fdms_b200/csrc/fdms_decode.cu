@@ -495,15 +495,27 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
       cur_hidx = mt.hidx;
       if constexpr (FP8) {
         // f16 q scaled by 2^a so that max |q| of the row is in [2^14, 2^15)
-        float amax = 0.f;
+        // (bf16 -> f16 is then exact). The 4 KS dims of lane column t are one
+        // run of the row (the K chunks of the column are adjacent): 16-byte loads.
+        constexpr int NQ = 4 * KS;   // q values of this lane
+        static_assert(RB <= 128 && NQ == T::KCPT * T::EC, "one run of adjacent K chunks");
+        uint32_t qw[NQ / 2];          // bf16 pairs, in k-slot order
         if (g < G) {
+          const uint4* src = reinterpret_cast<const uint4*>(Qs + g * D + NQ * t);
 #pragma unroll
-          for (int s2 = 0; s2 < KS; ++s2)
+          for (int i = 0; i < NQ / 8; ++i) {
+            const uint4 x = src[i];
+            qw[4 * i] = x.x; qw[4 * i + 1] = x.y; qw[4 * i + 2] = x.z; qw[4 * i + 3] = x.w;
+          }
+        } else {
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              amax = fmaxf(amax,
-                           fabsf(__uint_as_float((uint32_t)Qs[g * D + T::kdim(t, s2, e)] << 16)));
+          for (int i = 0; i < NQ / 2; ++i) qw[i] = 0u;
         }
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < NQ / 2; ++i)
+          amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(qw[i] << 16)),
+                                   fabsf(__uint_as_float(qw[i] & 0xFFFF0000u))));
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
         int ex = 0;
@@ -514,13 +526,10 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
         qmul = qscale * down;
 #pragma unroll
         for (int s2 = 0; s2 < KS; ++s2) {
-          float v4[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            v4[e] = g < G ? __uint_as_float((uint32_t)Qs[g * D + T::kdim(t, s2, e)] << 16) * up
-                          : 0.f;
-          qa[s2][0] = pack2<true>(v4[0], v4[1]);
-          qa[s2][1] = pack2<true>(v4[2], v4[3]);
+          qa[s2][0] = pack2<true>(__uint_as_float(qw[2 * s2] << 16) * up,
+                                  __uint_as_float(qw[2 * s2] & 0xFFFF0000u) * up);
+          qa[s2][1] = pack2<true>(__uint_as_float(qw[2 * s2 + 1] << 16) * up,
+                                  __uint_as_float(qw[2 * s2 + 1] & 0xFFFF0000u) * up);
         }
       } else {
         qmul = qscale;
