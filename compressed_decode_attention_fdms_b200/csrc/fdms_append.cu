@@ -1,4 +1,4 @@
-// Append + evict + compact: one CTA per (seq, kv head) of the call.
+// Append + evict + compact.
 //
 // What it applies (FastDMS announcement, aiwitness.kr/community/1t3vlrx, the
 // paragraphs on DMS per-head token eviction and on the compact store that
@@ -8,17 +8,24 @@
 //      r0 .. n1-W-1 are resolved now: in position order, those with keep = 1
 //      are appended to the head's compact store, the rest are dropped;
 //   3. the still-unresolved new tokens are written to the ring (staging).
-// Resolution is a stable stream compaction: each 256-position chunk takes a
-// warp ballot of the keep bits, a popcount prefix inside each warp, and an
-// exclusive scan of the 8 warp totals, so survivors keep their order.
-// Store blocks for all survivors of the call are taken from the pool with one
-// atomic bump before any row is written; if the pool cannot cover them the
-// head is left unchanged and FDMS_ERR_OUT_OF_BLOCKS is latched.
+// Resolution is a stable stream compaction (warp ballot of the keep bits, a
+// popcount prefix inside each warp, a scan of warp totals), so survivors keep
+// their order. Store blocks for all survivors of a head are taken from the pool
+// with one atomic bump before any row is written; if the pool cannot cover them
+// the head is left unchanged and FDMS_ERR_OUT_OF_BLOCKS is latched.
+//
+// Three paths, one result: decode steps (k_append_step: a warp per head, the
+// loads ordered for latency), calls of up to 16 tokens per sequence
+// (k_append_small: a warp per head) and bulk calls such as prefill (four
+// launches spread over many CTAs per head, below).
 //
 // FP8 cache: a sequence's first append fixes each head's K and V scales
 // (max(amax, 2^-126) / 448 of the call's values, or the caller's); every new
-// row is stored as e4m3_rne_satfinite(fp32(x) / scale) with the division in
-// IEEE fp32 and the rounding by the hardware conversion.
+// row is stored as e4m3_rne_satfinite(fp32(x) / scale) with the quotient
+// correctly rounded in IEEE fp32 and the rounding to E4M3 by the hardware
+// conversion.
+#include <algorithm>
+
 #include "fdms_internal.cuh"
 
 namespace fdms {
@@ -38,37 +45,35 @@ __device__ __forceinline__ float block_max(float x, float* red) {
   return m;
 }
 
-// Absolute maximum over m rows of D bf16 values (row stride `stride` elements).
-__device__ float rows_amax(const uint16_t* base, int m, int D, long long stride, float* red) {
-  float a = 0.0f;
-  const int vpr = D / 8;   // 16-byte vectors per row
-  for (long long i = threadIdx.x; i < (long long)m * vpr; i += kAppendThreads) {
-    const long long row = i / vpr;
-    const int vec = (int)(i % vpr);
-    const uint4 x = *reinterpret_cast<const uint4*>(base + row * stride + vec * 8);
-    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      a = fmaxf(a, fabsf(bf16lo_to_f32(w[j])));
-      a = fmaxf(a, fabsf(bf16hi_to_f32(w[j])));
-    }
-  }
-  return block_max(a, red);
+// x / s in IEEE binary32, rounded to nearest even, for finite x and a normal
+// s > 0, given r = RN(1/s): q = RN(x r), then one correction with the exact
+// residual x - q s (one FMA). This is Markstein's division (IBM J. Res. Dev.
+// 34(1), 1990): with r correctly rounded and q within an ulp of x / s, the
+// corrected quotient is the correctly rounded one. Where the quotient
+// overflows, q itself is returned (both saturate when converted); quotients
+// below the normal range convert to an E4M3 zero whatever their rounding.
+__device__ __forceinline__ float div_rn(float x, float s, float r) {
+  const float q = x * r;
+  const float q1 = fmaf(fmaf(-q, s, x), r, q);
+  return isfinite(q1) ? q1 : q;
 }
 
 // 8 bf16 (one 16-byte vector) / scale -> 8 E4M3 codes; counts clipped values.
 __device__ __forceinline__ uint2 quantise8(uint4 x, float scale, unsigned& sat) {
   const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+  const bool tiny = scale < 1.0e-30f;   // 1 / scale might overflow: plain division
+  const float r = tiny ? 0.f : __frcp_rn(scale);
   uint32_t out[2];
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
+    const float x4[4] = {bf16lo_to_f32(w[2 * j]), bf16hi_to_f32(w[2 * j]),
+                         bf16lo_to_f32(w[2 * j + 1]), bf16hi_to_f32(w[2 * j + 1])};
     float f[4];
-    f[0] = __fdiv_rn(bf16lo_to_f32(w[2 * j]), scale);
-    f[1] = __fdiv_rn(bf16hi_to_f32(w[2 * j]), scale);
-    f[2] = __fdiv_rn(bf16lo_to_f32(w[2 * j + 1]), scale);
-    f[3] = __fdiv_rn(bf16hi_to_f32(w[2 * j + 1]), scale);
 #pragma unroll
-    for (int t = 0; t < 4; ++t) sat += fabsf(f[t]) > 448.0f ? 1u : 0u;
+    for (int t = 0; t < 4; ++t) {
+      f[t] = tiny ? __fdiv_rn(x4[t], scale) : div_rn(x4[t], scale, r);
+      sat += fabsf(f[t]) > 448.0f ? 1u : 0u;
+    }
     out[j] = (uint32_t)f32x2_to_e4m3x2(f[0], f[1]) | ((uint32_t)f32x2_to_e4m3x2(f[2], f[3]) << 16);
   }
   return make_uint2(out[0], out[1]);
@@ -103,175 +108,380 @@ __device__ __forceinline__ void move_vec(uint8_t* dst_row, int dst_r, const uint
   }
 }
 
+// ================================================================ bulk append
+// Calls with more than kSmallMax new tokens per sequence (prefill): four
+// launches, the data-moving ones spread over many CTAs per (seq, kv head),
+// with the same result as the warp paths.
+//   1. k_bulk_count (head x chunk): survivors of each chunk of kChunkPositions
+//      of the positions resolved now; on a sequence's first FP8 append, the
+//      call's max |K| and |V| (atomicMax on the bits of non-negative floats).
+//   2. k_bulk_alloc (one warp per head): exclusive prefix of the chunk counts,
+//      one atomic bump for the store blocks of all survivors, the FP8 scales,
+//      and the head's new lengths; the state before the call goes to the
+//      workspace header, which the next two kernels read instead.
+//   3. k_bulk_write (head x chunk): the chunk's survivors to the store, in
+//      order, at len0 + prefix + rank (warp ballot/popc, scan of warp totals).
+//   4. k_bulk_ring (head): the still-unresolved new tokens to the ring, once
+//      every ring row that (3) resolves has been read.
+enum : int { kHdrM, kHdrN0, kHdrR0, kHdrLen0, kHdrN1, kHdrR1, kHdrNb0, kHdrStatus, kHdrBlkLo,
+             kHdrBlkHi, kHdrSk, kHdrSv };
+enum : int { kBulkGo = 0, kBulkSkip = 1 };
+
+struct BulkIn {
+  const int32_t* n_new;
+  const uint16_t* k_in;
+  const uint16_t* v_in;
+  const uint8_t* keep_in;
+  const float* kv_scale;
+  int batch, max_new, layer;
+};
+
+// max |x| over rows [r_lo, r_hi) of D bf16 values (row stride `stride`), CTA-wide
+__device__ float rows_amax_range(const uint16_t* base, int r_lo, int r_hi, int D, long long stride,
+                                 float* red) {
+  float a = 0.0f;
+  const int vpr = D / 8;
+  for (long long i = threadIdx.x; i < (long long)(r_hi - r_lo) * vpr; i += kAppendThreads) {
+    const long long row = r_lo + i / vpr;
+    const int vec = (int)(i % vpr);
+    const uint4 x = *reinterpret_cast<const uint4*>(base + row * stride + vec * 8);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      a = fmaxf(a, fabsf(bf16lo_to_f32(w[j])));
+      a = fmaxf(a, fabsf(bf16hi_to_f32(w[j])));
+    }
+  }
+  return block_max(a, red);
+}
+
 template <bool FP8>
 __global__ void __launch_bounds__(kAppendThreads)
-k_append_evict(CacheView c, int layer, const int32_t* __restrict__ n_new, int max_new,
-               const uint16_t* __restrict__ k_in, const uint16_t* __restrict__ v_in,
-               const uint8_t* __restrict__ keep_in, const float* __restrict__ kv_scale) {
+k_bulk_count(CacheView c, AppendWork aw, BulkIn in) {
   __shared__ float s_red[kWarps];
-  __shared__ int s_warp[kWarps];
-  __shared__ int s_src[kAppendThreads];   // survivors of the current chunk: positions
-  __shared__ int s_fail;
-  __shared__ long long s_base_blk;
-  __shared__ float s_scale[2];
-
-  const int b = blockIdx.x / c.Hkv, h = blockIdx.x % c.Hkv;
-  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const long long hi = head_index(c, layer, b, h);
   pdl_wait();                 // the previous kernel's writes are visible from here on
   pdl_launch_dependents();
-  const int m = n_new[b];
-  if (m < 0 || m > max_new) {
-    if (tid == 0) latch_error(c.ctr, FDMS_ERR_DEVICE);
+  const int hid = blockIdx.x, ch = blockIdx.y, nch = gridDim.y, tid = threadIdx.x;
+  const int b = hid / c.Hkv, h = hid % c.Hkv;
+  const long long hi = head_index(c, in.layer, b, h);
+  const int m = in.n_new[b];
+  const int n0 = c.tok_n[hi], r0 = c.tok_r[hi];
+  int cnt = 0;
+  if (m > 0 && m <= in.max_new && (long long)n0 + m <= c.max_seq_len) {
+    const int n1 = n0 + m;
+    const int r1 = (n1 - c.W - r0 >= c.P) ? n1 - c.W : r0;
+    const uint8_t* rkeep = c.ring_keep + hi * c.Rpad;
+    const uint8_t* keep_rows = in.keep_in + (long long)b * in.max_new * c.Hkv + h;
+    const int p_lo = r0 + ch * kChunkPositions, p_hi = min(r1, p_lo + kChunkPositions);
+    for (int base = p_lo; base < p_hi; base += kAppendThreads) {
+      const int p = base + tid;
+      int keep = 0;
+      if (p < p_hi)
+        keep = p < n0 ? (rkeep[p % c.R] != 0) : (keep_rows[(long long)(p - n0) * c.Hkv] != 0);
+      cnt += __syncthreads_count(keep);
+    }
+    if constexpr (FP8) {
+      if (n0 == 0 && !in.kv_scale) {   // rows [ch rpc, (ch + 1) rpc) of the call
+        const long long in_stride = (long long)c.Hkv * c.D;
+        const long long off = ((long long)b * in.max_new * c.Hkv + h) * c.D;
+        const int rpc = (m + nch - 1) / nch;
+        const int lo = min(m, ch * rpc), hi_r = min(m, lo + rpc);
+        const float ak = rows_amax_range(in.k_in + off, lo, hi_r, c.D, in_stride, s_red);
+        const float av = rows_amax_range(in.v_in + off, lo, hi_r, c.D, in_stride, s_red);
+        if (tid == 0) {
+          atomicMax(&aw.amax[hid * 2], __float_as_uint(ak));
+          atomicMax(&aw.amax[hid * 2 + 1], __float_as_uint(av));
+        }
+      }
+    }
+  }
+  if (tid == 0) aw.counts[(long long)hid * aw.max_chunks + ch] = cnt;
+}
+
+template <bool FP8>
+__global__ void __launch_bounds__(32)
+k_bulk_alloc(CacheView c, AppendWork aw, BulkIn in, int nch) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int hid = blockIdx.x, lane = threadIdx.x;
+  const int b = hid / c.Hkv, h = hid % c.Hkv;
+  const long long hi = head_index(c, in.layer, b, h);
+  int* hd = aw.hdr + (long long)hid * kHdrInts;
+  const int m = in.n_new[b];
+  const int n0 = c.tok_n[hi], r0 = c.tok_r[hi], len0 = c.store_len[hi];
+  unsigned ak_bits = 0, av_bits = 0;
+  if constexpr (FP8) {
+    ak_bits = aw.amax[hid * 2];
+    av_bits = aw.amax[hid * 2 + 1];
+  }
+  __syncwarp();
+  if (FP8 && lane == 0) {   // ready for the next call
+    aw.amax[hid * 2] = 0u;
+    aw.amax[hid * 2 + 1] = 0u;
+  }
+  if (m < 0 || m > in.max_new || (long long)n0 + m > c.max_seq_len) {
+    if (lane == 0) {
+      latch_error(c.ctr, FDMS_ERR_DEVICE);
+      hd[kHdrStatus] = kBulkSkip;
+    }
     return;
   }
-  if (m == 0) return;
-  const int n0 = c.tok_n[hi], r0 = c.tok_r[hi], len0 = c.store_len[hi];
-  if ((long long)n0 + m > c.max_seq_len) {
-    if (tid == 0) latch_error(c.ctr, FDMS_ERR_DEVICE);
+  if (m == 0) {
+    if (lane == 0) hd[kHdrStatus] = kBulkSkip;
     return;
   }
   const int n1 = n0 + m;
   const int r1 = (n1 - c.W - r0 >= c.P) ? n1 - c.W : r0;
-  const long long in_stride = (long long)c.Hkv * c.D;          // elements between tokens
-  const uint16_t* k_rows = k_in + ((long long)b * max_new * c.Hkv + h) * c.D;
-  const uint16_t* v_rows = v_in + ((long long)b * max_new * c.Hkv + h) * c.D;
-  const uint8_t* keep_rows = keep_in + (long long)b * max_new * c.Hkv + h;
-  uint8_t* rkeep = c.ring_keep + hi * c.Rpad;
-
-  // ---- FP8 scales
+  // exclusive prefix of the chunk counts
+  int* cnt = aw.counts + (long long)hid * aw.max_chunks;
+  int running = 0;
+  for (int base = 0; base < nch; base += 32) {
+    const int i = base + lane;
+    const int x = i < nch ? cnt[i] : 0;
+    int incl = x;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    if (i < nch) cnt[i] = running + incl - x;
+    running += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  const int len1 = len0 + running;
+  // FP8 scales: a sequence's first append fixes them
   float sk = 1.0f, sv = 1.0f;
   if constexpr (FP8) {
     if (n0 == 0) {
-      if (kv_scale) {
-        sk = kv_scale[((long long)b * c.Hkv + h) * 2];
-        sv = kv_scale[((long long)b * c.Hkv + h) * 2 + 1];
+      if (in.kv_scale) {
+        sk = in.kv_scale[((long long)b * c.Hkv + h) * 2];
+        sv = in.kv_scale[((long long)b * c.Hkv + h) * 2 + 1];
       } else {
-        const float ak = rows_amax(k_rows, m, c.D, in_stride, s_red);
-        const float av = rows_amax(v_rows, m, c.D, in_stride, s_red);
-        sk = __fdiv_rn(fmaxf(ak, 1.17549435e-38f), 448.0f);
-        sv = __fdiv_rn(fmaxf(av, 1.17549435e-38f), 448.0f);
+        sk = __fdiv_rn(fmaxf(__uint_as_float(ak_bits), 1.17549435e-38f), 448.0f);
+        sv = __fdiv_rn(fmaxf(__uint_as_float(av_bits), 1.17549435e-38f), 448.0f);
       }
-      if (tid == 0) {
+      if (lane == 0) {
         c.head_scale[hi * 2] = sk;
         c.head_scale[hi * 2 + 1] = sv;
       }
     } else {
-      if (tid == 0) {
-        s_scale[0] = c.head_scale[hi * 2];
-        s_scale[1] = c.head_scale[hi * 2 + 1];
-      }
-      __syncthreads();
-      sk = s_scale[0];
-      sv = s_scale[1];
+      sk = c.head_scale[hi * 2];
+      sv = c.head_scale[hi * 2 + 1];
     }
   }
-
-  auto keep_of = [&](int p) -> int {
-    return p < n0 ? (rkeep[p % c.R] != 0) : (keep_rows[(long long)(p - n0) * c.Hkv] != 0);
-  };
-
-  // ---- pass 1: how many survivors, and their blocks
-  int total = 0;
-  for (int base = r0; base < r1; base += kAppendThreads) {
-    const int p = base + tid;
-    total += __syncthreads_count(p < r1 && keep_of(p));
-  }
-  const int len1 = len0 + total;
+  // store blocks for all survivors: one atomic bump
   const int nb0 = (len0 + kBlockSlots - 1) / kBlockSlots;
   const int nb1 = (len1 + kBlockSlots - 1) / kBlockSlots;
-  if (tid == 0) {
-    s_fail = 0;
-    s_base_blk = 0;
-    if (nb1 > nb0) {
+  long long base_blk = 0;
+  if (nb1 > nb0) {
+    int fail = 0;
+    if (lane == 0) {
       const unsigned long long need = (unsigned long long)(nb1 - nb0);
       const unsigned long long base = atomicAdd(&c.ctr->blocks_next, need);
       if (base + need > (unsigned long long)c.num_blocks) {
         latch_error(c.ctr, FDMS_ERR_OUT_OF_BLOCKS);
-        s_fail = 1;
+        fail = 1;
       } else {
-        s_base_blk = (long long)base;
+        base_blk = (long long)base;
       }
     }
-  }
-  __syncthreads();
-  if (s_fail) return;
-  int32_t* bt = c.block_table + hi * c.max_blocks;
-  float* bts = c.bt_scale + hi * c.max_blocks * 2;
-  for (int j = nb0 + tid; j < nb1; j += kAppendThreads) {
-    bt[j] = (int32_t)(s_base_blk + (j - nb0));
-    bts[2 * j] = sk;
-    bts[2 * j + 1] = sv;
-  }
-  __syncthreads();
-
-  const int VPR = c.D / 8;      // 16-byte input vectors per row (8 bf16 each)
-  unsigned sat = 0;
-
-  // ---- pass 2: stable compaction of positions r0 .. r1-1 into the store
-  int written = 0;
-  for (int base = r0; base < r1; base += kAppendThreads) {
-    const int p = base + tid;
-    const int bit = (p < r1) ? keep_of(p) : 0;
-    const unsigned ball = __ballot_sync(0xffffffffu, bit);
-    const int in_warp = __popc(ball & ((1u << lane) - 1u));
-    if (lane == 0) s_warp[warp] = __popc(ball);
-    __syncthreads();
-    int warp_off = 0, chunk = 0;
-    for (int i = 0; i < kWarps; ++i) {
-      warp_off += (i < warp) ? s_warp[i] : 0;
-      chunk += s_warp[i];
+    if (__shfl_sync(0xffffffffu, fail, 0)) {
+      if (lane == 0) hd[kHdrStatus] = kBulkSkip;
+      return;
     }
-    if (bit) s_src[warp_off + in_warp] = p;
-    __syncthreads();
-    // copy the chunk's survivors: (survivor, vector) pairs over the CTA
-    for (int i = tid; i < chunk * VPR; i += kAppendThreads) {
-      const int sidx = i / VPR, vec = i % VPR;
-      const int src = s_src[sidx];
-      const int d = len0 + written + sidx;
-      const long long blk = bt[d / kBlockSlots];
-      const int row = d % kBlockSlots;
-      uint8_t* kd = block_k(c, blk) + (long long)row * c.RB;
-      uint8_t* vd = block_v(c, blk) + (long long)row * c.RB;
-      if (src < n0) {   // from the ring: already in cache format
-        const int slot = src % c.R;
-        move_vec<FP8>(kd, row, ring_k(c, hi) + (long long)slot * c.RB, slot, vec, c.RB, false);
-        move_vec<FP8>(vd, row, ring_v(c, hi) + (long long)slot * c.RB, slot, vec, c.RB, true);
-      } else {          // straight from this call's input
-        const long long t = src - n0;
-        put_input_vec<FP8>(kd, k_rows + t * in_stride, vec, sk, sat, c.RB, false, row);
-        put_input_vec<FP8>(vd, v_rows + t * in_stride, vec, sv, sat, c.RB, true, row);
-      }
-      if (vec == 0) c.blk_pos[blk * kBlockSlots + row] = src;
+    base_blk = __shfl_sync(0xffffffffu, base_blk, 0);
+    int32_t* bt = c.block_table + hi * c.max_blocks;
+    float* bts = c.bt_scale + hi * c.max_blocks * 2;
+    for (int j = nb0 + lane; j < nb1; j += 32) {
+      bt[j] = (int32_t)(base_blk + (j - nb0));
+      bts[2 * j] = sk;
+      bts[2 * j + 1] = sv;
     }
-    written += chunk;
-    __syncthreads();
   }
-
-  // ---- ring: unresolved new tokens (after all ring reads above)
-  const int w0 = r1 > n0 ? r1 : n0;
-  for (long long i = tid; i < (long long)(n1 - w0) * VPR; i += kAppendThreads) {
-    const int p = w0 + (int)(i / VPR), vec = (int)(i % VPR);
-    const long long t = p - n0;
-    const int slot = p % c.R;
-    put_input_vec<FP8>(ring_k(c, hi) + (long long)slot * c.RB, k_rows + t * in_stride, vec, sk, sat,
-                       c.RB, false, slot);
-    put_input_vec<FP8>(ring_v(c, hi) + (long long)slot * c.RB, v_rows + t * in_stride, vec, sv, sat,
-                       c.RB, true, slot);
-    if (vec == 0) rkeep[slot] = keep_rows[t * c.Hkv] ? 1 : 0;
-  }
-
-  if constexpr (FP8) {
-    for (int off = 16; off > 0; off >>= 1) sat += __shfl_xor_sync(0xffffffffu, sat, off);
-    if (lane == 0 && sat) atomicAdd(&c.ctr->saturations, (unsigned long long)sat);
-  }
-  if (tid == 0) {
+  if (lane == 0) {
+    hd[kHdrM] = m;
+    hd[kHdrN0] = n0;
+    hd[kHdrR0] = r0;
+    hd[kHdrLen0] = len0;
+    hd[kHdrN1] = n1;
+    hd[kHdrR1] = r1;
+    hd[kHdrNb0] = nb0;
+    hd[kHdrStatus] = kBulkGo;
+    hd[kHdrSk] = __float_as_int(sk);
+    hd[kHdrSv] = __float_as_int(sv);
     c.store_len[hi] = len1;
     c.tok_n[hi] = n1;
     c.tok_r[hi] = r1;
   }
 }
 
+template <bool FP8>
+__global__ void __launch_bounds__(kAppendThreads)
+k_bulk_write(CacheView c, AppendWork aw, BulkIn in) {
+  __shared__ int s_warp[kWarps];
+  __shared__ int s_src[kChunkPositions];   // survivors of the chunk, in order
+  __shared__ int s_total;
+  pdl_wait();
+  pdl_launch_dependents();
+  const int hid = blockIdx.x, ch = blockIdx.y, tid = threadIdx.x, warp = tid / 32,
+            lane = tid % 32;
+  const int* hd = aw.hdr + (long long)hid * kHdrInts;
+  if (hd[kHdrStatus] != kBulkGo) return;
+  const int n0 = hd[kHdrN0], r0 = hd[kHdrR0], len0 = hd[kHdrLen0], r1 = hd[kHdrR1];
+  const float sk = __int_as_float(hd[kHdrSk]), sv = __int_as_float(hd[kHdrSv]);
+  const int p_lo = r0 + ch * kChunkPositions, p_hi = min(r1, p_lo + kChunkPositions);
+  if (p_lo >= p_hi) return;
+  const int b = hid / c.Hkv, h = hid % c.Hkv;
+  const long long hi = head_index(c, in.layer, b, h);
+  const long long in_stride = (long long)c.Hkv * c.D;
+  const uint16_t* k_rows = in.k_in + ((long long)b * in.max_new * c.Hkv + h) * c.D;
+  const uint16_t* v_rows = in.v_in + ((long long)b * in.max_new * c.Hkv + h) * c.D;
+  const uint8_t* keep_rows = in.keep_in + (long long)b * in.max_new * c.Hkv + h;
+  const uint8_t* rkeep = c.ring_keep + hi * c.Rpad;
+  const int32_t* bt = c.block_table + hi * c.max_blocks;
+  const int VPR = c.D / 8;
+  unsigned sat = 0;
+  // survivors of the chunk, in position order: ballot inside warps, scan of
+  // the warp totals, 256 positions at a time
+  if (tid == 0) s_total = 0;
+  __syncthreads();
+  for (int base = p_lo; base < p_hi; base += kAppendThreads) {
+    const int p = base + tid;
+    int bit = 0;
+    if (p < p_hi)
+      bit = p < n0 ? (rkeep[p % c.R] != 0) : (keep_rows[(long long)(p - n0) * c.Hkv] != 0);
+    const unsigned ball = __ballot_sync(0xffffffffu, bit);
+    const int in_warp = __popc(ball & ((1u << lane) - 1u));
+    if (lane == 0) s_warp[warp] = __popc(ball);
+    __syncthreads();
+    int warp_off = s_total, round = 0;
+    for (int i = 0; i < kWarps; ++i) {
+      warp_off += (i < warp) ? s_warp[i] : 0;
+      round += s_warp[i];
+    }
+    if (bit) s_src[warp_off + in_warp] = p;
+    __syncthreads();
+    if (tid == 0) s_total += round;
+    __syncthreads();
+  }
+  const int total = s_total;
+  const int first = len0 + aw.counts[(long long)hid * aw.max_chunks + ch];   // store row
+  // copy: (survivor, vector) pairs over the CTA, four loads in flight per thread
+  for (int i0 = tid; i0 < total * VPR; i0 += 4 * kAppendThreads) {
+    uint4 xk[4], xv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * kAppendThreads;
+      if (i >= total * VPR) break;
+      const int src = s_src[i / VPR], vec = i % VPR;
+      if (src < n0) {   // from the ring: already in cache format
+        const int slot = src % c.R;
+        const uint8_t* ks = ring_k(c, hi) + (long long)slot * c.RB;
+        const uint8_t* vs = ring_v(c, hi) + (long long)slot * c.RB;
+        if constexpr (FP8) {
+          const uint2 a = *reinterpret_cast<const uint2*>(ks + swz_byte(c.RB, false, slot, vec * 8));
+          const uint2 bb = *reinterpret_cast<const uint2*>(vs + swz_byte(c.RB, true, slot, vec * 8));
+          xk[u] = make_uint4(a.x, a.y, 0u, 0u);
+          xv[u] = make_uint4(bb.x, bb.y, 0u, 0u);
+        } else {
+          xk[u] = *reinterpret_cast<const uint4*>(ks + swz_byte(c.RB, false, slot, vec * 16));
+          xv[u] = *reinterpret_cast<const uint4*>(vs + swz_byte(c.RB, true, slot, vec * 16));
+        }
+      } else {          // straight from this call's input
+        const long long t = src - n0;
+        xk[u] = *reinterpret_cast<const uint4*>(k_rows + t * in_stride + vec * 8);
+        xv[u] = *reinterpret_cast<const uint4*>(v_rows + t * in_stride + vec * 8);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * kAppendThreads;
+      if (i >= total * VPR) break;
+      const int sidx = i / VPR, vec = i % VPR;
+      const int src = s_src[sidx];
+      const int d = first + sidx;
+      const long long blk = bt[d / kBlockSlots];
+      const int row = d % kBlockSlots;
+      uint8_t* kd = block_k(c, blk) + (long long)row * c.RB;
+      uint8_t* vd = block_v(c, blk) + (long long)row * c.RB;
+      if constexpr (FP8) {
+        const uint2 ok = src < n0 ? make_uint2(xk[u].x, xk[u].y) : quantise8(xk[u], sk, sat);
+        const uint2 ov = src < n0 ? make_uint2(xv[u].x, xv[u].y) : quantise8(xv[u], sv, sat);
+        *reinterpret_cast<uint2*>(kd + swz_byte(c.RB, false, row, vec * 8)) = ok;
+        *reinterpret_cast<uint2*>(vd + swz_byte(c.RB, true, row, vec * 8)) = ov;
+      } else {
+        *reinterpret_cast<uint4*>(kd + swz_byte(c.RB, false, row, vec * 16)) = xk[u];
+        *reinterpret_cast<uint4*>(vd + swz_byte(c.RB, true, row, vec * 16)) = xv[u];
+      }
+      if (vec == 0) c.blk_pos[blk * kBlockSlots + row] = src;
+    }
+  }
+  if constexpr (FP8) {
+    for (int off = 16; off > 0; off >>= 1) sat += __shfl_xor_sync(0xffffffffu, sat, off);
+    if (lane == 0 && sat) atomicAdd(&c.ctr->saturations, (unsigned long long)sat);
+  }
+}
+
+template <bool FP8>
+__global__ void __launch_bounds__(kAppendThreads)
+k_bulk_ring(CacheView c, AppendWork aw, BulkIn in) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int hid = blockIdx.x, tid = threadIdx.x, lane = tid % 32;
+  const int* hd = aw.hdr + (long long)hid * kHdrInts;
+  if (hd[kHdrStatus] != kBulkGo) return;
+  const int n0 = hd[kHdrN0], n1 = hd[kHdrN1], r1 = hd[kHdrR1];
+  const float sk = __int_as_float(hd[kHdrSk]), sv = __int_as_float(hd[kHdrSv]);
+  const int b = hid / c.Hkv, h = hid % c.Hkv;
+  const long long hi = head_index(c, in.layer, b, h);
+  const long long in_stride = (long long)c.Hkv * c.D;
+  const uint16_t* k_rows = in.k_in + ((long long)b * in.max_new * c.Hkv + h) * c.D;
+  const uint16_t* v_rows = in.v_in + ((long long)b * in.max_new * c.Hkv + h) * c.D;
+  const uint8_t* keep_rows = in.keep_in + (long long)b * in.max_new * c.Hkv + h;
+  uint8_t* rkeep = c.ring_keep + hi * c.Rpad;
+  const int VPR = c.D / 8;
+  unsigned sat = 0;
+  // vectors of rows w0 .. n1-1, spread over the gridDim.y CTAs of the head;
+  // each thread loads its (up to) 4 input vectors before any store
+  const int w0 = r1 > n0 ? r1 : n0;
+  const long long nvec = (long long)(n1 - w0) * VPR;
+  const long long stride = (long long)gridDim.y * kAppendThreads;
+  for (long long i0 = (long long)blockIdx.y * kAppendThreads + tid; i0 < nvec; i0 += 4 * stride) {
+    uint4 xk[4], xv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const long long i = i0 + u * stride;
+      if (i < nvec) {
+        const long long t = w0 + i / VPR - n0;
+        const int vec = (int)(i % VPR);
+        xk[u] = *reinterpret_cast<const uint4*>(k_rows + t * in_stride + vec * 8);
+        xv[u] = *reinterpret_cast<const uint4*>(v_rows + t * in_stride + vec * 8);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const long long i = i0 + u * stride;
+      if (i >= nvec) break;
+      const int p = w0 + (int)(i / VPR), vec = (int)(i % VPR);
+      const int slot = p % c.R;
+      uint8_t* kd = ring_k(c, hi) + (long long)slot * c.RB;
+      uint8_t* vd = ring_v(c, hi) + (long long)slot * c.RB;
+      if constexpr (FP8) {
+        *reinterpret_cast<uint2*>(kd + swz_byte(c.RB, false, slot, vec * 8)) =
+            quantise8(xk[u], sk, sat);
+        *reinterpret_cast<uint2*>(vd + swz_byte(c.RB, true, slot, vec * 8)) =
+            quantise8(xv[u], sv, sat);
+      } else {
+        *reinterpret_cast<uint4*>(kd + swz_byte(c.RB, false, slot, vec * 16)) = xk[u];
+        *reinterpret_cast<uint4*>(vd + swz_byte(c.RB, true, slot, vec * 16)) = xv[u];
+      }
+      if (vec == 0) rkeep[slot] = keep_rows[(p - n0) * c.Hkv] ? 1 : 0;
+    }
+  }
+  if constexpr (FP8) {
+    for (int off = 16; off > 0; off >>= 1) sat += __shfl_xor_sync(0xffffffffu, sat, off);
+    if (lane == 0 && sat) atomicAdd(&c.ctr->saturations, (unsigned long long)sat);
+  }
+}
 
 constexpr int kSmallMax = 16;
 constexpr int kSmallWarps = 8;
@@ -378,7 +588,7 @@ __device__ void warp_resolve(const CacheView& c, long long hi, int lane, int n0,
 }
 
 // Decode-step path: one warp per (seq, kv head), for calls that bring at most
-// kSmallMax tokens per sequence. Same semantics as k_append_evict; the loads
+// kSmallMax tokens per sequence. Same semantics as the bulk path; the loads
 // whose addresses are known are issued together, so a decode step costs about
 // two dependent memory round trips.
 
@@ -704,12 +914,56 @@ fdms_status fdms_launch_append(fdms_cache* cache, int layer, int batch, const in
               : cudaLaunchKernelEx(&cfg, k_append_small<false>, c, layer, batch, n_new, max_new,
                                    kk, vv, keep, sc);
   } else {
-    cfg.gridDim = dim3((unsigned)(batch * c.Hkv));
+    const AppendWork& aw = cache->awork;
+    const BulkIn in{n_new, kk, vv, keep, sc, batch, max_new, layer};
+    const long long span = (long long)max_new + c.W + c.P;   // bound on positions resolved
+    const int nch = (int)((span + kChunkPositions - 1) / kChunkPositions);
+    if (nch > aw.max_chunks) return FDMS_ERR_INVALID_ARG;
+    const unsigned heads = (unsigned)(batch * c.Hkv);
+    cfg.gridDim = dim3(heads, (unsigned)nch);
     cfg.blockDim = dim3(kAppendThreads);
-    e = c.fp8 ? cudaLaunchKernelEx(&cfg, k_append_evict<true>, c, layer, n_new, max_new, kk, vv,
-                                   keep, sc)
-              : cudaLaunchKernelEx(&cfg, k_append_evict<false>, c, layer, n_new, max_new, kk, vv,
-                                   keep, sc);
+    e = c.fp8 ? cudaLaunchKernelEx(&cfg, k_bulk_count<true>, c, aw, in)
+              : cudaLaunchKernelEx(&cfg, k_bulk_count<false>, c, aw, in);
+    if (e == cudaSuccess) {
+      cfg.gridDim = dim3(heads);
+      cfg.blockDim = dim3(32);
+      e = c.fp8 ? cudaLaunchKernelEx(&cfg, k_bulk_alloc<true>, c, aw, in, nch)
+                : cudaLaunchKernelEx(&cfg, k_bulk_alloc<false>, c, aw, in, nch);
+    }
+    if (e == cudaSuccess) {
+      cfg.gridDim = dim3(heads, (unsigned)nch);
+      cfg.blockDim = dim3(kAppendThreads);
+      e = c.fp8 ? cudaLaunchKernelEx(&cfg, k_bulk_write<true>, c, aw, in)
+                : cudaLaunchKernelEx(&cfg, k_bulk_write<false>, c, aw, in);
+    }
+    if (e == cudaSuccess) {   // ring rows: at most W + P - 1 + max_new per head
+      const long long rvec = (long long)min((long long)max_new, (long long)c.W + c.P) * (c.D / 8);
+      const int ry = (int)std::min<long long>(16, (rvec + 4LL * kAppendThreads - 1) /
+                                                    (4LL * kAppendThreads));
+      cfg.gridDim = dim3(heads, (unsigned)std::max(1, ry));
+      e = c.fp8 ? cudaLaunchKernelEx(&cfg, k_bulk_ring<true>, c, aw, in)
+                : cudaLaunchKernelEx(&cfg, k_bulk_ring<false>, c, aw, in);
+    }
   }
   return e == cudaSuccess ? FDMS_OK : FDMS_ERR_CUDA;
+}
+
+fdms_status fdms_append_setup(fdms_cache* cache) {
+  const CacheView& c = cache->view;
+  AppendWork& aw = cache->awork;
+  const long long span = (long long)c.max_seq_len + c.W + c.P;
+  aw.max_chunks = (int)((span + kChunkPositions - 1) / kChunkPositions);
+  const size_t heads = (size_t)c.Bmax * c.Hkv;
+  void* p = nullptr;
+  auto take = [&](size_t bytes) -> void* {
+    if (cudaMalloc(&p, bytes) != cudaSuccess) return nullptr;
+    cache->allocs[cache->nallocs++] = p;
+    cache->bytes_reserved += bytes;
+    if (cudaMemset(p, 0, bytes) != cudaSuccess) return nullptr;
+    return p;
+  };
+  aw.counts = static_cast<int*>(take(heads * aw.max_chunks * sizeof(int)));
+  aw.hdr = static_cast<int*>(take(heads * kHdrInts * sizeof(int)));
+  aw.amax = static_cast<unsigned*>(take(heads * 2 * sizeof(unsigned)));
+  return aw.counts && aw.hdr && aw.amax ? FDMS_OK : FDMS_ERR_CUDA;
 }

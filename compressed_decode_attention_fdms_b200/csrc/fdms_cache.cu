@@ -177,6 +177,7 @@ fdms_status fdms_cache_create(const fdms_config* cfg, int device, void* stream,
   A(&v.ctr, sizeof(DevCounters));
   if (e == cudaSuccess) {
     fdms_status st = fdms_decode_setup(c);   // sizes the split grid and its workspace
+    if (st == FDMS_OK) st = fdms_append_setup(c);
     if (st != FDMS_OK) {
       free_all(c);
       delete c;

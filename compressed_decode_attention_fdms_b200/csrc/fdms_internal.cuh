@@ -97,6 +97,16 @@ struct DecodeWork {
   int max_ctas;
 };
 
+// Workspace of the bulk (prefill) append, per (seq, kv head) of the call.
+constexpr int kChunkPositions = 1024;  // positions per chunk of the bulk append
+constexpr int kHdrInts = 16;
+struct AppendWork {
+  int* counts;            // [heads][max_chunks]: survivors per chunk, then their prefix
+  int* hdr;               // [heads][kHdrInts]: state before the call, allocation, scales
+  unsigned* amax;         // [heads][2]: bits of max |x| over the call's K / V (FP8)
+  int max_chunks;
+};
+
 __device__ inline void latch_error(DevCounters* ctr, int code) {
   atomicCAS(&ctr->error, 0, code);
 }
@@ -194,6 +204,7 @@ struct fdms_cache {
   int num_sms;
   fdms::CacheView view;
   fdms::DecodeWork work;
+  fdms::AppendWork awork;
   size_t bytes_reserved;
   // allocations (freed at destroy)
   void* allocs[32];
@@ -210,3 +221,4 @@ fdms_status fdms_launch_append(fdms_cache* c, int layer, int batch, const int32_
 fdms_status fdms_launch_decode(fdms_cache* c, int layer, int batch, const void* q, void* out,
                                int out_f32, float* lse, cudaStream_t s);
 fdms_status fdms_decode_setup(fdms_cache* c);
+fdms_status fdms_append_setup(fdms_cache* c);
