@@ -136,20 +136,30 @@ struct BulkIn {
   int batch, max_new, layer;
 };
 
-// max |x| over rows [r_lo, r_hi) of D bf16 values (row stride `stride`), CTA-wide
+// max |x| over rows [r_lo, r_hi) of D bf16 values (row stride `stride`),
+// CTA-wide; eight 16-byte loads in flight per thread
 __device__ float rows_amax_range(const uint16_t* base, int r_lo, int r_hi, int D, long long stride,
                                  float* red) {
   float a = 0.0f;
   const int vpr = D / 8;
-  for (long long i = threadIdx.x; i < (long long)(r_hi - r_lo) * vpr; i += kAppendThreads) {
-    const long long row = r_lo + i / vpr;
-    const int vec = (int)(i % vpr);
-    const uint4 x = *reinterpret_cast<const uint4*>(base + row * stride + vec * 8);
-    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+  const long long nv = (long long)(r_hi - r_lo) * vpr;
+  for (long long i0 = threadIdx.x; i0 < nv; i0 += 8LL * kAppendThreads) {
+    uint4 x[8];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      a = fmaxf(a, fabsf(bf16lo_to_f32(w[j])));
-      a = fmaxf(a, fabsf(bf16hi_to_f32(w[j])));
+    for (int u = 0; u < 8; ++u) {
+      const long long i = i0 + (long long)u * kAppendThreads;
+      x[u] = i < nv ? *reinterpret_cast<const uint4*>(base + (r_lo + i / vpr) * stride +
+                                                       (i % vpr) * 8)
+                    : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const uint32_t w[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        a = fmaxf(a, fabsf(bf16lo_to_f32(w[j])));
+        a = fmaxf(a, fabsf(bf16hi_to_f32(w[j])));
+      }
     }
   }
   return block_max(a, red);
