@@ -287,38 +287,56 @@ def run_native(args, wl):
     row = 2 * wl.head_dim * elt
     qo_bytes = 2 * B * wl.q_heads * wl.head_dim * 2      # q read + out written, bf16
 
-    # prefill: every layer's append in one CUDA graph, replayed once between
-    # events (the inputs are generated first), with the bytes the appends must
-    # move: keep bits, the input rows they read (all of them for the FP8 scale
-    # pass of a first append, else survivors and ring rows) and the rows,
-    # positions and keep bytes they write
-    pre_bytes = 0.0
-    with torch.cuda.stream(stream):
-        pre_in = [wk.prefill_inputs(wl, layer, device=dev) for layer in range(L)]
-        for inp in pre_in:
-            n = inp["n_new"].to(torch.int64)
-            res = torch.where(n - wl.window >= wl.period, n - wl.window, torch.zeros_like(n))
-            pos = torch.arange(inp["max_new"], device=dev).view(1, -1, 1)
-            surv = int(((inp["keep"] != 0) & (pos < res.view(-1, 1, 1))).sum())
-            ring_rows = int((n - res).sum()) * wl.kv_heads
-            in_row = 2 * wl.head_dim * 2                  # K + V, bf16
-            read_rows = int(n.sum()) * wl.kv_heads if elt == 1 else surv + ring_rows
-            pre_bytes += (int(n.sum()) * wl.kv_heads + read_rows * in_row
-                          + (surv + ring_rows) * row + surv * 4 + ring_rows)
-    stream.synchronize()
-    graph_pre = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(stream):
-        with torch.cuda.graph(graph_pre, stream=stream):
-            for layer, inp in enumerate(pre_in):
+    # prefill, timed on the device, with the bytes the appends must move: keep
+    # bits, the input rows they read (all of them for the FP8 scale pass of a
+    # first append, else survivors and ring rows) and the rows, positions and
+    # keep bytes they write
+    def prefill_bytes(inp):
+        n = inp["n_new"].to(torch.int64)
+        res = torch.where(n - wl.window >= wl.period, n - wl.window, torch.zeros_like(n))
+        pos = torch.arange(inp["max_new"], device=dev).view(1, -1, 1)
+        surv = int(((inp["keep"] != 0) & (pos < res.view(-1, 1, 1))).sum())
+        ring_rows = int((n - res).sum()) * wl.kv_heads
+        in_row = 2 * wl.head_dim * 2                      # K + V, bf16
+        read_rows = int(n.sum()) * wl.kv_heads if elt == 1 else surv + ring_rows
+        return (int(n.sum()) * wl.kv_heads + read_rows * in_row
+                + (surv + ring_rows) * row + surv * 4 + ring_rows)
+
+    in_bytes = 2 * B * wl.max_ctx * wl.kv_heads * wl.head_dim * 2 * L
+    pre_bytes, pre_ms = 0.0, 0.0
+    if in_bytes <= 24e9:   # all layers' inputs fit: one graph, no launch gaps
+        pre_how = "CUDA events around one graph of every layer's fdms_append_evict"
+        with torch.cuda.stream(stream):
+            pre_in = [wk.prefill_inputs(wl, layer, device=dev) for layer in range(L)]
+            pre_bytes = float(sum(prefill_bytes(inp) for inp in pre_in))
+        stream.synchronize()
+        graph_pre = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(graph_pre, stream=stream):
+                for layer, inp in enumerate(pre_in):
+                    fd.fdms_append_evict(cache, layer, B, inp["n_new"], inp["max_new"], inp["k"],
+                                         inp["v"], inp["keep"], stream=stream)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            graph_pre.replay()
+            e1.record(stream)
+        stream.synchronize()
+        pre_ms = e0.elapsed_time(e1)
+        del graph_pre, pre_in
+    else:                  # one layer's inputs at a time, each append between events
+        pre_how = "CUDA events around each layer's fdms_append_evict, inputs made between"
+        for layer in range(L):
+            with torch.cuda.stream(stream):
+                inp = wk.prefill_inputs(wl, layer, device=dev)
+                pre_bytes += prefill_bytes(inp)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
                 fd.fdms_append_evict(cache, layer, B, inp["n_new"], inp["max_new"], inp["k"],
                                      inp["v"], inp["keep"], stream=stream)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        graph_pre.replay()
-        e1.record(stream)
-    stream.synchronize()
-    pre_ms = e0.elapsed_time(e1)
-    del graph_pre, pre_in
+                e1.record(stream)
+            stream.synchronize()
+            pre_ms += e0.elapsed_time(e1)
+            del inp
     with torch.cuda.stream(stream):
         # decode inputs of the device-timed steps, resident in HBM before timing
         steps_in = [[wk.decode_inputs(wl, l, s, device=dev) for l in range(L)]
@@ -434,8 +452,7 @@ def run_native(args, wl):
                         "us_per_layer": 1e3 * pre_ms / L, "gb_per_layer": pre_bytes / L / 1e9,
                         "achieved_gbs": pre_bytes / (pre_ms * 1e-3) / 1e9,
                         "frac": pre_bytes / (pre_ms * 1e-3) / 1e9 / peak,
-                        "timing": "CUDA events around one graph of every layer's "
-                                  "fdms_append_evict (4 launches each)"},
+                        "timing": pre_how + " (4 launches per layer)"},
             "kv_gb_per_step": kv_bytes / K / 1e9,
             "decode_share_of_step": dec_avg_ms * L * K / elapsed_ms,
         }
