@@ -411,6 +411,18 @@ def run_native(args, wl):
         t_max, bytes_all = float(tt.item()), float(bb.item())
     value = bytes_all / (t_max * 1e-3) / 1e9
 
+    # ---- KV memory after prefill and every step so far (the pages' memory
+    # table: compact store + ring against a dense cache of the same tokens)
+    st = fd.fdms_cache_stats(cache, stream)
+    dense_bf16 = st["tokens_appended"] * wl.kv_heads * 2 * wl.head_dim * 2
+    memory = {"compact_gib": st["bytes_compact"] / 2**30,
+              "dense_same_dtype_gib": st["bytes_dense_equiv"] / 2**30,
+              "dense_bf16_gib": dense_bf16 / 2**30,
+              "compression_same_dtype": st["bytes_dense_equiv"] / max(1, st["bytes_compact"]),
+              "compression_vs_bf16": dense_bf16 / max(1, st["bytes_compact"]),
+              "reserved_gib": st["bytes_reserved"] / 2**30,
+              "tokens_per_seq": st["tokens_appended"] // max(1, wl.layers * wl.batch)}
+
     # ---- end to end through the public API with pinned host buffers
     e2e = None
     if KE > 0:
@@ -454,6 +466,7 @@ def run_native(args, wl):
                         "frac": pre_bytes / (pre_ms * 1e-3) / 1e9 / peak,
                         "timing": pre_how + " (4 launches per layer)"},
             "kv_gb_per_step": kv_bytes / K / 1e9,
+            "memory": memory,
             "decode_share_of_step": dec_avg_ms * L * K / elapsed_ms,
         }
         if e2e:

@@ -140,11 +140,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 }
 
 
-// a / b for 0 <= a, 0 < b: 32-bit division when both fit (a short sequence),
-// the 64-bit one (a long software sequence) otherwise.
-__device__ __forceinline__ long long udiv(long long a, long long b) {
-  if (a < (1LL << 32) && b < (1LL << 32)) return (long long)((unsigned)a / (unsigned)b);
-  return a / b;
+// Tiles of one head: its store pages (tile = TR rows of a page), then the
+// TR-row frames its ring slots r .. n-1 fall in.
+template <int TR>
+__device__ __forceinline__ int head_tiles(int len, int n, int r) {
+  const int live = n - r;
+  return (len + TR - 1) / TR + (live > 0 ? (live + (r % TR) + TR - 1) / TR : 0);
+}
+// Tiles per warp for P tiles over n_ranges warps: ceil(P / n_ranges), at least
+// 1; an fp64 estimate of the quotient (inv = 1 / n_ranges) made exact by
+// integer correction.
+__device__ __forceinline__ int tiles_per_warp(int P, int n_ranges, double inv) {
+  long long qq = (long long)((double)P * inv);
+  while (qq * n_ranges > P) --qq;
+  while ((qq + 1) * n_ranges <= P) ++qq;
+  const int S = (int)qq + (qq * n_ranges < P ? 1 : 0);
+  return S > 1 ? S : 1;
 }
 
 // ------------------------------------------------------------- MMA helpers
@@ -259,9 +270,7 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
     const int h0 = tid * per, h1 = min(NH, h0 + per);
     long long su = 0;
     int sp = 0;
-    auto pages = [](int len, int live, int r) {
-      return (len + TR - 1) / TR + (live > 0 ? (live + (r % TR) + TR - 1) / TR : 0);
-    };
+    auto pages = [](int len, int live, int r) { return head_tiles<TR>(len, r + live, r); };
     for (int h = h0; h < h1; ++h) {
       const int len = c.store_len[hi0 + h], n = c.tok_n[hi0 + h], r = c.tok_r[hi0 + h];
       s_len[h] = len;
@@ -304,21 +313,10 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   // Warp v reads tiles [v S, (v + 1) S), S = ceil(P / ranges): a tile costs
   // the same compute full or not, so whole tiles are what gets balanced. The
   // quotient is an fp64 estimate made exact by integer correction.
-  int S;
-  {
-    long long qq = (long long)((double)P * inv_ranges);
-    while (qq * n_ranges > P) --qq;
-    while ((qq + 1) * n_ranges <= P) ++qq;
-    S = (int)qq + (qq * n_ranges < P ? 1 : 0);
-    S = S > 1 ? S : 1;
-  }
-  if (blockIdx.x == 0) {   // the plan the combine kernel reads back
-    for (int h = tid; h <= NH; h += T::NT) w.head_off[h] = page_off[h];
-    if (tid == 0) {
-      *w.span = S;
-      c.ctr->slots_decoded += (unsigned long long)total;   // one thread, launches are ordered
-      c.ctr->decode_calls += 1ull;
-    }
+  const int S = tiles_per_warp(P, n_ranges, inv_ranges);
+  if (blockIdx.x == 0 && tid == 0) {   // one thread, launches are ordered
+    c.ctr->slots_decoded += (unsigned long long)total;
+    c.ctr->decode_calls += 1ull;
   }
   // heads without a single slot get zeros (nobody else writes them)
   for (int h = blockIdx.x; h < NH; h += gridDim.x) {
@@ -807,19 +805,56 @@ __device__ __forceinline__ void merge_mlo(float& M, float& L, float& O, float M2
   M = mx;
 }
 
-template <int D, int G>
+template <int D, int G, int TR>
 __global__ void __launch_bounds__(Combine<D, G>::NT)
-k_decode_combine(DecodeWork w, int Hkv, int Hq, int batch, OutArgs oa) {
+k_decode_combine(CacheView c, DecodeWork w, int layer, int batch, OutArgs oa, int n_ranges,
+                 double inv_ranges) {
   using C = Combine<D, G>;
   constexpr int kChunk = 16, TPE = C::TPE;
-  pdl_wait();
   pdl_launch_dependents();
   const int hidx = blockIdx.x / C::CPH, tid = threadIdx.x, sub = tid % TPE;
-  // the head's tiles and the tiles per warp of the split
-  const long long hs = w.head_off[hidx], he = w.head_off[hidx + 1], S = *w.span;
+  // ---- the split's plan, rebuilt before the wait: it depends only on the
+  // head lengths, which no kernel between the split and this one changes (the
+  // append that set them had finished before the split began)
+  __shared__ int s_sum[C::NT / 32];
+  __shared__ int s_head[2];   // tile prefix at hidx and hidx + 1
+  __shared__ int s_total;
+  {
+    const int NH = batch * c.Hkv;
+    const long long hi0 = (long long)layer * c.Bmax * c.Hkv;
+    const int per = (NH + C::NT - 1) / C::NT;
+    const int h0 = min(NH, tid * per), h1 = min(NH, h0 + per);
+    int sp = 0, sp_at = 0, sp_next = 0;
+    for (int h = h0; h < h1; ++h) {
+      if (h == hidx) sp_at = sp;
+      if (h == hidx + 1) sp_next = sp;
+      sp += head_tiles<TR>(c.store_len[hi0 + h], c.tok_n[hi0 + h], c.tok_r[hi0 + h]);
+    }
+    const int lane = tid % 32, warp = tid / 32;
+    int incl = sp;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    if (lane == 31) s_sum[warp] = incl;
+    __syncthreads();
+    int excl = incl - sp;
+    for (int i = 0; i < warp; ++i) excl += s_sum[i];
+    if (hidx >= h0 && hidx < h1) s_head[0] = excl + sp_at;
+    if (hidx + 1 >= h0 && hidx + 1 < h1) s_head[1] = excl + sp_next;
+    if (tid == C::NT - 1) s_total = excl + sp;
+    __syncthreads();
+    if (hidx + 1 == NH && tid == 0) s_head[1] = s_total;
+    __syncthreads();
+  }
+  const int hs = s_head[0], he = s_head[1];
+  const int S = tiles_per_warp(s_total, n_ranges, inv_ranges);
+  pdl_wait();
   if (he == hs) return;
-  const long long r0 = udiv(hs, S), r1 = udiv(he - 1, S);
+  const long long r0 = hs / S, r1 = (he - 1) / S;
   if (r0 == r1) return;
+  const int Hkv = c.Hkv, Hq = c.Hq;
   const int kb = hidx / Hkv, kh = hidx % Hkv;
   const int idx = (blockIdx.x % C::CPH) * C::EPC + tid / TPE;
   const int h = idx / D, d = idx % D;
@@ -887,8 +922,8 @@ fdms_status launch_split_t(fdms_cache* cache, const DecodeWork& w, OutArgs oa, i
   cfg.gridDim = dim3((unsigned)(nh * Combine<T::D, T::G>::CPH));
   cfg.blockDim = dim3(Combine<T::D, T::G>::NT);
   cfg.dynamicSmemBytes = 0;
-  e = cudaLaunchKernelEx(&cfg, k_decode_combine<T::D, T::G>, w, cache->view.Hkv, cache->view.Hq,
-                         batch, oa);
+  e = cudaLaunchKernelEx(&cfg, k_decode_combine<T::D, T::G, T::TR>, cache->view, w, layer, batch,
+                         oa, n_ranges, 1.0 / (double)n_ranges);
   return e == cudaSuccess ? FDMS_OK : FDMS_ERR_CUDA;
 }
 
@@ -953,9 +988,7 @@ fdms_status fdms_decode_setup(fdms_cache* cache) {
   };
   w.part_o = static_cast<float*>(take((size_t)w.max_parts * c.G * c.D * sizeof(float)));
   w.part_ml = static_cast<float*>(take((size_t)w.max_parts * c.G * 2 * sizeof(float)));
-  w.head_off = static_cast<long long*>(take((size_t)(c.Bmax * c.Hkv + 1) * sizeof(long long)));
-  w.span = static_cast<long long*>(take(sizeof(long long)));
-  if (!w.part_o || !w.part_ml || !w.head_off || !w.span) return FDMS_ERR_CUDA;
+  if (!w.part_o || !w.part_ml) return FDMS_ERR_CUDA;
   return FDMS_OK;
 }
 
@@ -1006,14 +1039,13 @@ extern "C" fdms_status fdms_decode_attn_noalloc(fdms_cache* cache, int layer, in
   if (!q_dev || !out_dev || (((uintptr_t)q_dev | (uintptr_t)out_dev) & 15))
     return FDMS_ERR_INVALID_ARG;
   if (cache->device < 0 || cache->device >= kMaxDevices) return FDMS_ERR_UNSUPPORTED;
-  // layout of the scratch for this call: the plan (head prefix, ranges used),
-  // partials (o), partials (m, l); everything is written before it is read
+  // layout of the scratch for this call: partials (o), then partials (m, l);
+  // everything is written before it is read
   const long long parts = (long long)cache->decode_ctas * cache->ranges_per_cta +
                           (long long)batch * c.Hkv;
-  const size_t plan_bytes = align256((size_t)(batch * c.Hkv + 1) * sizeof(long long) + 16);
   const size_t o_bytes = align256((size_t)parts * c.G * c.D * sizeof(float));
   const size_t ml_bytes = align256((size_t)parts * c.G * 2 * sizeof(float));
-  const size_t need = plan_bytes + o_bytes + ml_bytes;
+  const size_t need = o_bytes + ml_bytes;
   if (need > FDMS_STATIC_SCRATCH_BYTES) return FDMS_ERR_INVALID_ARG;
 
   int prev = -1;
@@ -1027,10 +1059,8 @@ extern "C" fdms_status fdms_decode_attn_noalloc(fdms_cache* cache, int layer, in
   } else {
     unsigned char* b = static_cast<unsigned char*>(base);
     DecodeWork w;
-    w.head_off = reinterpret_cast<long long*>(b);
-    w.span = reinterpret_cast<long long*>(b + plan_bytes - 16);
-    w.part_o = reinterpret_cast<float*>(b + plan_bytes);
-    w.part_ml = reinterpret_cast<float*>(b + plan_bytes + o_bytes);
+    w.part_o = reinterpret_cast<float*>(b);
+    w.part_ml = reinterpret_cast<float*>(b + o_bytes);
     w.max_parts = (int)parts;
     w.max_ctas = cache->decode_ctas;
     // the array keeps the previous call's contents; nothing in it needs to

@@ -87,12 +87,10 @@ __host__ __device__ inline uint8_t* ring_v(const CacheView& c, long long hi) {
   return ring_k(c, hi) + (long long)c.R * c.RB;
 }
 
-// Decode workspace (split partials and the plan the combine reads back).
+// Decode workspace: the split partials (warp v's partial of head h at v + h).
 struct DecodeWork {
   float* part_o;          // [max_parts][G][D], unnormalised sum of p * v
   float* part_ml;         // [max_parts][G][2]: running max (log2 domain) and sum
-  long long* head_off;    // [heads + 1]: prefix of tiles over the call's heads
-  long long* span;        // tiles per warp range of the last split
   int max_parts;
   int max_ctas;
 };

@@ -179,12 +179,11 @@ fdms_status fdms_decode_attn_f32(fdms_cache* cache, int layer, int batch,
  * which fdms_decode_attn keeps in workspace the cache allocated, go instead
  * into one static array of FDMS_STATIC_SCRATCH_BYTES compiled into the library;
  * every device that loads the library holds that array until the process exits.
- *   - Needs (split warps + batch x Hkv) x G x (4 D + 8) bytes plus the
- *     per-head plan (at most one partial per split warp and head it shares
- *     with another warp; 8 split warps per decode CTA, 4 when G x D >= 1024);
- *     a call that needs more than the array returns FDMS_ERR_INVALID_ARG and
- *     queues nothing.
- *     Every value the call reads from the array it first writes itself.
+ *   - Needs (split warps + batch x Hkv) x G x (4 D + 8) bytes (at most one
+ *     partial per split warp and head it shares with another warp; 8 split
+ *     warps per decode CTA, 4 when G x D >= 1024); a call that needs more than
+ *     the array returns FDMS_ERR_INVALID_ARG and queues nothing. Every value
+ *     the call reads from the array it first writes itself.
  *   - The first call on a device looks up the array's device address (a
  *     runtime query, no allocation); make that first call before any stream
  *     capture.
