@@ -309,3 +309,33 @@ def test_mixed_append_sizes(kv_dtype, window, period):
         p.check_stats()
     finally:
         p.close()
+
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "fp8_e4m3"])
+@pytest.mark.parametrize("window,period", [(16, 1), (300, 64)])
+def test_large_appends_span_chunks(kv_dtype, window, period):
+    """Bulk appends of thousands of tokens onto sequences that already hold
+    tokens: the positions resolved at once come from the ring and from the
+    call's input and span several 1024-position chunks, whose boundaries fall
+    anywhere in the store's pages; single-token steps in between."""
+    rng = np.random.default_rng(window + period)
+    wl = wk.scaled(wk.get("tiny"), batch=3, ctx=40, steps=0, window=window, period=period,
+                   kv_dtype=kv_dtype, rate=0.35)
+    p = Pair(wl, max_seq_len=9000, oracle_capacity=9000)
+    try:
+        step = 0
+        for m in [700, 1, 2500, 1, 1, 3100, 1]:
+            big = wk.scaled(wl, ctx=m)
+            inp = wk.prefill_inputs(big, 0)
+            n = [m, max(m - int(rng.integers(1, 300)), 0) if m > 1 else 1, m // 3]
+            inp = {**inp, "n_new": torch.tensor(n, dtype=torch.int32)}
+            p.append(0, inp)
+            p.check_heads(0)
+            q = wk.decode_query(wl, 0, step)
+            step += 1
+            out = p.decode(0, q)
+            assert _max_err(out, p.oracle_out(0, q)) <= (TOL_BF16 if kv_dtype == "bf16" else
+                                                          TOL_FP8_MIRROR)
+        p.check_stats()
+    finally:
+        p.close()
