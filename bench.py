@@ -473,7 +473,8 @@ def run_native(args, wl):
             result["e2e"] = {"value": e2e["bytes"] / (e2e["ms"] * 1e-3) / 1e9, "unit": "GB/s",
                              "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                              "us_per_step": 1e3 * e2e["ms"] / KE, "steps": KE,
-                             "path": "Python binding -> C ABI, eager calls per layer"}
+                             "path": "Python binding -> C ABI, eager calls per layer; one packed "
+                                     "H2D of the step's inputs and one D2H of all outputs"}
         if not args.no_cpu_baseline and world == 1:
             bps, times, desc = oracle_sample(wl, args.cpu_seconds)
             result["cpu_baseline"] = {"value": bps / 1e9, "unit": "GB/s", "cores": 1,
@@ -490,35 +491,51 @@ def run_native(args, wl):
 
 
 def run_e2e(fd, cache, wl, stream, dev, s0, warm, steps, row):
-    """Steps through the public API with host buffers: H2D of the step's inputs
-    from pinned memory, every layer's append + decode, D2H of every output."""
+    """Steps through the public API with host buffers: every step, one copy of
+    all its inputs (every layer's new token, keep bits and query, packed in
+    one pinned buffer) to the device, every layer's fdms_append_evict +
+    fdms_decode_attn on views of that buffer, and one copy of every layer's
+    output back to pinned host memory."""
     L, B = wl.layers, wl.batch
+    # packed layout of one step: per layer n_new, k, v, keep, q, 16-byte aligned
+    shapes = [("n_new", torch.int32, (B,)),
+              ("k", torch.bfloat16, (B, 1, wl.kv_heads, wl.head_dim)),
+              ("v", torch.bfloat16, (B, 1, wl.kv_heads, wl.head_dim)),
+              ("keep", torch.uint8, (B, 1, wl.kv_heads)),
+              ("q", torch.bfloat16, (B, wl.q_heads, wl.head_dim))]
+    layout, off = [], 0
+    for layer in range(L):
+        per = {}
+        for name, dt, shp in shapes:
+            n = int(np.prod(shp)) * torch.tensor([], dtype=dt).element_size()
+            per[name] = (off, n, dt, shp)
+            off += (n + 15) // 16 * 16
+        layout.append(per)
+    step_bytes = off
     host = []
     for s in range(s0, s0 + warm + steps):
-        per = []
+        buf = torch.empty(step_bytes, dtype=torch.uint8).pin_memory()
         for layer in range(L):
             inp = wk.decode_inputs(wl, layer, s)
-            q = wk.decode_query(wl, layer, s)
-            per.append({k: v.pin_memory() for k, v in
-                        (("n_new", inp["n_new"]), ("k", inp["k"]), ("v", inp["v"]),
-                         ("keep", inp["keep"]), ("q", q))})
-        host.append(per)
-    dbuf = [{k: torch.empty_like(v, device=dev) for k, v in host[0][l].items()} for l in range(L)]
-    dout = [torch.empty((B, wl.q_heads, wl.head_dim), dtype=torch.bfloat16, device=dev)
-            for _ in range(L)]
-    hout = [torch.empty_like(dout[0], device="cpu").pin_memory() for _ in range(L)]
-    h2d = sum(v.numel() * v.element_size() for v in host[0][0].values()) * L
-    d2h = sum(o.numel() * o.element_size() for o in dout)
+            src = {"n_new": inp["n_new"], "k": inp["k"], "v": inp["v"], "keep": inp["keep"],
+                   "q": wk.decode_query(wl, layer, s)}
+            for name, (o, n, dt, shp) in layout[layer].items():
+                buf[o:o + n].view(dt).view(shp).copy_(src[name])
+        host.append(buf)
+    dbuf = torch.empty(step_bytes, dtype=torch.uint8, device=dev)
+    views = [{name: dbuf[o:o + n].view(dt).view(shp) for name, (o, n, dt, shp) in per.items()}
+             for per in layout]
+    dout = torch.empty((L, B, wl.q_heads, wl.head_dim), dtype=torch.bfloat16, device=dev)
+    hout = torch.empty_like(dout, device="cpu").pin_memory()
 
     def one(s):
+        dbuf.copy_(host[s], non_blocking=True)
         for layer in range(L):
-            for k, v in host[s][layer].items():
-                dbuf[layer][k].copy_(v, non_blocking=True)
-            d = dbuf[layer]
+            d = views[layer]
             fd.fdms_append_evict(cache, layer, B, d["n_new"], 1, d["k"], d["v"], d["keep"],
                                  stream=stream)
             fd.fdms_decode_attn(cache, layer, B, d["q"], dout[layer], stream=stream)
-            hout[layer].copy_(dout[layer], non_blocking=True)
+        hout.copy_(dout, non_blocking=True)
 
     with torch.cuda.stream(stream):
         for s in range(warm):
@@ -536,7 +553,7 @@ def run_e2e(fd, cache, wl, stream, dev, s0, warm, steps, row):
     torch.cuda.synchronize()
     st1 = fd.fdms_cache_stats(cache, stream)
     return {"ms": t0.elapsed_time(t1), "bytes": (st1["slots_decoded"] - st0["slots_decoded"]) * row,
-            "h2d": h2d, "d2h": d2h}
+            "h2d": step_bytes, "d2h": dout.numel() * dout.element_size()}
 
 
 def main():

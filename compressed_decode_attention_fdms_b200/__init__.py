@@ -172,13 +172,14 @@ def fdms_cache_destroy(cache: Cache):
 
 
 def _dev_tensor(t, dtype, shape, name, device):
+    """Device pointer of a tensor after checking what the C ABI assumes."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name}: expected a torch.Tensor")
-    if t.device.type != "cuda" or t.device.index != device:
+    if not t.is_cuda or t.get_device() != device:
         raise ValueError(f"{name}: must live on cuda:{device}")
     if t.dtype != dtype:
         raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
-    if tuple(t.shape) != tuple(shape):
+    if t.shape != shape:
         raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
     if not t.is_contiguous():
         raise ValueError(f"{name}: must be contiguous")
@@ -189,32 +190,30 @@ def fdms_append_evict(cache: Cache, layer: int, batch: int, n_new: torch.Tensor,
                       k: torch.Tensor, v: torch.Tensor, keep: torch.Tensor,
                       kv_scale: Optional[torch.Tensor] = None, stream=None):
     c = cache.config
-    H, D = c.num_kv_heads, c.head_dim
-    args = (
-        _dev_tensor(n_new, torch.int32, (batch,), "n_new", cache.device),
-        max_new,
-        _dev_tensor(k, torch.bfloat16, (batch, max_new, H, D), "k", cache.device),
-        _dev_tensor(v, torch.bfloat16, (batch, max_new, H, D), "v", cache.device),
-        _dev_tensor(keep, torch.uint8, (batch, max_new, H), "keep", cache.device),
+    H, D, dev = c.num_kv_heads, c.head_dim, cache.device
+    kv = (batch, max_new, H, D)
+    st = load_library().fdms_append_evict(
+        cache.handle, layer, batch, _dev_tensor(n_new, torch.int32, (batch,), "n_new", dev),
+        max_new, _dev_tensor(k, torch.bfloat16, kv, "k", dev),
+        _dev_tensor(v, torch.bfloat16, kv, "v", dev),
+        _dev_tensor(keep, torch.uint8, kv[:3], "keep", dev),
         None if kv_scale is None else
-        _dev_tensor(kv_scale, torch.float32, (batch, H, 2), "kv_scale", cache.device),
-    )
-    _check(load_library().fdms_append_evict(
-        ctypes.c_void_p(cache.handle), layer, batch, ctypes.c_void_p(args[0]), args[1],
-        ctypes.c_void_p(args[2]), ctypes.c_void_p(args[3]), ctypes.c_void_p(args[4]),
-        ctypes.c_void_p(args[5]), ctypes.c_void_p(_stream_ptr(stream, cache.device))),
-        "fdms_append_evict")
+        _dev_tensor(kv_scale, torch.float32, (batch, H, 2), "kv_scale", dev),
+        _stream_ptr(stream, dev))
+    if st != FDMS_OK:
+        raise FdmsError(st, "fdms_append_evict")
 
 
 def fdms_decode_attn(cache: Cache, layer: int, batch: int, q: torch.Tensor, out: torch.Tensor,
                      stream=None):
     c = cache.config
     shape = (batch, c.num_q_heads, c.head_dim)
-    qp = _dev_tensor(q, torch.bfloat16, shape, "q", cache.device)
-    op = _dev_tensor(out, torch.bfloat16, shape, "out", cache.device)
-    _check(load_library().fdms_decode_attn(
-        ctypes.c_void_p(cache.handle), layer, batch, ctypes.c_void_p(qp), ctypes.c_void_p(op),
-        ctypes.c_void_p(_stream_ptr(stream, cache.device))), "fdms_decode_attn")
+    dev = cache.device
+    st = load_library().fdms_decode_attn(
+        cache.handle, layer, batch, _dev_tensor(q, torch.bfloat16, shape, "q", dev),
+        _dev_tensor(out, torch.bfloat16, shape, "out", dev), _stream_ptr(stream, dev))
+    if st != FDMS_OK:
+        raise FdmsError(st, "fdms_decode_attn")
 
 
 def fdms_decode_attn_f32(cache: Cache, layer: int, batch: int, q: torch.Tensor,
