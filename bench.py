@@ -72,6 +72,19 @@ def load_peaks():
     return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (no MEASURED_PEAKS.json)"
 
 
+def code_hash(path):
+    """First 16 hex digits of the sha256 of a source file's code: // comments,
+    trailing blanks and empty lines removed, so that comment edits keep it."""
+    import hashlib
+    import re
+    lines = []
+    for line in open(path, encoding="utf-8"):
+        line = re.sub(r"//.*$", "", line.rstrip("\n")).rstrip()
+        if line:
+            lines.append(line)
+    return hashlib.sha256("\n".join(lines).encode()).hexdigest()[:16]
+
+
 def load_traffic(workload):
     """DRAM bytes of one decode call from the committed ncu summary, if it was
     taken on the decode sources as they are now; else None."""
@@ -80,8 +93,7 @@ def load_traffic(workload):
     if not os.path.exists(p):
         return None, "no capture"
     src = os.path.join(ROOT, "compressed_decode_attention_fdms_b200", "csrc")
-    now = [hashlib.sha256(open(os.path.join(src, f), "rb").read()).hexdigest()[:16]
-           for f in ("fdms_decode.cu", "fdms_internal.cuh")]
+    now = [code_hash(os.path.join(src, f)) for f in ("fdms_decode.cu", "fdms_internal.cuh")]
     for line in open(p):
         f = line.split()
         if not f or f[0].startswith("#") or f[0] != workload:

@@ -37,8 +37,12 @@
 //   - A head that lies whole inside one warp's range is written by that warp;
 //     heads with no slot get zeros. Every other head has one partial
 //     (m, l, o) per warp that covered part of it, written to a workspace; a
-//     combine kernel merges them, one output element per thread, loading the
-//     partials together: o = sum_w 2^(m_w - M) o_w / sum_w 2^(m_w - M) l_w.
+//     combine kernel merges them, four threads per output element, loading
+//     all partials of the head at once:
+//         o = sum_w 2^(m_w - M) o_w / sum_w 2^(m_w - M) l_w.
+//     The combine rebuilds the split's tile plan from the head lengths itself
+//     (nothing changes them between the two kernels), before its dependency
+//     wait.
 //   - Both kernels allow programmatic dependent launch: set-up that reads no
 //     data of the previous kernel runs while that kernel finishes.
 #include <cfloat>
