@@ -106,6 +106,25 @@ def load_traffic(workload):
     return None, "no capture for this workload"
 
 
+def rank_workload(wl, rank, world):
+    """The workload a rank runs: every rank its own sequences (replicas; the
+    path has no exchange step), so rank r draws from seed + 7919 r."""
+    return wk.scaled(wl, seed=wl.seed + 7919 * rank) if world > 1 else wl
+
+
+def over_ranks(t_ms, nbytes, world, device):
+    """Whole-job figures: the longest time over ranks and the bytes of all of
+    them (every rank takes the same two collective steps, in the same order)."""
+    if world <= 1:
+        return float(t_ms), float(nbytes)
+    import torch.distributed as dist
+    t = torch.tensor([float(t_ms)], dtype=torch.float64, device=device)
+    b = torch.tensor([float(nbytes)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(b, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(b.item())
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -282,8 +301,7 @@ def run_native(args, wl):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        wl = wk.scaled(wl, seed=wl.seed + 7919 * rank)   # each rank: its own sequences
+    wl = rank_workload(wl, rank, world)
 
     W, K = args.warmup, args.steps
     KE = 0 if args.no_e2e else args.e2e_steps
@@ -413,14 +431,7 @@ def run_native(args, wl):
     per_launch_bytes = dec_slots * row / dec_calls + qo_bytes
 
     # whole-job numbers: max time over ranks, bytes summed over ranks
-    t_max, bytes_all = elapsed_ms, float(kv_bytes)
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        bb = torch.tensor([float(kv_bytes)], dtype=torch.float64, device=dev)
-        dist.all_reduce(bb, op=dist.ReduceOp.SUM)
-        t_max, bytes_all = float(tt.item()), float(bb.item())
+    t_max, bytes_all = over_ranks(elapsed_ms, kv_bytes, world, dev)
     value = bytes_all / (t_max * 1e-3) / 1e9
 
     # ---- KV memory after prefill and every step so far (the pages' memory
@@ -439,12 +450,7 @@ def run_native(args, wl):
     e2e = None
     if KE > 0:
         e2e = run_e2e(fd, cache, wl, stream, dev, W + K, WE, KE, row)
-        if world > 1:
-            import torch.distributed as dist
-            tt = torch.tensor([e2e["ms"], e2e["bytes"]], dtype=torch.float64, device=dev)
-            dist.all_reduce(tt[0:1], op=dist.ReduceOp.MAX)
-            dist.all_reduce(tt[1:2], op=dist.ReduceOp.SUM)
-            e2e["ms"], e2e["bytes"] = float(tt[0]), float(tt[1])
+        e2e["ms"], e2e["bytes"] = over_ranks(e2e["ms"], e2e["bytes"], world, dev)
 
     peak, peak_src = load_peaks()
     traffic, traffic_src = load_traffic(wl.name)
