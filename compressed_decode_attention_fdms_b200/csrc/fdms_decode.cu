@@ -409,12 +409,17 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
     const uint32_t nb = (uint32_t)(row1 - row0) * RB;
     const long long voff =
         (long long)((mt.rows >> 16) & kRing ? c.R : kBlockSlots) * RB;
-    mbar_arrive_expect_tx(&full[s], 2u * nb + (uint32_t)T::Q_BYTES);
+    // q only with a warp's first tile of a head: the tiles after it keep the
+    // head's q fragments in registers (each bulk copy costs issue time)
+    const bool with_q = ((mt.rows >> 16) & kFirst) != 0;
+    mbar_arrive_expect_tx(&full[s], 2u * nb + (with_q ? (uint32_t)T::Q_BYTES : 0u));
     bulk_g2s(kdst + row0 * RB, mt.ksrc, nb, &full[s]);
     bulk_g2s(vdst + row0 * RB, mt.ksrc + voff, nb, &full[s]);
-    const int b = mt.hidx / c.Hkv, h = mt.hidx % c.Hkv;
-    bulk_g2s(vdst + T::KV_BYTES, q + ((long long)b * c.Hq + (long long)h * G) * D, T::Q_BYTES,
-             &full[s]);
+    if (with_q) {
+      const int b = mt.hidx / c.Hkv, h = mt.hidx % c.Hkv;
+      bulk_g2s(vdst + T::KV_BYTES, q + ((long long)b * c.Hq + (long long)h * G) * D,
+               T::Q_BYTES, &full[s]);
+    }
   };
   // descriptors of tiles [k0, k0 + 32) into the warp's ring
   auto fill = [&](int k0) {
