@@ -677,25 +677,35 @@ k_append_small(CacheView c, int layer, int batch, const int32_t* __restrict__ n_
 
 // Decode steps proper: at most kStepVecs 16-byte input vectors per sequence
 // (max_new * D / 8 <= 32), one warp per (seq, kv head). Same result as
-// k_append_small; ordered for latency: the head's state, the call's rows and
-// keep bits and the head's FP8 scales are loaded together (they do not depend
-// on each other), then the keep bits and ring rows of the positions resolved
-// now and the store's partly filled block, again together; every write comes
-// after. A step costs two round trips to memory (three when the store needs a
-// new block) where the general order takes five. Resolutions larger than two
-// vectors per lane take the general path.
+// k_append_small; ordered for latency. A head's own state (lengths, FP8
+// scales, ring keep bits and rows, block table) is written only by appends to
+// its layer. When the host knows that the kernel just before this one on the
+// stream is not such an append (`state_early`), the last one has finished by
+// the time this grid starts: every kernel of this library calls the dependency
+// wait before it lets its successor start, except the combine, which is itself
+// started only after its split has waited for the append before it. The state,
+// and the ring rows of every position the call could resolve, are then read
+// before the wait, while the previous kernel still runs, and only the call's
+// own inputs are read after it: a step costs one round trip to memory after
+// the wait (two when the store needs a new block). Without `state_early` the
+// same loads come after the wait, in two round trips. Resolutions larger than
+// two vectors per lane take the general path.
 constexpr int kStepVecs = 32;
 
 template <bool FP8>
-__global__ void __launch_bounds__(kSmallWarps * 32)
+__global__ void __maxnreg__(128)   // room for the rows read early (the default target spills)
 k_append_step(CacheView c, int layer, int batch, const int32_t* __restrict__ n_new, int max_new,
               const uint16_t* __restrict__ k_in, const uint16_t* __restrict__ v_in,
-              const uint8_t* __restrict__ keep_in, const float* __restrict__ kv_scale) {
-  pdl_wait();                 // the previous kernel's writes are visible from here on
-  pdl_launch_dependents();
+              const uint8_t* __restrict__ keep_in, const float* __restrict__ kv_scale,
+              int state_early) {
+  if (!state_early) pdl_wait();   // the previous kernel's writes are visible from here on
   const int lane = threadIdx.x & 31;
   const int hid = blockIdx.x * kSmallWarps + (threadIdx.x >> 5);
-  if (hid >= batch * c.Hkv) return;
+  if (hid >= batch * c.Hkv) {
+    if (state_early) pdl_wait();
+    pdl_launch_dependents();
+    return;
+  }
   const int b = hid / c.Hkv, h = hid % c.Hkv;
   const long long hi = head_index(c, layer, b, h);
   const long long in_stride = (long long)c.Hkv * c.D;   // elements between tokens
@@ -703,12 +713,60 @@ k_append_step(CacheView c, int layer, int batch, const int32_t* __restrict__ n_n
   const uint16_t* v_rows = v_in + ((long long)b * max_new * c.Hkv + h) * c.D;
   const uint8_t* keep_rows = keep_in + (long long)b * max_new * c.Hkv + h;
   uint8_t* rkeep = c.ring_keep + hi * c.Rpad;
+  int32_t* bt = c.block_table + hi * c.max_blocks;
   const int VPR = c.D / 8;    // 16-byte input vectors per row
   constexpr unsigned kAll = 0xffffffffu;
+  constexpr int EV = FP8 ? 8 : 16;   // bytes of one vector in the cache
 
-  // ---- round trip 1: state, the call's rows (vector `lane`), keep bits, scales
-  const int m = n_new[b];
+  // ---- the head's state and the ring rows the call may resolve
   const int n0 = c.tok_n[hi], r0 = c.tok_r[hi], len0 = c.store_len[hi];
+  float sk = 1.0f, sv = 1.0f;
+  if constexpr (FP8) {
+    sk = c.head_scale[hi * 2];
+    sv = c.head_scale[hi * 2 + 1];
+  }
+  // positions resolved if the sequence brings max_new tokens: resolution is
+  // monotone in the count, so these cover what any count up to max_new resolves
+  const int nm = n0 + max_new;
+  const int res_m = (nm - c.W - r0 >= c.P) ? nm - c.W - r0 : 0;
+  const bool fast = res_m <= 32 && res_m * VPR <= 2 * 32;
+  int kring = 0;
+  uint4 rk[2], rv[2];
+  long long tail_blk = 0;
+#pragma unroll
+  for (int j = 0; j < 2; ++j) rk[j] = rv[j] = make_uint4(0u, 0u, 0u, 0u);
+  if (fast) {
+    if (lane < res_m && r0 + lane < n0) kring = rkeep[(r0 + lane) % c.R] != 0;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int i = lane + 32 * j;
+      if (i < res_m * VPR) {
+        const int p = r0 + i / VPR, vec = i % VPR;
+        if (p < n0) {
+          const int slot = p % c.R;
+          const uint8_t* ks = ring_k(c, hi) + (long long)slot * c.RB;
+          const uint8_t* vs = ring_v(c, hi) + (long long)slot * c.RB;
+          if constexpr (FP8) {
+            const uint2 a =
+                *reinterpret_cast<const uint2*>(ks + swz_byte(c.RB, false, slot, vec * EV));
+            const uint2 bb =
+                *reinterpret_cast<const uint2*>(vs + swz_byte(c.RB, true, slot, vec * EV));
+            rk[j] = make_uint4(a.x, a.y, 0u, 0u);
+            rv[j] = make_uint4(bb.x, bb.y, 0u, 0u);
+          } else {
+            rk[j] = *reinterpret_cast<const uint4*>(ks + swz_byte(c.RB, false, slot, vec * EV));
+            rv[j] = *reinterpret_cast<const uint4*>(vs + swz_byte(c.RB, true, slot, vec * EV));
+          }
+        }
+      }
+    }
+    if (len0 % kBlockSlots) tail_blk = bt[(len0 - 1) / kBlockSlots];   // partly filled block
+  }
+  if (state_early) pdl_wait();
+  pdl_launch_dependents();
+
+  // ---- the call's inputs: count, rows (vector `lane`), keep bits
+  const int m = n_new[b];
   uint4 xk = make_uint4(0u, 0u, 0u, 0u), xv = xk;
   if (lane < max_new * VPR) {
     const int t = lane / VPR, vec = lane % VPR;
@@ -716,11 +774,6 @@ k_append_step(CacheView c, int layer, int batch, const int32_t* __restrict__ n_n
     xv = *reinterpret_cast<const uint4*>(v_rows + t * in_stride + vec * 8);
   }
   const int knew = lane < max_new ? (keep_rows[(long long)lane * c.Hkv] != 0) : 0;
-  float sk = 1.0f, sv = 1.0f;
-  if constexpr (FP8) {
-    sk = c.head_scale[hi * 2];
-    sv = c.head_scale[hi * 2 + 1];
-  }
   if (m < 0 || m > max_new || (long long)n0 + m > c.max_seq_len) {
     if (lane == 0) latch_error(c.ctr, FDMS_ERR_DEVICE);
     return;
@@ -756,45 +809,17 @@ k_append_step(CacheView c, int layer, int batch, const int32_t* __restrict__ n_n
       }
     }
   }
-  const int nres = r1 - r0;
-  if (nres > 32 || nres * VPR > 2 * 32) {
+  const int nres = r1 - r0;   // <= res_m
+  if (!fast) {
     warp_resolve<FP8>(c, hi, lane, n0, r0, len0, n1, r1, sk, sv, k_rows, v_rows, keep_rows,
                       in_stride);
     return;
   }
 
-  // ---- round trip 2: keep bits and ring rows of positions r0 .. r1-1, the
-  // store's partly filled block
+  // keep bits of the resolved positions: ring bits read above, the call's own
   const int p_l = r0 + lane;
   const int knew_p = __shfl_sync(kAll, knew, (p_l - n0) & 31);
-  int kp = 0;
-  if (lane < nres) kp = p_l < n0 ? (rkeep[p_l % c.R] != 0) : knew_p;
-  constexpr int EV = FP8 ? 8 : 16;   // bytes of one vector in the cache
-  uint4 rk[2], rv[2];
-#pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    rk[j] = rv[j] = make_uint4(0u, 0u, 0u, 0u);
-    const int i = lane + 32 * j;
-    if (i < nres * VPR) {
-      const int p = r0 + i / VPR, vec = i % VPR;
-      if (p < n0) {
-        const int slot = p % c.R;
-        const uint8_t* ks = ring_k(c, hi) + (long long)slot * c.RB;
-        const uint8_t* vs = ring_v(c, hi) + (long long)slot * c.RB;
-        if constexpr (FP8) {
-          const uint2 a = *reinterpret_cast<const uint2*>(ks + swz_byte(c.RB, false, slot, vec * EV));
-          const uint2 bb = *reinterpret_cast<const uint2*>(vs + swz_byte(c.RB, true, slot, vec * EV));
-          rk[j] = make_uint4(a.x, a.y, 0u, 0u);
-          rv[j] = make_uint4(bb.x, bb.y, 0u, 0u);
-        } else {
-          rk[j] = *reinterpret_cast<const uint4*>(ks + swz_byte(c.RB, false, slot, vec * EV));
-          rv[j] = *reinterpret_cast<const uint4*>(vs + swz_byte(c.RB, true, slot, vec * EV));
-        }
-      }
-    }
-  }
-  int32_t* bt = c.block_table + hi * c.max_blocks;
-  const long long tail_blk = (len0 % kBlockSlots) ? bt[(len0 - 1) / kBlockSlots] : 0;
+  const int kp = lane < nres ? (p_l < n0 ? kring : knew_p) : 0;
   const unsigned ball = __ballot_sync(kAll, kp != 0);
   const int len1 = len0 + __popc(ball);
   const int nb0 = (len0 + kBlockSlots - 1) / kBlockSlots;
@@ -901,6 +926,10 @@ fdms_status fdms_launch_append(fdms_cache* cache, int layer, int batch, const in
   const uint16_t* kk = static_cast<const uint16_t*>(k);
   const uint16_t* vv = static_cast<const uint16_t*>(v);
   const float* sc = c.fp8 ? kv_scale : nullptr;
+  // the kernel before this one on the stream may still be writing this layer's
+  // state only if it is an append to the same layer
+  const int early = cache->last_append_layer != layer;
+  cache->last_append_layer = layer;
   cudaLaunchConfig_t cfg = {};
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -913,9 +942,9 @@ fdms_status fdms_launch_append(fdms_cache* cache, int layer, int batch, const in
     cfg.gridDim = dim3((unsigned)((batch * c.Hkv + kSmallWarps - 1) / kSmallWarps));
     cfg.blockDim = dim3(kSmallWarps * 32);
     e = c.fp8 ? cudaLaunchKernelEx(&cfg, k_append_step<true>, c, layer, batch, n_new, max_new,
-                                   kk, vv, keep, sc)
+                                   kk, vv, keep, sc, early)
               : cudaLaunchKernelEx(&cfg, k_append_step<false>, c, layer, batch, n_new, max_new,
-                                   kk, vv, keep, sc);
+                                   kk, vv, keep, sc, early);
   } else if (max_new <= kSmallMax) {
     cfg.gridDim = dim3((unsigned)((batch * c.Hkv + kSmallWarps - 1) / kSmallWarps));
     cfg.blockDim = dim3(kSmallWarps * 32);

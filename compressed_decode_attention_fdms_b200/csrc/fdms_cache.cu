@@ -130,6 +130,7 @@ fdms_status fdms_cache_create(const fdms_config* cfg, int device, void* stream,
   std::memset(c, 0, sizeof(*c));
   c->cfg = *cfg;
   c->device = device;
+  c->last_append_layer = -1;
   if (cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) {
     delete c;
     return FDMS_ERR_CUDA;

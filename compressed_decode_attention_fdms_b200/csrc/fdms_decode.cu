@@ -928,6 +928,7 @@ fdms_status launch_split_t(fdms_cache* cache, const DecodeWork& w, OutArgs oa, i
                                      static_cast<const uint16_t*>(q), n_ranges,
                                      1.0 / (double)n_ranges);
   if (e != cudaSuccess) return FDMS_ERR_CUDA;
+  cache->last_append_layer = -1;   // the split waits for every append queued before it
   cfg.gridDim = dim3((unsigned)(nh * Combine<T::D, T::G>::CPH));
   cfg.blockDim = dim3(Combine<T::D, T::G>::NT);
   cfg.dynamicSmemBytes = 0;

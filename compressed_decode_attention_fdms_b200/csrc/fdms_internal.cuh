@@ -210,6 +210,10 @@ struct fdms_cache {
   int decode_ctas;        // split grid used
   int ctas_per_sm;
   int ranges_per_cta;     // warps per split CTA (one unit range each)
+  // layer of the last append queued on this cache if no decode call was queued
+  // after it, else -1: an append to another layer may read its head state
+  // before its dependency wait (see k_append_step)
+  int last_append_layer;
 };
 
 // launchers (defined in their .cu files)

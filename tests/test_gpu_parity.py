@@ -339,3 +339,49 @@ def test_large_appends_span_chunks(kv_dtype, window, period):
         p.check_stats()
     finally:
         p.close()
+
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "fp8_e4m3"])
+@pytest.mark.parametrize("window,period", [(4, 1), (0, 1), (3, 5), (2, 40)])
+def test_step_appends_back_to_back(kv_dtype, window, period):
+    """Step-sized appends (one or two tokens) queued with no other work between
+    them: several in a row to one layer, each of which must see the state the
+    one before it left, and alternating between two layers with no decode
+    between them; one decode per layer at the end. Inputs are staged on the
+    device first, so the append kernels follow each other directly on the
+    stream."""
+    import compressed_decode_attention_fdms_b200 as fd
+    dev = torch.device("cuda", 0)
+    wl = wk.scaled(wk.get("tiny"), layers=2, batch=3, ctx=30, steps=0, window=window,
+                   period=period, kv_dtype=kv_dtype, rate=0.4)
+    p = Pair(wl, max_seq_len=96, oracle_capacity=96)
+    tol = TOL_BF16 if kv_dtype == "bf16" else TOL_FP8_MIRROR
+    try:
+        for layer in range(2):
+            p.append(layer, wk.prefill_inputs(wl, layer))
+        order = [0, 0, 0, 1, 0, 1, 1, 0, 1, 1, 1, 0, 0, 1, 0, 0]
+        staged = []
+        for i, layer in enumerate(order):
+            if i % 3 == 2:   # two tokens for some sequences, none for one
+                inp = wk.prefill_inputs(wk.scaled(wl, ctx=2), layer)
+                n = [2, 1, 0]
+                inp = {**inp, "n_new": torch.tensor(n[i % 3:] + n[:i % 3], dtype=torch.int32)}
+            else:
+                inp = wk.decode_inputs(wl, layer, i)
+            d = {k: (t.to(dev).contiguous() if torch.is_tensor(t) else t) for k, t in inp.items()}
+            staged.append((layer, inp, d))
+        torch.cuda.synchronize()
+        for layer, _, d in staged:
+            fd.fdms_append_evict(p.cache, layer, wl.batch, d["n_new"].to(torch.int32),
+                                 d["max_new"], d["k"], d["v"], d["keep"])
+        torch.cuda.synchronize()
+        for layer, inp, _ in staged:
+            p.oc.append(layer, inp["n_new"].to(torch.int32).numpy(), bits(inp["k"]),
+                        bits(inp["v"]), inp["keep"].numpy())
+        for layer in range(2):
+            p.check_heads(layer)
+            q = wk.decode_query(wl, layer, 99)
+            assert _max_err(p.decode(layer, q), p.oracle_out(layer, q)) <= tol
+        p.check_stats()
+    finally:
+        p.close()
