@@ -58,25 +58,37 @@ __device__ __forceinline__ float div_rn(float x, float s, float r) {
   return isfinite(q1) ? q1 : q;
 }
 
+// The reciprocal div_rn takes: RN(1 / scale), or 0 where 1 / scale might
+// overflow (scale < 1e-30), which sends quantise8 to plain division. Computed
+// once per scale, not per vector.
+__device__ __forceinline__ float quant_recip(float scale) {
+  return scale < 1.0e-30f ? 0.f : __frcp_rn(scale);
+}
+
 // 8 bf16 (one 16-byte vector) / scale -> 8 E4M3 codes; counts clipped values.
-__device__ __forceinline__ uint2 quantise8(uint4 x, float scale, unsigned& sat) {
+// r = quant_recip(scale).
+__device__ __forceinline__ uint2 quantise8(uint4 x, float scale, float r, unsigned& sat) {
   const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-  const bool tiny = scale < 1.0e-30f;   // 1 / scale might overflow: plain division
-  const float r = tiny ? 0.f : __frcp_rn(scale);
-  uint32_t out[2];
+  float f[8];
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const float x4[4] = {bf16lo_to_f32(w[2 * j]), bf16hi_to_f32(w[2 * j]),
-                         bf16lo_to_f32(w[2 * j + 1]), bf16hi_to_f32(w[2 * j + 1])};
-    float f[4];
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      f[t] = tiny ? __fdiv_rn(x4[t], scale) : div_rn(x4[t], scale, r);
-      sat += fabsf(f[t]) > 448.0f ? 1u : 0u;
-    }
-    out[j] = (uint32_t)f32x2_to_e4m3x2(f[0], f[1]) | ((uint32_t)f32x2_to_e4m3x2(f[2], f[3]) << 16);
+  for (int j = 0; j < 4; ++j) {
+    f[2 * j] = bf16lo_to_f32(w[j]);
+    f[2 * j + 1] = bf16hi_to_f32(w[j]);
   }
-  return make_uint2(out[0], out[1]);
+  if (r != 0.f) {   // one branch for the vector: the common path has no division
+#pragma unroll
+    for (int t = 0; t < 8; ++t) f[t] = div_rn(f[t], scale, r);
+  } else {
+#pragma unroll
+    for (int t = 0; t < 8; ++t) f[t] = __fdiv_rn(f[t], scale);
+  }
+#pragma unroll
+  for (int t = 0; t < 8; ++t) sat += fabsf(f[t]) > 448.0f ? 1u : 0u;
+  const uint32_t lo = (uint32_t)f32x2_to_e4m3x2(f[0], f[1]) |
+                      ((uint32_t)f32x2_to_e4m3x2(f[2], f[3]) << 16);
+  const uint32_t hi = (uint32_t)f32x2_to_e4m3x2(f[4], f[5]) |
+                      ((uint32_t)f32x2_to_e4m3x2(f[6], f[7]) << 16);
+  return make_uint2(lo, hi);
 }
 
 // Copy one 16-byte vector `vec` (8 bf16 values) of an input row into row `row`
@@ -84,12 +96,12 @@ __device__ __forceinline__ uint2 quantise8(uint4 x, float scale, unsigned& sat) 
 // place in the page's chunk permutation.
 template <bool FP8>
 __device__ __forceinline__ void put_input_vec(uint8_t* dst_row, const uint16_t* src_row, int vec,
-                                              float scale, unsigned& sat, int RB, bool is_v,
-                                              int row) {
+                                              float scale, float r, unsigned& sat, int RB,
+                                              bool is_v, int row) {
   const uint4 x = *reinterpret_cast<const uint4*>(src_row + vec * 8);
   if constexpr (FP8) {
     *reinterpret_cast<uint2*>(dst_row + swz_byte(RB, is_v, row, vec * 8)) =
-        quantise8(x, scale, sat);
+        quantise8(x, scale, r, sat);
   } else {
     *reinterpret_cast<uint4*>(dst_row + swz_byte(RB, is_v, row, vec * 16)) = x;
   }
@@ -338,6 +350,7 @@ k_bulk_write(CacheView c, AppendWork aw, BulkIn in) {
   if (hd[kHdrStatus] != kBulkGo) return;
   const int n0 = hd[kHdrN0], r0 = hd[kHdrR0], len0 = hd[kHdrLen0], r1 = hd[kHdrR1];
   const float sk = __int_as_float(hd[kHdrSk]), sv = __int_as_float(hd[kHdrSv]);
+  const float qk = FP8 ? quant_recip(sk) : 0.f, qv = FP8 ? quant_recip(sv) : 0.f;
   const int p_lo = r0 + ch * kChunkPositions, p_hi = min(r1, p_lo + kChunkPositions);
   if (p_lo >= p_hi) return;
   const int b = hid / c.Hkv, h = hid % c.Hkv;
@@ -414,8 +427,10 @@ k_bulk_write(CacheView c, AppendWork aw, BulkIn in) {
       uint8_t* kd = block_k(c, blk) + (long long)row * c.RB;
       uint8_t* vd = block_v(c, blk) + (long long)row * c.RB;
       if constexpr (FP8) {
-        const uint2 ok = src < n0 ? make_uint2(xk[u].x, xk[u].y) : quantise8(xk[u], sk, sat);
-        const uint2 ov = src < n0 ? make_uint2(xv[u].x, xv[u].y) : quantise8(xv[u], sv, sat);
+        const uint2 ok =
+            src < n0 ? make_uint2(xk[u].x, xk[u].y) : quantise8(xk[u], sk, qk, sat);
+        const uint2 ov =
+            src < n0 ? make_uint2(xv[u].x, xv[u].y) : quantise8(xv[u], sv, qv, sat);
         *reinterpret_cast<uint2*>(kd + swz_byte(c.RB, false, row, vec * 8)) = ok;
         *reinterpret_cast<uint2*>(vd + swz_byte(c.RB, true, row, vec * 8)) = ov;
       } else {
@@ -441,6 +456,7 @@ k_bulk_ring(CacheView c, AppendWork aw, BulkIn in) {
   if (hd[kHdrStatus] != kBulkGo) return;
   const int n0 = hd[kHdrN0], n1 = hd[kHdrN1], r1 = hd[kHdrR1];
   const float sk = __int_as_float(hd[kHdrSk]), sv = __int_as_float(hd[kHdrSv]);
+  const float qk = FP8 ? quant_recip(sk) : 0.f, qv = FP8 ? quant_recip(sv) : 0.f;
   const int b = hid / c.Hkv, h = hid % c.Hkv;
   const long long hi = head_index(c, in.layer, b, h);
   const long long in_stride = (long long)c.Hkv * c.D;
@@ -477,9 +493,9 @@ k_bulk_ring(CacheView c, AppendWork aw, BulkIn in) {
       uint8_t* vd = ring_v(c, hi) + (long long)slot * c.RB;
       if constexpr (FP8) {
         *reinterpret_cast<uint2*>(kd + swz_byte(c.RB, false, slot, vec * 8)) =
-            quantise8(xk[u], sk, sat);
+            quantise8(xk[u], sk, qk, sat);
         *reinterpret_cast<uint2*>(vd + swz_byte(c.RB, true, slot, vec * 8)) =
-            quantise8(xv[u], sv, sat);
+            quantise8(xv[u], sv, qv, sat);
       } else {
         *reinterpret_cast<uint4*>(kd + swz_byte(c.RB, false, slot, vec * 16)) = xk[u];
         *reinterpret_cast<uint4*>(vd + swz_byte(c.RB, true, slot, vec * 16)) = xv[u];
@@ -506,6 +522,7 @@ __device__ void warp_resolve(const CacheView& c, long long hi, int lane, int n0,
                              const uint8_t* keep_rows, long long in_stride) {
   uint8_t* rkeep = c.ring_keep + hi * c.Rpad;
   const int VPR = c.D / 8;    // 16-byte input vectors per row
+  const float qk = FP8 ? quant_recip(sk) : 0.f, qv = FP8 ? quant_recip(sv) : 0.f;
   auto keep_of = [&](int p) -> int {
     return p < n0 ? (rkeep[p % c.R] != 0) : (keep_rows[(long long)(p - n0) * c.Hkv] != 0);
   };
@@ -565,8 +582,8 @@ __device__ void warp_resolve(const CacheView& c, long long hi, int lane, int n0,
         move_vec<FP8>(vd, row, ring_v(c, hi) + (long long)slot * c.RB, slot, vec, c.RB, true);
       } else {
         const long long t = src - n0;
-        put_input_vec<FP8>(kd, k_rows + t * in_stride, vec, sk, sat, c.RB, false, row);
-        put_input_vec<FP8>(vd, v_rows + t * in_stride, vec, sv, sat, c.RB, true, row);
+        put_input_vec<FP8>(kd, k_rows + t * in_stride, vec, sk, qk, sat, c.RB, false, row);
+        put_input_vec<FP8>(vd, v_rows + t * in_stride, vec, sv, qv, sat, c.RB, true, row);
       }
       if (vec == 0) c.blk_pos[blk * kBlockSlots + row] = src;
     }
@@ -580,9 +597,9 @@ __device__ void warp_resolve(const CacheView& c, long long hi, int lane, int n0,
     const long long t = p - n0;
     const int slot = p % c.R;
     put_input_vec<FP8>(ring_k(c, hi) + (long long)slot * c.RB, k_rows + t * in_stride, vec, sk,
-                       sat, c.RB, false, slot);
+                       qk, sat, c.RB, false, slot);
     put_input_vec<FP8>(ring_v(c, hi) + (long long)slot * c.RB, v_rows + t * in_stride, vec, sv,
-                       sat, c.RB, true, slot);
+                       qv, sat, c.RB, true, slot);
     if (vec == 0) rkeep[slot] = keep_rows[t * c.Hkv] ? 1 : 0;
   }
   if constexpr (FP8) {
@@ -720,10 +737,12 @@ k_append_step(CacheView c, int layer, int batch, const int32_t* __restrict__ n_n
 
   // ---- the head's state and the ring rows the call may resolve
   const int n0 = c.tok_n[hi], r0 = c.tok_r[hi], len0 = c.store_len[hi];
-  float sk = 1.0f, sv = 1.0f;
+  float sk = 1.0f, sv = 1.0f, qk = 0.f, qv = 0.f;
   if constexpr (FP8) {
     sk = c.head_scale[hi * 2];
     sv = c.head_scale[hi * 2 + 1];
+    qk = quant_recip(sk);
+    qv = quant_recip(sv);
   }
   // positions resolved if the sequence brings max_new tokens: resolution is
   // monotone in the count, so these cover what any count up to max_new resolves
@@ -807,6 +826,8 @@ k_append_step(CacheView c, int layer, int batch, const int32_t* __restrict__ n_n
         c.head_scale[hi * 2] = sk;
         c.head_scale[hi * 2 + 1] = sv;
       }
+      qk = quant_recip(sk);
+      qv = quant_recip(sv);
     }
   }
   const int nres = r1 - r0;   // <= res_m
@@ -873,8 +894,8 @@ k_append_step(CacheView c, int layer, int batch, const int32_t* __restrict__ n_n
       }
     } else {   // a token of this call resolved at once (window shorter than the call)
       const long long t = p - n0;
-      put_input_vec<FP8>(kd, k_rows + t * in_stride, vec, sk, sat, c.RB, false, row);
-      put_input_vec<FP8>(vd, v_rows + t * in_stride, vec, sv, sat, c.RB, true, row);
+      put_input_vec<FP8>(kd, k_rows + t * in_stride, vec, sk, qk, sat, c.RB, false, row);
+      put_input_vec<FP8>(vd, v_rows + t * in_stride, vec, sv, qv, sat, c.RB, true, row);
     }
     if (vec == 0) c.blk_pos[blk * kBlockSlots + row] = p;
   }
@@ -892,9 +913,9 @@ k_append_step(CacheView c, int layer, int batch, const int32_t* __restrict__ n_n
       uint8_t* vd = ring_v(c, hi) + (long long)slot * c.RB;
       if constexpr (FP8) {
         *reinterpret_cast<uint2*>(kd + swz_byte(c.RB, false, slot, vec * EV)) =
-            quantise8(xk, sk, sat);
+            quantise8(xk, sk, qk, sat);
         *reinterpret_cast<uint2*>(vd + swz_byte(c.RB, true, slot, vec * EV)) =
-            quantise8(xv, sv, sat);
+            quantise8(xv, sv, qv, sat);
       } else {
         *reinterpret_cast<uint4*>(kd + swz_byte(c.RB, false, slot, vec * EV)) = xk;
         *reinterpret_cast<uint4*>(vd + swz_byte(c.RB, true, slot, vec * EV)) = xv;
