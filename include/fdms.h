@@ -43,6 +43,14 @@
  * streams) and keeps them alive until the work queued on the stream is done.
  * No call allocates device memory after creation.
  *
+ * Ordering and threads: queue the calls on one cache in program order on one
+ * stream, or order streams with events. Consecutive kernels on a stream overlap
+ * through programmatic dependent launch; each kernel reads data its
+ * predecessor writes only after waiting for it. A cache keeps host-side state
+ * (which layer the last append went to, which decides how early the next append
+ * may read its head state), so calls on one cache must not run concurrently
+ * from several host threads; different caches are independent.
+ *
  * Errors: every call validates its arguments on the host and returns a status
  * before queuing any work. Calls that queue kernels are asynchronous; errors
  * found by the device (pool exhausted, sequence too long) are latched into a
