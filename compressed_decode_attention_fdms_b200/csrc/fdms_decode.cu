@@ -333,8 +333,10 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
       if (oa.lse && i % D == 0) oa.lse[(long long)b * c.Hq + kh * G + i / D] = -INFINITY;
     }
   }
-  const long long v_range = (long long)blockIdx.x * NCW + warp;
-  if ((long long)blockIdx.x * NCW * S >= P) return;
+  // Range v goes to warp v / gridDim.x of CTA v % gridDim.x: when fewer
+  // ranges than warps hold tiles, the busy ones are spread over every SM.
+  const long long v_range = (long long)warp * gridDim.x + blockIdx.x;
+  if ((long long)blockIdx.x * S >= P) return;
 
   // ---- this warp's tiles [gp0, gp0 + nt) and the heads h_gs .. h_ge they
   // belong to (the number of heads h >= 1 with page_off[h] <= page)
