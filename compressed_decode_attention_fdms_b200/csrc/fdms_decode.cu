@@ -218,8 +218,7 @@ __global__ void __launch_bounds__(T::NT, 1)
 k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
                const uint16_t* __restrict__ q, int n_ranges, double inv_ranges) {
   constexpr int D = T::D, G = T::G, RB = T::RB, TR = T::TR, NSTAGE = T::NSTAGE,
-                NCW = T::NCW, SPW = T::SPW, NJ = T::NJ, NU = T::NU, KS = T::KS, MT = T::MT,
-                NMR = T::NMR;
+                SPW = T::SPW, NJ = T::NJ, NU = T::NU, KS = T::KS, MT = T::MT, NMR = T::NMR;
   constexpr bool FP8 = T::FP8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 127) & ~(uintptr_t)127);
