@@ -37,6 +37,15 @@ resolved. Per kv head h, every token j carries keep[j] in {0, 1}.
   caller's values. Every store block and the ring use that scale, so a
   per-block scale field holds the same number in every block of a head.
 * Stored value of a slot: the bf16 value, or E4M3 value * scale (exact in fp64).
+* Second FP8 reading ("fp8_e4m3_block"). The configs' "one fp32 scale per
+  (layer, kv head, 64-token block)" can also mean a scale computed from each
+  block's own values. Store slot i (in store order) belongs to block i // 64. A
+  block is sealed once it holds 64 survivors; its K scale and its V scale are
+  max(amax over the block's 64 K (resp. V) values, 2^-126) / 448, and its rows
+  are stored as E4M3 with those scales (the same quotient and rounding rule as
+  above). Until then they stay in staging as bf16, as do the ring's rows, so
+  the store's partly filled last block and the ring decode exactly. A sealed
+  block never changes.
 * Decode happens after the token of the step is appended, so it attends to
   itself.
 * FP8 saturation counter: the number of elements written into the cache (store
@@ -69,11 +78,12 @@ class OracleCache:
     def __init__(self, layers, batch, q_heads, kv_heads, head_dim, window, period,
                  kv_dtype="bf16", capacity=1024, softmax_scale=None):
         assert q_heads % kv_heads == 0
-        assert kv_dtype in ("bf16", "fp8_e4m3")
+        assert kv_dtype in ("bf16", "fp8_e4m3", "fp8_e4m3_block")
         self.L, self.B, self.Hq, self.Hkv, self.D = layers, batch, q_heads, kv_heads, head_dim
         self.W, self.P = window, period
         self.kv_dtype = kv_dtype
         self.elt = 2 if kv_dtype == "bf16" else 1
+        self.block = kv_dtype == "fp8_e4m3_block"
         self.cap = capacity
         self.scale = (1.0 / np.sqrt(head_dim)) if softmax_scale is None else float(softmax_scale)
         shape = (layers, batch, capacity, kv_heads, head_dim)
@@ -138,7 +148,10 @@ class OracleCache:
 
     # ----------------------------------------------------------------- views
     def _payload(self, layer, b, h, pos):
-        if self.kv_dtype == "bf16":
+        """Stored payload: bf16 bits, or E4M3 codes (first FP8 reading). The
+        second FP8 reading returns the bf16 bits here; its sealed blocks' codes
+        and scales come from ``sealed_blocks``."""
+        if self.kv_dtype == "bf16" or self.block:
             return self.k[layer, b, pos, h], self.v[layer, b, pos, h]
         return self.kq[layer, b, pos, h], self.vq[layer, b, pos, h]
 
@@ -156,6 +169,35 @@ class OracleCache:
         kp, vp = self._payload(layer, b, h, pos)
         return pos, kp, vp, self.keep[layer, b, r:n, h].copy()
 
+    BLOCK = 64
+
+    def sealed_blocks(self, layer, b, h):
+        """Second FP8 reading: the sealed store blocks of one head.
+
+        Returns (positions int32 [nb*64], K codes uint8 [nb*64][D], V codes,
+        scales float32 [nb][2] (K, V), clipped count), nb = store_len // 64.
+        Built from the set definition on every call: a block's content depends
+        only on its 64 positions, so sealing is final by construction.
+        """
+        r = int(self.r[layer, b])
+        pos = np.flatnonzero(self.keep[layer, b, :r, h])
+        nb = len(pos) // self.BLOCK
+        pos = pos[:nb * self.BLOCK]
+        kq = np.zeros((len(pos), self.D), np.uint8)
+        vq = np.zeros((len(pos), self.D), np.uint8)
+        scales = np.zeros((nb, 2), np.float32)
+        clipped = 0
+        for j in range(nb):
+            rows = pos[j * self.BLOCK:(j + 1) * self.BLOCK]
+            kb, vb = self.k[layer, b, rows, h], self.v[layer, b, rows, h]
+            sk = nm.calibration_scale(np.max(np.abs(nm.bf16_to_f32(kb))))
+            sv = nm.calibration_scale(np.max(np.abs(nm.bf16_to_f32(vb))))
+            kq[j * self.BLOCK:(j + 1) * self.BLOCK], c1 = nm.quantise_e4m3(kb, sk)
+            vq[j * self.BLOCK:(j + 1) * self.BLOCK], c2 = nm.quantise_e4m3(vb, sv)
+            scales[j] = (sk, sv)
+            clipped += c1 + c2
+        return pos.astype(np.int32), kq, vq, scales, clipped
+
     def visible(self, layer, b, h):
         """Bool mask over positions 0..n-1: recent window or kept."""
         n = int(self.n[layer, b])
@@ -171,6 +213,18 @@ class OracleCache:
         if self.kv_dtype == "bf16" or mode == "true":
             return (nm.bf16_to_f64(self.k[layer, b, pos, h]),
                     nm.bf16_to_f64(self.v[layer, b, pos, h]))
+        if self.block:   # sealed rows dequantised, staged and ring rows exact
+            kk = nm.bf16_to_f64(self.k[layer, b, pos, h])
+            vv = nm.bf16_to_f64(self.v[layer, b, pos, h])
+            spos, kq, vq, scales, _ = self.sealed_blocks(layer, b, h)
+            where = {int(p): i for i, p in enumerate(spos)}
+            for out_i, p in enumerate(np.asarray(pos).reshape(-1)):
+                i = where.get(int(p))
+                if i is not None:
+                    sk, sv = scales[i // self.BLOCK]
+                    kk[out_i] = nm.e4m3_to_f64(kq[i]) * np.float64(sk)
+                    vv[out_i] = nm.e4m3_to_f64(vq[i]) * np.float64(sv)
+            return kk, vv
         sk, sv = self.kv_scale[layer, b, h]
         return (nm.e4m3_to_f64(self.kq[layer, b, pos, h]) * np.float64(sk),
                 nm.e4m3_to_f64(self.vq[layer, b, pos, h]) * np.float64(sv))
@@ -208,11 +262,23 @@ class OracleCache:
         slots_ring = int(np.sum(self.n - self.r)) * self.Hkv
         tokens = int(np.sum(self.n))
         row = 2 * self.D * self.elt
+        compact = (slots_store + slots_ring) * row
+        saturations = int(self.saturations)
+        if self.block:   # sealed slots in E4M3, staged and ring slots in bf16
+            sealed = 0
+            saturations = 0
+            for layer in range(self.L):
+                for b in range(self.B):
+                    for h in range(self.Hkv):
+                        spos, _, _, _, clipped = self.sealed_blocks(layer, b, h)
+                        sealed += len(spos)
+                        saturations += clipped
+            compact = sealed * row + (slots_store - sealed + slots_ring) * 2 * row
         return {
             "tokens_appended": tokens,
             "slots_store": slots_store,
             "slots_ring": slots_ring,
-            "bytes_compact": (slots_store + slots_ring) * row,
+            "bytes_compact": compact,
             "bytes_dense_equiv": dense_kv_bytes(tokens, 1, self.Hkv, self.D, self.elt),
-            "fp8_saturations": int(self.saturations),
+            "fp8_saturations": saturations,
         }
