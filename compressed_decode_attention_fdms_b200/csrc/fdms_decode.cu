@@ -313,7 +313,7 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   }
   const long long total = head_off[NH];
   const int P = page_off[NH];   // tiles of the call
-  // Warp v reads tiles [v S, (v + 1) S), S = ceil(P / ranges): a tile costs
+  // Range v holds tiles [v S, (v + 1) S), S = ceil(P / ranges): a tile costs
   // the same compute full or not, so whole tiles are what gets balanced. The
   // quotient is an fp64 estimate made exact by integer correction.
   const int S = tiles_per_warp(P, n_ranges, inv_ranges);
@@ -989,7 +989,7 @@ fdms_status fdms_decode_setup(fdms_cache* cache) {
   const CacheView& c = cache->view;
   DecodeWork& w = cache->work;
   w.max_ctas = ctas;
-  w.max_parts = ctas * cache->ranges_per_cta + c.Bmax * c.Hkv;   // warp v, head h: v + h
+  w.max_parts = ctas * cache->ranges_per_cta + c.Bmax * c.Hkv;   // range v, head h: v + h
   void* p = nullptr;
   auto take = [&](size_t bytes) -> void* {
     if (cudaMalloc(&p, bytes) != cudaSuccess) return nullptr;
