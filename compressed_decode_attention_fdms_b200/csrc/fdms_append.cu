@@ -1016,9 +1016,7 @@ fdms_status fdms_append_setup(fdms_cache* cache) {
   const size_t heads = (size_t)c.Bmax * c.Hkv;
   void* p = nullptr;
   auto take = [&](size_t bytes) -> void* {
-    if (cudaMalloc(&p, bytes) != cudaSuccess) return nullptr;
-    cache->allocs[cache->nallocs++] = p;
-    cache->bytes_reserved += bytes;
+    if (cudaMalloc(&p, bytes) != cudaSuccess || !fdms_track(cache, p, bytes)) return nullptr;
     if (cudaMemset(p, 0, bytes) != cudaSuccess) return nullptr;
     return p;
   };

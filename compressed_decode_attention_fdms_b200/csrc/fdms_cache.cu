@@ -39,8 +39,7 @@ cudaError_t alloc(fdms_cache* c, T** p, size_t bytes) {
   void* q = nullptr;
   cudaError_t e = cudaMalloc(&q, bytes);
   if (e != cudaSuccess) return e;
-  c->allocs[c->nallocs++] = q;
-  c->bytes_reserved += bytes;
+  if (!fdms_track(c, q, bytes)) return cudaErrorMemoryAllocation;
   *p = static_cast<T*>(q);
   return cudaSuccess;
 }

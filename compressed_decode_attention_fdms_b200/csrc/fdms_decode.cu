@@ -992,9 +992,7 @@ fdms_status fdms_decode_setup(fdms_cache* cache) {
   w.max_parts = ctas * cache->ranges_per_cta + c.Bmax * c.Hkv;   // range v, head h: v + h
   void* p = nullptr;
   auto take = [&](size_t bytes) -> void* {
-    if (cudaMalloc(&p, bytes) != cudaSuccess) return nullptr;
-    cache->allocs[cache->nallocs++] = p;
-    cache->bytes_reserved += bytes;
+    if (cudaMalloc(&p, bytes) != cudaSuccess || !fdms_track(cache, p, bytes)) return nullptr;
     return p;
   };
   w.part_o = static_cast<float*>(take((size_t)w.max_parts * c.G * c.D * sizeof(float)));

@@ -216,6 +216,18 @@ struct fdms_cache {
   int last_append_layer;
 };
 
+// Record a device allocation of the cache (freed at destroy). Frees `p` and
+// returns false when the table is full.
+inline bool fdms_track(fdms_cache* c, void* p, size_t bytes) {
+  if (c->nallocs >= (int)(sizeof(c->allocs) / sizeof(c->allocs[0]))) {
+    cudaFree(p);
+    return false;
+  }
+  c->allocs[c->nallocs++] = p;
+  c->bytes_reserved += bytes;
+  return true;
+}
+
 // launchers (defined in their .cu files)
 fdms_status fdms_launch_append(fdms_cache* c, int layer, int batch, const int32_t* n_new,
                                int max_new, const void* k, const void* v, const uint8_t* keep,
