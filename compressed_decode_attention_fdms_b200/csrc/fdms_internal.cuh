@@ -178,7 +178,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
   return ok != 0;
 }
-// global -> shared bulk copy (no multicast), completion counted on `bar`
+// global -> shared bulk copy into this CTA's own shared memory, completion counted on `bar`
 __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src, uint32_t bytes,
                                          uint64_t* bar) {
   asm volatile(
