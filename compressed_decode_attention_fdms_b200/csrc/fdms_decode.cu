@@ -54,6 +54,10 @@
 namespace fdms {
 namespace {
 
+#ifndef FDMS_CLUSTER_DECODE
+#define FDMS_CLUSTER_DECODE 1
+#endif
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
 
@@ -109,6 +113,15 @@ struct Dec {
     return 128 + OFF_HEADS + (size_t)(nh + 1) * 8 + (size_t)(nh + 1) * 4 +
            (size_t)nh * 4 * 3 + (size_t)nh * 8 + 64;
   }
+  // per-head (cluster) mode: a merge area after the head arrays, one slot of
+  // (o [G][D], m [G], l [G]) per warp and one for the CTA
+  static constexpr int SLOT = G * D + 2 * G;   // floats
+  __host__ __device__ static size_t merge_off(int nh) {
+    return ((size_t)OFF_HEADS + (size_t)(nh + 1) * 12 + (size_t)nh * 20 + 15) / 16 * 16;
+  }
+  static size_t smem_bytes_cluster(int nh) {
+    return 128 + merge_off(nh) + (size_t)(NCW + 1) * SLOT * 4 + 64;
+  }
 
   // unpermuted 16-byte K chunk i (0 .. KCPT-1) of lane column t
   __device__ static int kchunk(int t, int i) { return RB == 256 ? t + 4 * i : KCPT * t + i; }
@@ -162,6 +175,23 @@ __device__ __forceinline__ int tiles_per_warp(int P, int n_ranges, double inv) {
   return S > 1 ? S : 1;
 }
 
+// ------------------------------------------------------------ cluster helpers
+// All threads of every CTA of the cluster arrive, then wait: shared-memory
+// writes before it are visible to every CTA of the cluster after it.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// fp32 at the same shared-memory offset as `local` in CTA `rank` of the cluster
+__device__ __forceinline__ float ld_cluster_f32(const float* local, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+               : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
+
 // ------------------------------------------------------------- MMA helpers
 template <bool F16>
 __device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2,
@@ -213,7 +243,13 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return r;
 }
 
-template <class T>
+// CS = 0: one plan over every head of the call, cut into equal tile ranges,
+// partials merged by k_decode_combine. CS > 0 (calls with few heads): one
+// cluster of CS CTAs per head; the CTAs split the head's tiles, each merges its
+// warps' partials in shared memory, and the cluster merges the CTAs' partials
+// through distributed shared memory and writes the output: no global plan, no
+// workspace, no combine kernel.
+template <class T, int CS>
 __global__ void __launch_bounds__(T::NT, 1)
 k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
                const uint16_t* __restrict__ q, int n_ranges, double inv_ranges) {
@@ -268,7 +304,23 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   pdl_launch_dependents();
 
   // ---- units and pages of every head of the call; exclusive prefix
-  {
+  const int hsel = CS > 0 ? (int)(blockIdx.x / (CS > 0 ? CS : 1)) : 0;   // cluster mode: its head
+  if constexpr (CS > 0) {
+    if (tid == 0) {
+      const long long hi = hi0 + hsel;
+      const int len = c.store_len[hi], n = c.tok_n[hi], r = c.tok_r[hi];
+      s_len[hsel] = len;
+      s_n[hsel] = n;
+      s_r[hsel] = r;
+      s_hscale[2 * hsel] = FP8 ? c.head_scale[hi * 2] : 1.0f;
+      s_hscale[2 * hsel + 1] = FP8 ? c.head_scale[hi * 2 + 1] : 1.0f;
+      head_off[hsel] = 0;
+      head_off[hsel + 1] = len + (n - r);
+      page_off[hsel] = 0;
+      page_off[hsel + 1] = head_tiles<TR>(len, n, r);
+    }
+    __syncthreads();
+  } else {
     const int per = (NH + T::NT - 1) / T::NT;
     const int h0 = tid * per, h1 = min(NH, h0 + per);
     long long su = 0;
@@ -311,6 +363,28 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
     }
     __syncthreads();
   }
+  int gp0 = 0, nt = 0, h_gs = 0, h_ge = 0;
+  long long v_range = 0;
+  float* mslot = reinterpret_cast<float*>(smem + T::merge_off(NH));   // cluster mode
+  if constexpr (CS > 0) {
+    // the head's tiles, split evenly over the cluster's CTAs, then over warps
+    const int P = page_off[hsel + 1];
+    const int crank = (int)(blockIdx.x % CS);
+    const int per_c = (P + CS - 1) / CS;
+    const int c0 = min(P, crank * per_c), c1 = min(P, c0 + per_c);
+    const int per_w = (c1 - c0 + T::NCW - 1) / T::NCW;
+    gp0 = min(c1, c0 + warp * per_w);
+    nt = min(c1, gp0 + per_w) - gp0;
+    h_gs = h_ge = hsel;
+    if (crank == 0 && tid == 0) {
+      atomicAdd(&c.ctr->slots_decoded, (unsigned long long)head_off[hsel + 1]);
+      if (blockIdx.x == 0) atomicAdd(&c.ctr->decode_calls, 1ull);
+    }
+    if (lane < G) {   // an empty partial until the warp's last tile replaces it
+      mslot[warp * T::SLOT + G * D + lane] = -INFINITY;
+      mslot[warp * T::SLOT + G * D + G + lane] = 0.f;
+    }
+  } else {
   const long long total = head_off[NH];
   const int P = page_off[NH];   // tiles of the call
   // Range v holds tiles [v S, (v + 1) S), S = ceil(P / ranges): a tile costs
@@ -334,14 +408,13 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   }
   // Range v goes to warp v / gridDim.x of CTA v % gridDim.x: when fewer
   // ranges than warps hold tiles, the busy ones are spread over every SM.
-  const long long v_range = (long long)warp * gridDim.x + blockIdx.x;
+  v_range = (long long)warp * gridDim.x + blockIdx.x;
   if ((long long)blockIdx.x * S >= P) return;
 
   // ---- this warp's tiles [gp0, gp0 + nt) and the heads h_gs .. h_ge they
   // belong to (the number of heads h >= 1 with page_off[h] <= page)
-  const int gp0 = (int)min(v_range * S, (long long)P);
-  const int nt = min(gp0 + S, P) - gp0;
-  int h_gs = 0, h_ge = 0;
+  gp0 = (int)min(v_range * S, (long long)P);
+  nt = min(gp0 + S, P) - gp0;
   if (nt > 0) {
     for (int base = 1; base < NH; base += 32) {
       const int h = base + lane;
@@ -349,6 +422,7 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
       h_gs += __popc(__ballot_sync(0xffffffffu, po <= gp0));
       h_ge += __popc(__ballot_sync(0xffffffffu, po <= gp0 + nt - 1));
     }
+  }
   }
 
   // descriptor of this warp's tile k (one lane per tile)
@@ -737,7 +811,24 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
       l += __shfl_xor_sync(0xffffffffu, l, 2);
       const int hidx = mt.hidx;
       const int kb = hidx / c.Hkv, kh = hidx % c.Hkv;
-      if (page_off[hidx] >= gp0 && page_off[hidx + 1] <= gp0 + nt) {
+      if constexpr (CS > 0) {   // the warp's partial, for the CTA's merge
+        float* po = mslot + warp * T::SLOT;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int h = 2 * t + e;
+          if (h < G) {
+#pragma unroll
+            for (int i = 0; i < MT; ++i) {
+              po[h * D + T::vdim(g, i, 0)] = oacc[i][e] * mt.vhead;
+              po[h * D + T::vdim(g, i, 1)] = oacc[i][2 + e] * mt.vhead;
+            }
+          }
+        }
+        if (t == 0 && g < G) {
+          po[G * D + g] = m_run;
+          po[G * D + G + g] = l;
+        }
+      } else if (page_off[hidx] >= gp0 && page_off[hidx + 1] <= gp0 + nt) {
         // the whole head lies in this warp's range: write the output now
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
@@ -784,6 +875,67 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
         }
       }
     }
+  }
+
+  if constexpr (CS > 0) {
+    // ---- merge: the warps' partials into the CTA's (shared memory), then the
+    // CTAs' partials across the cluster; each CTA writes 1/CS of the head's
+    // output. o = sum_w 2^(m_w - M) o_w / sum_w 2^(m_w - M) l_w.
+    __syncthreads();
+    float* cp = mslot + T::NCW * T::SLOT;
+    for (int e = tid; e < G * D; e += T::NT) {
+      const int h = e / D;
+      float M = -INFINITY;
+#pragma unroll
+      for (int v = 0; v < T::NCW; ++v) M = fmaxf(M, mslot[v * T::SLOT + G * D + h]);
+      float L = 0.f, O = 0.f;
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int v = 0; v < T::NCW; ++v) {
+          const float mv = mslot[v * T::SLOT + G * D + h];
+          if (mv != -INFINITY) {   // empty partials hold no o values
+            const float bw = fast_exp2(mv - M);
+            L += mslot[v * T::SLOT + G * D + G + h] * bw;
+            O += mslot[v * T::SLOT + e] * bw;
+          }
+        }
+      }
+      cp[e] = O;
+      if (e % D == 0) {
+        cp[G * D + h] = M;
+        cp[G * D + G + h] = L;
+      }
+    }
+    __syncthreads();   // converged warps for the aligned cluster barrier
+    cluster_sync_all();
+    const int kb = hsel / c.Hkv, kh = hsel % c.Hkv;
+    const int crank = (int)(blockIdx.x % CS);
+    constexpr int PER = G * D / CS;
+    for (int e = crank * PER + tid; e < (crank + 1) * PER; e += T::NT) {
+      const int h = e / D, d = e % D;
+      float M = -INFINITY, L = 0.f, O = 0.f;
+#pragma unroll
+      for (int j = 0; j < CS; ++j) {
+        const float mj = ld_cluster_f32(cp + G * D + h, (uint32_t)j);
+        if (mj == -INFINITY) continue;
+        const float lj = ld_cluster_f32(cp + G * D + G + h, (uint32_t)j);
+        const float oj = ld_cluster_f32(cp + e, (uint32_t)j);
+        const float mx = fmaxf(M, mj);
+        const float a = fast_exp2(M - mx), bw = fast_exp2(mj - mx);   // a = 0 while M = -inf
+        L = L * a + lj * bw;
+        O = O * a + oj * bw;
+        M = mx;
+      }
+      const float o = M == -INFINITY ? 0.f : O / L;
+      const long long oi = ((long long)kb * c.Hq + (long long)kh * G + h) * D + d;
+      if (oa.f32) static_cast<float*>(oa.out)[oi] = o;
+      else static_cast<uint16_t*>(oa.out)[oi] = f32_to_bf16_rn(o);
+      if (oa.lse && d == 0)
+        oa.lse[(long long)kb * c.Hq + kh * G + h] =
+            M == -INFINITY ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
+    }
+    __syncthreads();
+    cluster_sync_all();   // no CTA leaves while another still reads its shared memory
   }
 }
 
@@ -910,10 +1062,56 @@ k_decode_combine(CacheView c, DecodeWork w, int layer, int batch, OutArgs oa, in
 }
 
 // ------------------------------------------------------------------ dispatch
+// Cluster size for a call of nh heads: the largest of 8, 4, 2 whose nh * CS
+// CTAs fit on the SMs at once, if the call has at most half as many heads as
+// there are SMs; 0 selects the global plan and the combine kernel.
+inline int cluster_size(const fdms_cache* cache, int nh) {
+#if FDMS_CLUSTER_DECODE
+  if (!cache->cluster_ok) return 0;
+  for (int cs = 8; cs >= 2; cs /= 2)
+    if ((long long)nh * cs <= cache->num_sms) return cs;
+#endif
+  (void)cache;
+  (void)nh;
+  return 0;
+}
+
+template <class T, int CS>
+fdms_status launch_cluster_t(fdms_cache* cache, const DecodeWork& w, OutArgs oa, int layer,
+                             int batch, const void* q, cudaStream_t s) {
+  const int nh = batch * cache->view.Hkv;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(nh * CS));
+  cfg.blockDim = dim3(T::NT);
+  cfg.dynamicSmemBytes = T::smem_bytes_cluster(nh);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = CS;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_decode_split<T, CS>, cache->view, w, oa,
+                                           layer, batch, static_cast<const uint16_t*>(q), 0,
+                                           0.0);
+  if (e != cudaSuccess) return FDMS_ERR_CUDA;
+  cache->last_append_layer = -1;   // the kernel waits for every append queued before it
+  return FDMS_OK;
+}
+
 template <class T>
 fdms_status launch_split_t(fdms_cache* cache, const DecodeWork& w, OutArgs oa, int layer,
                            int batch, const void* q, cudaStream_t s) {
   const int nh = batch * cache->view.Hkv;
+  switch (cluster_size(cache, nh)) {
+    case 8: return launch_cluster_t<T, 8>(cache, w, oa, layer, batch, q, s);
+    case 4: return launch_cluster_t<T, 4>(cache, w, oa, layer, batch, q, s);
+    case 2: return launch_cluster_t<T, 2>(cache, w, oa, layer, batch, q, s);
+    default: break;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)cache->decode_ctas);
   cfg.blockDim = dim3(T::NT);
@@ -925,7 +1123,7 @@ fdms_status launch_split_t(fdms_cache* cache, const DecodeWork& w, OutArgs oa, i
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const int n_ranges = cache->decode_ctas * T::NCW;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, k_decode_split<T>, cache->view, w, oa, layer, batch,
+  cudaError_t e = cudaLaunchKernelEx(&cfg, k_decode_split<T, 0>, cache->view, w, oa, layer, batch,
                                      static_cast<const uint16_t*>(q), n_ranges,
                                      1.0 / (double)n_ranges);
   if (e != cudaSuccess) return FDMS_ERR_CUDA;
@@ -943,15 +1141,26 @@ fdms_status setup_t(fdms_cache* cache) {
   const int nh = cache->view.Bmax * cache->view.Hkv;
   const size_t smem = T::smem_bytes(nh);
   if (smem > 227 * 1024) return FDMS_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(k_decode_split<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(k_decode_split<T, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return FDMS_ERR_UNSUPPORTED;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_decode_split<T>, T::NT, smem) !=
-          cudaSuccess || per_sm < 1)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_decode_split<T, 0>, T::NT,
+                                                    smem) != cudaSuccess || per_sm < 1)
     return FDMS_ERR_UNSUPPORTED;
   cache->ctas_per_sm = per_sm;
   cache->ranges_per_cta = T::NCW;
+  // per-head cluster mode: usable when every cluster size fits
+  const size_t csmem = T::smem_bytes_cluster(nh);
+  cache->cluster_ok =
+      csmem <= 227 * 1024 &&
+      cudaFuncSetAttribute(k_decode_split<T, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)csmem) == cudaSuccess &&
+      cudaFuncSetAttribute(k_decode_split<T, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)csmem) == cudaSuccess &&
+      cudaFuncSetAttribute(k_decode_split<T, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)csmem) == cudaSuccess;
+  cudaGetLastError();   // a refused attribute only turns the cluster mode off
   return FDMS_OK;
 }
 

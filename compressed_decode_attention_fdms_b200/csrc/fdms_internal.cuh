@@ -214,6 +214,7 @@ struct fdms_cache {
   // after it, else -1: an append to another layer may read its head state
   // before its dependency wait (see k_append_step)
   int last_append_layer;
+  int cluster_ok;         // the per-head cluster decode mode can be launched
 };
 
 // Record a device allocation of the cache (freed at destroy). Frees `p` and
