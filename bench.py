@@ -454,6 +454,14 @@ def run_native(args, wl):
 
     peak, peak_src = load_peaks()
     traffic, traffic_src = load_traffic(wl.name)
+    # the library's decode mode for this call shape: one cluster of CS CTAs per
+    # (seq, kv head) when there are at most half as many as SMs and no explicit
+    # split grid, else the global plan (split + combine)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    nh = wl.batch * wl.kv_heads
+    cs = next((c for c in (8, 4, 2) if nh * c <= sms), 0) if args.decode_ctas == 0 else 0
+    kernel = (f"fdms_decode_attn (k_decode_split, one cluster of {cs} CTAs per head, no combine)"
+              if cs else "fdms_decode_attn (k_decode_split + k_decode_combine)")
     achieved = per_launch_bytes / (dec_avg_ms * 1e-3) / 1e9
     result = None
     if rank == 0:
@@ -470,14 +478,14 @@ def run_native(args, wl):
             "roofline": {
                 "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": traffic, "traffic_source": traffic_src,
-                "kernel": "fdms_decode_attn (k_decode_split + k_decode_combine)",
+                "kernel": kernel,
                 "per_launch_bytes": per_launch_bytes, "launch_us": dec_avg_ms * 1e3,
                 "launch_timing": f"CUDA events around one graph of {K * L} back-to-back "
                                  "decode calls (all layers, K rounds); duration / calls",
                 "peak_source": peak_src,
             },
             "clocks": clocks,
-            "gpu_launches": K * L * 3,
+            "gpu_launches": K * L * (2 if cs else 3),
             "prefill": {"tokens_per_seq": int(wl.max_ctx), "layers": L,
                         "us_per_layer": 1e3 * pre_ms / L, "gb_per_layer": pre_bytes / L / 1e9,
                         "achieved_gbs": pre_bytes / (pre_ms * 1e-3) / 1e9,

@@ -1064,10 +1064,11 @@ k_decode_combine(CacheView c, DecodeWork w, int layer, int batch, OutArgs oa, in
 // ------------------------------------------------------------------ dispatch
 // Cluster size for a call of nh heads: the largest of 8, 4, 2 whose nh * CS
 // CTAs fit on the SMs at once, if the call has at most half as many heads as
-// there are SMs; 0 selects the global plan and the combine kernel.
+// there are SMs; 0 selects the global plan and the combine kernel, which a
+// cache created with an explicit split grid (decode_ctas > 0) always uses.
 inline int cluster_size(const fdms_cache* cache, int nh) {
 #if FDMS_CLUSTER_DECODE
-  if (!cache->cluster_ok) return 0;
+  if (!cache->cluster_ok || cache->cfg.decode_ctas > 0) return 0;
   for (int cs = 8; cs >= 2; cs /= 2)
     if ((long long)nh * cs <= cache->num_sms) return cs;
 #endif

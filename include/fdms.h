@@ -15,7 +15,9 @@
  *                        that leave the recent window, compact survivors;
  *   fdms_decode_attn   - single-token attention of every query head over the
  *                        survivors of its kv head (split over the GPU, then
- *                        merged);
+ *                        merged: through distributed shared memory inside a
+ *                        cluster of CTAs per head for calls with few heads, by
+ *                        a combine kernel otherwise);
  *   fdms_cache_stats   - counters, including compact vs dense-equivalent bytes
  *                        (the quantity of the pages' KV-memory table).
  *
@@ -98,7 +100,11 @@ typedef struct {
                             max_seq_len tokens in every (layer, seq, kv head) */
   fdms_kv_dtype kv_dtype;
   float softmax_scale;   /* 0 -> 1 / sqrt(head_dim) */
-  int decode_ctas;       /* split-kernel grid; 0 -> SM count x CTAs per SM */
+  int decode_ctas;       /* 0 -> automatic: a call with at most half as many
+                            (seq, kv head) pairs as SMs runs one cluster of 2-8
+                            CTAs per pair; other calls run one plan over SM
+                            count x CTAs per SM split CTAs. > 0 -> always the
+                            plan, over this many CTAs */
 } fdms_config;
 
 typedef struct {

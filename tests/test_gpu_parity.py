@@ -101,11 +101,19 @@ SMALL = {
 }
 
 
+# Decode modes: "auto" (decode_ctas = 0) runs these few-head calls as one
+# cluster of CTAs per head; "plan" (an explicit grid) forces the global tile
+# plan with the combine kernel, which calls with many heads use.
+MODES = {"auto": 0, "plan": 148}
+
+
+@pytest.mark.parametrize("mode", list(MODES))
 @pytest.mark.parametrize("name", list(SMALL))
-def test_scaled_workloads(name):
+def test_scaled_workloads(name, mode):
     wl = SMALL[name]
     true_tol = TOL_FP8_TRUE if name == "qwen_shape_fp8" else None
-    run_workload(wl, check_every=max(1, wl.steps // 3), true_tol=true_tol)
+    run_workload(wl, check_every=max(1, wl.steps // 3), true_tol=true_tol,
+                 decode_ctas=MODES[mode])
 
 
 # Edge cases: window / period / group / head dim / dtype sweeps on tiny shapes.
@@ -118,10 +126,11 @@ EDGE = [
 ]
 
 
+@pytest.mark.parametrize("mode", list(MODES))
 @pytest.mark.parametrize("i", range(len(EDGE)))
-def test_edge_shapes(i):
+def test_edge_shapes(i, mode):
     base = wk.scaled(wk.get("tiny"), ctx=200, steps=6, batch=2, rate=0.3)
-    run_workload(wk.scaled(base, **EDGE[i]))
+    run_workload(wk.scaled(base, **EDGE[i]), decode_ctas=MODES[mode])
 
 
 @pytest.mark.parametrize("ctx", [0, 1, 63, 64, 65, 127, 128, 129])
