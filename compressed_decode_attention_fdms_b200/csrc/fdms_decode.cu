@@ -1265,7 +1265,9 @@ extern "C" fdms_status fdms_decode_attn_noalloc(fdms_cache* cache, int layer, in
   const size_t o_bytes = align256((size_t)parts * c.G * c.D * sizeof(float));
   const size_t ml_bytes = align256((size_t)parts * c.G * 2 * sizeof(float));
   const size_t need = o_bytes + ml_bytes;
-  if (need > FDMS_STATIC_SCRATCH_BYTES) return FDMS_ERR_INVALID_ARG;
+  // a call that runs in per-head clusters keeps its partials in shared memory
+  if (cluster_size(cache, batch * c.Hkv) == 0 && need > FDMS_STATIC_SCRATCH_BYTES)
+    return FDMS_ERR_INVALID_ARG;
 
   int prev = -1;
   if (cudaGetDevice(&prev) != cudaSuccess) return FDMS_ERR_CUDA;

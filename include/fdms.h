@@ -58,7 +58,8 @@
  * found by the device (pool exhausted, sequence too long) are latched into a
  * sticky word with the first error code and the affected head is left
  * unchanged; fdms_cache_stats reports the word. Device code never traps or
- * waits without a bound.
+ * waits without a bound (the barriers of one CTA or one cluster aside, which
+ * every thread of it reaches).
  *
  * Layouts: all tensors are dense, row-major, in the order written; "bf16" is
  * the IEEE binary32 upper half. Device pointers must be 16-byte aligned.
@@ -195,7 +196,8 @@ fdms_status fdms_decode_attn_f32(fdms_cache* cache, int layer, int batch,
  * every device that loads the library holds that array until the process exits.
  *   - Needs (split warps + batch x Hkv) x G x (4 D + 8) bytes (at most one
  *     partial per split warp and head it shares with another warp; 8 split
- *     warps per decode CTA, 4 when G x D >= 1024); a call that needs more than
+ *     warps per decode CTA, 4 when G x D >= 1024), or none for a call that
+ *     runs in per-head clusters (see decode_ctas); a call that needs more than
  *     the array returns FDMS_ERR_INVALID_ARG and queues nothing. Every value
  *     the call reads from the array it first writes itself.
  *   - The first call on a device looks up the array's device address (a
