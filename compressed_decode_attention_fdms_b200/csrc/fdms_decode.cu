@@ -304,7 +304,8 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   pdl_launch_dependents();
 
   // ---- units and pages of every head of the call; exclusive prefix
-  const int hsel = CS > 0 ? (int)(blockIdx.x / (CS > 0 ? CS : 1)) : 0;   // cluster mode: its head
+  // cluster mode: the head of this CTA's cluster
+  const int hsel = CS > 0 ? (int)(blockIdx.x / (CS > 0 ? CS : 1)) : 0;
   if constexpr (CS > 0) {
     if (tid == 0) {
       const long long hi = hi0 + hsel;
