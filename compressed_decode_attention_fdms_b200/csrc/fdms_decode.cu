@@ -1,4 +1,4 @@
-// Decode attention over the compact store: split kernel + combine kernel.
+// Decode attention over the compact store: split kernel (+ combine kernel).
 //
 // FastDMS decodes over the survivors of per-head eviction only, reading 5-8x
 // less KV than a dense cache ("FastDMS: 6.4X KV-cache compression running
@@ -8,12 +8,18 @@
 // S_h = the head's compact store plus its visible ring slots.
 //
 // The kernel is memory bound: every byte of a visible K and V row is read once.
-//   - Work is balanced over the GPU by tiles, not by heads. The tiles of all
-//     heads of the call (a tile = up to 32 rows of one 64-slot page for
-//     128-byte rows: the head's store pages, then its ring slots) are laid end
-//     to end and cut into equal ranges, one per warp of the grid; a warp does
-//     the same number of tile steps whatever the mix of head lengths, and
-//     emits one partial (m, l, o) per head its range touches.
+//   - Two ways to spread the work, chosen per call on the host:
+//     * per-head clusters (calls with at most half as many heads as SMs): one
+//       thread-block cluster of 2-8 CTAs per (seq, kv head); the head's tiles
+//       (a tile = up to 32 rows of one 64-slot page for 128-byte rows: the
+//       head's store pages, then its ring slots) are split evenly over the
+//       cluster's CTAs and then their warps; the warps' partials (m, l, o) are
+//       merged in shared memory, the CTAs' through distributed shared memory,
+//       and the cluster writes the output. No plan, workspace or combine.
+//     * one plan (other calls): the tiles of all heads of the call are laid
+//       end to end and cut into equal ranges, one per warp of the grid; a warp
+//       does the same number of tile steps whatever the mix of head lengths,
+//       and emits one partial per head its range touches.
 //   - Each warp stages its own tiles (32 rows of a 64-slot page for 128-byte
 //     rows): the K rows, V rows and the head's q go to shared memory by 1-D
 //     bulk copies (cp.async.bulk, completion on an mbarrier) into one of the
@@ -34,8 +40,8 @@
 //     (cvt e4m3x2 -> f16x2) and q is brought into f16 range by a power of two
 //     that the score scale undoes; the page's K scale multiplies the scores
 //     and its V scale the probabilities, never the elements.
-//   - A head that lies whole inside one warp's range is written by that warp;
-//     heads with no slot get zeros. Every other head has one partial
+//   - Plan mode: a head that lies whole inside one warp's range is written by
+//     that warp; heads with no slot get zeros. Every other head has one partial
 //     (m, l, o) per warp that covered part of it, written to a workspace; a
 //     combine kernel merges them, four threads per output element, loading
 //     all partials of the head at once:
