@@ -3,7 +3,8 @@
 
 One step = for every layer: append one token per sequence with its keep bits
 (fdms_append_evict: ring write, eviction, compaction) and run decode attention
-for all query heads (fdms_decode_attn: split kernel + combine kernel). Inputs
+for all query heads (fdms_decode_attn: one kernel of per-head CTA clusters for
+calls with few heads, else a split kernel and a combine kernel). Inputs
 are the seeded synthetic workloads of ``workloads`` (shapes of the FastDMS
 announcement's benchmark: ctx 8192, Llama-3.2-1B / Qwen3-8B shapes, c = 1 or 8).
 
@@ -100,8 +101,7 @@ def load_traffic(workload):
             continue
         if f[2:4] == now:
             return float(f[1]), "ncu dram__bytes_read.sum + dram__bytes_write.sum of " \
-                                "k_decode_split + k_decode_combine, profiles/decode_step_" + \
-                                workload + ".md"
+                                "one decode call's kernels"
         return None, "decode kernels changed since the ncu capture"
     return None, "no capture for this workload"
 

@@ -10,9 +10,10 @@
 //   3. the still-unresolved new tokens are written to the ring (staging).
 // Resolution is a stable stream compaction (warp ballot of the keep bits, a
 // popcount prefix inside each warp, a scan of warp totals), so survivors keep
-// their order. Store blocks for all survivors of a head are taken from the pool
-// with one atomic bump before any row is written; if the pool cannot cover them
-// the head is left unchanged and FDMS_ERR_OUT_OF_BLOCKS is latched.
+// their order. Store blocks for all survivors of a head are reserved in one
+// step before any row is written; if the pool cannot cover them the head is
+// left unchanged, the pool counter does not move, and FDMS_ERR_OUT_OF_BLOCKS is
+// latched.
 //
 // Three paths, one result: decode steps (k_append_step: a warp per head, the
 // loads ordered for latency), calls of up to 16 tokens per sequence
@@ -43,6 +44,24 @@ __device__ __forceinline__ float block_max(float x, float* red) {
   float m = red[0];
   for (int i = 1; i < kWarps; ++i) m = fmaxf(m, red[i]);
   return m;
+}
+
+// Blocks [base, base + need) of the pool for one head, or -1 when the pool
+// cannot cover them. The counter never moves past num_blocks: a request that
+// does not fit leaves it as it was, so a later, smaller request can still be
+// served and the count of blocks handed out stays exact. A compare-and-swap
+// loop: warps of one kernel rarely contend (a decode step takes a new block
+// about once per 64 kept tokens of a head). Gives up (-1) after a bounded
+// number of lost races.
+__device__ long long take_blocks(DevCounters* ctr, unsigned long long need, long long num_blocks) {
+  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(&ctr->blocks_next);
+  for (int it = 0; it < (1 << 16); ++it) {
+    if (cur + need > (unsigned long long)num_blocks) return -1;
+    const unsigned long long prev = atomicCAS(&ctr->blocks_next, cur, cur + need);
+    if (prev == cur) return (long long)cur;
+    cur = prev;
+  }
+  return -1;
 }
 
 // x / s in IEEE binary32, rounded to nearest even, for finite x and a normal
@@ -127,16 +146,16 @@ __device__ __forceinline__ void move_vec(uint8_t* dst_row, int dst_r, const uint
 //   1. k_bulk_count (head x chunk): survivors of each chunk of kChunkPositions
 //      of the positions resolved now; on a sequence's first FP8 append, the
 //      call's max |K| and |V| (atomicMax on the bits of non-negative floats).
-//   2. k_bulk_alloc (one warp per head): exclusive prefix of the chunk counts,
-//      one atomic bump for the store blocks of all survivors, the FP8 scales,
-//      and the head's new lengths; the state before the call goes to the
-//      workspace header, which the next two kernels read instead.
+//   2. k_bulk_alloc (one CTA for the call): exclusive prefix of the chunk
+//      counts per head, the FP8 scales, the store blocks of all heads reserved
+//      in head order, and the heads' new lengths; the state before the call
+//      goes to the workspace header, which the next two kernels read instead.
 //   3. k_bulk_write (head x chunk): the chunk's survivors to the store, in
 //      order, at len0 + prefix + rank (warp ballot/popc, scan of warp totals).
 //   4. k_bulk_ring (head): the still-unresolved new tokens to the ring, once
 //      every ring row that (3) resolves has been read.
-enum : int { kHdrM, kHdrN0, kHdrR0, kHdrLen0, kHdrN1, kHdrR1, kHdrNb0, kHdrStatus, kHdrBlkLo,
-             kHdrBlkHi, kHdrSk, kHdrSv };
+enum : int { kHdrM, kHdrN0, kHdrR0, kHdrLen0, kHdrN1, kHdrR1, kHdrNb0, kHdrStatus, kHdrLen1,
+             kHdrSk, kHdrSv };
 enum : int { kBulkGo = 0, kBulkSkip = 1 };
 
 struct BulkIn {
@@ -220,119 +239,199 @@ k_bulk_count(CacheView c, AppendWork aw, BulkIn in) {
   if (tid == 0) aw.counts[(long long)hid * aw.max_chunks + ch] = cnt;
 }
 
+constexpr int kAllocThreads = 1024;
+constexpr int kAllocWarps = kAllocThreads / 32;
+constexpr int kMaxCallHeads = 4096;   // max_batch x num_kv_heads of a supported cache
+
+// One CTA for every head of the call, in three phases:
+//   1. a warp per head: exclusive prefix of the chunk counts, FP8 scales, the
+//      state before the call and after it (into the head's header), and the
+//      pool blocks the head needs;
+//   2. the blocks of all heads reserved at once, in head order; when the pool
+//      cannot cover them all, heads are served first-fit in head order, so a
+//      head that does not fit leaves the pool to the heads after it;
+//   3. a warp per head: block table entries and lengths, or the error for a
+//      head that got no blocks (left unchanged).
+// Allocations of different kernels never overlap (each runs after its
+// dependency wait), so inside this kernel the pool counter has one writer.
 template <bool FP8>
-__global__ void __launch_bounds__(32)
-k_bulk_alloc(CacheView c, AppendWork aw, BulkIn in, int nch) {
+__global__ void __launch_bounds__(kAllocThreads)
+k_bulk_alloc(CacheView c, AppendWork aw, BulkIn in, int nch, int heads) {
+  __shared__ int s_need[kMaxCallHeads];   // blocks a head needs; -1: nothing to do
+  __shared__ int s_blk[kMaxCallHeads];    // first block handed out; -1: none
+  __shared__ int s_wsum[kAllocWarps];
+  __shared__ long long s_base;
   pdl_wait();
   pdl_launch_dependents();
-  const int hid = blockIdx.x, lane = threadIdx.x;
-  const int b = hid / c.Hkv, h = hid % c.Hkv;
-  const long long hi = head_index(c, in.layer, b, h);
-  int* hd = aw.hdr + (long long)hid * kHdrInts;
-  const int m = in.n_new[b];
-  const int n0 = c.tok_n[hi], r0 = c.tok_r[hi], len0 = c.store_len[hi];
-  unsigned ak_bits = 0, av_bits = 0;
-  if constexpr (FP8) {
-    ak_bits = aw.amax[hid * 2];
-    av_bits = aw.amax[hid * 2 + 1];
-  }
-  __syncwarp();
-  if (FP8 && lane == 0) {   // ready for the next call
-    aw.amax[hid * 2] = 0u;
-    aw.amax[hid * 2 + 1] = 0u;
-  }
-  if (m < 0 || m > in.max_new || (long long)n0 + m > c.max_seq_len) {
-    if (lane == 0) {
-      latch_error(c.ctr, FDMS_ERR_DEVICE);
-      hd[kHdrStatus] = kBulkSkip;
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+
+  // ---- phase 1
+  for (int hid = warp; hid < heads; hid += kAllocWarps) {
+    const int b = hid / c.Hkv, h = hid % c.Hkv;
+    const long long hi = head_index(c, in.layer, b, h);
+    int* hd = aw.hdr + (long long)hid * kHdrInts;
+    const int m = in.n_new[b];
+    const int n0 = c.tok_n[hi], r0 = c.tok_r[hi], len0 = c.store_len[hi];
+    unsigned ak_bits = 0, av_bits = 0;
+    if constexpr (FP8) {
+      ak_bits = aw.amax[hid * 2];
+      av_bits = aw.amax[hid * 2 + 1];
     }
-    return;
-  }
-  if (m == 0) {
-    if (lane == 0) hd[kHdrStatus] = kBulkSkip;
-    return;
-  }
-  const int n1 = n0 + m;
-  const int r1 = (n1 - c.W - r0 >= c.P) ? n1 - c.W : r0;
-  // exclusive prefix of the chunk counts
-  int* cnt = aw.counts + (long long)hid * aw.max_chunks;
-  int running = 0;
-  for (int base = 0; base < nch; base += 32) {
-    const int i = base + lane;
-    const int x = i < nch ? cnt[i] : 0;
-    int incl = x;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += y;
+    __syncwarp();
+    if (FP8 && lane == 0) {   // ready for the next call
+      aw.amax[hid * 2] = 0u;
+      aw.amax[hid * 2 + 1] = 0u;
     }
-    if (i < nch) cnt[i] = running + incl - x;
-    running += __shfl_sync(0xffffffffu, incl, 31);
-  }
-  const int len1 = len0 + running;
-  // FP8 scales: a sequence's first append fixes them
-  float sk = 1.0f, sv = 1.0f;
-  if constexpr (FP8) {
-    if (n0 == 0) {
-      if (in.kv_scale) {
-        sk = in.kv_scale[((long long)b * c.Hkv + h) * 2];
-        sv = in.kv_scale[((long long)b * c.Hkv + h) * 2 + 1];
-      } else {
-        sk = __fdiv_rn(fmaxf(__uint_as_float(ak_bits), 1.17549435e-38f), 448.0f);
-        sv = __fdiv_rn(fmaxf(__uint_as_float(av_bits), 1.17549435e-38f), 448.0f);
-      }
+    if (m < 0 || m > in.max_new || (long long)n0 + m > c.max_seq_len || m == 0) {
       if (lane == 0) {
-        c.head_scale[hi * 2] = sk;
-        c.head_scale[hi * 2 + 1] = sv;
+        if (m != 0) latch_error(c.ctr, FDMS_ERR_DEVICE);
+        hd[kHdrStatus] = kBulkSkip;
+        s_need[hid] = -1;
       }
-    } else {
-      sk = c.head_scale[hi * 2];
-      sv = c.head_scale[hi * 2 + 1];
+      continue;
+    }
+    const int n1 = n0 + m;
+    const int r1 = (n1 - c.W - r0 >= c.P) ? n1 - c.W : r0;
+    // exclusive prefix of the chunk counts
+    int* cnt = aw.counts + (long long)hid * aw.max_chunks;
+    int running = 0;
+    for (int base = 0; base < nch; base += 32) {
+      const int i = base + lane;
+      const int x = i < nch ? cnt[i] : 0;
+      int incl = x;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      if (i < nch) cnt[i] = running + incl - x;
+      running += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    const int len1 = len0 + running;
+    // FP8 scales: a sequence's first append fixes them
+    float sk = 1.0f, sv = 1.0f;
+    if constexpr (FP8) {
+      if (n0 == 0) {
+        if (in.kv_scale) {
+          sk = in.kv_scale[((long long)b * c.Hkv + h) * 2];
+          sv = in.kv_scale[((long long)b * c.Hkv + h) * 2 + 1];
+        } else {
+          sk = __fdiv_rn(fmaxf(__uint_as_float(ak_bits), 1.17549435e-38f), 448.0f);
+          sv = __fdiv_rn(fmaxf(__uint_as_float(av_bits), 1.17549435e-38f), 448.0f);
+        }
+        if (lane == 0) {
+          c.head_scale[hi * 2] = sk;
+          c.head_scale[hi * 2 + 1] = sv;
+        }
+      } else {
+        sk = c.head_scale[hi * 2];
+        sv = c.head_scale[hi * 2 + 1];
+      }
+    }
+    const int nb0 = (len0 + kBlockSlots - 1) / kBlockSlots;
+    const int nb1 = (len1 + kBlockSlots - 1) / kBlockSlots;
+    if (lane == 0) {
+      hd[kHdrM] = m;
+      hd[kHdrN0] = n0;
+      hd[kHdrR0] = r0;
+      hd[kHdrLen0] = len0;
+      hd[kHdrN1] = n1;
+      hd[kHdrR1] = r1;
+      hd[kHdrNb0] = nb0;
+      hd[kHdrLen1] = len1;
+      hd[kHdrStatus] = kBulkGo;
+      hd[kHdrSk] = __float_as_int(sk);
+      hd[kHdrSv] = __float_as_int(sv);
+      s_need[hid] = nb1 - nb0;
     }
   }
-  // store blocks for all survivors: one atomic bump
-  const int nb0 = (len0 + kBlockSlots - 1) / kBlockSlots;
-  const int nb1 = (len1 + kBlockSlots - 1) / kBlockSlots;
-  long long base_blk = 0;
-  if (nb1 > nb0) {
-    int fail = 0;
-    if (lane == 0) {
-      const unsigned long long need = (unsigned long long)(nb1 - nb0);
-      const unsigned long long base = atomicAdd(&c.ctr->blocks_next, need);
-      if (base + need > (unsigned long long)c.num_blocks) {
-        latch_error(c.ctr, FDMS_ERR_OUT_OF_BLOCKS);
-        fail = 1;
+  __syncthreads();
+
+  // ---- phase 2: exclusive prefix of the needs in head order
+  constexpr int PER = kMaxCallHeads / kAllocThreads;
+  int mine[PER], sum = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int hid = tid * PER + i;
+    mine[i] = hid < heads ? max(s_need[hid], 0) : 0;
+    sum += mine[i];
+  }
+  int incl = sum;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) s_wsum[warp] = incl;
+  __syncthreads();
+  int excl = incl - sum, total = 0;
+  for (int i = 0; i < kAllocWarps; ++i) {
+    if (i < warp) excl += s_wsum[i];
+    total += s_wsum[i];
+  }
+  if (tid == 0) {
+    const long long cur = (long long)c.ctr->blocks_next;
+    if (cur + total <= c.num_blocks) {
+      s_base = cur;
+      c.ctr->blocks_next = (unsigned long long)(cur + total);
+    } else {
+      s_base = -1;
+    }
+  }
+  __syncthreads();
+  if (s_base >= 0) {
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int hid = tid * PER + i;
+      if (hid < heads) s_blk[hid] = (int)(s_base + excl);
+      excl += mine[i];
+    }
+  } else if (tid == 0) {   // the pool falls short: first fit in head order
+    long long cur = (long long)c.ctr->blocks_next;
+    for (int hid = 0; hid < heads; ++hid) {
+      const int need = s_need[hid];
+      if (need <= 0) {
+        s_blk[hid] = (int)cur;
+      } else if (cur + need <= c.num_blocks) {
+        s_blk[hid] = (int)cur;
+        cur += need;
       } else {
-        base_blk = (long long)base;
+        s_blk[hid] = -1;
       }
     }
-    if (__shfl_sync(0xffffffffu, fail, 0)) {
-      if (lane == 0) hd[kHdrStatus] = kBulkSkip;
-      return;
+    c.ctr->blocks_next = (unsigned long long)cur;
+  }
+  __syncthreads();
+
+  // ---- phase 3
+  for (int hid = warp; hid < heads; hid += kAllocWarps) {
+    const int need = s_need[hid];
+    if (need < 0) continue;
+    int* hd = aw.hdr + (long long)hid * kHdrInts;
+    const int b = hid / c.Hkv, h = hid % c.Hkv;
+    const long long hi = head_index(c, in.layer, b, h);
+    const long long base_blk = s_blk[hid];
+    if (base_blk < 0) {
+      if (lane == 0) {
+        latch_error(c.ctr, FDMS_ERR_OUT_OF_BLOCKS);
+        hd[kHdrStatus] = kBulkSkip;
+      }
+      continue;
     }
-    base_blk = __shfl_sync(0xffffffffu, base_blk, 0);
+    const int nb0 = hd[kHdrNb0];
+    const float sk = __int_as_float(hd[kHdrSk]), sv = __int_as_float(hd[kHdrSv]);
     int32_t* bt = c.block_table + hi * c.max_blocks;
     float* bts = c.bt_scale + hi * c.max_blocks * 2;
-    for (int j = nb0 + lane; j < nb1; j += 32) {
-      bt[j] = (int32_t)(base_blk + (j - nb0));
-      bts[2 * j] = sk;
-      bts[2 * j + 1] = sv;
+    for (int j = lane; j < need; j += 32) {
+      bt[nb0 + j] = (int32_t)(base_blk + j);
+      bts[2 * (nb0 + j)] = sk;
+      bts[2 * (nb0 + j) + 1] = sv;
     }
-  }
-  if (lane == 0) {
-    hd[kHdrM] = m;
-    hd[kHdrN0] = n0;
-    hd[kHdrR0] = r0;
-    hd[kHdrLen0] = len0;
-    hd[kHdrN1] = n1;
-    hd[kHdrR1] = r1;
-    hd[kHdrNb0] = nb0;
-    hd[kHdrStatus] = kBulkGo;
-    hd[kHdrSk] = __float_as_int(sk);
-    hd[kHdrSv] = __float_as_int(sv);
-    c.store_len[hi] = len1;
-    c.tok_n[hi] = n1;
-    c.tok_r[hi] = r1;
+    if (lane == 0) {
+      c.store_len[hi] = hd[kHdrLen1];
+      c.tok_n[hi] = hd[kHdrN1];
+      c.tok_r[hi] = hd[kHdrR1];
+    }
   }
 }
 
@@ -539,13 +638,10 @@ __device__ void warp_resolve(const CacheView& c, long long hi, int lane, int n0,
   if (nb1 > nb0) {
     int fail = 0;
     if (lane == 0) {
-      const unsigned long long need = (unsigned long long)(nb1 - nb0);
-      const unsigned long long base = atomicAdd(&c.ctr->blocks_next, need);
-      if (base + need > (unsigned long long)c.num_blocks) {
+      base_blk = take_blocks(c.ctr, (unsigned long long)(nb1 - nb0), c.num_blocks);
+      if (base_blk < 0) {
         latch_error(c.ctr, FDMS_ERR_OUT_OF_BLOCKS);
         fail = 1;
-      } else {
-        base_blk = (long long)base;
       }
     }
     if (__shfl_sync(0xffffffffu, fail, 0)) return;
@@ -846,16 +942,13 @@ k_append_step(CacheView c, int layer, int batch, const int32_t* __restrict__ n_n
   const int nb0 = (len0 + kBlockSlots - 1) / kBlockSlots;
   const int nb1 = (len1 + kBlockSlots - 1) / kBlockSlots;
   long long base_blk = 0;
-  if (nb1 > nb0) {   // new store blocks for this call (one atomic bump)
+  if (nb1 > nb0) {   // new store blocks for this call, reserved at once
     int fail = 0;
     if (lane == 0) {
-      const unsigned long long need = (unsigned long long)(nb1 - nb0);
-      const unsigned long long base = atomicAdd(&c.ctr->blocks_next, need);
-      if (base + need > (unsigned long long)c.num_blocks) {
+      base_blk = take_blocks(c.ctr, (unsigned long long)(nb1 - nb0), c.num_blocks);
+      if (base_blk < 0) {
         latch_error(c.ctr, FDMS_ERR_OUT_OF_BLOCKS);
         fail = 1;
-      } else {
-        base_blk = (long long)base;
       }
     }
     if (__shfl_sync(kAll, fail, 0)) return;
@@ -985,10 +1078,10 @@ fdms_status fdms_launch_append(fdms_cache* cache, int layer, int batch, const in
     e = c.fp8 ? cudaLaunchKernelEx(&cfg, k_bulk_count<true>, c, aw, in)
               : cudaLaunchKernelEx(&cfg, k_bulk_count<false>, c, aw, in);
     if (e == cudaSuccess) {
-      cfg.gridDim = dim3(heads);
-      cfg.blockDim = dim3(32);
-      e = c.fp8 ? cudaLaunchKernelEx(&cfg, k_bulk_alloc<true>, c, aw, in, nch)
-                : cudaLaunchKernelEx(&cfg, k_bulk_alloc<false>, c, aw, in, nch);
+      cfg.gridDim = dim3(1);
+      cfg.blockDim = dim3(kAllocThreads);
+      e = c.fp8 ? cudaLaunchKernelEx(&cfg, k_bulk_alloc<true>, c, aw, in, nch, (int)heads)
+                : cudaLaunchKernelEx(&cfg, k_bulk_alloc<false>, c, aw, in, nch, (int)heads);
     }
     if (e == cudaSuccess) {
       cfg.gridDim = dim3(heads, (unsigned)nch);

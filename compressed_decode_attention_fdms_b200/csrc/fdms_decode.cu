@@ -1,4 +1,4 @@
-// Decode attention over the compact store: split kernel (+ combine kernel).
+// Decode attention over the compact store.
 //
 // FastDMS decodes over the survivors of per-head eviction only, reading 5-8x
 // less KV than a dense cache ("FastDMS: 6.4X KV-cache compression running
@@ -8,48 +8,47 @@
 // S_h = the head's compact store plus its visible ring slots.
 //
 // The kernel is memory bound: every byte of a visible K and V row is read once.
+// A tile is 4 KB of K rows and 4 KB of V rows of one 64-slot page (32 rows of
+// 128 bytes): a store tile, or a ring frame (TR consecutive positions, which
+// sit in TR consecutive ring slots).
 //   - Two ways to spread the work, chosen per call on the host:
-//     * per-head clusters (calls with at most half as many heads as SMs): one
-//       thread-block cluster of 2-8 CTAs per (seq, kv head); the head's tiles
-//       (a tile = up to 32 rows of one 64-slot page for 128-byte rows: the
-//       head's store pages, then its ring slots) are split evenly over the
-//       cluster's CTAs and then their warps; the warps' partials (m, l, o) are
-//       merged in shared memory, the CTAs' through distributed shared memory,
-//       and the cluster writes the output. No plan, workspace or combine.
+//     * per-head clusters (calls with few (seq, kv head) pairs): one
+//       thread-block cluster of 2-8 CTAs per pair; the head's tiles are split
+//       over the cluster's warps in runs whose lengths differ by at most one;
+//       the warps' partials (m, l, o) are merged in shared memory, the CTAs'
+//       through distributed shared memory, and the cluster writes the output.
+//       No plan, workspace or combine kernel.
 //     * one plan (other calls): the tiles of all heads of the call are laid
-//       end to end and cut into equal ranges, one per warp of the grid; a warp
-//       does the same number of tile steps whatever the mix of head lengths,
-//       and emits one partial per head its range touches.
-//   - Each warp stages its own tiles (32 rows of a 64-slot page for 128-byte
-//     rows): the K rows, V rows and the head's q go to shared memory by 1-D
-//     bulk copies (cp.async.bulk, completion on an mbarrier) into one of the
-//     warp's two stages, and the warp refills a stage as soon as it has read
-//     it. The tile descriptors (head, rows, source address) are worked out 32
-//     at a time, one lane per tile, so the block-table reads of a warp's first
-//     tiles overlap. Rows keep their page row in shared memory, so the chunk
-//     permutation they are stored with makes the fragment loads below free of
-//     bank conflicts.
-//   - A warp computes the scores of a tile on the tensor cores
-//     (mma.sync m16n8k16, fp32 accumulate; the G query heads of the kv head
-//     are rows 0..G-1 of the 16-row A tile, keys are the columns), an online
-//     softmax in fp32 in the log2 domain, and o^T += V^T p^T on the tensor
-//     cores again (head dims are the rows, heads the columns, keys the
-//     reduction): the score accumulators already have the layout of p^T's B
-//     fragments. p is split into a 16-bit head and a 16-bit remainder so its
-//     rounding stays below 2^-16 relative. FP8 pages are converted exactly to f16
-//     (cvt e4m3x2 -> f16x2) and q is brought into f16 range by a power of two
-//     that the score scale undoes; the page's K scale multiplies the scores
-//     and its V scale the probabilities, never the elements.
-//   - Plan mode: a head that lies whole inside one warp's range is written by
-//     that warp; heads with no slot get zeros. Every other head has one partial
-//     (m, l, o) per warp that covered part of it, written to a workspace; a
-//     combine kernel merges them, four threads per output element, loading
-//     all partials of the head at once:
-//         o = sum_w 2^(m_w - M) o_w / sum_w 2^(m_w - M) l_w.
-//     The combine rebuilds the split's tile plan from the head lengths itself
-//     (nothing changes them between the two kernels), before its dependency
-//     wait.
-//   - Both kernels allow programmatic dependent launch: set-up that reads no
+//       end to end and cut into equal ranges, one per warp of the grid; heads
+//       shared by several warps are merged by a combine kernel.
+//   - The store is append-only and a ring slot keeps its row until the ring
+//     wraps past it, so everything a decode call saw of a head stays where it
+//     was. In cluster mode the call plans its tiles from what the previous
+//     decode of the same layer saw (a per-head snapshot) and issues the copies
+//     of those tiles before its dependency wait, while the kernel before it
+//     still runs; after the wait it reads the head's current lengths, masks
+//     ring rows that have been resolved since, extends the tiles at the end of
+//     the store and of the ring, and adds tiles for what is new.
+//   - Each warp stages its own tiles: K rows, V rows and the head's q go to
+//     shared memory by 1-D bulk copies (cp.async.bulk, completion on an
+//     mbarrier) into one of the warp's two stages; the warp refills a stage as
+//     soon as it has read it. Rows keep their page row in shared memory, so
+//     the chunk permutation they are stored with makes the matrix loads free
+//     of bank conflicts.
+//   - Tile arithmetic on the tensor cores (mma.sync m16n8k16, fp32
+//     accumulate), keys on the M side: S^T = K Q^T with 16 keys per MMA row
+//     block and the kv head's G query heads as columns; online softmax in fp32
+//     in the log2 domain per column; O^T += V^T P^T with 16 head dims per MMA
+//     row block. P is carried as a 16-bit head plus a 16-bit remainder, so its
+//     rounding stays below 2^-16 relative: with G <= 4 the remainder rides in
+//     the MMA's spare columns (column c < G: head of p for head c, G <= c < 2G:
+//     remainder of p for head c - G, their sum taken at the end), with G = 8 in
+//     a second MMA. The score accumulators are moved into the layout of P^T by
+//     an in-register transpose (movmatrix). FP8 pages are converted exactly to
+//     f16 (cvt e4m3x2 -> f16x2) and q is brought into f16 range by a power of
+//     two that the score scale undoes; the page's K scale multiplies the
+//     scores and its V scale the probabilities, never the elements.
+//   - Every kernel allows programmatic dependent launch: set-up that reads no
 //     data of the previous kernel runs while that kernel finishes.
 #include <cfloat>
 #include <cstdio>
@@ -70,11 +69,12 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
 enum : int { kFirst = 1, kLast = 2, kRing = 4, kPending = 8 };
 
 struct TileMeta {
-  const uint8_t* ksrc;   // first K row of the tile; its V rows follow the block's
-                         // (or the ring's) K rows
+  const uint8_t* ksrc;   // K row of frame row 0 (store: the tile's first row in its
+                         // block; ring: the frame's first slot); V rows follow the
+                         // block's (or the ring's) K rows
   int hidx;              // head of the call (b * Hkv + h)
   int rows;              // row0 | row1 << 8 | flags << 16: frame rows [row0, row1)
-  int p0;                // ring tiles: position of row row0
+  int p0;                // ring tiles: position of frame row 0
   float ks;              // K scale of the page
   float vrel;            // V scale of the page / the head's V scale
   int pad;
@@ -94,7 +94,7 @@ struct Dec {
   static constexpr int ELT = FP8 ? 1 : 2;
   static constexpr int RB = D * ELT;           // bytes per row
   static constexpr int TR = 4096 / RB;         // rows per tile: 4 KB of K, 4 KB of V
-  static constexpr int NCW = G * D >= 1024 ? 4 : 8;   // warps (one unit range each)
+  static constexpr int NCW = G * D >= 1024 ? 4 : 8;   // warps per CTA
   static constexpr int NT = NCW * 32;
   static constexpr int SPW = 2;                // stages per warp
   static constexpr int NSTAGE = NCW * SPW;
@@ -102,45 +102,32 @@ struct Dec {
   static constexpr int KV_BYTES = TR * RB;
   static constexpr int Q_BYTES = G * D * 2;
   static constexpr int STAGE_BYTES = 2 * KV_BYTES + ((Q_BYTES + 127) / 128) * 128;
-  static constexpr int NJ = TR / 8;            // score n-tiles (8 keys each)
-  static constexpr int NU = TR / 16;           // p.v k-steps (16 keys each)
-  static constexpr int KS = D / 16;            // q.k k-steps (16 dims each)
-  static constexpr int MT = D / 16;            // p.v m-tiles (16 dims each)
-  static constexpr int EC = 16 / ELT;          // elements per 16-byte chunk
-  static constexpr int KCPT = RB / 64;         // K chunks per lane column (1, 2 or 4)
-  static constexpr bool SPLIT = true;          // p = 16-bit head + 16-bit remainder
+  static constexpr int MK = TR / 16;           // 16-key row blocks per tile
+  static constexpr int KS = D / 16;            // score k-steps (16 dims each)
+  static constexpr int MT = D / 16;            // P.V row blocks (16 dims each)
+  static constexpr bool PACK = G <= 4;         // p remainder in the spare MMA columns
   static_assert(TR >= 16 && TR <= 64 && 64 % TR == 0, "tiles tile a page");
 
   static constexpr int OFF_META = NSTAGE * STAGE_BYTES;
   static constexpr int OFF_BAR = OFF_META + NCW * NMR * (int)sizeof(TileMeta);
   static constexpr int OFF_HEADS = OFF_BAR + NSTAGE * 8;
+  // global plan: head_off (i64), page_off (i32), len, n, r (i32), head scales (2 x f32)
   static size_t smem_bytes(int nh) {
-    // head_off (i64), page_off (i32), len, n, r (i32), head scales (2 x f32)
     return 128 + OFF_HEADS + (size_t)(nh + 1) * 8 + (size_t)(nh + 1) * 4 +
            (size_t)nh * 4 * 3 + (size_t)nh * 8 + 64;
   }
-  // per-head (cluster) mode: a merge area after the head arrays, one slot of
-  // (o [G][D], m [G], l [G]) per warp and one for the CTA
+  // per-head clusters: 16 ints of head state, then one slot of (o [G][D],
+  // m [G], l [G]) per warp and one for the CTA
   static constexpr int SLOT = G * D + 2 * G;   // floats
-  __host__ __device__ static size_t merge_off(int nh) {
-    return ((size_t)OFF_HEADS + (size_t)(nh + 1) * 12 + (size_t)nh * 20 + 15) / 16 * 16;
+  static constexpr int OFF_MERGE = OFF_HEADS + 64;
+  static size_t smem_bytes_cluster() {
+    return 128 + OFF_MERGE + (size_t)(NCW + 1) * SLOT * 4 + 64;
   }
-  static size_t smem_bytes_cluster(int nh) {
-    return 128 + merge_off(nh) + (size_t)(NCW + 1) * SLOT * 4 + 64;
-  }
-
-  // unpermuted 16-byte K chunk i (0 .. KCPT-1) of lane column t
-  __device__ static int kchunk(int t, int i) { return RB == 256 ? t + 4 * i : KCPT * t + i; }
-  // element (dim) behind q.k k-step s, slot e (0..3) of lane column t:
-  // e = 0, 1 are the fragment's k = 2t, 2t+1; e = 2, 3 are k = 2t+8, 2t+9
-  __device__ static int kdim(int t, int s, int e) {
-    const int se = 4 * s + e;
-    return kchunk(t, se / EC) * EC + se % EC;
-  }
-  // dim of row g (hi = 0) or row g + 8 (hi = 1) of p.v m-tile i
-  __device__ static int vdim(int g, int i, int hi) {
-    if (RB == 256) return (i < 4 ? 8 * g + 2 * i : 64 + 8 * g + 2 * (i - 4)) + hi;
-    return (D / 8) * g + 2 * i + hi;
+  // head dim of P.V accumulator row block i, lane group g, upper half hi:
+  // BF16 V^T comes from transposed 8x8 matrix loads (dims in order), FP8 V^T
+  // from byte pairs (dims 2g and 2g + 1 of the 16-dim chunk)
+  __host__ __device__ static int vdim(int i, int g, int hi) {
+    return FP8 ? 16 * i + 2 * g + hi : 16 * i + 8 * hi + g;
   }
 };
 
@@ -162,9 +149,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-
 // Tiles of one head: its store pages (tile = TR rows of a page), then the
-// TR-row frames its ring slots r .. n-1 fall in.
+// TR-position frames its ring slots r .. n-1 fall in.
 template <int TR>
 __device__ __forceinline__ int head_tiles(int len, int n, int r) {
   const int live = n - r;
@@ -188,13 +174,28 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n"
                "barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// fp32 at the same shared-memory offset as `local` in CTA `rank` of the cluster
-__device__ __forceinline__ float ld_cluster_f32(const float* local, uint32_t rank) {
+// The same rendezvous without ordering memory: every thread of the cluster has
+// got here (its earlier loads have returned their values).
+__device__ __forceinline__ void cluster_sync_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;\n"
+               "barrier.cluster.wait.aligned;" ::: "memory");
+}
+// shared-memory address of `local`'s counterpart in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t cluster_addr(const void* local, uint32_t rank) {
   uint32_t remote;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
                : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
+  return remote;
+}
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
   float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ int4 ld_dsmem_v4(uint32_t addr) {
+  int4 v;
+  asm volatile("ld.shared::cluster.v4.s32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr) : "memory");
   return v;
 }
 
@@ -215,6 +216,24 @@ __device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a1, uin
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
   }
+}
+// four 8x8 16-bit matrices from shared memory; lane i gives the address of row
+// i % 8 of matrix i / 8, register j receives matrix j
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+// the same, each matrix transposed
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+// transpose of an 8x8 16-bit matrix held one 32-bit pair per lane (lane 4g + t:
+// row g, columns 2t and 2t + 1)
+__device__ __forceinline__ uint32_t movm_t(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
 }
 
 // two f32 -> packed 16-bit pair (x0 in the low half), round to nearest even
@@ -248,31 +267,70 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
   return r;
 }
+// the 16-bit part a P^T column carries: 0 = head, 1 = remainder, 2 = none
+__device__ __forceinline__ uint32_t pick16(int role, uint32_t head, uint32_t rem) {
+  return role == 0 ? head : (role == 1 ? rem : 0u);
+}
+
+// Descriptor of one tile from the head's lengths (store length len, tokens n,
+// resolved r): store tile `idx` (kind 0) or ring frame `idx` (kind 1, the TR
+// positions from idx * TR). Ring frames keep only positions in [r, n).
+template <class T>
+__device__ __forceinline__ TileMeta tile_meta(const CacheView& c, long long hi, int hidx,
+                                              int kind, int idx, int len, int n, int r,
+                                              float hs_k, float hs_v) {
+  constexpr int TR = T::TR, RB = T::RB;
+  TileMeta mt;
+  mt.hidx = hidx;
+  mt.pad = 0;
+  int row0, row1, flags = 0;
+  if (kind == 0) {
+    const int j = idx * TR / kBlockSlots;
+    row0 = 0;
+    row1 = min(TR, len - idx * TR);
+    const long long blk = c.block_table[hi * c.max_blocks + j];
+    if (T::FP8) {
+      mt.ks = c.bt_scale[(hi * c.max_blocks + j) * 2];
+      mt.vrel = c.bt_scale[(hi * c.max_blocks + j) * 2 + 1] / hs_v;
+    } else {
+      mt.ks = mt.vrel = 1.0f;
+    }
+    mt.ksrc = block_k(c, blk) + (long long)((idx * TR) % kBlockSlots) * RB;
+    mt.p0 = 0;
+  } else {
+    const int f0 = idx * TR;
+    // clipped to the frame: a frame wholly below r (resolved since a snapshot
+    // planned it) or above n comes out empty
+    const int lo = min(max(f0, r), f0 + TR), hi_p = max(lo, min(f0 + TR, n));
+    row0 = lo - f0;
+    row1 = hi_p - f0;
+    flags = kRing | (lo < n - c.W ? kPending : 0);
+    mt.ks = hs_k;
+    mt.vrel = 1.0f;
+    mt.ksrc = ring_k(c, hi) + (long long)(f0 % c.R) * RB;
+    mt.p0 = f0;
+  }
+  mt.rows = row0 | row1 << 8 | flags << 16;
+  return mt;
+}
 
 // CS = 0: one plan over every head of the call, cut into equal tile ranges,
 // partials merged by k_decode_combine. CS > 0 (calls with few heads): one
-// cluster of CS CTAs per head; the CTAs split the head's tiles, each merges its
-// warps' partials in shared memory, and the cluster merges the CTAs' partials
-// through distributed shared memory and writes the output: no global plan, no
-// workspace, no combine kernel.
+// cluster of CS CTAs per head, planned from the head's snapshot when use_snap
+// (copies issued before the dependency wait); the cluster merges its warps'
+// partials in shared memory and across CTAs through distributed shared memory
+// and writes the output: no global plan, no workspace, no combine kernel.
 template <class T, int CS>
 __global__ void __launch_bounds__(T::NT, 1)
 k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
-               const uint16_t* __restrict__ q, int n_ranges, double inv_ranges) {
-  constexpr int D = T::D, G = T::G, RB = T::RB, TR = T::TR, NSTAGE = T::NSTAGE,
-                SPW = T::SPW, NJ = T::NJ, NU = T::NU, KS = T::KS, MT = T::MT, NMR = T::NMR;
-  constexpr bool FP8 = T::FP8;
+               const uint16_t* __restrict__ q, int n_ranges, double inv_ranges, int use_snap) {
+  constexpr int D = T::D, G = T::G, RB = T::RB, TR = T::TR, SPW = T::SPW, MK = T::MK,
+                KS = T::KS, MT = T::MT, NMR = T::NMR, NCW = T::NCW;
+  constexpr bool FP8 = T::FP8, PACK = T::PACK;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 127) & ~(uintptr_t)127);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + T::OFF_BAR);
   const int NH = batch * c.Hkv;
-  long long* head_off = reinterpret_cast<long long*>(smem + T::OFF_HEADS);   // [NH + 1]
-  int* page_off = reinterpret_cast<int*>(head_off + NH + 1);                 // [NH + 1]
-  int* s_len = page_off + NH + 1;
-  int* s_n = s_len + NH;
-  int* s_r = s_n + NH;
-  float* s_hscale = reinterpret_cast<float*>(s_r + NH);                      // [NH][2]
-
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const long long hi0 = (long long)layer * c.Bmax * c.Hkv;   // first head of this layer
   TileMeta* ring = reinterpret_cast<TileMeta*>(smem + T::OFF_META) + warp * NMR;
@@ -281,58 +339,192 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   // that kernel. Stale V rows of a stage are multiplied by p = 0, so they must
   // hold numbers: start from zeros, not from whatever bits shared memory held
   // (stale K rows only produce scores that are then masked).
-  for (int i = tid; i < NSTAGE * (T::KV_BYTES / 16); i += T::NT) {
+  for (int i = tid; i < T::NSTAGE * (T::KV_BYTES / 16); i += T::NT) {
     const int st = i / (T::KV_BYTES / 16), off = i % (T::KV_BYTES / 16);
     reinterpret_cast<uint4*>(smem + st * T::STAGE_BYTES + T::KV_BYTES)[off] =
         make_uint4(0u, 0u, 0u, 0u);
   }
-  // warm L2 with this layer's lengths and block tables (read after the wait)
-  {
-    const int NHL = batch * c.Hkv;
-    const long long bt_lines = ((long long)NHL * c.max_blocks * 4 + 127) / 128;
-    const char* btp = reinterpret_cast<const char*>(c.block_table + hi0 * c.max_blocks);
-    for (long long i = (long long)blockIdx.x * T::NT + tid; i < bt_lines;
-         i += (long long)gridDim.x * T::NT)
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(btp + i * 128));
-    if (tid < 4 && blockIdx.x < 8) {
-      const char* arr = tid == 0   ? reinterpret_cast<const char*>(c.store_len + hi0)
-                        : tid == 1 ? reinterpret_cast<const char*>(c.tok_n + hi0)
-                        : tid == 2 ? reinterpret_cast<const char*>(c.tok_r + hi0)
-                                   : reinterpret_cast<const char*>(c.head_scale + hi0 * 2);
-      const int bytes = tid == 3 ? NHL * 8 : NHL * 4;   // this layer's slice only
-      for (int j = blockIdx.x; j * 128 < bytes; j += 8)
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(arr + j * 128));
-    }
-  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // before any bulk copy
   if (lane < SPW) mbar_init(&full[warp * SPW + lane], 1);
   fence_mbar_init();
-  pdl_wait();                 // the previous kernel's writes are visible from here on
-  pdl_launch_dependents();
 
-  // ---- units and pages of every head of the call; exclusive prefix
-  // cluster mode: the head of this CTA's cluster
+  // stage the K and V rows [row0, row1) of `mt` for tile k (one lane). phase 0:
+  // the whole tile (arrive + K/V + q with a head's first tile); 1: K/V only, no
+  // arrival (before the dependency wait); 2: the arrival and q of a tile whose
+  // K/V phase 1 issued
+  auto issue = [&](const TileMeta& mt, int k, int phase) {
+    const int s = warp * SPW + k % SPW;
+    uint8_t* kdst = smem + s * T::STAGE_BYTES;
+    uint8_t* vdst = kdst + T::KV_BYTES;
+    const int row0 = mt.rows & 0xFF, row1 = (mt.rows >> 8) & 0xFF;
+    const uint32_t nb = row1 > row0 ? (uint32_t)(row1 - row0) * RB : 0u;
+    const long long voff = (long long)((mt.rows >> 16) & kRing ? c.R : kBlockSlots) * RB;
+    // q only with a warp's first tile of a head: the tiles after it keep the
+    // head's q fragments in registers
+    const bool with_q = ((mt.rows >> 16) & kFirst) != 0;
+    const uint32_t qb = with_q ? (uint32_t)T::Q_BYTES : 0u;
+    if (phase == 0) mbar_arrive_expect_tx(&full[s], 2u * nb + qb);
+    if (phase == 1) mbar_expect_tx(&full[s], 2u * nb);
+    if (phase == 2) mbar_arrive_expect_tx(&full[s], qb);
+    if (phase != 2 && nb > 0) {
+      bulk_g2s(kdst + row0 * RB, mt.ksrc + (long long)row0 * RB, nb, &full[s]);
+      bulk_g2s(vdst + row0 * RB, mt.ksrc + voff + (long long)row0 * RB, nb, &full[s]);
+    }
+    if (with_q && phase != 1) {
+      const int b = mt.hidx / c.Hkv, h = mt.hidx % c.Hkv;
+      bulk_g2s(vdst + T::KV_BYTES, q + ((long long)b * c.Hq + (long long)h * G) * D,
+               T::Q_BYTES, &full[s]);
+    }
+  };
+
+  // ================================================= plan: this warp's tiles
+  int nt = 0;                       // tiles of this warp
+  unsigned pre_mask = 0;            // tiles k < SPW whose K/V went out before the wait
+  TileMeta pre_mt;                  // lane k < SPW: what went out for tile k
+  // cluster mode
+  int* cst = reinterpret_cast<int*>(smem + T::OFF_HEADS);
+  float* mslot = reinterpret_cast<float*>(smem + T::OFF_MERGE);
   const int hsel = CS > 0 ? (int)(blockIdx.x / (CS > 0 ? CS : 1)) : 0;
+  const int crank = CS > 0 ? (int)(blockIdx.x % (CS > 0 ? CS : 1)) : 0;
+  int sp_s = 0, f0_s = 0, a_first = 0, cnt = 0, e0 = 0, E_store = 0, fx0 = 0;
+  // global plan
+  long long* head_off = reinterpret_cast<long long*>(smem + T::OFF_HEADS);
+  int* page_off = reinterpret_cast<int*>(head_off + NH + 1);
+  int* s_len = page_off + NH + 1;
+  int* s_n = s_len + NH;
+  int* s_r = s_n + NH;
+  float* s_hscale = reinterpret_cast<float*>(s_r + NH);
+  int gp0 = 0, h_gs = 0, h_ge = 0;
+  long long v_range = 0;
+
   if constexpr (CS > 0) {
+    constexpr int NW = CS * NCW;              // warps of the cluster
+    const int v = crank * NCW + warp;
+    const long long hi = hi0 + hsel;
+    // cst: [0..3] rank 0's copy of the snapshot, [4..6] snapshot planned on,
+    // [8..10] lengths now, [12..13] FP8 head scales
+    auto split = [&](int len_s, int n_s, int r_s) {
+      sp_s = (len_s + TR - 1) / TR;
+      f0_s = r_s / TR;
+      const int P_s = head_tiles<TR>(len_s, n_s, r_s);
+      const int qq = P_s / NW, rem = P_s % NW;
+      cnt = qq + (v < rem ? 1 : 0);
+      a_first = v * qq + min(v, rem);
+      e0 = (v - rem + NW) % NW;               // extra tiles continue the round
+    };
+    // warm L2 with the head's block-table row and lengths (read after the wait)
+    if (warp == NCW - 1) {
+      const char* btp = reinterpret_cast<const char*>(c.block_table + hi * c.max_blocks);
+      for (int i = lane; i * 128 < c.max_blocks * 4; i += 32)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(btp + i * 128));
+      if (lane == 0) {
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(c.store_len + hi));
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(c.tok_n + hi));
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(c.tok_r + hi));
+      }
+    }
+    if (use_snap) {
+      // ---- before the wait: the snapshot (one copy for the whole cluster)
+      if (crank == 0 && tid == 0) {
+        int4 sv = w.snap[hi];
+        if (!(sv.x >= 0 && sv.x <= sv.z && sv.z <= sv.y && sv.y <= c.max_seq_len &&
+              sv.y - sv.z <= c.R))
+          sv = make_int4(0, 0, 0, 0);
+        *reinterpret_cast<int4*>(cst) = sv;
+      }
+      cluster_sync_all();
+      if (tid == 0) {
+        const int4 sv = ld_dsmem_v4(cluster_addr(cst, 0));
+        cst[4] = sv.x;
+        cst[5] = sv.y;
+        cst[6] = sv.z;
+      }
+      __syncthreads();
+      const int len_s = cst[4], n_s = cst[5], r_s = cst[6];
+      split(len_s, n_s, r_s);
+      // the warp's first tiles, unless they can still grow (the last store
+      // tile and the last ring frame when partly filled)
+      const int k = lane;
+      bool pre = false;
+      if (k < SPW && k < cnt) {
+        const int item = a_first + k;
+        const int kind = item < sp_s ? 0 : 1;
+        const int idx = kind == 0 ? item : f0_s + (item - sp_s);
+        const bool edge = kind == 0 ? (idx == sp_s - 1 && len_s % TR != 0)
+                                    : (idx == (n_s - 1) / TR && n_s % TR != 0);
+        if (!edge) {
+          pre_mt = tile_meta<T>(c, hi, hsel, kind, idx, len_s, n_s, r_s, 1.f, 1.f);
+          pre_mt.rows |= (k == 0 ? kFirst : 0) << 16;
+          issue(pre_mt, k, 1);
+          pre = true;
+        }
+      }
+      pre_mask = __ballot_sync(0xffffffffu, pre);
+    }
+    pdl_wait();                 // the previous kernel's writes are visible from here on
+    pdl_launch_dependents();
+    // the arrivals (and q, an input of this call) of the tiles issued early
+    if ((pre_mask >> lane) & 1) issue(pre_mt, lane, 2);
     if (tid == 0) {
-      const long long hi = hi0 + hsel;
       const int len = c.store_len[hi], n = c.tok_n[hi], r = c.tok_r[hi];
-      s_len[hsel] = len;
-      s_n[hsel] = n;
-      s_r[hsel] = r;
-      s_hscale[2 * hsel] = FP8 ? c.head_scale[hi * 2] : 1.0f;
-      s_hscale[2 * hsel + 1] = FP8 ? c.head_scale[hi * 2 + 1] : 1.0f;
-      head_off[hsel] = 0;
-      head_off[hsel + 1] = len + (n - r);
-      page_off[hsel] = 0;
-      page_off[hsel + 1] = head_tiles<TR>(len, n, r);
+      cst[8] = len;
+      cst[9] = n;
+      cst[10] = r;
+      reinterpret_cast<float*>(cst)[12] = FP8 ? c.head_scale[hi * 2] : 1.0f;
+      reinterpret_cast<float*>(cst)[13] = FP8 ? c.head_scale[hi * 2 + 1] : 1.0f;
+      if (!use_snap) {
+        cst[4] = len;
+        cst[5] = n;
+        cst[6] = r;
+      }
+      if (crank == 0) {
+        if (w.snap) w.snap[hi] = make_int4(len, n, r, 0);
+        atomicAdd(&c.ctr->slots_decoded, (unsigned long long)(len + (n - r)));
+        if (blockIdx.x == 0) atomicAdd(&c.ctr->decode_calls, 1ull);
+      }
     }
     __syncthreads();
+    const int len_s = cst[4], n_s = cst[5], r_s = cst[6];
+    const int len = cst[8], n = cst[9], r = cst[10];
+    if (!use_snap) split(len_s, n_s, r_s);
+    // tiles that are new since the snapshot: store tiles past its last one,
+    // ring frames past its last one (and not below the current first)
+    const int sp_c = (len + TR - 1) / TR;
+    E_store = max(0, sp_c - sp_s);
+    const int nfr_s = head_tiles<TR>(0, n_s, r_s);
+    fx0 = max(nfr_s > 0 ? f0_s + nfr_s : r / TR, r / TR);
+    const int E_ring = n > r ? max(0, (n - 1) / TR - fx0 + 1) : 0;
+    const int E = E_store + E_ring;
+    nt = cnt + (E > e0 ? (E - e0 + NW - 1) / NW : 0);
+    if (lane < G) {   // an empty partial until the warp's last tile replaces it
+      mslot[warp * T::SLOT + G * D + lane] = -INFINITY;
+      mslot[warp * T::SLOT + G * D + G + lane] = 0.f;
+    }
   } else {
+    // warm L2 with this layer's lengths and block tables (read after the wait)
+    {
+      const long long bt_lines = ((long long)NH * c.max_blocks * 4 + 127) / 128;
+      const char* btp = reinterpret_cast<const char*>(c.block_table + hi0 * c.max_blocks);
+      for (long long i = (long long)blockIdx.x * T::NT + tid; i < bt_lines;
+           i += (long long)gridDim.x * T::NT)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(btp + i * 128));
+      if (tid < 4 && blockIdx.x < 8) {
+        const char* arr = tid == 0   ? reinterpret_cast<const char*>(c.store_len + hi0)
+                          : tid == 1 ? reinterpret_cast<const char*>(c.tok_n + hi0)
+                          : tid == 2 ? reinterpret_cast<const char*>(c.tok_r + hi0)
+                                     : reinterpret_cast<const char*>(c.head_scale + hi0 * 2);
+        const int bytes = tid == 3 ? NH * 8 : NH * 4;   // this layer's slice only
+        for (int j = blockIdx.x; j * 128 < bytes; j += 8)
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(arr + j * 128));
+      }
+    }
+    pdl_wait();
+    pdl_launch_dependents();
+    // ---- units and pages of every head of the call; exclusive prefix
     const int per = (NH + T::NT - 1) / T::NT;
     const int h0 = tid * per, h1 = min(NH, h0 + per);
     long long su = 0;
     int sp = 0;
-    auto pages = [](int len, int live, int r) { return head_tiles<TR>(len, r + live, r); };
     for (int h = h0; h < h1; ++h) {
       const int len = c.store_len[hi0 + h], n = c.tok_n[hi0 + h], r = c.tok_r[hi0 + h];
       s_len[h] = len;
@@ -341,7 +533,7 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
       s_hscale[2 * h] = FP8 ? c.head_scale[(hi0 + h) * 2] : 1.0f;
       s_hscale[2 * h + 1] = FP8 ? c.head_scale[(hi0 + h) * 2 + 1] : 1.0f;
       su += len + (n - r);
-      sp += pages(len, n - r, r);
+      sp += head_tiles<TR>(len, n, r);
     }
     long long iu = su;
     int ip = sp;
@@ -362,191 +554,126 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
       head_off[h] = eu;
       page_off[h] = ep;
       eu += s_len[h] + (s_n[h] - s_r[h]);
-      ep += pages(s_len[h], s_n[h] - s_r[h], s_r[h]);
+      ep += head_tiles<TR>(s_len[h], s_n[h], s_r[h]);
     }
     if (tid == T::NT - 1) {
       head_off[NH] = eu;
       page_off[NH] = ep;
     }
     __syncthreads();
-  }
-  int gp0 = 0, nt = 0, h_gs = 0, h_ge = 0;
-  long long v_range = 0;
-  float* mslot = reinterpret_cast<float*>(smem + T::merge_off(NH));   // cluster mode
-  if constexpr (CS > 0) {
-    // the head's tiles, split evenly over the cluster's CTAs, then over warps
-    const int P = page_off[hsel + 1];
-    const int crank = (int)(blockIdx.x % CS);
-    const int per_c = (P + CS - 1) / CS;
-    const int c0 = min(P, crank * per_c), c1 = min(P, c0 + per_c);
-    const int per_w = (c1 - c0 + T::NCW - 1) / T::NCW;
-    gp0 = min(c1, c0 + warp * per_w);
-    nt = min(c1, gp0 + per_w) - gp0;
-    h_gs = h_ge = hsel;
-    if (crank == 0 && tid == 0) {
-      atomicAdd(&c.ctr->slots_decoded, (unsigned long long)head_off[hsel + 1]);
-      if (blockIdx.x == 0) atomicAdd(&c.ctr->decode_calls, 1ull);
+    const long long total = head_off[NH];
+    const int P = page_off[NH];   // tiles of the call
+    // Range v holds tiles [v S, (v + 1) S), S = ceil(P / ranges): a tile costs
+    // the same compute full or not, so whole tiles are what gets balanced.
+    const int S = tiles_per_warp(P, n_ranges, inv_ranges);
+    if (blockIdx.x == 0 && tid == 0) {   // one thread, launches are ordered
+      c.ctr->slots_decoded += (unsigned long long)total;
+      c.ctr->decode_calls += 1ull;
     }
-    if (lane < G) {   // an empty partial until the warp's last tile replaces it
-      mslot[warp * T::SLOT + G * D + lane] = -INFINITY;
-      mslot[warp * T::SLOT + G * D + G + lane] = 0.f;
+    // heads without a single slot get zeros (nobody else writes them)
+    for (int h = blockIdx.x; h < NH; h += gridDim.x) {
+      if (page_off[h + 1] != page_off[h]) continue;
+      const int b = h / c.Hkv, kh = h % c.Hkv;
+      for (int i = tid; i < G * D; i += T::NT) {
+        const long long oi = ((long long)b * c.Hq + (long long)kh * G) * D + i;
+        if (oa.f32) static_cast<float*>(oa.out)[oi] = 0.f;
+        else static_cast<uint16_t*>(oa.out)[oi] = 0;
+        if (oa.lse && i % D == 0) oa.lse[(long long)b * c.Hq + kh * G + i / D] = -INFINITY;
+      }
     }
-  } else {
-  const long long total = head_off[NH];
-  const int P = page_off[NH];   // tiles of the call
-  // Range v holds tiles [v S, (v + 1) S), S = ceil(P / ranges): a tile costs
-  // the same compute full or not, so whole tiles are what gets balanced. The
-  // quotient is an fp64 estimate made exact by integer correction.
-  const int S = tiles_per_warp(P, n_ranges, inv_ranges);
-  if (blockIdx.x == 0 && tid == 0) {   // one thread, launches are ordered
-    c.ctr->slots_decoded += (unsigned long long)total;
-    c.ctr->decode_calls += 1ull;
-  }
-  // heads without a single slot get zeros (nobody else writes them)
-  for (int h = blockIdx.x; h < NH; h += gridDim.x) {
-    if (page_off[h + 1] != page_off[h]) continue;
-    const int b = h / c.Hkv, kh = h % c.Hkv;
-    for (int i = tid; i < G * D; i += T::NT) {
-      const long long oi = ((long long)b * c.Hq + (long long)kh * G) * D + i;
-      if (oa.f32) static_cast<float*>(oa.out)[oi] = 0.f;
-      else static_cast<uint16_t*>(oa.out)[oi] = 0;
-      if (oa.lse && i % D == 0) oa.lse[(long long)b * c.Hq + kh * G + i / D] = -INFINITY;
+    // Range v goes to warp v / gridDim.x of CTA v % gridDim.x: when fewer
+    // ranges than warps hold tiles, the busy ones are spread over every SM.
+    v_range = (long long)warp * gridDim.x + blockIdx.x;
+    if ((long long)blockIdx.x * S >= P) return;
+    // ---- this warp's tiles [gp0, gp0 + nt) and the heads h_gs .. h_ge they
+    // belong to (the number of heads h >= 1 with page_off[h] <= page)
+    gp0 = (int)min(v_range * S, (long long)P);
+    nt = min(gp0 + S, P) - gp0;
+    if (nt > 0) {
+      for (int base = 1; base < NH; base += 32) {
+        const int h = base + lane;
+        const int po = h < NH ? page_off[h] : P;
+        h_gs += __popc(__ballot_sync(0xffffffffu, po <= gp0));
+        h_ge += __popc(__ballot_sync(0xffffffffu, po <= gp0 + nt - 1));
+      }
     }
-  }
-  // Range v goes to warp v / gridDim.x of CTA v % gridDim.x: when fewer
-  // ranges than warps hold tiles, the busy ones are spread over every SM.
-  v_range = (long long)warp * gridDim.x + blockIdx.x;
-  if ((long long)blockIdx.x * S >= P) return;
-
-  // ---- this warp's tiles [gp0, gp0 + nt) and the heads h_gs .. h_ge they
-  // belong to (the number of heads h >= 1 with page_off[h] <= page)
-  gp0 = (int)min(v_range * S, (long long)P);
-  nt = min(gp0 + S, P) - gp0;
-  if (nt > 0) {
-    for (int base = 1; base < NH; base += 32) {
-      const int h = base + lane;
-      const int po = h < NH ? page_off[h] : P;
-      h_gs += __popc(__ballot_sync(0xffffffffu, po <= gp0));
-      h_ge += __popc(__ballot_sync(0xffffffffu, po <= gp0 + nt - 1));
-    }
-  }
   }
 
-  // descriptor of this warp's tile k (one lane per tile)
+  // descriptor of this warp's tile k (one lane per tile), from the lengths now
   auto make_meta = [&](int k) -> TileMeta {
     TileMeta mt;
-    const int gp = gp0 + k;
-    // head of page gp: the last h in [h_gs, h_ge] with page_off[h] <= gp
-    int h_lo = h_gs, h_hi = h_ge;
-    while (h_lo < h_hi) {
-      const int mid = (h_lo + h_hi + 1) >> 1;
-      if (page_off[mid] <= gp) h_lo = mid; else h_hi = mid - 1;
-    }
-    const int hidx = h_lo;
-    const int lp = gp - page_off[hidx];
-    const int len = s_len[hidx], n = s_n[hidx], r = s_r[hidx];
-    const int sp = (len + TR - 1) / TR;
-    const long long hi = hi0 + hidx;
-    int flags = (k == 0 || lp == 0 ? kFirst : 0) |
-                (k == nt - 1 || gp + 1 == page_off[hidx + 1] ? kLast : 0);
-    int row0, row1;
-    mt.hidx = hidx;
-    mt.p0 = 0;
-    mt.pad = 0;
-    if (lp < sp) {   // store tile lp: block lp * TR / 64, rows from (lp * TR) % 64
-      const int j = lp * TR / kBlockSlots;
-      const int rb = (lp * TR) % kBlockSlots;          // block row of frame row 0
-      row0 = 0;
-      row1 = min(TR, len - lp * TR);
-      const long long blk = c.block_table[hi * c.max_blocks + j];
-      if (FP8) {
-        mt.ks = c.bt_scale[(hi * c.max_blocks + j) * 2];
-        mt.vrel = c.bt_scale[(hi * c.max_blocks + j) * 2 + 1] / s_hscale[2 * hidx + 1];
+    if constexpr (CS > 0) {
+      const int len = cst[8], n = cst[9], r = cst[10];
+      int kind, idx;
+      if (k < cnt) {
+        const int item = a_first + k;
+        kind = item < sp_s ? 0 : 1;
+        idx = kind == 0 ? item : f0_s + (item - sp_s);
       } else {
-        mt.ks = mt.vrel = 1.0f;
+        const int e = e0 + (k - cnt) * CS * NCW;
+        kind = e < E_store ? 0 : 1;
+        idx = kind == 0 ? sp_s + e : fx0 + (e - E_store);
       }
-      mt.ksrc = block_k(c, blk) + (long long)rb * RB;
-    } else {         // ring tile: live units [TR*rp - off, TR*(rp+1) - off)
-      const int rp = lp - sp, off = r % TR, live = n - r;
-      const int a = max(TR * rp - off, 0), b = min(TR * (rp + 1) - off, live);
-      const int p0 = r + a;
-      const int slot0 = p0 % c.R;
-      row0 = slot0 % TR;
-      row1 = row0 + (b - a);
-      mt.p0 = p0;
-      flags |= kRing | (p0 < n - c.W ? kPending : 0);
-      mt.ks = s_hscale[2 * hidx];
-      mt.vrel = 1.0f;
-      mt.ksrc = ring_k(c, hi) + (long long)slot0 * RB;
+      const float* hs = reinterpret_cast<const float*>(cst) + 12;
+      mt = tile_meta<T>(c, hi0 + hsel, hsel, kind, idx, len, n, r, hs[0], hs[1]);
+      mt.rows |= ((k == 0 ? kFirst : 0) | (k == nt - 1 ? kLast : 0)) << 16;
+    } else {
+      const int gp = gp0 + k;
+      // head of page gp: the last h in [h_gs, h_ge] with page_off[h] <= gp
+      int h_lo = h_gs, h_hi = h_ge;
+      while (h_lo < h_hi) {
+        const int mid = (h_lo + h_hi + 1) >> 1;
+        if (page_off[mid] <= gp) h_lo = mid; else h_hi = mid - 1;
+      }
+      const int hidx = h_lo;
+      const int lp = gp - page_off[hidx];
+      const int len = s_len[hidx], n = s_n[hidx], r = s_r[hidx];
+      const int sp = (len + TR - 1) / TR;
+      mt = tile_meta<T>(c, hi0 + hidx, hidx, lp < sp ? 0 : 1, lp < sp ? lp : r / TR + (lp - sp),
+                        len, n, r, s_hscale[2 * hidx], s_hscale[2 * hidx + 1]);
+      mt.rows |= ((k == 0 || lp == 0 ? kFirst : 0) |
+                  (k == nt - 1 || gp + 1 == page_off[hidx + 1] ? kLast : 0)) << 16;
     }
-    mt.rows = row0 | row1 << 8 | flags << 16;
     return mt;
-  };
-  // stage the K rows, V rows and q of tile k (one lane)
-  auto issue = [&](const TileMeta& mt, int k) {
-    const int s = warp * SPW + k % SPW;
-    uint8_t* kdst = smem + s * T::STAGE_BYTES;
-    uint8_t* vdst = kdst + T::KV_BYTES;
-    const int row0 = mt.rows & 0xFF, row1 = (mt.rows >> 8) & 0xFF;
-    const uint32_t nb = (uint32_t)(row1 - row0) * RB;
-    const long long voff =
-        (long long)((mt.rows >> 16) & kRing ? c.R : kBlockSlots) * RB;
-    // q only with a warp's first tile of a head: the tiles after it keep the
-    // head's q fragments in registers (each bulk copy costs issue time)
-    const bool with_q = ((mt.rows >> 16) & kFirst) != 0;
-    mbar_arrive_expect_tx(&full[s], 2u * nb + (with_q ? (uint32_t)T::Q_BYTES : 0u));
-    bulk_g2s(kdst + row0 * RB, mt.ksrc, nb, &full[s]);
-    bulk_g2s(vdst + row0 * RB, mt.ksrc + voff, nb, &full[s]);
-    if (with_q) {
-      const int b = mt.hidx / c.Hkv, h = mt.hidx % c.Hkv;
-      bulk_g2s(vdst + T::KV_BYTES, q + ((long long)b * c.Hq + (long long)h * G) * D,
-               T::Q_BYTES, &full[s]);
-    }
   };
   // descriptors of tiles [k0, k0 + 32) into the warp's ring
   auto fill = [&](int k0) {
     const int k = k0 + lane;
     if (k < nt) ring[k % NMR] = make_meta(k);
   };
-  // first descriptors; lanes 0 .. SPW-1 stage their tiles at once
-  {
-    const int k = lane;
-    if (k < nt) {
-      const TileMeta mt = make_meta(k);
-      ring[k] = mt;
-      if (k < SPW) issue(mt, k);
-    }
-    fill(32);
-    __syncwarp();
-  }
+  fill(0);
+  fill(32);
+  __syncwarp();
+  if (lane < SPW && lane < nt && !((pre_mask >> lane) & 1)) issue(ring[lane], lane, 0);
+
 
   // ================= tiles of this warp
   const int g = lane >> 2, t = lane & 3;
   const float qscale = c.softmax_scale * kLog2e;
+  // P^T columns 2t and 2t + 1 of this lane: head, remainder or nothing
+  const int role0 = PACK ? (2 * t < G ? 0 : (2 * t < 2 * G ? 1 : 2)) : 0;
+  const int role1 = PACK ? (2 * t + 1 < G ? 0 : (2 * t + 1 < 2 * G ? 1 : 2)) : 0;
+  const int qh = PACK ? g % G : g;   // query head of this lane's q column
+  // This lane's row address for a matrix load: row 16 m + 8 ((lane >> 3) & 1) +
+  // (lane & 7), chunk cb + (lane >> 4), so registers 0..3 receive the matrices
+  // (rows 0-7, chunk cb), (rows 8-15, cb), (rows 0-7, cb + 1), (rows 8-15, cb + 1)
+  // of row block m. Row blocks start at multiples of 8 rows, so the chunk
+  // permutation of the row is that of lane & 7.
+  const int lrow = 8 * ((lane >> 3) & 1) + (lane & 7);
+  const int lsub = lane >> 4;
+  const int lx = RB == 64 ? ((lane & 7) >> 1) & 3 : (lane & 7);
+  auto lm_addr = [&](uint32_t base, int m, int cb) -> uint32_t {
+    return base + (uint32_t)((16 * m + lrow) * RB + 16 * ((cb + lsub) ^ lx));
+  };
+  constexpr int NKL = FP8 ? KS / 2 : KS;   // K matrix loads per row block
+  constexpr int NVL = FP8 ? MT / 2 : MT;   // V matrix loads per row block
 
-  // shared-memory byte offsets of this lane's fragment loads inside a tile:
-  // K rows 8j + g (the row permutation bits are g for every j), V rows
-  // 16u + 2t + {0, 1, 8, 9} (permutation bits 2t + {0, 1})
-  int koff[T::KCPT];
-#pragma unroll
-  for (int i = 0; i < T::KCPT; ++i)
-    koff[i] = g * RB + 16 * swz_chunk(RB, false, g, T::kchunk(t, i));
-  constexpr int VCHK = RB == 256 ? 2 : 1;
-  int voff[4][VCHK];
-#pragma unroll
-  for (int q4 = 0; q4 < 4; ++q4) {
-    const int rr = 2 * t + (q4 & 1) + 8 * (q4 >> 1);
-#pragma unroll
-    for (int ci = 0; ci < VCHK; ++ci)
-      voff[q4][ci] = rr * RB + (RB == 64 ? 8 * g
-                                          : 16 * swz_chunk(RB, true, rr, RB == 256 ? g + 8 * ci : g));
-  }
-
-  uint32_t qa[KS][2];          // q A-fragments (row g, k-steps)
-  float qmul = 0.f;            // score multiplier of row g (scale, log2 e, q's power of two)
+  uint32_t qb[KS][2];          // q B-fragments (column g, k-steps)
+  float qmul0 = 0.f, qmul1 = 0.f;   // score multipliers of columns 2t, 2t + 1
   int cur_hidx = -1;
-  float m_run = -INFINITY, l_run = 0.f;    // softmax state of head g (shared by its quad)
-  float oacc[MT][4];           // o^T: [dims g, g+8 of m-tile i] x [heads 2t, 2t+1]
+  float m0 = -INFINITY, m1 = -INFINITY;   // running max of columns 2t, 2t + 1
+  float l0 = 0.f, l1 = 0.f;               // this lane's part of their sums
+  float oacc[MT][4];           // o^T: [dims of row block i] x [columns 2t, 2t + 1]
 #pragma unroll
   for (int i = 0; i < MT; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
 
@@ -554,57 +681,42 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
     const int s = warp * SPW + (k % SPW);
     const bool ok = mbar_wait(&full[s], (k / SPW) & 1);
     if (!__all_sync(0xffffffffu, ok)) {
-      if (lane == 0) latch_error(c.ctr, FDMS_ERR_DEVICE);
+      // a copy did not land in time: latch the error, give the warp's other
+      // stage in flight one more bounded wait so that no copy is left pending
+      // into shared memory when the CTA leaves, and stop
+      if (lane == 0) {
+        latch_error(c.ctr, FDMS_ERR_DEVICE);
+        if (k + 1 < nt) mbar_wait(&full[warp * SPW + ((k + 1) % SPW)], ((k + 1) / SPW) & 1);
+      }
+      __syncwarp();
       break;
     }
     const TileMeta tm = ring[k % NMR];
-    struct {
-      int hidx, row0, row1, flags, p0, thresh, R;
-      float ks, vrel, vhead;
-      long long keep_base;
-    } mt;
-    mt.hidx = tm.hidx;
-    mt.row0 = tm.rows & 0xFF;
-    mt.row1 = (tm.rows >> 8) & 0xFF;
-    mt.flags = tm.rows >> 16;
-    mt.p0 = tm.p0;
-    mt.thresh = s_n[tm.hidx] - c.W;
-    mt.R = c.R;
-    mt.ks = tm.ks;
-    mt.vrel = tm.vrel;
-    mt.vhead = s_hscale[2 * tm.hidx + 1];
-    mt.keep_base = (hi0 + tm.hidx) * c.Rpad;
+    const int row0 = tm.rows & 0xFF, row1 = (tm.rows >> 8) & 0xFF, flags = tm.rows >> 16;
+    const int hidx = tm.hidx;
     const uint8_t* Ks = smem + s * T::STAGE_BYTES;
     const uint8_t* Vs = Ks + T::KV_BYTES;
     const uint16_t* Qs = reinterpret_cast<const uint16_t*>(Vs + T::KV_BYTES);
-    const int row0 = mt.row0, row1 = mt.row1;
+    const uint32_t ks_base = smem_addr(Ks), vs_base = smem_addr(Vs);
 
     // ---- q fragments of the head (only when the head changes)
-    if (mt.hidx != cur_hidx) {
-      cur_hidx = mt.hidx;
+    if (hidx != cur_hidx) {
+      cur_hidx = hidx;
       if constexpr (FP8) {
-        // f16 q scaled by 2^a so that max |q| of the row is in [2^14, 2^15)
-        // (bf16 -> f16 is then exact). The 4 KS dims of lane column t are one
-        // run of the row (the K chunks of the column are adjacent): 16-byte loads.
-        constexpr int NQ = 4 * KS;   // q values of this lane
-        static_assert(RB <= 128 && NQ == T::KCPT * T::EC, "one run of adjacent K chunks");
-        uint32_t qw[NQ / 2];          // bf16 pairs, in k-slot order
-        if (g < G) {
-          const uint4* src = reinterpret_cast<const uint4*>(Qs + g * D + NQ * t);
-#pragma unroll
-          for (int i = 0; i < NQ / 8; ++i) {
-            const uint4 x = src[i];
-            qw[4 * i] = x.x; qw[4 * i + 1] = x.y; qw[4 * i + 2] = x.z; qw[4 * i + 3] = x.w;
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < NQ / 2; ++i) qw[i] = 0u;
-        }
+        // f16 q scaled by 2^a so that max |q| of the head is in [2^14, 2^15)
+        // (bf16 -> f16 is then exact). K-slots 2t, 2t + 1, 2t + 8, 2t + 9 of
+        // k-step s are dims 16 s + 4t .. 16 s + 4t + 3 (the order the E4M3 K
+        // matrices give); the four lanes of a lane group hold a whole head.
+        uint2 qw[KS];
         float amax = 0.f;
 #pragma unroll
-        for (int i = 0; i < NQ / 2; ++i)
-          amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(qw[i] << 16)),
-                                   fabsf(__uint_as_float(qw[i] & 0xFFFF0000u))));
+        for (int s2 = 0; s2 < KS; ++s2) {
+          qw[s2] = *reinterpret_cast<const uint2*>(Qs + qh * D + 16 * s2 + 4 * t);
+          amax = fmaxf(amax, fmaxf(fmaxf(fabsf(__uint_as_float(qw[s2].x << 16)),
+                                         fabsf(__uint_as_float(qw[s2].x & 0xFFFF0000u))),
+                                   fmaxf(fabsf(__uint_as_float(qw[s2].y << 16)),
+                                         fabsf(__uint_as_float(qw[s2].y & 0xFFFF0000u)))));
+        }
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
         int ex = 0;
@@ -612,193 +724,202 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
         ex = max(-126, min(126, ex));
         const float up = __uint_as_float((uint32_t)(ex + 127) << 23);
         const float down = __uint_as_float((uint32_t)(127 - ex) << 23);
-        qmul = qscale * down;
+        const float qm = qscale * down;
 #pragma unroll
         for (int s2 = 0; s2 < KS; ++s2) {
-          qa[s2][0] = pack2<true>(__uint_as_float(qw[2 * s2] << 16) * up,
-                                  __uint_as_float(qw[2 * s2] & 0xFFFF0000u) * up);
-          qa[s2][1] = pack2<true>(__uint_as_float(qw[2 * s2 + 1] << 16) * up,
-                                  __uint_as_float(qw[2 * s2 + 1] & 0xFFFF0000u) * up);
+          qb[s2][0] = pack2<true>(__uint_as_float(qw[s2].x << 16) * up,
+                                  __uint_as_float(qw[s2].x & 0xFFFF0000u) * up);
+          qb[s2][1] = pack2<true>(__uint_as_float(qw[s2].y << 16) * up,
+                                  __uint_as_float(qw[s2].y & 0xFFFF0000u) * up);
         }
+        // column c carries query head c % G (c when G = 8); lane 4c holds its multiplier
+        qmul0 = __shfl_sync(0xffffffffu, qm, 4 * (2 * t));
+        qmul1 = __shfl_sync(0xffffffffu, qm, 4 * (2 * t + 1));
       } else {
-        qmul = qscale;
+        qmul0 = qmul1 = qscale;
 #pragma unroll
         for (int s2 = 0; s2 < KS; ++s2) {
-          const int d0 = T::kdim(t, s2, 0), d2 = T::kdim(t, s2, 2);
-          qa[s2][0] = g < G ? *reinterpret_cast<const uint32_t*>(Qs + g * D + d0) : 0u;
-          qa[s2][1] = g < G ? *reinterpret_cast<const uint32_t*>(Qs + g * D + d2) : 0u;
+          qb[s2][0] = *reinterpret_cast<const uint32_t*>(Qs + qh * D + 16 * s2 + 2 * t);
+          qb[s2][1] = *reinterpret_cast<const uint32_t*>(Qs + qh * D + 16 * s2 + 8 + 2 * t);
         }
       }
     }
-    if (mt.flags & kFirst) {
-      m_run = -INFINITY;
-      l_run = 0.f;
+    if (flags & kFirst) {
+      m0 = m1 = -INFINITY;
+      l0 = l1 = 0.f;
 #pragma unroll
       for (int i = 0; i < MT; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
     }
 
     // ---- visible rows of the tile frame: [row0, row1), less the pending ring
     // rows whose keep bit is 0 (one ring_keep byte per row, read only then)
-    const bool pend = (mt.flags & kPending) != 0;
+    const bool pend = (flags & kPending) != 0;
     const bool full_tile = row0 == 0 && row1 == TR && !pend;
     unsigned long long vmask = ~0ull;
     if (!full_tile) {
       vmask = (row1 >= 64 ? ~0ull : (1ull << row1) - 1ull) & ~((1ull << row0) - 1ull);
       if (pend) {
+        const int thresh = (CS > 0 ? cst[9] : s_n[hidx]) - c.W;
+        const long long keep_base = (hi0 + hidx) * c.Rpad;
 #pragma unroll
         for (int h2 = 0; h2 < (TR + 31) / 32; ++h2) {
           const int row = 32 * h2 + lane;
           bool drop = false;
           if (row < TR && row >= row0 && row < row1) {
-            const int p = mt.p0 + (row - row0);
-            drop = p < mt.thresh && c.ring_keep[mt.keep_base + p % mt.R] == 0;
+            const int p = tm.p0 + row;
+            drop = p < thresh && c.ring_keep[keep_base + p % c.R] == 0;
           }
           const unsigned bd = __ballot_sync(0xffffffffu, drop);
           vmask &= ~((unsigned long long)bd << (32 * h2));
         }
       }
-      vmask >>= 2 * t;   // bit 8j + e: row 8j + 2t + e of this lane
     }
 
-    // ---- scores of rows 8j + (0..7): S[head g][keys 8j + 2t, 8j + 2t + 1]
-    float sc[NJ][2];
-    const float mul = qmul * mt.ks;
+    // ---- scores S^T[key][column]: keys 16 m + g (elements 0, 1) and
+    // 16 m + g + 8 (elements 2, 3) of row block m, columns 2t and 2t + 1
+    float sc[MK][4];
+    {
+      uint32_t ka[MK][NKL][4];
 #pragma unroll
-    for (int j = 0; j < NJ; ++j) {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t kw[T::KCPT][4];   // key row 8j + g, this lane's chunks
+      for (int m = 0; m < MK; ++m)
 #pragma unroll
-      for (int i = 0; i < T::KCPT; ++i) {
-        const uint4 x = *reinterpret_cast<const uint4*>(Ks + 8 * j * RB + koff[i]);
-        kw[i][0] = x.x; kw[i][1] = x.y; kw[i][2] = x.z; kw[i][3] = x.w;
+        for (int j = 0; j < NKL; ++j) ldsm_x4(ka[m][j], lm_addr(ks_base, m, 2 * j));
+      float acc[MK][4];
+#pragma unroll
+      for (int m = 0; m < MK; ++m) acc[m][0] = acc[m][1] = acc[m][2] = acc[m][3] = 0.f;
+      if constexpr (FP8) {
+        // load j covers k-steps 2j (registers 0, 1) and 2j + 1 (registers 2, 3);
+        // a register holds E4M3 dims 4t .. 4t + 3 of its key row: the low pair
+        // is k-slots 2t, 2t + 1, the high pair k-slots 2t + 8, 2t + 9
+#pragma unroll
+        for (int j = 0; j < NKL; ++j)
+#pragma unroll
+          for (int hc = 0; hc < 2; ++hc)
+#pragma unroll
+            for (int m = 0; m < MK; ++m) {
+              const uint32_t r0 = ka[m][j][2 * hc], r8 = ka[m][j][2 * hc + 1];
+              mma16816<true>(acc[m], e4m3x2_to_f16x2(r0 & 0xFFFF), e4m3x2_to_f16x2(r8 & 0xFFFF),
+                             e4m3x2_to_f16x2(r0 >> 16), e4m3x2_to_f16x2(r8 >> 16),
+                             qb[2 * j + hc][0], qb[2 * j + hc][1]);
+            }
+      } else {
+        // load s is k-step s: chunks 2s (dims 16s .. 16s + 7) and 2s + 1
+#pragma unroll
+        for (int s2 = 0; s2 < KS; ++s2)
+#pragma unroll
+          for (int m = 0; m < MK; ++m)
+            mma16816<false>(acc[m], ka[m][s2][0], ka[m][s2][1], ka[m][s2][2], ka[m][s2][3],
+                            qb[s2][0], qb[s2][1]);
       }
+      const float mul0 = qmul0 * tm.ks, mul1 = qmul1 * tm.ks;
 #pragma unroll
-      for (int s2 = 0; s2 < KS; ++s2) {
-        uint32_t b0, b1;
-        if constexpr (FP8) {
-          const uint32_t wv = kw[(4 * s2) / 16][((4 * s2) % 16) / 4];   // 4 codes
-          b0 = e4m3x2_to_f16x2(wv & 0xFFFF);
-          b1 = e4m3x2_to_f16x2(wv >> 16);
-        } else {
-          const int se = 4 * s2;                      // span elements 4 s2 .. 4 s2 + 3
-          b0 = kw[se / 8][(se % 8) / 2];
-          b1 = kw[se / 8][(se % 8) / 2 + 1];
-        }
-        mma16816<FP8>(acc, qa[s2][0], 0u, qa[s2][1], 0u, b0, b1);
+      for (int m = 0; m < MK; ++m) {
+        sc[m][0] = acc[m][0] * mul0;
+        sc[m][1] = acc[m][1] * mul1;
+        sc[m][2] = acc[m][2] * mul0;
+        sc[m][3] = acc[m][3] * mul1;
       }
-      sc[j][0] = acc[0] * mul;
-      sc[j][1] = acc[1] * mul;
     }
     if (!full_tile) {
 #pragma unroll
-      for (int j = 0; j < NJ; ++j)
-#pragma unroll
-        for (int e = 0; e < 2; ++e)
-          if (!((vmask >> (8 * j + e)) & 1ull)) sc[j][e] = -INFINITY;
+      for (int m = 0; m < MK; ++m) {
+        if (!((vmask >> (16 * m + g)) & 1ull)) sc[m][0] = sc[m][1] = -INFINITY;
+        if (!((vmask >> (16 * m + g + 8)) & 1ull)) sc[m][2] = sc[m][3] = -INFINITY;
+      }
     }
 
-    // ---- online softmax for row (head) g; the 4 lanes of a quad share it.
-    // With no visible key so far the reference point is 0: every p is then
+    // ---- online softmax per column (the 8 lanes with this t share it). With
+    // no visible key so far the reference point is 0: every p is then
     // 2^-inf = 0 and so is the rescale of the (empty) accumulators.
-    float mx = -INFINITY;
+    float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < NJ; ++j) mx = fmaxf(mx, fmaxf(sc[j][0], sc[j][1]));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    const float mn = fmaxf(m_run, mx);
-    const float mref = mn == -INFINITY ? 0.f : mn;
-    const float alpha = fast_exp2(m_run - mref);
-    float pr[NJ][2];
-    float ls = 0.f;
-#pragma unroll
-    for (int j = 0; j < NJ; ++j) {
-      pr[j][0] = fast_exp2(sc[j][0] - mref);
-      pr[j][1] = fast_exp2(sc[j][1] - mref);
-      ls += pr[j][0] + pr[j][1];
+    for (int m = 0; m < MK; ++m) {
+      mx0 = fmaxf(mx0, fmaxf(sc[m][0], sc[m][2]));
+      mx1 = fmaxf(mx1, fmaxf(sc[m][1], sc[m][3]));
     }
-    l_run = l_run * alpha + ls;
-    m_run = mn;
-    // o^T columns are heads 2t, 2t+1: their rescale factors live in quads 2t, 2t+1
-    const float al_e = __shfl_sync(0xffffffffu, alpha, 8 * t);
-    const float al_o = __shfl_sync(0xffffffffu, alpha, 8 * t + 4);
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    }
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+    const float mr0 = mn0 == -INFINITY ? 0.f : mn0, mr1 = mn1 == -INFINITY ? 0.f : mn1;
+    const float al0 = fast_exp2(m0 - mr0), al1 = fast_exp2(m1 - mr1);
+    float pr[MK][4];
+    float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+    for (int m = 0; m < MK; ++m) {
+      pr[m][0] = fast_exp2(sc[m][0] - mr0);
+      pr[m][1] = fast_exp2(sc[m][1] - mr1);
+      pr[m][2] = fast_exp2(sc[m][2] - mr0);
+      pr[m][3] = fast_exp2(sc[m][3] - mr1);
+      ls0 += pr[m][0] + pr[m][2];
+      ls1 += pr[m][1] + pr[m][3];
+    }
+    l0 = l0 * al0 + ls0;
+    l1 = l1 * al1 + ls1;
+    m0 = mn0;
+    m1 = mn1;
 #pragma unroll
     for (int i = 0; i < MT; ++i) {
-      oacc[i][0] *= al_e;
-      oacc[i][1] *= al_o;
-      oacc[i][2] *= al_e;
-      oacc[i][3] *= al_o;
+      oacc[i][0] *= al0;
+      oacc[i][1] *= al1;
+      oacc[i][2] *= al0;
+      oacc[i][3] *= al1;
     }
 
-    // ---- o^T += V^T p^T, keys 16u .. 16u + 15 per k-step
+    // ---- P^T B-fragments: 16-bit head and remainder of p * (page V scale /
+    // head V scale), moved from the S^T layout (lane 4g + t: key g, columns
+    // 2t, 2t + 1) to the B layout (lane 4g + t: keys 2t, 2t + 1 of column g)
+    uint32_t bh[MK][2], bl[MK][2];
 #pragma unroll
-    for (int u = 0; u < NU; ++u) {
-      // p^T B fragment: (keys 16u + 2t, +1) and (16u + 8 + 2t, +1) of head g
-      const float p0 = pr[2 * u][0] * mt.vrel, p1 = pr[2 * u][1] * mt.vrel;
-      const float p2 = pr[2 * u + 1][0] * mt.vrel, p3 = pr[2 * u + 1][1] * mt.vrel;
-      const uint32_t bh0 = pack2<FP8>(p0, p1), bh1 = pack2<FP8>(p2, p3);
-      uint32_t bl0 = 0u, bl1 = 0u;
-      if constexpr (T::SPLIT) {
-        const float2 f0 = unpack2<FP8>(bh0), f1 = unpack2<FP8>(bh1);
-        bl0 = pack2<FP8>(p0 - f0.x, p1 - f0.y);
-        bl1 = pack2<FP8>(p2 - f1.x, p3 - f1.y);
-      }
-      // V rows 16u + 2t + {0, 1, 8, 9}: the dims of lane group g
-      const uint8_t* Vu = Vs + 16 * u * RB;
-      if constexpr (RB == 64) {     // FP8, D = 64: 8 bytes (8 dims) of lane group g per row
-        uint2 x[4];
+    for (int m = 0; m < MK; ++m) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) x[i] = *reinterpret_cast<const uint2*>(Vu + voff[i][0]);
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {            // word e: dims 8g + 4e .. +3 = m-tiles 2e, 2e+1
-          const uint32_t w0 = e ? x[0].y : x[0].x, w1 = e ? x[1].y : x[1].x;
-          const uint32_t w8 = e ? x[2].y : x[2].x, w9 = e ? x[3].y : x[3].x;
-          const uint32_t lo01 = prmt(w0, w1, 0x5140), hi01 = prmt(w0, w1, 0x7362);
-          const uint32_t lo89 = prmt(w8, w9, 0x5140), hi89 = prmt(w8, w9, 0x7362);
-          const uint32_t A0 = e4m3x2_to_f16x2(lo01 & 0xFFFF), A1 = e4m3x2_to_f16x2(lo01 >> 16);
-          const uint32_t A2 = e4m3x2_to_f16x2(lo89 & 0xFFFF), A3 = e4m3x2_to_f16x2(lo89 >> 16);
-          const uint32_t B0 = e4m3x2_to_f16x2(hi01 & 0xFFFF), B1 = e4m3x2_to_f16x2(hi01 >> 16);
-          const uint32_t B2 = e4m3x2_to_f16x2(hi89 & 0xFFFF), B3 = e4m3x2_to_f16x2(hi89 >> 16);
-          mma16816<true>(oacc[2 * e], A0, A1, A2, A3, bh0, bh1);
-          mma16816<true>(oacc[2 * e], A0, A1, A2, A3, bl0, bl1);
-          mma16816<true>(oacc[2 * e + 1], B0, B1, B2, B3, bh0, bh1);
-          mma16816<true>(oacc[2 * e + 1], B0, B1, B2, B3, bl0, bl1);
+      for (int hh = 0; hh < 2; ++hh) {   // keys g (hh = 0) and g + 8 (hh = 1)
+        const float p0 = pr[m][2 * hh] * tm.vrel, p1 = pr[m][2 * hh + 1] * tm.vrel;
+        const uint32_t hw = pack2<FP8>(p0, p1);
+        const float2 hf = unpack2<FP8>(hw);
+        const uint32_t rw = pack2<FP8>(p0 - hf.x, p1 - hf.y);
+        if constexpr (PACK) {
+          const uint32_t x = (pick16(role0, hw, rw) & 0xFFFFu) |
+                             (pick16(role1, hw, rw) & 0xFFFF0000u);
+          bh[m][hh] = movm_t(x);
+          bl[m][hh] = 0u;
+        } else {
+          bh[m][hh] = movm_t(hw);
+          bl[m][hh] = movm_t(rw);
         }
-      } else {
-        constexpr int VCH = RB == 256 ? 2 : 1;   // 16-byte chunks of a lane group per row
+      }
+    }
+
+    // ---- o^T += V^T P^T, 16 keys (row block m) per k-step
 #pragma unroll
-        for (int ci = 0; ci < VCH; ++ci) {
-          uint4 x[4];
+    for (int m = 0; m < MK; ++m) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) x[i] = *reinterpret_cast<const uint4*>(Vu + voff[i][ci]);
-          const uint32_t w0[4] = {x[0].x, x[0].y, x[0].z, x[0].w};
-          const uint32_t w1[4] = {x[1].x, x[1].y, x[1].z, x[1].w};
-          const uint32_t w8[4] = {x[2].x, x[2].y, x[2].z, x[2].w};
-          const uint32_t w9[4] = {x[3].x, x[3].y, x[3].z, x[3].w};
+      for (int j = 0; j < NVL; ++j) {
+        uint32_t va[4];
+        ldsm_x4_t(va, lm_addr(vs_base, m, 2 * j));
+        if constexpr (FP8) {
+          // load j covers dim chunks 2j (registers 0, 1) and 2j + 1 (2, 3),
+          // each one row block of 16 dims; a transposed register holds the
+          // byte pairs (dims 2g, 2g + 1) of keys 2t and 2t + 1: row g of the
+          // block is dim 2g, row g + 8 dim 2g + 1
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if constexpr (FP8) {     // word e: 4 dims = m-tiles 2e, 2e + 1
-              const uint32_t lo01 = prmt(w0[e], w1[e], 0x5140), hi01 = prmt(w0[e], w1[e], 0x7362);
-              const uint32_t lo89 = prmt(w8[e], w9[e], 0x5140), hi89 = prmt(w8[e], w9[e], 0x7362);
-              const uint32_t A0 = e4m3x2_to_f16x2(lo01 & 0xFFFF),
-                             A1 = e4m3x2_to_f16x2(lo01 >> 16);
-              const uint32_t A2 = e4m3x2_to_f16x2(lo89 & 0xFFFF),
-                             A3 = e4m3x2_to_f16x2(lo89 >> 16);
-              const uint32_t B0 = e4m3x2_to_f16x2(hi01 & 0xFFFF),
-                             B1 = e4m3x2_to_f16x2(hi01 >> 16);
-              const uint32_t B2 = e4m3x2_to_f16x2(hi89 & 0xFFFF),
-                             B3 = e4m3x2_to_f16x2(hi89 >> 16);
-              mma16816<true>(oacc[2 * e], A0, A1, A2, A3, bh0, bh1);
-              mma16816<true>(oacc[2 * e], A0, A1, A2, A3, bl0, bl1);
-              mma16816<true>(oacc[2 * e + 1], B0, B1, B2, B3, bh0, bh1);
-              mma16816<true>(oacc[2 * e + 1], B0, B1, B2, B3, bl0, bl1);
-            } else {                 // word e: 2 dims = m-tile 4 ci + e (rows g, g + 8)
-              const int i = 4 * ci + e;
-              const uint32_t a0 = prmt(w0[e], w1[e], 0x5410), a1 = prmt(w0[e], w1[e], 0x7632);
-              const uint32_t a2 = prmt(w8[e], w9[e], 0x5410), a3 = prmt(w8[e], w9[e], 0x7632);
-              mma16816<false>(oacc[i], a0, a1, a2, a3, bh0, bh1);
-              mma16816<false>(oacc[i], a0, a1, a2, a3, bl0, bl1);
-            }
+          for (int hc = 0; hc < 2; ++hc) {
+            const int i = 2 * j + hc;
+            const uint32_t x = prmt(va[2 * hc], va[2 * hc + 1], 0x6420);
+            const uint32_t y = prmt(va[2 * hc], va[2 * hc + 1], 0x7531);
+            const uint32_t a0 = e4m3x2_to_f16x2(x & 0xFFFF), a2 = e4m3x2_to_f16x2(x >> 16);
+            const uint32_t a1 = e4m3x2_to_f16x2(y & 0xFFFF), a3 = e4m3x2_to_f16x2(y >> 16);
+            mma16816<true>(oacc[i], a0, a1, a2, a3, bh[m][0], bh[m][1]);
+            if constexpr (!PACK) mma16816<true>(oacc[i], a0, a1, a2, a3, bl[m][0], bl[m][1]);
           }
+        } else {
+          // load j is row block j: chunks 2j (dims 16j .. 16j + 7, registers
+          // 0, 1) and 2j + 1 (dims 16j + 8 .. 16j + 15, registers 2, 3)
+          mma16816<false>(oacc[j], va[0], va[2], va[1], va[3], bh[m][0], bh[m][1]);
+          if constexpr (!PACK) mma16816<false>(oacc[j], va[0], va[2], va[1], va[3], bl[m][0],
+                                               bl[m][1]);
         }
       }
     }
@@ -809,76 +930,86 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
       fill(k + 33);
       __syncwarp();
     }
-    if (lane == 0 && k + SPW < nt) issue(ring[(k + SPW) % NMR], k + SPW);
+    if (lane == 0 && k + SPW < nt) issue(ring[(k + SPW) % NMR], k + SPW, 0);
 
     // ---- end of this head inside the range
-    if (mt.flags & kLast) {
-      float l = l_run;
-      l += __shfl_xor_sync(0xffffffffu, l, 1);
-      l += __shfl_xor_sync(0xffffffffu, l, 2);
-      const int hidx = mt.hidx;
+    if (flags & kLast) {
+      float L0 = l0, L1 = l1;
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        L0 += __shfl_xor_sync(0xffffffffu, L0, off);
+        L1 += __shfl_xor_sync(0xffffffffu, L1, off);
+      }
+      // a head's p head and remainder columns summed: columns h and h + G
+      float o[MT][4];
+#pragma unroll
+      for (int i = 0; i < MT; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float x = oacc[i][e];
+          if constexpr (G == 4) x += __shfl_xor_sync(0xffffffffu, x, 2);
+          if constexpr (G == 2) x += __shfl_xor_sync(0xffffffffu, x, 1);
+          o[i][e] = x;
+        }
+      if constexpr (G == 1) {
+#pragma unroll
+        for (int i = 0; i < MT; ++i) {
+          o[i][0] += o[i][1];
+          o[i][2] += o[i][3];
+        }
+      }
+      float vhead;
+      if constexpr (CS > 0) vhead = reinterpret_cast<const float*>(cst)[13];
+      else vhead = s_hscale[2 * hidx + 1];
       const int kb = hidx / c.Hkv, kh = hidx % c.Hkv;
-      if constexpr (CS > 0) {   // the warp's partial, for the CTA's merge
-        float* po = mslot + warp * T::SLOT;
+      // lane 4g + t holds heads 2t (element 0) and 2t + 1 (element 1)
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int h = 2 * t + e;
-          if (h < G) {
+      for (int e = 0; e < 2; ++e) {
+        const int h = 2 * t + e;
+        if (h >= G) continue;
+        const float mh = e ? m1 : m0, lh = e ? L1 : L0;
+        if constexpr (CS > 0) {   // the warp's partial, for the CTA's merge
+          float* po = mslot + warp * T::SLOT;
 #pragma unroll
-            for (int i = 0; i < MT; ++i) {
-              po[h * D + T::vdim(g, i, 0)] = oacc[i][e] * mt.vhead;
-              po[h * D + T::vdim(g, i, 1)] = oacc[i][2 + e] * mt.vhead;
+          for (int i = 0; i < MT; ++i) {
+            po[h * D + T::vdim(i, g, 0)] = o[i][e] * vhead;
+            po[h * D + T::vdim(i, g, 1)] = o[i][2 + e] * vhead;
+          }
+          if (g == 0) {
+            po[G * D + h] = mh;
+            po[G * D + G + h] = lh;
+          }
+        } else if (page_off[hidx] >= gp0 && page_off[hidx + 1] <= gp0 + nt) {
+          // the whole head lies in this warp's range: write the output now
+          const float inv = mh == -INFINITY ? 0.f : vhead / lh;
+          const long long ob = ((long long)kb * c.Hq + (long long)kh * G + h) * D;
+#pragma unroll
+          for (int i = 0; i < MT; ++i)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+              const float ov = o[i][2 * hf + e] * inv;
+              const long long oi = ob + T::vdim(i, g, hf);
+              if (oa.f32) static_cast<float*>(oa.out)[oi] = ov;
+              else static_cast<uint16_t*>(oa.out)[oi] = f32_to_bf16_rn(ov);
             }
+          if (oa.lse && g == 0)
+            oa.lse[(long long)kb * c.Hq + kh * G + h] =
+                mh == -INFINITY ? -INFINITY : (mh + log2f(lh)) * 0.6931471805599453f;
+        } else {
+          // shared with other warps: this warp's partial goes to the workspace,
+          // at v + hidx (unique: a warp's heads are consecutive, and later
+          // warps never go back to earlier heads)
+          const long long part = v_range + hidx;
+          float* po = w.part_o + (part * G + h) * D;
+#pragma unroll
+          for (int i = 0; i < MT; ++i) {
+            po[T::vdim(i, g, 0)] = o[i][e] * vhead;
+            po[T::vdim(i, g, 1)] = o[i][2 + e] * vhead;
           }
-        }
-        if (t == 0 && g < G) {
-          po[G * D + g] = m_run;
-          po[G * D + G + g] = l;
-        }
-      } else if (page_off[hidx] >= gp0 && page_off[hidx + 1] <= gp0 + nt) {
-        // the whole head lies in this warp's range: write the output now
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int h = 2 * t + e;
-          const float lh = __shfl_sync(0xffffffffu, l, 4 * (h & 7));
-          const float mh = __shfl_sync(0xffffffffu, m_run, 4 * (h & 7));
-          if (h < G) {
-            const float inv = mh == -INFINITY ? 0.f : mt.vhead / lh;
-            const long long ob = ((long long)kb * c.Hq + (long long)kh * G + h) * D;
-#pragma unroll
-            for (int i = 0; i < MT; ++i)
-#pragma unroll
-              for (int hi = 0; hi < 2; ++hi) {
-                const float o = oacc[i][2 * hi + e] * inv;
-                const long long oi = ob + T::vdim(g, i, hi);
-                if (oa.f32) static_cast<float*>(oa.out)[oi] = o;
-                else static_cast<uint16_t*>(oa.out)[oi] = f32_to_bf16_rn(o);
-              }
-            if (oa.lse && g == 0)
-              oa.lse[(long long)kb * c.Hq + kh * G + h] =
-                  mh == -INFINITY ? -INFINITY : (mh + log2f(lh)) * 0.6931471805599453f;
+          if (g == 0) {
+            w.part_ml[(part * G + h) * 2] = mh;
+            w.part_ml[(part * G + h) * 2 + 1] = lh;
           }
-        }
-      } else {
-        // shared with other warps: this warp's partial goes to the workspace,
-        // at v + hidx (unique: a warp's heads are consecutive, and later
-        // warps never go back to earlier heads)
-        const long long part = v_range + hidx;
-        float* po = w.part_o + part * G * D;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int h = 2 * t + e;
-          if (h < G) {
-#pragma unroll
-            for (int i = 0; i < MT; ++i) {
-              po[h * D + T::vdim(g, i, 0)] = oacc[i][e] * mt.vhead;
-              po[h * D + T::vdim(g, i, 1)] = oacc[i][2 + e] * mt.vhead;
-            }
-          }
-        }
-        if (t == 0 && g < G) {
-          w.part_ml[(part * G + g) * 2] = m_run;
-          w.part_ml[(part * G + g) * 2 + 1] = l;
         }
       }
     }
@@ -889,49 +1020,59 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
     // CTAs' partials across the cluster; each CTA writes 1/CS of the head's
     // output. o = sum_w 2^(m_w - M) o_w / sum_w 2^(m_w - M) l_w.
     __syncthreads();
-    float* cp = mslot + T::NCW * T::SLOT;
+    float* cpart = mslot + NCW * T::SLOT;
     for (int e = tid; e < G * D; e += T::NT) {
       const int h = e / D;
-      float M = -INFINITY;
+      float mv[NCW], M = -INFINITY;
 #pragma unroll
-      for (int v = 0; v < T::NCW; ++v) M = fmaxf(M, mslot[v * T::SLOT + G * D + h]);
+      for (int v = 0; v < NCW; ++v) {
+        mv[v] = mslot[v * T::SLOT + G * D + h];
+        M = fmaxf(M, mv[v]);
+      }
       float L = 0.f, O = 0.f;
       if (M != -INFINITY) {
 #pragma unroll
-        for (int v = 0; v < T::NCW; ++v) {
-          const float mv = mslot[v * T::SLOT + G * D + h];
-          if (mv != -INFINITY) {   // empty partials hold no o values
-            const float bw = fast_exp2(mv - M);
+        for (int v = 0; v < NCW; ++v) {
+          if (mv[v] != -INFINITY) {   // empty partials hold no o values
+            const float bw = fast_exp2(mv[v] - M);
             L += mslot[v * T::SLOT + G * D + G + h] * bw;
             O += mslot[v * T::SLOT + e] * bw;
           }
         }
       }
-      cp[e] = O;
+      cpart[e] = O;
       if (e % D == 0) {
-        cp[G * D + h] = M;
-        cp[G * D + G + h] = L;
+        cpart[G * D + h] = M;
+        cpart[G * D + G + h] = L;
       }
     }
     __syncthreads();   // converged warps for the aligned cluster barrier
     cluster_sync_all();
+    uint32_t rbase[CS];
+#pragma unroll
+    for (int j = 0; j < CS; ++j) rbase[j] = cluster_addr(cpart, (uint32_t)j);
     const int kb = hsel / c.Hkv, kh = hsel % c.Hkv;
-    const int crank = (int)(blockIdx.x % CS);
     constexpr int PER = G * D / CS;
     for (int e = crank * PER + tid; e < (crank + 1) * PER; e += T::NT) {
       const int h = e / D, d = e % D;
-      float M = -INFINITY, L = 0.f, O = 0.f;
+      float mj[CS], lj[CS], oj[CS];
 #pragma unroll
-      for (int j = 0; j < CS; ++j) {
-        const float mj = ld_cluster_f32(cp + G * D + h, (uint32_t)j);
-        if (mj == -INFINITY) continue;
-        const float lj = ld_cluster_f32(cp + G * D + G + h, (uint32_t)j);
-        const float oj = ld_cluster_f32(cp + e, (uint32_t)j);
-        const float mx = fmaxf(M, mj);
-        const float a = fast_exp2(M - mx), bw = fast_exp2(mj - mx);   // a = 0 while M = -inf
-        L = L * a + lj * bw;
-        O = O * a + oj * bw;
-        M = mx;
+      for (int j = 0; j < CS; ++j) {   // every load first, then the arithmetic
+        mj[j] = ld_dsmem_f32(rbase[j] + 4u * (uint32_t)(G * D + h));
+        lj[j] = ld_dsmem_f32(rbase[j] + 4u * (uint32_t)(G * D + G + h));
+        oj[j] = ld_dsmem_f32(rbase[j] + 4u * (uint32_t)e);
+      }
+      float M = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < CS; ++j) M = fmaxf(M, mj[j]);
+      float L = 0.f, O = 0.f;
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int j = 0; j < CS; ++j) {
+          const float bw = mj[j] == -INFINITY ? 0.f : fast_exp2(mj[j] - M);
+          L += lj[j] * bw;
+          O += oj[j] * bw;
+        }
       }
       const float o = M == -INFINITY ? 0.f : O / L;
       const long long oi = ((long long)kb * c.Hq + (long long)kh * G + h) * D + d;
@@ -941,8 +1082,8 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
         oa.lse[(long long)kb * c.Hq + kh * G + h] =
             M == -INFINITY ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
     }
-    __syncthreads();
-    cluster_sync_all();   // no CTA leaves while another still reads its shared memory
+    __syncwarp();
+    cluster_sync_relaxed();   // no CTA leaves while another still reads its shared memory
   }
 }
 
@@ -1069,15 +1210,16 @@ k_decode_combine(CacheView c, DecodeWork w, int layer, int batch, OutArgs oa, in
 }
 
 // ------------------------------------------------------------------ dispatch
-// Cluster size for a call of nh heads: the largest of 8, 4, 2 whose nh * CS
-// CTAs fit on the SMs at once, if the call has at most half as many heads as
-// there are SMs; 0 selects the global plan and the combine kernel, which a
-// cache created with an explicit split grid (decode_ctas > 0) always uses.
+// Cluster size for a call of nh heads: the largest of 8, 4, 2 with nh clusters
+// of that size resident at once on this device (cudaOccupancyMaxActiveClusters,
+// queried at set-up: clusters live inside one GPC, so fewer fit than SMs / CS);
+// 0 selects the global plan and the combine kernel, which a cache created with
+// an explicit split grid (decode_ctas > 0) always uses.
 inline int cluster_size(const fdms_cache* cache, int nh) {
 #if FDMS_CLUSTER_DECODE
   if (!cache->cluster_ok || cache->cfg.decode_ctas > 0) return 0;
-  for (int cs = 8; cs >= 2; cs /= 2)
-    if ((long long)nh * cs <= cache->num_sms) return cs;
+  for (int i = 3; i >= 1; --i)
+    if (nh <= cache->max_clusters[i]) return 1 << i;
 #endif
   (void)cache;
   (void)nh;
@@ -1085,13 +1227,13 @@ inline int cluster_size(const fdms_cache* cache, int nh) {
 }
 
 template <class T, int CS>
-fdms_status launch_cluster_t(fdms_cache* cache, const DecodeWork& w, OutArgs oa, int layer,
+cudaError_t launch_cluster_t(fdms_cache* cache, const DecodeWork& w, OutArgs oa, int layer,
                              int batch, const void* q, cudaStream_t s) {
   const int nh = batch * cache->view.Hkv;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(nh * CS));
   cfg.blockDim = dim3(T::NT);
-  cfg.dynamicSmemBytes = T::smem_bytes_cluster(nh);
+  cfg.dynamicSmemBytes = T::smem_bytes_cluster();
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1102,23 +1244,24 @@ fdms_status launch_cluster_t(fdms_cache* cache, const DecodeWork& w, OutArgs oa,
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_decode_split<T, CS>, cache->view, w, oa,
-                                           layer, batch, static_cast<const uint16_t*>(q), 0,
-                                           0.0);
-  if (e != cudaSuccess) return FDMS_ERR_CUDA;
-  cache->last_append_layer = -1;   // the kernel waits for every append queued before it
-  return FDMS_OK;
+  return cudaLaunchKernelEx(&cfg, k_decode_split<T, CS>, cache->view, w, oa, layer, batch,
+                            static_cast<const uint16_t*>(q), 0, 0.0, w.snap ? 1 : 0);
 }
 
 template <class T>
 fdms_status launch_split_t(fdms_cache* cache, const DecodeWork& w, OutArgs oa, int layer,
                            int batch, const void* q, cudaStream_t s) {
   const int nh = batch * cache->view.Hkv;
-  switch (cluster_size(cache, nh)) {
-    case 8: return launch_cluster_t<T, 8>(cache, w, oa, layer, batch, q, s);
-    case 4: return launch_cluster_t<T, 4>(cache, w, oa, layer, batch, q, s);
-    case 2: return launch_cluster_t<T, 2>(cache, w, oa, layer, batch, q, s);
-    default: break;
+  const int cs = cluster_size(cache, nh);
+  if (cs > 0) {
+    const cudaError_t e = cs == 8   ? launch_cluster_t<T, 8>(cache, w, oa, layer, batch, q, s)
+                          : cs == 4 ? launch_cluster_t<T, 4>(cache, w, oa, layer, batch, q, s)
+                                    : launch_cluster_t<T, 2>(cache, w, oa, layer, batch, q, s);
+    if (e == cudaSuccess) {
+      cache->last_append_layer = -1;   // the kernel waits for every append queued before it
+      return FDMS_OK;
+    }
+    cudaGetLastError();   // a refused cluster launch falls back to the global plan
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)cache->decode_ctas);
@@ -1133,7 +1276,7 @@ fdms_status launch_split_t(fdms_cache* cache, const DecodeWork& w, OutArgs oa, i
   const int n_ranges = cache->decode_ctas * T::NCW;
   cudaError_t e = cudaLaunchKernelEx(&cfg, k_decode_split<T, 0>, cache->view, w, oa, layer, batch,
                                      static_cast<const uint16_t*>(q), n_ranges,
-                                     1.0 / (double)n_ranges);
+                                     1.0 / (double)n_ranges, 0);
   if (e != cudaSuccess) return FDMS_ERR_CUDA;
   cache->last_append_layer = -1;   // the split waits for every append queued before it
   cfg.gridDim = dim3((unsigned)(nh * Combine<T::D, T::G>::CPH));
@@ -1142,6 +1285,27 @@ fdms_status launch_split_t(fdms_cache* cache, const DecodeWork& w, OutArgs oa, i
   e = cudaLaunchKernelEx(&cfg, k_decode_combine<T::D, T::G, T::TR>, cache->view, w, layer, batch,
                          oa, n_ranges, 1.0 / (double)n_ranges);
   return e == cudaSuccess ? FDMS_OK : FDMS_ERR_CUDA;
+}
+
+template <class T, int CS>
+int max_active_clusters() {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(CS * 64));
+  cfg.blockDim = dim3(T::NT);
+  cfg.dynamicSmemBytes = T::smem_bytes_cluster();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaFuncSetAttribute(k_decode_split<T, CS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)T::smem_bytes_cluster()) != cudaSuccess ||
+      cudaOccupancyMaxActiveClusters(&n, k_decode_split<T, CS>, &cfg) != cudaSuccess)
+    n = 0;
+  return n;
 }
 
 template <class T>
@@ -1158,17 +1322,13 @@ fdms_status setup_t(fdms_cache* cache) {
     return FDMS_ERR_UNSUPPORTED;
   cache->ctas_per_sm = per_sm;
   cache->ranges_per_cta = T::NCW;
-  // per-head cluster mode: usable when every cluster size fits
-  const size_t csmem = T::smem_bytes_cluster(nh);
-  cache->cluster_ok =
-      csmem <= 227 * 1024 &&
-      cudaFuncSetAttribute(k_decode_split<T, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)csmem) == cudaSuccess &&
-      cudaFuncSetAttribute(k_decode_split<T, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)csmem) == cudaSuccess &&
-      cudaFuncSetAttribute(k_decode_split<T, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)csmem) == cudaSuccess;
-  cudaGetLastError();   // a refused attribute only turns the cluster mode off
+  // per-head cluster mode: how many clusters of each size fit at once
+  cache->max_clusters[0] = 0;
+  cache->max_clusters[1] = max_active_clusters<T, 2>();
+  cache->max_clusters[2] = max_active_clusters<T, 4>();
+  cache->max_clusters[3] = max_active_clusters<T, 8>();
+  cache->cluster_ok = T::smem_bytes_cluster() <= 227 * 1024 && cache->max_clusters[1] > 0;
+  cudaGetLastError();   // a refused query only turns the cluster mode off
   return FDMS_OK;
 }
 
@@ -1212,9 +1372,12 @@ fdms_status fdms_decode_setup(fdms_cache* cache) {
     if (cudaMalloc(&p, bytes) != cudaSuccess || !fdms_track(cache, p, bytes)) return nullptr;
     return p;
   };
+  const size_t heads = (size_t)c.L * c.Bmax * c.Hkv;
   w.part_o = static_cast<float*>(take((size_t)w.max_parts * c.G * c.D * sizeof(float)));
   w.part_ml = static_cast<float*>(take((size_t)w.max_parts * c.G * 2 * sizeof(float)));
-  if (!w.part_o || !w.part_ml) return FDMS_ERR_CUDA;
+  w.snap = static_cast<int4*>(take(heads * sizeof(int4)));
+  if (!w.part_o || !w.part_ml || !w.snap) return FDMS_ERR_CUDA;
+  if (cudaMemset(w.snap, 0, heads * sizeof(int4)) != cudaSuccess) return FDMS_ERR_CUDA;
   return FDMS_OK;
 }
 
@@ -1227,9 +1390,9 @@ fdms_status fdms_launch_decode(fdms_cache* cache, int layer, int batch, const vo
 }
 
 // ------------------------------------------------- decode without allocation
-// A fixed scratch array for fdms_decode_attn_noalloc: the split plan and the
-// split partials. Host code only learns its device address through
-// cudaGetSymbolAddress (the host-side name is a stand-in, not a device
+// A fixed scratch array for fdms_decode_attn_noalloc: the split partials of
+// calls that run the global plan. Host code only learns its device address
+// through cudaGetSymbolAddress (the host-side name is a stand-in, not a device
 // pointer); device code never names it, it receives the address as arguments.
 static __device__ __align__(256) unsigned char fdms_noalloc_scratch[FDMS_STATIC_SCRATCH_BYTES];
 
@@ -1291,6 +1454,7 @@ extern "C" fdms_status fdms_decode_attn_noalloc(fdms_cache* cache, int layer, in
     w.part_ml = reinterpret_cast<float*>(b + o_bytes);
     w.max_parts = (int)parts;
     w.max_ctas = cache->decode_ctas;
+    w.snap = cache->work.snap;   // the cache's own memory, not scratch
     // the array keeps the previous call's contents; nothing in it needs to
     // start at zero (every value is written by this call before it is read)
     OutArgs oa{out_dev, nullptr, 0};

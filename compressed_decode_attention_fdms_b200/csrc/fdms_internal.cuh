@@ -56,14 +56,17 @@ struct CacheView {
 
 // Row layout inside a 64-row page (a store block, or 64 ring slots): the 16-byte
 // chunks of row r are stored XOR-permuted by r, so that the decode kernel's
-// tensor-core fragment loads from shared memory touch every bank once. Rows
-// keep their page-row index r in shared memory, so the permutation survives a
-// straight bulk copy. K and V rows use different permutations when rows are 256
-// bytes, the same one when they are 128 bytes, none when they are 64 bytes.
+// matrix loads from shared memory (ldmatrix: eight consecutive rows, one
+// 16-byte chunk each) touch every bank once. Rows keep their page-row index r
+// in shared memory, so the permutation survives a straight bulk copy. The
+// permutation depends on r mod 8 only: 128- and 256-byte rows XOR the chunk
+// index with r mod 8 (eight rows, eight distinct 16-byte bank groups); 64-byte
+// rows, two to a 128-byte line, XOR it with (r / 2) mod 4. K and V rows use
+// the same permutation.
 __host__ __device__ inline int swz_chunk(int RB, bool is_v, int row, int chunk) {
-  if (RB == 128) return chunk ^ (row & 7);
-  if (RB == 256) return is_v ? (chunk ^ (row & 6)) : (chunk ^ ((row & 1) << 2));
-  return chunk;
+  (void)is_v;
+  if (RB == 64) return chunk ^ ((row >> 1) & 3);
+  return chunk ^ (row & 7);
 }
 // Byte offset inside a row of the logical byte b (the chunk permutation keeps
 // the byte's place inside its chunk).
@@ -93,6 +96,8 @@ struct DecodeWork {
   float* part_ml;         // [max_parts][G][2]: running max (log2 domain) and sum
   int max_parts;
   int max_ctas;
+  int4* snap;             // per head of the cache: (store_len, n, r, 0) the last
+                          // per-head-cluster decode of it saw; null: not kept
 };
 
 // Workspace of the bulk (prefill) append, per (seq, kv head) of the call.
@@ -168,6 +173,12 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
                ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
 }
+// raise the transaction count of the current phase without arriving (the
+// arrival comes later)
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;"
+               ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
+}
 // returns true once the phase with the given parity has completed
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
@@ -215,6 +226,7 @@ struct fdms_cache {
   // before its dependency wait (see k_append_step)
   int last_append_layer;
   int cluster_ok;         // the per-head cluster decode mode can be launched
+  int max_clusters[4];    // clusters of 2, 4, 8 CTAs (index 1..3) resident at once
 };
 
 // Record a device allocation of the cache (freed at destroy). Frees `p` and

@@ -2,13 +2,17 @@
 bench.py times (needs a B200).
 
 The GPU cache holds every sequence of the workload at full context length and
-runs the default decode grid (one split CTA per SM); the fp64 oracle follows a
+runs the default decode launch (llama1b_c8 and qwen8b_c8_fp8: one cluster of
+CTAs per (seq, kv head); qwen8b_long_fp8, 256 heads: the global tile plan with
+its combine kernel); the fp64 oracle follows a
 few sampled sequences one by one (a one-sequence oracle each, fed that
 sequence's inputs, which do not depend on the other sequences). One layer: the
 kernels' launch configuration and per-call sizes do not depend on the number
 of layers. Checked after the prefill and after each decode step: the sampled
 sequences' heads (store and ring) bit-exact, and their decode outputs within
-the bars of test_gpu_parity.
+the bars of test_gpu_parity; FP8 outputs also within the stated 3e-2 of the
+oracle fed the unquantised bf16 values (the method's own E4M3 error, which
+averages out over the thousands of tokens these heads see).
 """
 import numpy as np
 import pytest
@@ -27,6 +31,7 @@ from _pair import bits  # noqa: E402
 
 TOL_BF16 = 3e-3
 TOL_FP8_MIRROR = 3e-3
+TOL_FP8_TRUE = 3e-2   # the stated FP8 bar, against the unquantised bf16 inputs
 STEPS = 3
 
 
@@ -99,6 +104,10 @@ def test_full_size_sampled_sequences(name):
                 ref = ocs[b].attention(0, 0, bits(q[b]))
                 err = float(np.max(np.abs(g[b] - ref) - _half_ulp_bf16(ref)))
                 assert err <= tol, (name, step, b, err)
+                if wl.kv_dtype == "fp8_e4m3":
+                    ref_t = ocs[b].attention(0, 0, bits(q[b]), mode="true")
+                    err_t = float(np.max(np.abs(g[b] - ref_t) - _half_ulp_bf16(ref_t)))
+                    assert err_t <= TOL_FP8_TRUE, (name, step, b, err_t)
                 for h in range(wl.kv_heads):
                     _check_head(cache, ocs[b], b, h, 0, b, wl.kv_dtype)
         assert fd.fdms_cache_stats(cache)["error"] == 0

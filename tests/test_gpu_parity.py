@@ -238,18 +238,49 @@ def test_caller_fp8_scales():
 
 
 def test_pool_exhaustion_latches_error_and_leaves_head_unchanged():
+    """A head whose survivors do not fit is left unchanged, the pool counter
+    does not move past the blocks handed out, and a later, smaller request
+    still gets the blocks that are left."""
     import compressed_decode_attention_fdms_b200 as fd
     wl = wk.scaled(wk.get("tiny"), ctx=500, steps=0, window=0, rate=1.0)
-    p = Pair(wl, num_blocks=9)      # 2 heads x 8 blocks needed
+    p = Pair(wl, num_blocks=9, max_seq_len=640, oracle_capacity=640)   # 2 heads x 8 blocks
+    dev = "cuda:0"
     try:
         p.append(0, wk.prefill_inputs(wl, 0))
         st = fd.fdms_cache_stats(p.cache)
         assert st["error"] == fd.FDMS_ERR_OUT_OF_BLOCKS
         infos = [fd.fdms_cache_read_head(p.cache, 0, 0, h) for h in range(2)]
-        done = [i for i in infos if i["num_tokens"] == 500]
-        untouched = [i for i in infos if i["num_tokens"] == 0]
-        assert len(done) == 1 and len(untouched) == 1
-        assert untouched[0]["store_len"] == 0
+        assert infos[0]["num_tokens"] == 500 and infos[0]["store_len"] == 500
+        assert infos[1]["num_tokens"] == 0 and infos[1]["store_len"] == 0   # first fit, head order
+        assert st["blocks_used"] == 8 and st["blocks_free"] == 1
+        # 30 more tokens: head 0 keeps none (no block needed), head 1 keeps all
+        # (one block): the block left over goes to head 1
+        more = wk.prefill_inputs(wk.scaled(wl, ctx=30), 0)
+        keep = more["keep"].clone()
+        keep[:, :, 0] = 0
+        keep[:, :, 1] = 1
+        fd.fdms_append_evict(p.cache, 0, 1, more["n_new"].to(dev), more["max_new"],
+                             more["k"].to(dev), more["v"].to(dev), keep.to(dev))
+        st = fd.fdms_cache_stats(p.cache)
+        assert st["blocks_used"] == 9 and st["blocks_free"] == 0
+        h1 = fd.fdms_cache_read_head(p.cache, 0, 0, 1)
+        assert h1["num_tokens"] == 30 and h1["store_len"] == 30
+        assert np.array_equal(h1["pos"][:30], np.arange(30))
+        assert np.array_equal(h1["k"].view(np.uint16).reshape(30, -1),
+                              bits(more["k"][0, :30, 1]).reshape(30, -1))
+        h0 = fd.fdms_cache_read_head(p.cache, 0, 0, 0)
+        assert h0["num_tokens"] == 530 and h0["store_len"] == 500
+        # the pool is now full: a step that needs a block fails and changes nothing
+        step = wk.decode_inputs(wl, 0, 0)
+        skeep = step["keep"].clone()
+        skeep[:] = 1
+        for _ in range(40):     # head 1 fills its block (64 slots) and needs another
+            fd.fdms_append_evict(p.cache, 0, 1, step["n_new"].to(dev), 1, step["k"].to(dev),
+                                 step["v"].to(dev), skeep.to(dev))
+        st = fd.fdms_cache_stats(p.cache)
+        assert st["blocks_used"] == 9 and st["blocks_free"] == 0
+        h1 = fd.fdms_cache_read_head(p.cache, 0, 0, 1)
+        assert h1["store_len"] == 64 and h1["num_tokens"] == 64
     finally:
         p.close()
 
