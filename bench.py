@@ -56,12 +56,14 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="llama1b_c8", choices=sorted(wk.WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="budget of the oracle's timed sample")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-ctas", type=int, default=0)
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other workloads' decode calls in the default run")
     return ap.parse_args()
 
 
@@ -254,21 +256,85 @@ def oracle_sample(wl, budget_s: float, min_steps=1, max_steps=None, warmup=0):
     return bytes_ / sum(times), times, desc
 
 
+def oracle_seq_worker(job):
+    """Time the fp64 oracle on some sequences of layer 0, in a process of its
+    own (one thread): prefill, then decode steps (append + attention) until
+    the time budget is spent or `steps` are done. Returns (bytes, seconds,
+    steps) of the timed steps."""
+    name, seqs, steps, budget_s = job
+    from threadpoolctl import threadpool_limits
+    from oracle.cache import OracleCache
+    torch.set_num_threads(1)
+    wl = wk.get(name)
+    ctx = wk.context_lengths(wl)
+    elt = 1 if wl.kv_dtype == "fp8_e4m3" else 2
+    row = 2 * wl.head_dim * elt
+    with threadpool_limits(limits=1):
+        ocs = {}
+        for b in seqs:
+            pre = wk.prefill_inputs(wl, 0, seqs=[b])
+            oc = OracleCache(1, 1, wl.q_heads, wl.kv_heads, wl.head_dim, wl.window, wl.period,
+                             wl.kv_dtype, capacity=int(ctx[b]) + steps + 1)
+            n = int(ctx[b])
+            oc.append(0, np.array([n]), to_bits(pre["k"][b:b + 1, :n]),
+                      to_bits(pre["v"][b:b + 1, :n]), pre["keep"][b:b + 1, :n].numpy())
+            ocs[b] = oc
+        total, nbytes, done = 0.0, 0, 0
+        for step in range(steps):
+            inp = wk.decode_inputs(wl, 0, step)
+            q = to_bits(wk.decode_query(wl, 0, step))
+            kb, vb, keep = to_bits(inp["k"]), to_bits(inp["v"]), inp["keep"].numpy()
+            t0 = time.perf_counter()
+            for b in seqs:
+                ocs[b].append(0, np.array([1]), kb[b:b + 1], vb[b:b + 1], keep[b:b + 1])
+                ocs[b].attention(0, 0, q[b])
+            total += time.perf_counter() - t0
+            done += 1
+            for b in seqs:
+                oc = ocs[b]
+                units = int(oc.n[0, 0] - oc.r[0, 0]) * wl.kv_heads
+                units += int(np.count_nonzero(oc.keep[0, 0, :int(oc.r[0, 0])]))
+                nbytes += units * row
+            if total >= budget_s:
+                break
+    return nbytes, total, done
+
+
+def oracle_parallel(wl, budget_s, steps=None):
+    """The fp64 oracle on this host's cores: one spawned process per group of
+    sequences of layer 0 (as many processes as cores, at most one per
+    sequence), all running at once; bytes of every process / the longest
+    process time. Spawned, not forked: this process has a CUDA context."""
+    import multiprocessing as mp
+    cores = max(1, min(os.cpu_count() or 1, wl.batch))
+    groups = [list(range(i, wl.batch, cores)) for i in range(cores)]
+    n_steps = steps if steps is not None else wl.steps
+    jobs = [(wl.name, g, n_steps, budget_s) for g in groups]
+    with mp.get_context("spawn").Pool(cores) as pool:
+        res = pool.map(oracle_seq_worker, jobs)
+    nbytes = sum(r[0] for r in res)
+    t = max(r[1] for r in res)
+    done = min(r[2] for r in res)
+    desc = (f"fp64 numpy oracle, layer 0 of {wl.layers}, all {wl.batch} sequences x "
+            f"{wl.kv_heads} kv heads, {done}+ decode steps (append + attention) after the "
+            f"prefill; {cores} processes of one thread each (host has {os.cpu_count()} cores)")
+    return {"value": nbytes / t / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": desc, "seconds": t}
+
+
 def run_reference(args, wl):
     world, rank, _ = dist_env()
     if rank != 0:
         return 0
-    bps, times, desc = oracle_sample(wl, budget_s=1e9, min_steps=args.steps,
-                                     max_steps=args.steps, warmup=args.warmup)
-    gbs = bps / 1e9
-    ms = 1e3 * sum(times) / len(times)
+    cb = oracle_parallel(wl, budget_s=1e9, steps=args.warmup + args.steps)
+    gbs = cb["value"]
     line = {
         "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s",
-        "n_gpus": args.gpus, "steps": len(times), "warmup": args.warmup, "ms_per_step": ms,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * cb["seconds"] / max(1, args.warmup + args.steps),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": {**config_dict(wl), "step": "one layer, all sequences"},
-        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": desc},
+        "cpu_baseline": cb,
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -292,20 +358,10 @@ def pool_blocks(wl, steps_total):
     return int(np.sum(np.ceil(np.minimum(n, mean + 6 * sd + 64) / 64) + 1))
 
 
-def run_native(args, wl):
-    import compressed_decode_attention_fdms_b200 as fd
-
-    world, rank, local = dist_env()
-    if world > 1:
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    wl = rank_workload(wl, rank, world)
-
-    W, K = args.warmup, args.steps
-    KE = 0 if args.no_e2e else args.e2e_steps
-    WE = 0 if args.no_e2e else 3
+def measure(fd, args, wl, dev, local, world, K, W, KE, WE):
+    """One workload on this rank: prefill, W warm-up steps, K timed steps (one
+    CUDA graph), K rounds of decode calls alone (the per-launch duration), and
+    KE end-to-end steps. Returns the figures (whole-job bytes over ranks)."""
     steps_total = W + K + WE + KE
     cfg = fd.make_config(wl.layers, wl.batch, wl.q_heads, wl.kv_heads, wl.head_dim, wl.window,
                          wl.period, wl.max_ctx + steps_total, pool_blocks(wl, steps_total),
@@ -454,47 +510,87 @@ def run_native(args, wl):
 
     peak, peak_src = load_peaks()
     traffic, traffic_src = load_traffic(wl.name)
-    # the library's decode mode for this call shape: one cluster of CS CTAs per
-    # (seq, kv head) when there are at most half as many as SMs and no explicit
-    # split grid, else the global plan (split + combine)
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    nh = wl.batch * wl.kv_heads
-    cs = next((c for c in (8, 4, 2) if nh * c <= sms), 0) if args.decode_ctas == 0 else 0
-    kernel = (f"fdms_decode_attn (k_decode_split, one cluster of {cs} CTAs per head, no combine)"
-              if cs else "fdms_decode_attn (k_decode_split + k_decode_combine)")
     achieved = per_launch_bytes / (dec_avg_ms * 1e-3) / 1e9
+    res = {
+        "value": value, "t_max": t_max, "kv_bytes": kv_bytes, "elapsed_ms": elapsed_ms,
+        "clocks": clk.summary(), "memory": memory, "e2e": e2e, "cs": fd.decode_cluster_size(cache, B),
+        "roofline": {
+            "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "traffic": traffic, "traffic_source": traffic_src,
+            "per_launch_bytes": per_launch_bytes, "launch_us": dec_avg_ms * 1e3,
+            "launch_timing": f"CUDA events around one graph of {K * L} back-to-back "
+                             "decode calls (all layers, K rounds); duration / calls",
+            "peak_source": peak_src,
+        },
+        "prefill": {"tokens_per_seq": int(wl.max_ctx), "layers": L,
+                    "us_per_layer": 1e3 * pre_ms / L, "gb_per_layer": pre_bytes / L / 1e9,
+                    "achieved_gbs": pre_bytes / (pre_ms * 1e-3) / 1e9,
+                    "frac": pre_bytes / (pre_ms * 1e-3) / 1e9 / peak,
+                    "timing": pre_how + " (4 launches per layer)"},
+        "decode_share_of_step": dec_avg_ms * L * K / elapsed_ms,
+    }
+    del graph, graph_dec
+    fd.fdms_cache_destroy(cache)
+    return res
+
+
+def decode_kernel_desc(cs):
+    return (f"fdms_decode_attn (k_decode_split, one cluster of {cs} CTAs per (seq, kv head), "
+            "no combine)" if cs else "fdms_decode_attn (k_decode_split + k_decode_combine)")
+
+
+# workloads reported next to the headline one in the default run (their decode
+# call and step at a shorter run; BASELINE's other single-GPU configs)
+EXTRA_WORKLOADS = ("qwen8b_c8_fp8", "llama1b_c1")
+
+
+def run_native(args, wl):
+    import compressed_decode_attention_fdms_b200 as fd
+
+    world, rank, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = rank_workload(wl, rank, world)
+    W, K = args.warmup, args.steps
+    KE = 0 if args.no_e2e else args.e2e_steps
+    WE = 0 if args.no_e2e else 3
+    m = measure(fd, args, wl, dev, local, world, K, W, KE, WE)
+    extras = {}
+    if world == 1 and not args.no_extras and args.workload == "llama1b_c8":
+        for name in EXTRA_WORKLOADS:
+            x = measure(fd, args, wk.get(name), dev, local, world, min(K, 20), W, 0, 0)
+            extras[name] = {
+                "config": config_dict(wk.get(name)), "value": x["value"], "unit": "GB/s",
+                "us_per_step": 1e3 * x["t_max"] / min(K, 20), "roofline": x["roofline"],
+                "kernel": decode_kernel_desc(x["cs"]), "clocks": x["clocks"],
+                "memory": x["memory"], "kv_gb_per_step": x["kv_bytes"] / min(K, 20) / 1e9}
     result = None
     if rank == 0:
-        clocks = clk.summary()
+        roof = dict(m["roofline"])
+        roof["kernel"] = decode_kernel_desc(m["cs"])
         result = {
-            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
-            "warmup": W, "ms_per_step": t_max / K, "us_per_step": 1e3 * t_max / K,
+            "metric": METRIC, "value": m["value"], "unit": "GB/s", "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": m["t_max"] / K, "us_per_step": 1e3 * m["t_max"] / K,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
             "config": {**config_dict(wl), "parallelism": f"replicas{world}" if world > 1 else "1gpu",
                        "l2": "inputs larger than L2: every step reads "
-                             f"{kv_bytes / K / 1e6:.0f} MB of compact KV (L2 126 MB)",
+                             f"{m['kv_bytes'] / K / 1e6:.0f} MB of compact KV (L2 126 MB)",
                        "timing": "K steps in one CUDA graph; events around each decode call"},
-            "roofline": {
-                "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": traffic, "traffic_source": traffic_src,
-                "kernel": kernel,
-                "per_launch_bytes": per_launch_bytes, "launch_us": dec_avg_ms * 1e3,
-                "launch_timing": f"CUDA events around one graph of {K * L} back-to-back "
-                                 "decode calls (all layers, K rounds); duration / calls",
-                "peak_source": peak_src,
-            },
-            "clocks": clocks,
-            "gpu_launches": K * L * (2 if cs else 3),
-            "prefill": {"tokens_per_seq": int(wl.max_ctx), "layers": L,
-                        "us_per_layer": 1e3 * pre_ms / L, "gb_per_layer": pre_bytes / L / 1e9,
-                        "achieved_gbs": pre_bytes / (pre_ms * 1e-3) / 1e9,
-                        "frac": pre_bytes / (pre_ms * 1e-3) / 1e9 / peak,
-                        "timing": pre_how + " (4 launches per layer)"},
-            "kv_gb_per_step": kv_bytes / K / 1e9,
-            "memory": memory,
-            "decode_share_of_step": dec_avg_ms * L * K / elapsed_ms,
+            "roofline": roof,
+            "clocks": m["clocks"],
+            "gpu_launches": K * wl.layers * (2 if m["cs"] else 3),
+            "prefill": m["prefill"],
+            "kv_gb_per_step": m["kv_bytes"] / K / 1e9,
+            "memory": m["memory"],
+            "decode_share_of_step": m["decode_share_of_step"],
         }
+        if extras:
+            result["workloads"] = extras
+        e2e = m["e2e"]
         if e2e:
             result["e2e"] = {"value": e2e["bytes"] / (e2e["ms"] * 1e-3) / 1e9, "unit": "GB/s",
                              "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
@@ -502,11 +598,13 @@ def run_native(args, wl):
                              "path": "Python binding -> C ABI, eager calls per layer; one packed "
                                      "H2D of the step's inputs and one D2H of all outputs"}
         if not args.no_cpu_baseline and world == 1:
-            bps, times, desc = oracle_sample(wl, args.cpu_seconds)
-            result["cpu_baseline"] = {"value": bps / 1e9, "unit": "GB/s", "cores": 1,
-                                      "kind": "oracle", "sample": desc}
-    del graph, graph_dec
-    fd.fdms_cache_destroy(cache)
+            # decode steps past the workload's own count so that the budget,
+            # not the step count, ends the sample
+            cb = oracle_parallel(wl, args.cpu_seconds, steps=4096)
+            cb1 = oracle_sample(wl, args.cpu_seconds / 2)
+            result["cpu_baseline"] = cb
+            result["cpu_baseline_1thread"] = {"value": cb1[0] / 1e9, "unit": "GB/s", "cores": 1,
+                                              "kind": "oracle", "sample": cb1[2]}
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

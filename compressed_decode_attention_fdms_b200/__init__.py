@@ -29,7 +29,7 @@ FDMS_KV_BF16, FDMS_KV_FP8_E4M3 = 0, 1
 EXPORTED = (
     "fdms_status_string", "fdms_cache_create", "fdms_cache_destroy", "fdms_append_evict",
     "fdms_decode_attn", "fdms_decode_attn_f32", "fdms_cache_stats", "fdms_cache_read_head",
-    "fdms_decode_attn_noalloc",
+    "fdms_decode_attn_noalloc", "fdms_decode_layout",
 )
 
 
@@ -96,6 +96,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fdms_decode_attn_f32.argtypes = [P, I, I, P, P, P, P]
     lib.fdms_decode_attn_noalloc.restype = I
     lib.fdms_decode_attn_noalloc.argtypes = [P, I, I, P, P, P]
+    lib.fdms_decode_layout.restype = I
+    lib.fdms_decode_layout.argtypes = [P, I, ctypes.POINTER(I), ctypes.POINTER(I)]
     lib.fdms_cache_stats.restype = I
     lib.fdms_cache_stats.argtypes = [P, ctypes.POINTER(fdms_stats), P]
     lib.fdms_cache_read_head.restype = I
@@ -239,6 +241,20 @@ def fdms_decode_attn_noalloc(cache: Cache, layer: int, batch: int, q: torch.Tens
     _check(load_library().fdms_decode_attn_noalloc(
         ctypes.c_void_p(cache.handle), layer, batch, ctypes.c_void_p(qp), ctypes.c_void_p(op),
         ctypes.c_void_p(_stream_ptr(stream, cache.device))), "fdms_decode_attn_noalloc")
+
+
+def fdms_decode_layout(cache: Cache, batch: int) -> dict:
+    """How a decode call of `batch` sequences runs: cluster CTAs per head (0 =
+    global plan) and the split grid of the plan."""
+    cl, sp = ctypes.c_int(), ctypes.c_int()
+    _check(load_library().fdms_decode_layout(ctypes.c_void_p(cache.handle), batch,
+                                             ctypes.byref(cl), ctypes.byref(sp)),
+           "fdms_decode_layout")
+    return {"cluster_ctas": cl.value, "split_ctas": sp.value}
+
+
+def decode_cluster_size(cache: Cache, batch: int) -> int:
+    return fdms_decode_layout(cache, batch)["cluster_ctas"]
 
 
 def fdms_cache_stats(cache: Cache, stream=None) -> dict:

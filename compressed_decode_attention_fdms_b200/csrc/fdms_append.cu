@@ -242,23 +242,34 @@ k_bulk_count(CacheView c, AppendWork aw, BulkIn in) {
 constexpr int kAllocThreads = 1024;
 constexpr int kAllocWarps = kAllocThreads / 32;
 constexpr int kMaxCallHeads = 4096;   // max_batch x num_kv_heads of a supported cache
+constexpr int kAllocPer = kMaxCallHeads / kAllocThreads;
+
+// Dynamic shared memory of k_bulk_alloc for a call of `heads` heads: blocks
+// needed, first block, first new block-table entry, FP8 scales (K, V).
+inline size_t bulk_alloc_smem(int heads) { return (size_t)heads * 5 * sizeof(int); }
 
 // One CTA for every head of the call, in three phases:
-//   1. a warp per head: exclusive prefix of the chunk counts, FP8 scales, the
-//      state before the call and after it (into the head's header), and the
-//      pool blocks the head needs;
+//   1. a thread per head (heads tid, tid + 1024, ...): exclusive prefix of the
+//      chunk counts, FP8 scales, the state before the call and after it (into
+//      the head's header, for the kernels after this one; the thread keeps it
+//      in registers), and the pool blocks the head needs;
 //   2. the blocks of all heads reserved at once, in head order; when the pool
 //      cannot cover them all, heads are served first-fit in head order, so a
 //      head that does not fit leaves the pool to the heads after it;
-//   3. a warp per head: block table entries and lengths, or the error for a
-//      head that got no blocks (left unchanged).
+//   3. the owning thread writes the head's new lengths, or the error for a
+//      head that got no blocks (left unchanged); then a warp per head writes
+//      the block-table entries and their scales.
 // Allocations of different kernels never overlap (each runs after its
 // dependency wait), so inside this kernel the pool counter has one writer.
 template <bool FP8>
 __global__ void __launch_bounds__(kAllocThreads)
 k_bulk_alloc(CacheView c, AppendWork aw, BulkIn in, int nch, int heads) {
-  __shared__ int s_need[kMaxCallHeads];   // blocks a head needs; -1: nothing to do
-  __shared__ int s_blk[kMaxCallHeads];    // first block handed out; -1: none
+  extern __shared__ int s_alloc[];
+  int* s_need = s_alloc;               // blocks a head needs; -1: nothing to do
+  int* s_blk = s_need + heads;         // first block handed out; -1: none
+  int* s_nb0 = s_blk + heads;          // first new block-table entry
+  float* s_sk = reinterpret_cast<float*>(s_nb0 + heads);
+  float* s_sv = s_sk + heads;
   __shared__ int s_wsum[kAllocWarps];
   __shared__ long long s_base;
   pdl_wait();
@@ -266,7 +277,12 @@ k_bulk_alloc(CacheView c, AppendWork aw, BulkIn in, int nch, int heads) {
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
 
   // ---- phase 1
-  for (int hid = warp; hid < heads; hid += kAllocWarps) {
+  int st_len1[kAllocPer], st_n1[kAllocPer], st_r1[kAllocPer];
+#pragma unroll
+  for (int i = 0; i < kAllocPer; ++i) {
+    const int hid = tid + i * kAllocThreads;
+    st_len1[i] = st_n1[i] = st_r1[i] = 0;
+    if (hid >= heads) continue;
     const int b = hid / c.Hkv, h = hid % c.Hkv;
     const long long hi = head_index(c, in.layer, b, h);
     int* hd = aw.hdr + (long long)hid * kHdrInts;
@@ -276,36 +292,29 @@ k_bulk_alloc(CacheView c, AppendWork aw, BulkIn in, int nch, int heads) {
     if constexpr (FP8) {
       ak_bits = aw.amax[hid * 2];
       av_bits = aw.amax[hid * 2 + 1];
-    }
-    __syncwarp();
-    if (FP8 && lane == 0) {   // ready for the next call
-      aw.amax[hid * 2] = 0u;
+      aw.amax[hid * 2] = 0u;   // ready for the next call
       aw.amax[hid * 2 + 1] = 0u;
     }
     if (m < 0 || m > in.max_new || (long long)n0 + m > c.max_seq_len || m == 0) {
-      if (lane == 0) {
-        if (m != 0) latch_error(c.ctr, FDMS_ERR_DEVICE);
-        hd[kHdrStatus] = kBulkSkip;
-        s_need[hid] = -1;
-      }
+      if (m != 0) latch_error(c.ctr, FDMS_ERR_DEVICE);
+      hd[kHdrStatus] = kBulkSkip;
+      s_need[hid] = -1;
       continue;
     }
     const int n1 = n0 + m;
     const int r1 = (n1 - c.W - r0 >= c.P) ? n1 - c.W : r0;
-    // exclusive prefix of the chunk counts
+    // exclusive prefix of the chunk counts, eight loads in flight
     int* cnt = aw.counts + (long long)hid * aw.max_chunks;
     int running = 0;
-    for (int base = 0; base < nch; base += 32) {
-      const int i = base + lane;
-      const int x = i < nch ? cnt[i] : 0;
-      int incl = x;
+    for (int base = 0; base < nch; base += 8) {
+      int x[8];
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += y;
+      for (int u = 0; u < 8; ++u) x[u] = base + u < nch ? cnt[base + u] : 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (base + u < nch) cnt[base + u] = running;
+        running += x[u];
       }
-      if (i < nch) cnt[i] = running + incl - x;
-      running += __shfl_sync(0xffffffffu, incl, 31);
     }
     const int len1 = len0 + running;
     // FP8 scales: a sequence's first append fixes them
@@ -319,10 +328,8 @@ k_bulk_alloc(CacheView c, AppendWork aw, BulkIn in, int nch, int heads) {
           sk = __fdiv_rn(fmaxf(__uint_as_float(ak_bits), 1.17549435e-38f), 448.0f);
           sv = __fdiv_rn(fmaxf(__uint_as_float(av_bits), 1.17549435e-38f), 448.0f);
         }
-        if (lane == 0) {
-          c.head_scale[hi * 2] = sk;
-          c.head_scale[hi * 2 + 1] = sv;
-        }
+        c.head_scale[hi * 2] = sk;
+        c.head_scale[hi * 2 + 1] = sv;
       } else {
         sk = c.head_scale[hi * 2];
         sv = c.head_scale[hi * 2 + 1];
@@ -330,29 +337,33 @@ k_bulk_alloc(CacheView c, AppendWork aw, BulkIn in, int nch, int heads) {
     }
     const int nb0 = (len0 + kBlockSlots - 1) / kBlockSlots;
     const int nb1 = (len1 + kBlockSlots - 1) / kBlockSlots;
-    if (lane == 0) {
-      hd[kHdrM] = m;
-      hd[kHdrN0] = n0;
-      hd[kHdrR0] = r0;
-      hd[kHdrLen0] = len0;
-      hd[kHdrN1] = n1;
-      hd[kHdrR1] = r1;
-      hd[kHdrNb0] = nb0;
-      hd[kHdrLen1] = len1;
-      hd[kHdrStatus] = kBulkGo;
-      hd[kHdrSk] = __float_as_int(sk);
-      hd[kHdrSv] = __float_as_int(sv);
-      s_need[hid] = nb1 - nb0;
-    }
+    hd[kHdrM] = m;
+    hd[kHdrN0] = n0;
+    hd[kHdrR0] = r0;
+    hd[kHdrLen0] = len0;
+    hd[kHdrN1] = n1;
+    hd[kHdrR1] = r1;
+    hd[kHdrNb0] = nb0;
+    hd[kHdrLen1] = len1;
+    hd[kHdrStatus] = kBulkGo;
+    hd[kHdrSk] = __float_as_int(sk);
+    hd[kHdrSv] = __float_as_int(sv);
+    s_need[hid] = nb1 - nb0;
+    s_nb0[hid] = nb0;
+    s_sk[hid] = sk;
+    s_sv[hid] = sv;
+    st_len1[i] = len1;
+    st_n1[i] = n1;
+    st_r1[i] = r1;
   }
   __syncthreads();
 
-  // ---- phase 2: exclusive prefix of the needs in head order
-  constexpr int PER = kMaxCallHeads / kAllocThreads;
-  int mine[PER], sum = 0;
+  // ---- phase 2: exclusive prefix of the needs in head order (thread tid
+  // holds heads tid * kAllocPer .. tid * kAllocPer + kAllocPer - 1)
+  int mine[kAllocPer], sum = 0;
 #pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    const int hid = tid * PER + i;
+  for (int i = 0; i < kAllocPer; ++i) {
+    const int hid = tid * kAllocPer + i;
     mine[i] = hid < heads ? max(s_need[hid], 0) : 0;
     sum += mine[i];
   }
@@ -381,8 +392,8 @@ k_bulk_alloc(CacheView c, AppendWork aw, BulkIn in, int nch, int heads) {
   __syncthreads();
   if (s_base >= 0) {
 #pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      const int hid = tid * PER + i;
+    for (int i = 0; i < kAllocPer; ++i) {
+      const int hid = tid * kAllocPer + i;
       if (hid < heads) s_blk[hid] = (int)(s_base + excl);
       excl += mine[i];
     }
@@ -403,34 +414,34 @@ k_bulk_alloc(CacheView c, AppendWork aw, BulkIn in, int nch, int heads) {
   }
   __syncthreads();
 
-  // ---- phase 3
-  for (int hid = warp; hid < heads; hid += kAllocWarps) {
-    const int need = s_need[hid];
-    if (need < 0) continue;
-    int* hd = aw.hdr + (long long)hid * kHdrInts;
-    const int b = hid / c.Hkv, h = hid % c.Hkv;
-    const long long hi = head_index(c, in.layer, b, h);
-    const long long base_blk = s_blk[hid];
-    if (base_blk < 0) {
-      if (lane == 0) {
-        latch_error(c.ctr, FDMS_ERR_OUT_OF_BLOCKS);
-        hd[kHdrStatus] = kBulkSkip;
-      }
+  // ---- phase 3: lengths (owning thread), then block tables (warp per head)
+#pragma unroll
+  for (int i = 0; i < kAllocPer; ++i) {
+    const int hid = tid + i * kAllocThreads;
+    if (hid >= heads || s_need[hid] < 0) continue;
+    const long long hi = head_index(c, in.layer, hid / c.Hkv, hid % c.Hkv);
+    if (s_blk[hid] < 0) {
+      latch_error(c.ctr, FDMS_ERR_OUT_OF_BLOCKS);
+      aw.hdr[(long long)hid * kHdrInts + kHdrStatus] = kBulkSkip;
       continue;
     }
-    const int nb0 = hd[kHdrNb0];
-    const float sk = __int_as_float(hd[kHdrSk]), sv = __int_as_float(hd[kHdrSv]);
+    c.store_len[hi] = st_len1[i];
+    c.tok_n[hi] = st_n1[i];
+    c.tok_r[hi] = st_r1[i];
+  }
+  for (int hid = warp; hid < heads; hid += kAllocWarps) {
+    const int need = s_need[hid];
+    const long long base_blk = s_blk[hid];
+    if (need <= 0 || base_blk < 0) continue;
+    const long long hi = head_index(c, in.layer, hid / c.Hkv, hid % c.Hkv);
+    const int nb0 = s_nb0[hid];
+    const float sk = s_sk[hid], sv = s_sv[hid];
     int32_t* bt = c.block_table + hi * c.max_blocks;
     float* bts = c.bt_scale + hi * c.max_blocks * 2;
     for (int j = lane; j < need; j += 32) {
       bt[nb0 + j] = (int32_t)(base_blk + j);
       bts[2 * (nb0 + j)] = sk;
       bts[2 * (nb0 + j) + 1] = sv;
-    }
-    if (lane == 0) {
-      c.store_len[hi] = hd[kHdrLen1];
-      c.tok_n[hi] = hd[kHdrN1];
-      c.tok_r[hi] = hd[kHdrR1];
     }
   }
 }
@@ -792,17 +803,14 @@ k_append_small(CacheView c, int layer, int batch, const int32_t* __restrict__ n_
 // (max_new * D / 8 <= 32), one warp per (seq, kv head). Same result as
 // k_append_small; ordered for latency. A head's own state (lengths, FP8
 // scales, ring keep bits and rows, block table) is written only by appends to
-// its layer. When the host knows that the kernel just before this one on the
-// stream is not such an append (`state_early`), the last one has finished by
-// the time this grid starts: every kernel of this library calls the dependency
-// wait before it lets its successor start, except the combine, which is itself
-// started only after its split has waited for the append before it. The state,
-// and the ring rows of every position the call could resolve, are then read
-// before the wait, while the previous kernel still runs, and only the call's
-// own inputs are read after it: a step costs one round trip to memory after
-// the wait (two when the store needs a new block). Without `state_early` the
-// same loads come after the wait, in two round trips. Resolutions larger than
-// two vectors per lane take the general path.
+// its layer. When the host knows that the last append to this layer has
+// finished by the time this grid starts (`state_early`), the state, and the
+// ring rows of every position the call could resolve, are read before the
+// wait, while the previous kernel still runs, and only the call's own inputs
+// are read after it: a step costs one round trip to memory after the wait
+// (two when the store needs a new block). Without `state_early` the same loads
+// come after the wait, in two round trips. Resolutions larger than two
+// vectors per lane take the general path.
 constexpr int kStepVecs = 32;
 
 template <bool FP8>
@@ -811,12 +819,15 @@ k_append_step(CacheView c, int layer, int batch, const int32_t* __restrict__ n_n
               const uint16_t* __restrict__ k_in, const uint16_t* __restrict__ v_in,
               const uint8_t* __restrict__ keep_in, const float* __restrict__ kv_scale,
               int state_early) {
+  // The next kernel may start at once: it reads nothing this one writes
+  // before its own dependency wait (the host keeps track of which kernels have
+  // certainly finished when deciding what may be read early).
+  pdl_launch_dependents();
   if (!state_early) pdl_wait();   // the previous kernel's writes are visible from here on
   const int lane = threadIdx.x & 31;
   const int hid = blockIdx.x * kSmallWarps + (threadIdx.x >> 5);
   if (hid >= batch * c.Hkv) {
     if (state_early) pdl_wait();
-    pdl_launch_dependents();
     return;
   }
   const int b = hid / c.Hkv, h = hid % c.Hkv;
@@ -878,7 +889,6 @@ k_append_step(CacheView c, int layer, int batch, const int32_t* __restrict__ n_n
     if (len0 % kBlockSlots) tail_blk = bt[(len0 - 1) / kBlockSlots];   // partly filled block
   }
   if (state_early) pdl_wait();
-  pdl_launch_dependents();
 
   // ---- the call's inputs: count, rows (vector `lane`), keep bits
   const int m = n_new[b];
@@ -1040,10 +1050,10 @@ fdms_status fdms_launch_append(fdms_cache* cache, int layer, int batch, const in
   const uint16_t* kk = static_cast<const uint16_t*>(k);
   const uint16_t* vv = static_cast<const uint16_t*>(v);
   const float* sc = c.fp8 ? kv_scale : nullptr;
-  // the kernel before this one on the stream may still be writing this layer's
-  // state only if it is an append to the same layer
-  const int early = cache->last_append_layer != layer;
-  cache->last_append_layer = layer;
+  // this layer's state may be read before the dependency wait when its last
+  // writer (the last append to the layer) has certainly finished
+  const int early = fdms_log_finished(cache, cache->append_at[layer]) ? 1 : 0;
+  long long last = 0;
   cudaLaunchConfig_t cfg = {};
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -1059,6 +1069,7 @@ fdms_status fdms_launch_append(fdms_cache* cache, int layer, int batch, const in
                                    kk, vv, keep, sc, early)
               : cudaLaunchKernelEx(&cfg, k_append_step<false>, c, layer, batch, n_new, max_new,
                                    kk, vv, keep, sc, early);
+    last = fdms_log_launch(cache, false);   // lets its successor start at once
   } else if (max_new <= kSmallMax) {
     cfg.gridDim = dim3((unsigned)((batch * c.Hkv + kSmallWarps - 1) / kSmallWarps));
     cfg.blockDim = dim3(kSmallWarps * 32);
@@ -1066,6 +1077,7 @@ fdms_status fdms_launch_append(fdms_cache* cache, int layer, int batch, const in
                                    kk, vv, keep, sc)
               : cudaLaunchKernelEx(&cfg, k_append_small<false>, c, layer, batch, n_new, max_new,
                                    kk, vv, keep, sc);
+    last = fdms_log_launch(cache, true);
   } else {
     const AppendWork& aw = cache->awork;
     const BulkIn in{n_new, kk, vv, keep, sc, batch, max_new, layer};
@@ -1077,17 +1089,22 @@ fdms_status fdms_launch_append(fdms_cache* cache, int layer, int batch, const in
     cfg.blockDim = dim3(kAppendThreads);
     e = c.fp8 ? cudaLaunchKernelEx(&cfg, k_bulk_count<true>, c, aw, in)
               : cudaLaunchKernelEx(&cfg, k_bulk_count<false>, c, aw, in);
+    last = fdms_log_launch(cache, true);
     if (e == cudaSuccess) {
       cfg.gridDim = dim3(1);
       cfg.blockDim = dim3(kAllocThreads);
+      cfg.dynamicSmemBytes = bulk_alloc_smem((int)heads);
       e = c.fp8 ? cudaLaunchKernelEx(&cfg, k_bulk_alloc<true>, c, aw, in, nch, (int)heads)
                 : cudaLaunchKernelEx(&cfg, k_bulk_alloc<false>, c, aw, in, nch, (int)heads);
+      last = fdms_log_launch(cache, true);
     }
     if (e == cudaSuccess) {
       cfg.gridDim = dim3(heads, (unsigned)nch);
       cfg.blockDim = dim3(kAppendThreads);
+      cfg.dynamicSmemBytes = 0;
       e = c.fp8 ? cudaLaunchKernelEx(&cfg, k_bulk_write<true>, c, aw, in)
                 : cudaLaunchKernelEx(&cfg, k_bulk_write<false>, c, aw, in);
+      last = fdms_log_launch(cache, true);
     }
     if (e == cudaSuccess) {   // ring rows: at most W + P - 1 + max_new per head
       const long long rvec = (long long)min((long long)max_new, (long long)c.W + c.P) * (c.D / 8);
@@ -1096,7 +1113,12 @@ fdms_status fdms_launch_append(fdms_cache* cache, int layer, int batch, const in
       cfg.gridDim = dim3(heads, (unsigned)std::max(1, ry));
       e = c.fp8 ? cudaLaunchKernelEx(&cfg, k_bulk_ring<true>, c, aw, in)
                 : cudaLaunchKernelEx(&cfg, k_bulk_ring<false>, c, aw, in);
+      last = fdms_log_launch(cache, true);
     }
+  }
+  if (last > 0) {
+    cache->append_at[layer] = last;
+    cache->tokens_since[layer] += max_new;
   }
   return e == cudaSuccess ? FDMS_OK : FDMS_ERR_CUDA;
 }
@@ -1116,5 +1138,11 @@ fdms_status fdms_append_setup(fdms_cache* cache) {
   aw.counts = static_cast<int*>(take(heads * aw.max_chunks * sizeof(int)));
   aw.hdr = static_cast<int*>(take(heads * kHdrInts * sizeof(int)));
   aw.amax = static_cast<unsigned*>(take(heads * 2 * sizeof(unsigned)));
+  const int smem = (int)bulk_alloc_smem((int)heads);
+  if (cudaFuncSetAttribute(k_bulk_alloc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem) != cudaSuccess ||
+      cudaFuncSetAttribute(k_bulk_alloc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem) != cudaSuccess)
+    return FDMS_ERR_UNSUPPORTED;
   return aw.counts && aw.hdr && aw.amax ? FDMS_OK : FDMS_ERR_CUDA;
 }

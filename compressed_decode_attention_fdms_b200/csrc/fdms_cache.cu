@@ -47,6 +47,13 @@ cudaError_t alloc(fdms_cache* c, T** p, size_t bytes) {
 void free_all(fdms_cache* c) {
   for (int i = 0; i < c->nallocs; ++i) cudaFree(c->allocs[i]);
   c->nallocs = 0;
+  delete[] c->append_at;
+  delete[] c->decode_at;
+  delete[] c->tokens_since;
+  delete[] c->decode_batch;
+  delete[] c->decode_count;
+  c->append_at = c->decode_at = c->tokens_since = c->decode_count = nullptr;
+  c->decode_batch = nullptr;
 }
 
 bool valid_config(const fdms_config* cfg) {
@@ -129,8 +136,13 @@ fdms_status fdms_cache_create(const fdms_config* cfg, int device, void* stream,
   std::memset(c, 0, sizeof(*c));
   c->cfg = *cfg;
   c->device = device;
-  c->last_append_layer = -1;
+  c->append_at = new long long[cfg->num_layers]();
+  c->decode_at = new long long[cfg->num_layers]();
+  c->tokens_since = new long long[cfg->num_layers]();
+  c->decode_batch = new int[cfg->num_layers]();
+  c->decode_count = new long long[cfg->num_layers]();
   if (cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) {
+    free_all(c);
     delete c;
     return FDMS_ERR_CUDA;
   }
@@ -156,6 +168,7 @@ fdms_status fdms_cache_create(const fdms_config* cfg, int device, void* stream,
   const long long heads = (long long)v.L * v.Bmax * v.Hkv;
   v.num_blocks = cfg->num_blocks > 0 ? cfg->num_blocks : heads * v.max_blocks;
   if (v.num_blocks >= (1LL << 31)) {
+    free_all(c);
     delete c;
     return FDMS_ERR_INVALID_ARG;
   }

@@ -96,8 +96,13 @@ struct DecodeWork {
   float* part_ml;         // [max_parts][G][2]: running max (log2 domain) and sum
   int max_parts;
   int max_ctas;
-  int4* snap;             // per head of the cache: (store_len, n, r, 0) the last
-                          // per-head-cluster decode of it saw; null: not kept
+  int4* snap;             // [2][L * Bmax * Hkv]: per head, (store_len, n, r, 0) as a
+                          // decode of it saw them; two copies, so that the kernel
+                          // that writes one never races its own reads of the other
+  int4* snap_rd;          // this call's copies (set per call): the one it reads
+  int4* snap_wr;          // and the one it writes for the next decode of the layer
+  int* head_cnt;          // [Bmax * Hkv]: partials of a head merged so far (global
+                          // plan); back to 0 once merged
 };
 
 // Workspace of the bulk (prefill) append, per (seq, kv head) of the call.
@@ -197,6 +202,38 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src, uint32
       ::"r"(smem_addr(dst_smem)), "l"(src), "r"(bytes), "r"(smem_addr(bar)) : "memory");
 }
 
+// 4-byte global -> shared copy in the background (LDGSTS), and an arrival on
+// `bar` once every such copy this thread issued has landed (the barrier counts
+// one arrival per thread that calls it)
+__device__ __forceinline__ void cp_async4(void* dst_smem, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst_smem)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar))
+               : "memory");
+}
+// atomic add with release and acquire semantics at GPU scope: writes this
+// thread made (or saw, e.g. through a warp barrier) before it are visible to
+// a thread that reads its result, and that thread sees them after it
+__device__ __forceinline__ int atom_add_acq_rel(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v)
+               : "memory");
+  return old;
+}
+
+// add without a result, with release semantics at GPU scope (the writes this
+// thread made or saw before it are visible to whoever acquires the sum)
+__device__ __forceinline__ void red_add_release(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // Programmatic dependent launch: wait for the preceding grid's memory, and let
 // the next grid start its prologue.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -221,13 +258,37 @@ struct fdms_cache {
   int decode_ctas;        // split grid used
   int ctas_per_sm;
   int ranges_per_cta;     // warps per split CTA (one unit range each)
-  // layer of the last append queued on this cache if no decode call was queued
-  // after it, else -1: an append to another layer may read its head state
-  // before its dependency wait (see k_append_step)
-  int last_append_layer;
   int cluster_ok;         // the per-head cluster decode mode can be launched
   int max_clusters[4];    // clusters of 2, 4, 8 CTAs (index 1..3) resident at once
+  int plan_ctas_per_sm;   // global-plan split CTAs that fit on one SM
+  // Kernels queued on the cache, numbered from 1 in launch order. A kernel
+  // that lets its successor start only after its own dependency wait ("waits
+  // first": every decode kernel, the bulk and small appends) has seen every
+  // kernel before it finish when it passes that wait; the decode-step append
+  // lets its successor start at once. So when a new kernel starts, every
+  // kernel queued before the latest "waits first" one has finished: a head's
+  // state may be read before the dependency wait only if its last writer is
+  // one of those.
+  long long launches;         // kernels queued so far
+  long long last_wait_first;  // number of the latest "waits first" kernel, 0: none
+  long long* append_at;       // [L]: number of the last append kernel to the layer
+  long long* decode_at;       // [L]: number of the last decode kernel of the layer
+  long long* tokens_since;    // [L]: tokens per sequence appended since that decode
+  int* decode_batch;          // [L]: batch of that decode
+  long long* decode_count;    // [L]: decode calls of the layer so far (snapshot copy)
 };
+
+// Number a kernel just queued; `waits_first`: it lets its successor start only
+// after its own dependency wait.
+inline long long fdms_log_launch(fdms_cache* c, bool waits_first) {
+  const long long n = ++c->launches;
+  if (waits_first) c->last_wait_first = n;
+  return n;
+}
+// Kernel number n (0: none) has certainly finished when the next kernel starts.
+inline bool fdms_log_finished(const fdms_cache* c, long long n) {
+  return n < c->last_wait_first;
+}
 
 // Record a device allocation of the cache (freed at destroy). Frees `p` and
 // returns false when the table is full.

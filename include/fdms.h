@@ -17,7 +17,8 @@
  *                        survivors of its kv head (split over the GPU, then
  *                        merged: through distributed shared memory inside a
  *                        cluster of CTAs per head for calls with few heads, by
- *                        a combine kernel otherwise);
+ *                        the last split warp of each head to finish otherwise;
+ *                        one kernel either way);
  *   fdms_cache_stats   - counters, including compact vs dense-equivalent bytes
  *                        (the quantity of the pages' KV-memory table).
  *
@@ -47,11 +48,18 @@
  *
  * Ordering and threads: queue the calls on one cache in program order on one
  * stream, or order streams with events. Consecutive kernels on a stream overlap
- * through programmatic dependent launch; each kernel reads data its
- * predecessor writes only after waiting for it. A cache keeps host-side state
- * (which layer the last append went to, which decides how early the next append
- * may read its head state), so calls on one cache must not run concurrently
- * from several host threads; different caches are independent.
+ * through programmatic dependent launch: a kernel may start while the one
+ * before it finishes, and reads what that kernel writes only after its
+ * dependency wait. Before the wait a kernel reads only cache state that a
+ * kernel queued earlier has certainly finished writing: the cache keeps a
+ * host-side log of the kernels it queued, and every kernel that starts has
+ * seen each kernel before the last "wait-first" kernel (one whose every CTA
+ * waits before it lets its dependents start) complete. Kernels of other code
+ * queued between the library's calls keep that true as long as none of them
+ * lets its dependents start before its own dependency wait (kernels launched
+ * without programmatic dependent launch never do). Because of that host-side
+ * state, calls on one cache must not run concurrently from several host
+ * threads; different caches are independent.
  *
  * Errors: every call validates its arguments on the host and returns a status
  * before queuing any work. Calls that queue kernels are asynchronous; errors
@@ -101,11 +109,14 @@ typedef struct {
                             max_seq_len tokens in every (layer, seq, kv head) */
   fdms_kv_dtype kv_dtype;
   float softmax_scale;   /* 0 -> 1 / sqrt(head_dim) */
-  int decode_ctas;       /* 0 -> automatic: a call with at most half as many
-                            (seq, kv head) pairs as SMs runs one cluster of 2-8
-                            CTAs per pair; other calls run one plan over SM
-                            count x CTAs per SM split CTAs. > 0 -> always the
-                            plan, over this many CTAs */
+  int decode_ctas;       /* 0 -> automatic: a call whose (seq, kv head) pairs
+                            can all hold a cluster of 8, 4 or 2 CTAs at once on
+                            this device runs one cluster (of the largest such
+                            size) per pair; other calls run
+                            one plan over SM-count split CTAs (two may share an
+                            SM, so consecutive calls overlap). > 0 -> always
+                            the plan, over this many CTAs, at most as many
+                            as can be resident on the device at once */
 } fdms_config;
 
 typedef struct {
@@ -194,12 +205,14 @@ fdms_status fdms_decode_attn_f32(fdms_cache* cache, int layer, int batch,
  * which fdms_decode_attn keeps in workspace the cache allocated, go instead
  * into one static array of FDMS_STATIC_SCRATCH_BYTES compiled into the library;
  * every device that loads the library holds that array until the process exits.
- *   - Needs (split warps + batch x Hkv) x G x (4 D + 8) bytes (at most one
- *     partial per split warp and head it shares with another warp; 8 split
- *     warps per decode CTA, 4 when G x D >= 1024), or none for a call that
- *     runs in per-head clusters (see decode_ctas); a call that needs more than
- *     the array returns FDMS_ERR_INVALID_ARG and queues nothing. Every value
- *     the call reads from the array it first writes itself.
+ *   - Needs (split warps + batch x Hkv) x G x (4 D + 8) bytes plus
+ *     4 x batch x Hkv bytes of merge counters, each part rounded up to 256
+ *     (at most one partial per split warp and head it shares with another
+ *     warp; 4 to 6 split warps per decode CTA), or none for a call that runs in
+ *     per-head clusters (see decode_ctas); a call that needs more than the
+ *     array returns FDMS_ERR_INVALID_ARG and queues nothing. The call clears
+ *     the counters on its stream before its kernel; every other value it reads
+ *     from the array it first writes itself.
  *   - The first call on a device looks up the array's device address (a
  *     runtime query, no allocation); make that first call before any stream
  *     capture.
@@ -209,6 +222,14 @@ fdms_status fdms_decode_attn_f32(fdms_cache* cache, int layer, int batch,
  * Allocates nothing and calls no allocating routine. */
 fdms_status fdms_decode_attn_noalloc(fdms_cache* cache, int layer, int batch,
                                      const void* q_dev, void* out_dev, void* stream);
+
+/* How a decode call of `batch` sequences would run on this cache (no device
+ * work): *cluster_ctas_out receives the CTAs of the thread-block cluster per
+ * (seq, kv head) (2, 4 or 8), or 0 when the call runs the global plan, whose
+ * split grid (CTAs) goes to *split_ctas_out. Either pointer may be NULL.
+ * INVALID_ARG for a NULL cache or batch outside 1..max_batch. */
+fdms_status fdms_decode_layout(fdms_cache* cache, int batch, int* cluster_ctas_out,
+                               int* split_ctas_out);
 
 /* Gather the counters on `stream` and wait for them. */
 fdms_status fdms_cache_stats(fdms_cache* cache, fdms_stats* host_out, void* stream);
