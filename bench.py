@@ -64,6 +64,9 @@ def parse_args():
     ap.add_argument("--decode-ctas", type=int, default=0)
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the other workloads' decode calls in the default run")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="run only the workload's first N layers (a smaller case for "
+                         "profiling: one decode call's bytes do not depend on it)")
     return ap.parse_args()
 
 
@@ -102,8 +105,9 @@ def load_traffic(workload):
         if not f or f[0].startswith("#") or f[0] != workload:
             continue
         if f[2:4] == now:
-            return float(f[1]), "ncu dram__bytes_read.sum + dram__bytes_write.sum of " \
-                                "one decode call's kernels"
+            return float(f[1]), "ncu dram__bytes_read.sum + dram__bytes_write.sum per " \
+                                "decode call, mean over the calls of two full steps " \
+                                f"(profiles/k_decode_split_{workload}.md)"
         return None, "decode kernels changed since the ncu capture"
     return None, "no capture for this workload"
 
@@ -535,12 +539,14 @@ def measure(fd, args, wl, dev, local, world, K, W, KE, WE):
 
 
 def decode_kernel_desc(cs):
-    return (f"fdms_decode_attn (k_decode_split, one cluster of {cs} CTAs per (seq, kv head), "
-            "no combine)" if cs else "fdms_decode_attn (k_decode_split + k_decode_combine)")
+    return (f"fdms_decode_attn (k_decode_split: one cluster of {cs} CTAs per (seq, kv head), "
+            "merged through distributed shared memory)" if cs else
+            "fdms_decode_attn (k_decode_plan: one tile plan over the grid, each shared head "
+            "merged by the warp holding its last tile)")
 
 
 # workloads reported next to the headline one in the default run (their decode
-# call and step at a shorter run; BASELINE's other single-GPU configs)
+# call and step at a shorter run): the pages' other single-GPU workloads
 EXTRA_WORKLOADS = ("qwen8b_c8_fp8", "llama1b_c1")
 
 
@@ -683,6 +689,8 @@ def run_e2e(fd, cache, wl, stream, dev, s0, warm, steps, row):
 def main():
     args = parse_args()
     wl = wk.get(args.workload)
+    if args.layers > 0:
+        wl = wk.scaled(wl, layers=min(args.layers, wl.layers))
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_native(args, wl)
