@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(HERE, "libfdms.so")
 
 FDMS_OK, FDMS_ERR_INVALID_ARG, FDMS_ERR_OUT_OF_BLOCKS, FDMS_ERR_CUDA, \
     FDMS_ERR_UNSUPPORTED, FDMS_ERR_DEVICE = range(6)
-FDMS_KV_BF16, FDMS_KV_FP8_E4M3 = 0, 1
+FDMS_KV_BF16, FDMS_KV_FP8_E4M3, FDMS_KV_FP8_E4M3_BLOCK = 0, 1, 2
 
 # every symbol include/fdms.h declares
 EXPORTED = (
@@ -136,6 +136,8 @@ class Cache:
 
     @property
     def elt(self) -> int:
+        """Bytes per element of a row fdms_cache_read_head returns (a per-block
+        FP8 cache returns 2 D bytes per row: codes, or bf16 for staged rows)."""
         return 1 if self.config.kv_dtype == FDMS_KV_FP8_E4M3 else 2
 
     def __del__(self):
@@ -151,7 +153,8 @@ class Cache:
 def make_config(num_layers, max_batch, num_q_heads, num_kv_heads, head_dim, window,
                 compact_period=1, max_seq_len=8192, num_blocks=0, kv_dtype="bf16",
                 softmax_scale=0.0, decode_ctas=0) -> fdms_config:
-    dt = {"bf16": FDMS_KV_BF16, "fp8_e4m3": FDMS_KV_FP8_E4M3}[kv_dtype] \
+    dt = {"bf16": FDMS_KV_BF16, "fp8_e4m3": FDMS_KV_FP8_E4M3,
+          "fp8_e4m3_block": FDMS_KV_FP8_E4M3_BLOCK}[kv_dtype] \
         if isinstance(kv_dtype, str) else int(kv_dtype)
     return fdms_config(num_layers, max_batch, num_q_heads, num_kv_heads, head_dim, window,
                        compact_period, max_seq_len, num_blocks, dt, softmax_scale, decode_ctas)

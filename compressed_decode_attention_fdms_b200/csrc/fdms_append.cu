@@ -1038,6 +1038,193 @@ k_append_step(CacheView c, int layer, int batch, const int32_t* __restrict__ n_n
   }
 }
 
+
+// ===================================================== per-block FP8 append
+// FDMS_KV_FP8_E4M3_BLOCK: survivors go, in order, to the head's bf16 staging
+// block; when its 64th row is written the block is sealed: one pool block
+// (taken from the bump allocator for all of the call's seals at once, before
+// any write, so a head that does not fit is left unchanged), K and V scales
+// max(amax over the 64 rows, 2^-126) / 448, the rows quantised into it with the
+// same correctly rounded quotient as the other FP8 paths. New tokens that stay
+// unresolved go to the ring as bf16. A warp per head, any call size (the
+// survivors of a 32-position chunk cross at most one block boundary).
+
+// 16-byte bf16 vector `vec` of row `row` in a bf16 page of `rb`-byte rows
+__device__ __forceinline__ uint4* bf16_vec(uint8_t* page, int rb, bool is_v, int row, int vec) {
+  return reinterpret_cast<uint4*>(page + (long long)row * rb + swz_byte(rb, is_v, row, vec * 16));
+}
+
+__device__ __forceinline__ float amax8(uint4 x) {
+  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+  float a = 0.f;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    a = fmaxf(a, fmaxf(fabsf(bf16lo_to_f32(w[j])), fabsf(bf16hi_to_f32(w[j]))));
+  return a;
+}
+
+// Seal the staging block of head hi as store block jb in pool block blk.
+__device__ void seal_block(const CacheView& c, long long hi, int jb, long long blk, int lane,
+                           unsigned& sat) {
+  const int VPR = c.D / 8, SRB = 2 * c.D;
+  uint8_t* sk = stage_k(c, hi);
+  uint8_t* sv = stage_v(c, hi);
+  float ak = 0.f, av = 0.f;
+  for (int i = lane; i < kBlockSlots * VPR; i += 32) {
+    const int row = i / VPR, vec = i % VPR;
+    ak = fmaxf(ak, amax8(*bf16_vec(sk, SRB, false, row, vec)));
+    av = fmaxf(av, amax8(*bf16_vec(sv, SRB, true, row, vec)));
+  }
+  for (int off = 16; off > 0; off >>= 1) {
+    ak = fmaxf(ak, __shfl_xor_sync(0xffffffffu, ak, off));
+    av = fmaxf(av, __shfl_xor_sync(0xffffffffu, av, off));
+  }
+  const float sck = __fdiv_rn(fmaxf(ak, 1.17549435e-38f), 448.0f);
+  const float scv = __fdiv_rn(fmaxf(av, 1.17549435e-38f), 448.0f);
+  const float qk = quant_recip(sck), qv = quant_recip(scv);
+  uint8_t* dk = block_k(c, blk);
+  uint8_t* dv = block_v(c, blk);
+  for (int i = lane; i < kBlockSlots * VPR; i += 32) {
+    const int row = i / VPR, vec = i % VPR;
+    *reinterpret_cast<uint2*>(dk + (long long)row * c.RB + swz_byte(c.RB, false, row, vec * 8)) =
+        quantise8(*bf16_vec(sk, SRB, false, row, vec), sck, qk, sat);
+    *reinterpret_cast<uint2*>(dv + (long long)row * c.RB + swz_byte(c.RB, true, row, vec * 8)) =
+        quantise8(*bf16_vec(sv, SRB, true, row, vec), scv, qv, sat);
+  }
+  for (int row = lane; row < kBlockSlots; row += 32)
+    c.blk_pos[blk * kBlockSlots + row] = c.stage_pos[hi * kBlockSlots + row];
+  if (lane == 0) {
+    c.block_table[hi * c.max_blocks + jb] = (int32_t)blk;
+    c.bt_scale[(hi * c.max_blocks + jb) * 2] = sck;
+    c.bt_scale[(hi * c.max_blocks + jb) * 2 + 1] = scv;
+  }
+}
+
+__global__ void __launch_bounds__(kSmallWarps * 32)
+k_append_block(CacheView c, int layer, int batch, const int32_t* __restrict__ n_new,
+               int max_new, const uint16_t* __restrict__ k_in, const uint16_t* __restrict__ v_in,
+               const uint8_t* __restrict__ keep_in) {
+  pdl_wait();                 // the previous kernel's writes are visible from here on
+  pdl_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int hid = blockIdx.x * kSmallWarps + (threadIdx.x >> 5);
+  if (hid >= batch * c.Hkv) return;
+  const int b = hid / c.Hkv, h = hid % c.Hkv;
+  const long long hi = head_index(c, layer, b, h);
+  const long long in_stride = (long long)c.Hkv * c.D;   // elements between tokens
+  const uint16_t* k_rows = k_in + ((long long)b * max_new * c.Hkv + h) * c.D;
+  const uint16_t* v_rows = v_in + ((long long)b * max_new * c.Hkv + h) * c.D;
+  const uint8_t* keep_rows = keep_in + (long long)b * max_new * c.Hkv + h;
+  uint8_t* rkeep = c.ring_keep + hi * c.Rpad;
+  const int VPR = c.D / 8, SRB = 2 * c.D;
+  constexpr unsigned kAll = 0xffffffffu;
+
+  const int m = n_new[b];
+  const int n0 = c.tok_n[hi], r0 = c.tok_r[hi], len0 = c.store_len[hi];
+  if (m < 0 || m > max_new || (long long)n0 + m > c.max_seq_len) {
+    if (lane == 0) latch_error(c.ctr, FDMS_ERR_DEVICE);
+    return;
+  }
+  if (m == 0) return;
+  const int n1 = n0 + m;
+  const int r1 = (n1 - c.W - r0 >= c.P) ? n1 - c.W : r0;
+  auto keep_of = [&](int p) -> int {
+    return p < n0 ? (rkeep[p % c.R] != 0) : (keep_rows[(long long)(p - n0) * c.Hkv] != 0);
+  };
+
+  // survivors, and the pool blocks the call seals (one bump, before any write)
+  int total = 0;
+  for (int base = r0; base < r1; base += 32) {
+    const int p = base + lane;
+    total += __popc(__ballot_sync(kAll, p < r1 && keep_of(p)));
+  }
+  const int len1 = len0 + total;
+  const int nseal = len1 / kBlockSlots - len0 / kBlockSlots;
+  long long base_blk = 0;
+  if (nseal > 0) {
+    int fail = 0;
+    if (lane == 0) {
+      const long long base = take_blocks(c.ctr, (unsigned long long)nseal, c.num_blocks);
+      if (base < 0) {
+        latch_error(c.ctr, FDMS_ERR_OUT_OF_BLOCKS);
+        fail = 1;
+      } else {
+        base_blk = base;
+      }
+    }
+    if (__shfl_sync(kAll, fail, 0)) return;
+    base_blk = __shfl_sync(kAll, base_blk, 0);
+  }
+
+  // survivors to staging rows, in store order, sealing each block that fills
+  unsigned sat = 0;
+  uint8_t* sk = stage_k(c, hi);
+  uint8_t* sv = stage_v(c, hi);
+  int len = len0;
+  auto stage_rows = [&](unsigned ball, int base, int k0, int k1, int d0) {
+    // ranks k0 .. k1-1 of the chunk's survivors to store indices d0 + (rank - k0)
+    for (int i = lane; i < (k1 - k0) * VPR; i += 32) {
+      const int rank = k0 + i / VPR, vec = i % VPR;
+      const int src = base + (int)__fns(ball, 0, rank + 1);
+      const int row = (d0 + rank - k0) % kBlockSlots;
+      uint4 xk, xv;
+      if (src < n0) {
+        const int slot = src % c.R;
+        xk = *bf16_vec(ring_k(c, hi), SRB, false, slot, vec);
+        xv = *bf16_vec(ring_v(c, hi), SRB, true, slot, vec);
+      } else {
+        const long long t = src - n0;
+        xk = *reinterpret_cast<const uint4*>(k_rows + t * in_stride + vec * 8);
+        xv = *reinterpret_cast<const uint4*>(v_rows + t * in_stride + vec * 8);
+      }
+      *bf16_vec(sk, SRB, false, row, vec) = xk;
+      *bf16_vec(sv, SRB, true, row, vec) = xv;
+      if (vec == 0) c.stage_pos[hi * kBlockSlots + row] = src;
+    }
+  };
+  for (int base = r0; base < r1; base += 32) {
+    const int p = base + lane;
+    const unsigned ball = __ballot_sync(kAll, p < r1 && keep_of(p));
+    const int cnt = __popc(ball);
+    if (cnt == 0) continue;
+    const int first = min(cnt, kBlockSlots - len % kBlockSlots);   // fills the open block
+    stage_rows(ball, base, 0, first, len);
+    len += first;
+    if (len % kBlockSlots == 0) {
+      __syncwarp();
+      const int jb = len / kBlockSlots - 1;
+      seal_block(c, hi, jb, base_blk + (jb - len0 / kBlockSlots), lane, sat);
+      __syncwarp();   // the staging rows are read before the next ones are written
+    }
+    if (cnt > first) {
+      stage_rows(ball, base, first, cnt, len);
+      len += cnt - first;
+    }
+  }
+  __syncwarp();   // ring slots read above may be overwritten below
+
+  // the call's unresolved tokens to the ring, in bf16
+  const int w0 = r1 > n0 ? r1 : n0;
+  for (int i = lane; i < (n1 - w0) * VPR; i += 32) {
+    const int p = w0 + i / VPR, vec = i % VPR;
+    const long long t = p - n0;
+    const int slot = p % c.R;
+    *bf16_vec(ring_k(c, hi), SRB, false, slot, vec) =
+        *reinterpret_cast<const uint4*>(k_rows + t * in_stride + vec * 8);
+    *bf16_vec(ring_v(c, hi), SRB, true, slot, vec) =
+        *reinterpret_cast<const uint4*>(v_rows + t * in_stride + vec * 8);
+    if (vec == 0) rkeep[slot] = keep_rows[t * c.Hkv] ? 1 : 0;
+  }
+  for (int off = 16; off > 0; off >>= 1) sat += __shfl_xor_sync(kAll, sat, off);
+  if (lane == 0 && sat) atomicAdd(&c.ctr->saturations, (unsigned long long)sat);
+  __syncwarp();
+  if (lane == 0) {
+    c.store_len[hi] = len1;
+    c.tok_n[hi] = n1;
+    c.tok_r[hi] = r1;
+  }
+}
+
 }  // namespace
 }  // namespace fdms
 
@@ -1049,7 +1236,7 @@ fdms_status fdms_launch_append(fdms_cache* cache, int layer, int batch, const in
   const CacheView& c = cache->view;
   const uint16_t* kk = static_cast<const uint16_t*>(k);
   const uint16_t* vv = static_cast<const uint16_t*>(v);
-  const float* sc = c.fp8 ? kv_scale : nullptr;
+  const float* sc = c.fp8 && !c.blk ? kv_scale : nullptr;
   // this layer's state may be read before the dependency wait when its last
   // writer (the last append to the layer) has certainly finished
   const int early = fdms_log_finished(cache, cache->append_at[layer]) ? 1 : 0;
@@ -1062,7 +1249,12 @@ fdms_status fdms_launch_append(fdms_cache* cache, int layer, int batch, const in
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e;
-  if (max_new * (c.D / 8) <= kStepVecs) {
+  if (c.blk) {   // per-block FP8: one warp-per-head path for every call size
+    cfg.gridDim = dim3((unsigned)((batch * c.Hkv + kSmallWarps - 1) / kSmallWarps));
+    cfg.blockDim = dim3(kSmallWarps * 32);
+    e = cudaLaunchKernelEx(&cfg, k_append_block, c, layer, batch, n_new, max_new, kk, vv, keep);
+    last = fdms_log_launch(cache, true);
+  } else if (max_new * (c.D / 8) <= kStepVecs) {
     cfg.gridDim = dim3((unsigned)((batch * c.Hkv + kSmallWarps - 1) / kSmallWarps));
     cfg.blockDim = dim3(kSmallWarps * 32);
     e = c.fp8 ? cudaLaunchKernelEx(&cfg, k_append_step<true>, c, layer, batch, n_new, max_new,

@@ -62,7 +62,9 @@ bool valid_config(const fdms_config* cfg) {
   if (cfg->num_q_heads < 1 || cfg->num_q_heads % cfg->num_kv_heads != 0) return false;
   if (cfg->window < 0 || cfg->compact_period < 1 || cfg->max_seq_len < 1) return false;
   if (cfg->num_blocks < 0 || cfg->decode_ctas < 0) return false;
-  if (cfg->kv_dtype != FDMS_KV_BF16 && cfg->kv_dtype != FDMS_KV_FP8_E4M3) return false;
+  if (cfg->kv_dtype != FDMS_KV_BF16 && cfg->kv_dtype != FDMS_KV_FP8_E4M3 &&
+      cfg->kv_dtype != FDMS_KV_FP8_E4M3_BLOCK)
+    return false;
   if (!(cfg->softmax_scale >= 0.0f) || !std::isfinite(cfg->softmax_scale)) return false;
   if ((long long)cfg->window + cfg->compact_period > (1LL << 30)) return false;
   return true;
@@ -77,13 +79,14 @@ bool supported_config(const fdms_config* cfg) {
 }
 
 // Totals over all heads, one CTA (the stats call is not on the hot path).
-__global__ void k_stats(CacheView c) {
-  __shared__ unsigned long long s_tok[32], s_store[32], s_ring[32];
+__global__ void __launch_bounds__(1024) k_stats(CacheView c) {
+  __shared__ unsigned long long s_tok[32], s_store[32], s_ring[32], s_seal[32];
   const long long heads = (long long)c.L * c.Bmax * c.Hkv;
-  unsigned long long tok = 0, store = 0, ring = 0;
+  unsigned long long tok = 0, store = 0, ring = 0, seal = 0;
   for (long long hi = threadIdx.x; hi < heads; hi += blockDim.x) {
-    const int n = c.tok_n[hi], r = c.tok_r[hi];
-    store += (unsigned long long)c.store_len[hi];
+    const int n = c.tok_n[hi], r = c.tok_r[hi], len = c.store_len[hi];
+    store += (unsigned long long)len;
+    seal += (unsigned long long)(len / kBlockSlots * kBlockSlots);
     ring += (unsigned long long)(n - r);
     if (hi % c.Hkv == 0) tok += (unsigned long long)n;
   }
@@ -91,17 +94,112 @@ __global__ void k_stats(CacheView c) {
     tok += __shfl_xor_sync(0xffffffffu, tok, off);
     store += __shfl_xor_sync(0xffffffffu, store, off);
     ring += __shfl_xor_sync(0xffffffffu, ring, off);
+    seal += __shfl_xor_sync(0xffffffffu, seal, off);
   }
   const int w = threadIdx.x / 32, l = threadIdx.x % 32;
-  if (l == 0) { s_tok[w] = tok; s_store[w] = store; s_ring[w] = ring; }
+  if (l == 0) { s_tok[w] = tok; s_store[w] = store; s_ring[w] = ring; s_seal[w] = seal; }
   __syncthreads();
   if (threadIdx.x == 0) {
-    unsigned long long a = 0, b = 0, d = 0;
-    for (int i = 0; i < (int)(blockDim.x / 32); ++i) { a += s_tok[i]; b += s_store[i]; d += s_ring[i]; }
+    unsigned long long a = 0, b = 0, d = 0, e = 0;
+    for (int i = 0; i < (int)(blockDim.x / 32); ++i) {
+      a += s_tok[i]; b += s_store[i]; d += s_ring[i]; e += s_seal[i];
+    }
     c.ctr->tokens = a;
     c.ctr->slots_store = b;
     c.ctr->slots_ring = d;
+    c.ctr->slots_sealed = e;
   }
+}
+
+// fdms_cache_read_head for per-block FP8: host rows of 2 D bytes; sealed
+// entries carry their codes in the first D bytes and the block's scales, staged
+// and ring entries their bf16 values and scale 0.
+fdms_status read_head_block(const CacheView& v, long long hi, int n, int r, int len,
+                            int32_t* pos_host, uint8_t* keep_host, void* k_host, void* v_host,
+                            float* scale_host) {
+  const int RB = v.RB, SRB = 2 * v.D;
+  uint8_t* kh = static_cast<uint8_t*>(k_host);
+  uint8_t* vh = static_cast<uint8_t*>(v_host);
+  auto unswizzle = [](uint8_t* dst, const uint8_t* src, int rb, int row, bool is_v) {
+    for (int b = 0; b < rb; b += 16) std::memcpy(dst + b, src + swz_byte(rb, is_v, row, b), 16);
+  };
+  cudaError_t e = cudaSuccess;
+  const int nseal = len / kBlockSlots;
+  std::vector<int32_t> bt(nseal > 0 ? nseal : 1);
+  std::vector<float> bs(2 * (nseal > 0 ? nseal : 1));
+  if (nseal > 0) {
+    e = cudaMemcpy(bt.data(), v.block_table + hi * v.max_blocks, nseal * 4,
+                   cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess)
+      e = cudaMemcpy(bs.data(), v.bt_scale + hi * v.max_blocks * 2, nseal * 8,
+                     cudaMemcpyDeviceToHost);
+  }
+  std::vector<uint8_t> tmp((size_t)kBlockSlots * SRB);
+  for (int j = 0; j < nseal && e == cudaSuccess; ++j) {
+    const int base = j * kBlockSlots;
+    const long long blk = bt[j];
+    for (int which = 0; which < 2 && e == cudaSuccess; ++which) {
+      uint8_t* dst = which ? vh : kh;
+      if (!dst) continue;
+      e = cudaMemcpy(tmp.data(), which ? block_v(v, blk) : block_k(v, blk),
+                     (size_t)kBlockSlots * RB, cudaMemcpyDeviceToHost);
+      for (int i = 0; i < kBlockSlots; ++i) {
+        uint8_t* row = dst + (size_t)(base + i) * SRB;
+        std::memset(row, 0, SRB);
+        unswizzle(row, tmp.data() + (size_t)i * RB, RB, i, which == 1);
+      }
+    }
+    if (pos_host && e == cudaSuccess)
+      e = cudaMemcpy(pos_host + base, v.blk_pos + blk * kBlockSlots, kBlockSlots * 4,
+                     cudaMemcpyDeviceToHost);
+    for (int i = 0; i < kBlockSlots; ++i) {
+      if (keep_host) keep_host[base + i] = 1;
+      if (scale_host) {
+        scale_host[2 * (base + i)] = bs[2 * j];
+        scale_host[2 * (base + i) + 1] = bs[2 * j + 1];
+      }
+    }
+  }
+  // staged rows: the store's partly filled block
+  const int staged = len - nseal * kBlockSlots;
+  if (staged > 0 && e == cudaSuccess) {
+    const int base = nseal * kBlockSlots;
+    for (int which = 0; which < 2 && e == cudaSuccess; ++which) {
+      uint8_t* dst = which ? vh : kh;
+      if (!dst) continue;
+      e = cudaMemcpy(tmp.data(), which ? stage_v(v, hi) : stage_k(v, hi),
+                     (size_t)staged * SRB, cudaMemcpyDeviceToHost);
+      for (int i = 0; i < staged; ++i)
+        unswizzle(dst + (size_t)(base + i) * SRB, tmp.data() + (size_t)i * SRB, SRB, i,
+                  which == 1);
+    }
+    if (pos_host && e == cudaSuccess)
+      e = cudaMemcpy(pos_host + base, v.stage_pos + hi * kBlockSlots, (size_t)staged * 4,
+                     cudaMemcpyDeviceToHost);
+    for (int i = 0; i < staged; ++i) {
+      if (keep_host) keep_host[base + i] = 1;
+      if (scale_host) scale_host[2 * (base + i)] = scale_host[2 * (base + i) + 1] = 0.0f;
+    }
+  }
+  if (e != cudaSuccess) return FDMS_ERR_CUDA;
+  // ring, in position order r..n-1, bf16
+  if (n > r) {
+    std::vector<uint8_t> rk((size_t)v.R * SRB), rv((size_t)v.R * SRB), rkeep(v.R);
+    e = cudaMemcpy(rk.data(), ring_k(v, hi), rk.size(), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemcpy(rv.data(), ring_v(v, hi), rv.size(), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess)
+      e = cudaMemcpy(rkeep.data(), v.ring_keep + hi * v.Rpad, v.R, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return FDMS_ERR_CUDA;
+    for (int p = r; p < n; ++p) {
+      const int slot = p % v.R, i = len + (p - r);
+      if (pos_host) pos_host[i] = p;
+      if (keep_host) keep_host[i] = rkeep[slot];
+      if (kh) unswizzle(kh + (size_t)i * SRB, rk.data() + (size_t)slot * SRB, SRB, slot, false);
+      if (vh) unswizzle(vh + (size_t)i * SRB, rv.data() + (size_t)slot * SRB, SRB, slot, true);
+      if (scale_host) scale_host[2 * i] = scale_host[2 * i + 1] = 0.0f;
+    }
+  }
+  return FDMS_OK;
 }
 
 }  // namespace
@@ -153,8 +251,10 @@ fdms_status fdms_cache_create(const fdms_config* cfg, int device, void* stream,
   v.Hkv = cfg->num_kv_heads;
   v.G = v.Hq / v.Hkv;
   v.D = cfg->head_dim;
-  v.fp8 = cfg->kv_dtype == FDMS_KV_FP8_E4M3;
+  v.blk = cfg->kv_dtype == FDMS_KV_FP8_E4M3_BLOCK;
+  v.fp8 = cfg->kv_dtype == FDMS_KV_FP8_E4M3 || v.blk;
   v.RB = v.D * (v.fp8 ? 1 : 2);
+  v.RBR = v.blk ? 2 * v.D : v.RB;   // per-block FP8 stages its rows in bf16
   v.W = cfg->window;
   v.P = cfg->compact_period;
   // ring capacity: W + P - 1 unresolved tokens at most, rounded up to whole
@@ -184,7 +284,11 @@ fdms_status fdms_cache_create(const fdms_config* cfg, int device, void* stream,
   A(&v.store_len, (size_t)heads * sizeof(int32_t));
   A(&v.tok_n, (size_t)heads * sizeof(int32_t));
   A(&v.tok_r, (size_t)heads * sizeof(int32_t));
-  A(&v.ring, (size_t)heads * 2 * v.R * v.RB);
+  A(&v.ring, (size_t)heads * 2 * v.R * v.RBR);
+  if (v.blk) {
+    A(&v.stage, (size_t)heads * 2 * kBlockSlots * 2 * v.D);
+    A(&v.stage_pos, (size_t)heads * kBlockSlots * sizeof(int32_t));
+  }
   A(&v.ring_keep, (size_t)heads * v.Rpad);
   A(&v.head_scale, (size_t)heads * 2 * sizeof(float));
   A(&v.ctr, sizeof(DevCounters));
@@ -234,7 +338,7 @@ fdms_status fdms_append_evict(fdms_cache* c, int layer, int batch, const int32_t
   if (batch == 0 || max_new == 0) return FDMS_OK;
   if (!n_new_dev || !k_dev || !v_dev || !keep_dev) return FDMS_ERR_INVALID_ARG;
   if (((uintptr_t)k_dev | (uintptr_t)v_dev) & 15) return FDMS_ERR_INVALID_ARG;
-  if (kv_scale_dev && !v.fp8) return FDMS_ERR_INVALID_ARG;
+  if (kv_scale_dev && (!v.fp8 || v.blk)) return FDMS_ERR_INVALID_ARG;
   if (max_new > v.max_seq_len) return FDMS_ERR_INVALID_ARG;
   DeviceGuard guard(c->device);
   return fdms_launch_append(c, layer, batch, n_new_dev, max_new, k_dev, v_dev, keep_dev,
@@ -288,6 +392,9 @@ fdms_status fdms_cache_stats(fdms_cache* c, fdms_stats* out, void* stream) {
   out->blocks_used = used;
   out->blocks_free = v.num_blocks - used;
   out->bytes_compact = (out->slots_store + out->slots_ring) * row;
+  if (v.blk)   // sealed slots in E4M3, staged and ring slots in bf16
+    out->bytes_compact = (long long)h.slots_sealed * row +
+                         (out->slots_store - (long long)h.slots_sealed + out->slots_ring) * 2 * row;
   out->bytes_dense_equiv = out->tokens_appended * v.Hkv * row;
   out->bytes_reserved = (long long)c->bytes_reserved;
   out->fp8_saturations = (long long)h.saturations;
@@ -322,6 +429,8 @@ fdms_status fdms_cache_read_head(fdms_cache* c, int layer, int seq, int kv_head,
   const int total = len + (n - r);
   if (!pos_host && !keep_host && !k_host && !v_host && !scale_host) return FDMS_OK;
   if (capacity < total) return FDMS_ERR_INVALID_ARG;
+  if (v.blk) return read_head_block(v, hi, n, r, len, pos_host, keep_host, k_host, v_host,
+                                    scale_host);
   const int RB = v.RB;
   uint8_t* kh = static_cast<uint8_t*>(k_host);
   uint8_t* vh = static_cast<uint8_t*>(v_host);

@@ -71,7 +71,10 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
 
-enum : int { kFirst = 1, kLast = 2, kRing = 4, kPending = 8 };
+// tile flags: first / last tile of a head in a warp's list, a ring frame, ring
+// rows that may be pending (keep bit decides), bf16 rows of a per-block FP8
+// cache (the store's partly filled block, staged, or the ring)
+enum : int { kFirst = 1, kLast = 2, kRing = 4, kPending = 8, kBf16 = 16 };
 
 struct TileMeta {
   const uint8_t* ksrc;   // K row of frame row 0 (store: the tile's first row in its
@@ -313,6 +316,85 @@ __device__ __forceinline__ TileMeta tile_meta(const CacheView& c, long long hi, 
   return mt;
 }
 
+// Per-block FP8 cache (FDMS_KV_FP8_E4M3_BLOCK): a head's tiles are its sealed
+// store blocks (E4M3, TR rows of T per tile, each page with its own K and V
+// scale), then the store's partly filled block, staged in bf16 (kind 3), then
+// its ring frames, in bf16 (kind 1); the bf16 tiles use the geometry of T16,
+// the BF16 configuration of the same D and G (TR16 rows of 2 D bytes).
+template <int TR, int TR16>
+__host__ __device__ inline int blk_sealed_tiles(int len) {
+  return len / kBlockSlots * (kBlockSlots / TR);
+}
+template <int TR, int TR16>
+__host__ __device__ inline int blk_head_tiles(int len, int n, int r) {
+  const int staged = len % kBlockSlots, live = n - r;
+  return blk_sealed_tiles<TR, TR16>(len) + (staged + TR16 - 1) / TR16 +
+         (live > 0 ? (live + (r % TR16) + TR16 - 1) / TR16 : 0);
+}
+// Descriptor of bf16 tile idx of a per-block FP8 head: staged rows (kind 3:
+// rows idx * TR16 .. of the partly filled block) or ring frame idx (kind 1).
+template <class T16>
+__device__ __forceinline__ TileMeta tile_meta_b16(const CacheView& c, long long hi, int hidx,
+                                                  int kind, int idx, int len, int n, int r) {
+  constexpr int TR16 = T16::TR, RB16 = T16::RB;
+  TileMeta mt;
+  mt.hidx = hidx;
+  mt.pad = 0;
+  mt.ks = mt.vrel = 1.0f;
+  int row0, row1, flags = kBf16;
+  if (kind == 3) {
+    row0 = 0;
+    row1 = max(0, min(TR16, len % kBlockSlots - idx * TR16));
+    mt.ksrc = stage_k(c, hi) + (long long)idx * TR16 * RB16;
+    mt.p0 = 0;
+  } else {
+    const int f0 = idx * TR16;
+    const int lo = min(max(f0, r), f0 + TR16), hi_p = max(lo, min(f0 + TR16, n));
+    row0 = lo - f0;
+    row1 = hi_p - f0;
+    flags |= kRing | (lo < n - c.W ? kPending : 0);
+    mt.ksrc = ring_k(c, hi) + (long long)(f0 % c.R) * RB16;
+    mt.p0 = f0;
+  }
+  mt.rows = row0 | row1 << 8 | flags << 16;
+  return mt;
+}
+
+// The partial of a head's E4M3 tiles (o8, FP8 accumulator layout: dims
+// 16 i + 2 g + hf) and that of its bf16 tiles (o16, BF16 layout: dims
+// 16 i + 8 hf + g), of the same columns 2t, 2t + 1, merged into o8:
+//     o = 2^(m8 - M) s8 o8 + 2^(m16 - M) o16,  l likewise,  M = max(m8, m16),
+// s8 the V unit of the E4M3 partial. Each o16 value moves to the lane of the
+// FP8 layout that holds its dim (a lane-group shuffle).
+template <int MT>
+__device__ __forceinline__ void merge_kinds(float (&o8)[MT][4], float& m0, float& m1, float& L0,
+                                            float& L1, float s8, const float (&o16)[MT][4],
+                                            float n0, float n1, float K0, float K1, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  const float M0 = fmaxf(m0, n0), M1 = fmaxf(m1, n1);
+  const float a0 = m0 == -INFINITY ? 0.f : fast_exp2(m0 - M0) * s8;
+  const float a1 = m1 == -INFINITY ? 0.f : fast_exp2(m1 - M1) * s8;
+  const float b0 = n0 == -INFINITY ? 0.f : fast_exp2(n0 - M0);
+  const float b1 = n1 == -INFINITY ? 0.f : fast_exp2(n1 - M1);
+#pragma unroll
+  for (int i = 0; i < MT; ++i)
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const int d = 2 * g + hf, src = 4 * (d & 7) + t;   // dim 16 i + d in the BF16 layout
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float x0 = __shfl_sync(0xffffffffu, o16[i][e], src);
+        const float x1 = __shfl_sync(0xffffffffu, o16[i][2 + e], src);
+        const float x = (d >> 3) ? x1 : x0;
+        o8[i][2 * hf + e] = o8[i][2 * hf + e] * (e ? a1 : a0) + x * (e ? b1 : b0);
+      }
+    }
+  L0 = (m0 == -INFINITY ? 0.f : L0 * fast_exp2(m0 - M0)) + K0 * b0;
+  L1 = (m1 == -INFINITY ? 0.f : L1 * fast_exp2(m1 - M1)) + K1 * b1;
+  m0 = M0;
+  m1 = M1;
+}
+
 // ------------------------------------------------------------ a warp's tiles
 // One warp's online softmax over the tiles of one head at a time, and the
 // arithmetic of a tile staged in shared memory (K rows, V rows, the head's q).
@@ -353,6 +435,13 @@ struct WarpTiles {
     qmul0 = qmul1 = 0.f;
     cur_hidx = -1;
     q_raw = false;
+    m0 = m1 = -INFINITY;
+    l0 = l1 = 0.f;
+#pragma unroll
+    for (int i = 0; i < MT; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
+  }
+  // a new head: empty running state
+  __device__ __forceinline__ void reset() {
     m0 = m1 = -INFINITY;
     l0 = l1 = 0.f;
 #pragma unroll
@@ -1168,12 +1257,16 @@ struct PlanWarps {
   static constexpr int value = T::G * T::D >= 1024 ? 4 : (T::G * T::D > 256 ? 5 : 6);
 };
 
-template <class T, int NW>
+template <class T, int NW, bool BLK>
 __global__ void __launch_bounds__(NW * 32, 2)
 k_decode_plan(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
               const uint16_t* __restrict__ q, int n_ranges, double inv_ranges, int use_snap,
               int tok_since) {
   using PL = PlanL<T, NW>;
+  // per-block FP8 (BLK): sealed E4M3 tiles with T, bf16 tiles with T16; no
+  // snapshots (use_snap is 0)
+  using T16 = Dec<T::D, false, T::G>;
+  constexpr int TR16 = T16::TR;
   constexpr int D = T::D, G = T::G, TR = T::TR, SPW = T::SPW, MT = T::MT, NMR = PL::NMR,
                 HALF = PL::HALF, NT = PL::NT;
   constexpr bool FP8 = T::FP8;
@@ -1201,6 +1294,11 @@ k_decode_plan(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   uint64_t* len_bar = full + PL::NSTAGE;   // the lengths now have landed (every thread arrives)
   if (tid == 0) mbar_init(len_bar, NT);
   init_stages<T>(smem, full, PL::NSTAGE, NT, tid, warp, lane);
+  // the copies of a tile (bf16 tiles of a per-block FP8 cache have 2 D-byte rows)
+  auto stg = [&](uint8_t* dst, uint64_t* bar, const TileMeta& mt, int phase) {
+    if (BLK && ((mt.rows >> 16) & kBf16)) stage_tile<T16>(c, dst, bar, mt, phase);
+    else stage_tile<T>(c, dst, bar, mt, phase);
+  };
 
   // warm L2 with this layer's lengths and block tables (read after the wait)
   {
@@ -1228,9 +1326,11 @@ k_decode_plan(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   auto spares = [&](int h) -> int {
     return use_snap ? sp_base + (sn[h] == sr[h] ? 1 : 0) : 0;
   };
-  auto plan_tiles = [&](int h) -> int {
-    return max(1, head_tiles<TR>(sl[h], sn[h], sr[h]) + spares(h));
+  auto htiles = [&](int len, int n, int r) -> int {
+    if constexpr (BLK) return blk_head_tiles<TR, TR16>(len, n, r);
+    else return head_tiles<TR>(len, n, r);
   };
+  auto plan_tiles = [&](int h) -> int { return max(1, htiles(sl[h], sn[h], sr[h]) + spares(h)); };
   // exclusive prefix of the heads' plan tiles (sl, sn, sr filled)
   auto scan = [&]() {
     const int per = (NH + NT - 1) / NT;
@@ -1290,6 +1390,16 @@ k_decode_plan(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   // kind (0 store tile, 1 ring frame, 2 spare) and index of tile lp of head h
   // in the plan; whether it can still grow since the plan's lengths
   auto plan_item = [&](int h, int lp, int& kind, int& idx) -> bool {
+    if constexpr (BLK) {   // sealed tiles, staged tiles (kind 3), ring frames
+      const int n8 = blk_sealed_tiles<TR, TR16>(sl[h]);
+      const int nst = (sl[h] % kBlockSlots + TR16 - 1) / TR16;
+      const int nfr = sn[h] > sr[h] ? (sn[h] - sr[h] + sr[h] % TR16 + TR16 - 1) / TR16 : 0;
+      if (lp < n8) { kind = 0; idx = lp; }
+      else if (lp < n8 + nst) { kind = 3; idx = lp - n8; }
+      else if (lp < n8 + nst + nfr) { kind = 1; idx = sr[h] / TR16 + (lp - n8 - nst); }
+      else { kind = 2; idx = 0; }
+      return true;
+    }
     const int sp = (sl[h] + TR - 1) / TR, nfr = head_tiles<TR>(0, sn[h], sr[h]);
     if (lp < sp) {
       kind = 0;
@@ -1350,7 +1460,7 @@ k_decode_plan(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
         described = true;
         kept = kind == 0 && !grows;
         if (k < SPW && !grows) {
-          stage_tile<T>(c, smem + (warp * SPW + k) * T::STAGE_BYTES, &full[warp * SPW + k], mt,
+          stg(smem + (warp * SPW + k) * T::STAGE_BYTES, &full[warp * SPW + k], mt,
                         1);
           pre_mask |= 1u << k;
         }
@@ -1363,6 +1473,8 @@ k_decode_plan(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   __syncthreads();            // the lengths barrier is set up for every thread
   WarpTiles<T> wt;
   wt.init(lane, c.softmax_scale);
+  WarpTiles<T16> wt16;   // the bf16 tiles of a per-block FP8 head
+  if (BLK) wt16.init(lane, c.softmax_scale);
   // q of the kv head hidx of the call (its first query head's first element)
   auto q_of = [&](int hidx) -> const uint16_t* {
     return q + ((long long)(hidx / c.Hkv) * c.Hq + (long long)(hidx % c.Hkv) * G) * D;
@@ -1377,7 +1489,7 @@ k_decode_plan(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
     wt.fetch_q(q_of(h), h);
   }
   if ((pre_mask >> lane) & 1)
-    stage_tile<T>(c, smem + (warp * SPW + lane) * T::STAGE_BYTES, &full[warp * SPW + lane],
+    stg(smem + (warp * SPW + lane) * T::STAGE_BYTES, &full[warp * SPW + lane],
                   ring[lane], 2);
   // ---- lengths now of every head, and the FP8 head scales the snapshot could
   // not give (heads that held no token then): copied to shared memory in the
@@ -1390,6 +1502,9 @@ k_decode_plan(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
     cp_async4(&cr[h], c.tok_r + hh);
     if (!FP8) {
       if (!use_snap) hsc[2 * h] = hsc[2 * h + 1] = 1.0f;
+    } else if (BLK) {   // the V unit of the E4M3 tiles: the head's first block's V scale
+      hsc[2 * h] = 1.0f;
+      cp_async4(&hsc[2 * h + 1], c.bt_scale + hh * c.max_blocks * 2 + 1);
     } else if (!use_snap || sn[h] == 0) {
       cp_async4(&hsc[2 * h], c.head_scale + hh * 2);
       cp_async4(&hsc[2 * h + 1], c.head_scale + hh * 2 + 1);
@@ -1426,7 +1541,7 @@ k_decode_plan(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
     const int len = cl[h], n = cn[h], r = cr[h];
     TileMeta mt;
     if (!len_ok) kind = 2;
-    if (kind == 2 && len_ok) {   // a spare: the first new store tiles, then the new ring frames
+    if (!BLK && kind == 2 && len_ok) {   // a spare: the first new store tiles, then the new ring frames
       const int sp = (sl[h] + TR - 1) / TR, nfr = head_tiles<TR>(0, sn[h], sr[h]);
       const int E_store = max(0, (len + TR - 1) / TR - sp);
       const int fx = max(nfr > 0 ? sr[h] / TR + nfr : r / TR, r / TR);
@@ -1451,6 +1566,8 @@ k_decode_plan(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
     } else if (kind == 0 && pre) {
       mt = ring[k];
       mt.rows = min(TR, len - idx * TR) << 8;
+    } else if (BLK && kind != 0) {
+      mt = tile_meta_b16<T16>(c, hi0 + h, h, kind, idx, len, n, r);
     } else {
       mt = tile_meta<T>(c, hi0 + h, h, kind, idx, len, n, r, hsc[2 * h], hsc[2 * h + 1]);
     }
@@ -1484,7 +1601,7 @@ k_decode_plan(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   const unsigned first = (nt >= SPW ? (1u << SPW) - 1u : (1u << nt) - 1u) & ~pre_mask;
   ensure(first);
   if ((first >> lane) & 1)
-    stage_tile<T>(c, smem + (warp * SPW + lane) * T::STAGE_BYTES, &full[warp * SPW + lane],
+    stg(smem + (warp * SPW + lane) * T::STAGE_BYTES, &full[warp * SPW + lane],
                   ring[lane], 0);
 
   // ================= tiles of this warp
@@ -1515,8 +1632,19 @@ k_decode_plan(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
       // (only pending ring rows, which a tile described after the wait holds,
       // need the position count now)
       const int thresh = ((tm.rows >> 16) & kPending) ? cn[h] - c.W : 0;
-      if (h != wt.cur_hidx) wt.fetch_q(q_of(h), h);
-      wt.tile(smem + s * T::STAGE_BYTES, tm, thresh, c.ring_keep + (hi0 + h) * c.Rpad, c.R, lane);
+      if (BLK && ((tm.rows >> 16) & kFirst)) {   // a head starts: both running states empty
+        wt.reset();
+        wt16.reset();
+      }
+      if (BLK && ((tm.rows >> 16) & kBf16)) {
+        if (h != wt16.cur_hidx) wt16.fetch_q(q_of(h), h);
+        wt16.tile(smem + s * T::STAGE_BYTES, tm, thresh, c.ring_keep + (hi0 + h) * c.Rpad, c.R,
+                  lane);
+      } else {
+        if (h != wt.cur_hidx) wt.fetch_q(q_of(h), h);
+        wt.tile(smem + s * T::STAGE_BYTES, tm, thresh, c.ring_keep + (hi0 + h) * c.Rpad, c.R,
+                lane);
+      }
       __syncwarp();
       // descriptors come HALF at a time: those of tiles k + HALF + 1 .. k + NMR
       // once tile k + 1 starts a new HALF
@@ -1528,18 +1656,25 @@ k_decode_plan(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
       // the stage is free: refill it with tile k + SPW
       ensure(k + SPW < 32 ? 1u << (k + SPW) : 0u);
       if (lane == 0 && k + SPW < nt)
-        stage_tile<T>(c, smem + s * T::STAGE_BYTES, &full[s], ring[(k + SPW) % NMR], 0);
+        stg(smem + s * T::STAGE_BYTES, &full[s], ring[(k + SPW) % NMR], 0);
     } else if ((tm.rows >> 16) & kFirst) {
-      wt.m0 = wt.m1 = -INFINITY;   // an empty partial for the heads still to come
-      wt.l0 = wt.l1 = 0.f;
+      wt.reset();   // an empty partial for the heads still to come
+      if (BLK) wt16.reset();
     }
 
     // ---- end of this head inside the range
     if (!((tm.rows >> 16) & kLast)) continue;
     float o[MT][4], L0, L1;
     wt.finish(o, L0, L1);
+    float vhead = hsc[2 * h + 1];
+    if constexpr (BLK) {   // the bf16 tiles' partial joins, in the E4M3 layout and V unit 1
+      float o16[MT][4], K0, K1;
+      wt16.finish(o16, K0, K1);
+      merge_kinds<MT>(o, wt.m0, wt.m1, L0, L1, vhead, o16, wt16.m0, wt16.m1, K0, K1, lane);
+      vhead = 1.0f;
+      if (k + 1 < nt) wt16.fetch_q(q_of(h + 1), h + 1);
+    }
     if (k + 1 < nt) wt.fetch_q(q_of(h + 1), h + 1);   // the range's next head
-    const float vhead = hsc[2 * h + 1];
     const int kb = h / c.Hkv, kh = h % c.Hkv;
     if (page_off[h] >= gp0 && page_off[h + 1] <= gp0 + nt) {
       // the whole head lies in this warp's range: write the output now
@@ -1706,24 +1841,42 @@ fdms_status launch_split_t(fdms_cache* cache, const DecodeWork& w_in, OutArgs oa
     if (e != cudaSuccess) cudaGetLastError();   // a refused cluster launch falls back to the plan
   }
   if (e != cudaSuccess) {
-    constexpr int NW = PlanWarps<T>::value;
-    using PL = PlanL<T, NW>;
-    const int use_snap = prev > 0 && writer_done && batch <= cache->decode_batch[layer] &&
-                                 tokens <= kSnapMaxTokens ? 1 : 0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)cache->decode_ctas);
-    cfg.blockDim = dim3(PL::NT);
-    cfg.dynamicSmemBytes = PL::smem_bytes(nh);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const int n_ranges = cache->decode_ctas * NW;
-    e = cudaLaunchKernelEx(&cfg, k_decode_plan<T, NW>, cache->view, w, oa, layer, batch,
-                           static_cast<const uint16_t*>(q), n_ranges, 1.0 / (double)n_ranges,
-                           use_snap, (int)tokens);
+    bool done = false;
+    if constexpr (T::FP8) {
+      if (cache->view.blk) {
+        // per-block FP8: two tile kinds per head, four warps per CTA (registers
+        // for both running states), no snapshots (the staged block changes)
+        constexpr int NWB = 4;
+        using PL = PlanL<T, NWB>;
+        cfg.blockDim = dim3(PL::NT);
+        cfg.dynamicSmemBytes = PL::smem_bytes(nh);
+        const int n_ranges = cache->decode_ctas * NWB;
+        e = cudaLaunchKernelEx(&cfg, k_decode_plan<T, NWB, true>, cache->view, w, oa, layer,
+                               batch, static_cast<const uint16_t*>(q), n_ranges,
+                               1.0 / (double)n_ranges, 0, (int)tokens);
+        done = true;
+      }
+    }
+    if (!done) {
+      constexpr int NW = PlanWarps<T>::value;
+      using PL = PlanL<T, NW>;
+      const int use_snap = prev > 0 && writer_done && batch <= cache->decode_batch[layer] &&
+                                   tokens <= kSnapMaxTokens ? 1 : 0;
+      cfg.blockDim = dim3(PL::NT);
+      cfg.dynamicSmemBytes = PL::smem_bytes(nh);
+      const int n_ranges = cache->decode_ctas * NW;
+      e = cudaLaunchKernelEx(&cfg, k_decode_plan<T, NW, false>, cache->view, w, oa, layer, batch,
+                             static_cast<const uint16_t*>(q), n_ranges, 1.0 / (double)n_ranges,
+                             use_snap, (int)tokens);
+    }
   }
   if (e != cudaSuccess) return FDMS_ERR_CUDA;
   const long long n = fdms_log_launch(cache, true);   // every decode kernel waits first
@@ -1762,14 +1915,23 @@ fdms_status setup_t(fdms_cache* cache) {
   const int nh = cache->view.Bmax * cache->view.Hkv;
   const size_t smem = PL::smem_bytes(nh);
   if (smem > 227 * 1024) return FDMS_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(k_decode_plan<T, NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(k_decode_plan<T, NW, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return FDMS_ERR_UNSUPPORTED;
+  if constexpr (T::FP8) {
+    if (cache->view.blk) {   // the per-block FP8 variant (four warps)
+      const size_t smem_b = PlanL<T, 4>::smem_bytes(nh);
+      if (smem_b > 227 * 1024 ||
+          cudaFuncSetAttribute(k_decode_plan<T, 4, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b) != cudaSuccess)
+        return FDMS_ERR_UNSUPPORTED;
+    }
+  }
   // CTAs of the plan kernel resident per SM at the largest call (its merging
   // warps wait for the other parts of their head, so every CTA of a call must
   // be able to be resident at once)
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_decode_plan<T, NW>, PL::NT, smem) !=
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_decode_plan<T, NW, false>, PL::NT, smem) !=
           cudaSuccess ||
       per_sm < 1)
     return FDMS_ERR_UNSUPPORTED;
@@ -1781,7 +1943,9 @@ fdms_status setup_t(fdms_cache* cache) {
   cache->max_clusters[1] = max_active_clusters<T, 2>();
   cache->max_clusters[2] = max_active_clusters<T, 4>();
   cache->max_clusters[3] = max_active_clusters<T, 8>();
-  cache->cluster_ok = T::smem_bytes_cluster() <= 227 * 1024 && cache->max_clusters[3] > 0;
+  // (a per-block FP8 cache decodes in the global plan only)
+  cache->cluster_ok = !cache->view.blk && T::smem_bytes_cluster() <= 227 * 1024 &&
+                      cache->max_clusters[3] > 0;
   cudaGetLastError();   // a refused query only turns the cluster mode off
   return FDMS_OK;
 }

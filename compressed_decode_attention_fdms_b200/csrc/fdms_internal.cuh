@@ -21,7 +21,7 @@ struct DevCounters {
   unsigned long long slots_decoded;    // cumulative units scanned by decode calls
   unsigned long long decode_calls;
   // stats scratch (filled by the stats kernel)
-  unsigned long long tokens, slots_store, slots_ring;
+  unsigned long long tokens, slots_store, slots_ring, slots_sealed;
 };
 
 // Everything a kernel needs to find a head's data. Passed by value.
@@ -34,6 +34,9 @@ struct DevCounters {
 //              (position p lives in slot p % R; R is a multiple of 64)
 //   ring_keep: hi * Rpad bytes
 //   head_scale[hi * 2 + {0,1}]         FP8 scale of K / V
+//   per-block FP8 (blk): stage: hi * 2 * 64 * 2D bytes, bf16 K rows [64][2D]
+//              then V rows, the store's partly filled block; stage_pos[hi * 64
+//              + row] their positions; ring rows are bf16 too (RBR = 2D)
 // Pool block b: K rows [64][RB] at pool + b * 2 * 64 * RB, V rows right after;
 //   blk_pos[b * 64 + row] is the token position of each slot.
 struct CacheView {
@@ -48,9 +51,13 @@ struct CacheView {
   uint8_t* ring_keep;
   float* head_scale;
   DevCounters* ctr;
+  uint8_t* stage;         // per-block FP8 only
+  int32_t* stage_pos;     // per-block FP8 only
   long long num_blocks;
   int L, Bmax, Hq, Hkv, G, D, RB, W, P, R, Rpad, max_blocks, max_seq_len;
+  int RBR;                // bytes of a ring row (RB, or 2 D for per-block FP8)
   int fp8;
+  int blk;                // per-block FP8 scales (FDMS_KV_FP8_E4M3_BLOCK)
   float softmax_scale;
 };
 
@@ -84,10 +91,16 @@ __host__ __device__ inline uint8_t* block_v(const CacheView& c, long long blk) {
   return block_k(c, blk) + (long long)kBlockSlots * c.RB;
 }
 __host__ __device__ inline uint8_t* ring_k(const CacheView& c, long long hi) {
-  return c.ring + hi * 2LL * c.R * c.RB;
+  return c.ring + hi * 2LL * c.R * c.RBR;
 }
 __host__ __device__ inline uint8_t* ring_v(const CacheView& c, long long hi) {
-  return ring_k(c, hi) + (long long)c.R * c.RB;
+  return ring_k(c, hi) + (long long)c.R * c.RBR;
+}
+__host__ __device__ inline uint8_t* stage_k(const CacheView& c, long long hi) {
+  return c.stage + hi * 2LL * kBlockSlots * (2 * c.D);
+}
+__host__ __device__ inline uint8_t* stage_v(const CacheView& c, long long hi) {
+  return stage_k(c, hi) + (long long)kBlockSlots * (2 * c.D);
 }
 
 // Decode workspace: the split partials (warp v's partial of head h at v + h).

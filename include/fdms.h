@@ -94,7 +94,14 @@ typedef enum {
                                  max_seq_len, a bounded wait that ran out) */
 } fdms_status;
 
-typedef enum { FDMS_KV_BF16 = 0, FDMS_KV_FP8_E4M3 = 1 } fdms_kv_dtype;
+/* FDMS_KV_FP8_E4M3_BLOCK: E4M3 with one (K, V) scale pair per 64-slot store
+ * block, from that block's own maxima (max(amax, 2^-126) / 448), fixed when the
+ * block's 64th survivor arrives ("sealing"). Until then the store's partly
+ * filled block stays bf16 in a per-head staging block, and the ring holds bf16
+ * rows. Decode reads the sealed blocks as E4M3 with their own scales and the
+ * staged block and the ring as bf16; it always runs the global plan (four
+ * warps per CTA, no per-head clusters). */
+typedef enum { FDMS_KV_BF16 = 0, FDMS_KV_FP8_E4M3 = 1, FDMS_KV_FP8_E4M3_BLOCK = 2 } fdms_kv_dtype;
 
 typedef struct {
   int num_layers;        /* L >= 1 */
@@ -166,7 +173,7 @@ fdms_status fdms_cache_destroy(fdms_cache* cache);
  *   kv_scale_dev  FP8 only, optional: float [batch][Hkv][2] (K, V scales) used
  *                 for sequences that receive their first tokens in this call;
  *                 NULL = max(amax, 2^-126) / 448 of this call's values per head.
- *                 Must be NULL for a BF16 cache.
+ *                 Must be NULL for a BF16 or per-block FP8 cache.
  * A sequence that would exceed max_seq_len is left unchanged and latches DEVICE.
  * A head whose survivors do not fit in the pool is left unchanged and latches
  * OUT_OF_BLOCKS. */
@@ -241,8 +248,11 @@ fdms_status fdms_cache_stats(fdms_cache* cache, fdms_stats* host_out, void* stre
  *   pos_host     int32 [capacity]: token positions.
  *   keep_host    uint8 [capacity]: keep bits (1 for store entries).
  *   k_host/v_host  [capacity][D * element bytes]: stored payload (bf16 or E4M3).
+ *                FDMS_KV_FP8_E4M3_BLOCK: [capacity][2 D] bytes; a sealed entry
+ *                holds its D E4M3 codes in the first D bytes (the rest zero), a
+ *                staged or ring entry its D bf16 values.
  *   scale_host   float [capacity][2]: (K, V) scale applied to each entry
- *                (1.0 for BF16).
+ *                (1.0 for BF16; 0 for the bf16 entries of FDMS_KV_FP8_E4M3_BLOCK).
  *   info_host    counts, always filled.
  * Any pointer but info_host may be NULL to skip it. */
 fdms_status fdms_cache_read_head(fdms_cache* cache, int layer, int seq, int kv_head,
