@@ -212,6 +212,18 @@ def to_bits(t: torch.Tensor) -> np.ndarray:
     return t.contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
+def oracle_decode_bytes(oc, wl, b, row):
+    """K/V bytes a decode of sequence b of the oracle cache's layer 0 reads:
+    store and ring slots, one K row and one V row each (per-block FP8: sealed
+    slots in E4M3, the staged and ring slots in bf16, twice the row)."""
+    r, n = int(oc.r[0, b]), int(oc.n[0, b])
+    lens = np.count_nonzero(oc.keep[0, b, :r], axis=0)          # [Hkv]
+    if wl.kv_dtype != "fp8_e4m3_block":
+        return int(np.sum(lens) + (n - r) * wl.kv_heads) * row
+    sealed = lens // 64 * 64
+    return int(np.sum(sealed) * row + (np.sum(lens - sealed) + (n - r) * wl.kv_heads) * 2 * row)
+
+
 def oracle_sample(wl, budget_s: float, min_steps=1, max_steps=None, warmup=0):
     """Time the fp64 oracle on one layer of the workload, all sequences.
 
@@ -227,7 +239,7 @@ def oracle_sample(wl, budget_s: float, min_steps=1, max_steps=None, warmup=0):
     oc = OracleCache(1, wl.batch, wl.q_heads, wl.kv_heads, wl.head_dim, wl.window, wl.period,
                      wl.kv_dtype, capacity=int(ctx.max()) + n_steps + warmup + 1)
     pre = wk.prefill_inputs(wl, layer)
-    elt = 1 if wl.kv_dtype == "fp8_e4m3" else 2
+    elt = 1 if wl.kv_dtype.startswith("fp8") else 2
     row = 2 * wl.head_dim * elt
     times, bytes_ = [], 0
     with threadpool_limits(limits=1):
@@ -245,11 +257,7 @@ def oracle_sample(wl, budget_s: float, min_steps=1, max_steps=None, warmup=0):
             dt = time.perf_counter() - t0
             if step < warmup:
                 continue
-            units = int(np.sum((oc.n - oc.r)) * wl.kv_heads)
-            for b in range(wl.batch):
-                r = int(oc.r[0, b])
-                units += int(np.count_nonzero(oc.keep[0, b, :r]))
-            bytes_ += units * row
+            bytes_ += sum(oracle_decode_bytes(oc, wl, b, row) for b in range(wl.batch))
             times.append(dt)
             total_t += dt
             if len(times) >= min_steps and total_t >= budget_s:
@@ -271,7 +279,7 @@ def oracle_seq_worker(job):
     torch.set_num_threads(1)
     wl = wk.get(name)
     ctx = wk.context_lengths(wl)
-    elt = 1 if wl.kv_dtype == "fp8_e4m3" else 2
+    elt = 1 if wl.kv_dtype.startswith("fp8") else 2
     row = 2 * wl.head_dim * elt
     with threadpool_limits(limits=1):
         ocs = {}
@@ -296,9 +304,7 @@ def oracle_seq_worker(job):
             done += 1
             for b in seqs:
                 oc = ocs[b]
-                units = int(oc.n[0, 0] - oc.r[0, 0]) * wl.kv_heads
-                units += int(np.count_nonzero(oc.keep[0, 0, :int(oc.r[0, 0])]))
-                nbytes += units * row
+                nbytes += oracle_decode_bytes(oc, wl, 0, row)
             if total >= budget_s:
                 break
     return nbytes, total, done
@@ -350,7 +356,7 @@ def pool_blocks(wl, steps_total):
     """Blocks for the pool: worst case when it fits in 40 GB, else a bound
     from the keep rates with a 6-sigma margin per head."""
     ctx = wk.context_lengths(wl)
-    elt = 1 if wl.kv_dtype == "fp8_e4m3" else 2
+    elt = 1 if wl.kv_dtype.startswith("fp8") else 2
     block_bytes = 2 * 64 * wl.head_dim * elt
     n = ctx[None, :, None] + steps_total
     worst = int(np.sum(np.ceil(np.broadcast_to(n, (wl.layers, wl.batch, wl.kv_heads)) / 64)))
@@ -373,7 +379,7 @@ def measure(fd, args, wl, dev, local, world, K, W, KE, WE):
     stream = torch.cuda.Stream(dev)
     cache = fd.fdms_cache_create(cfg, local, stream)
     L, B = wl.layers, wl.batch
-    elt = 1 if wl.kv_dtype == "fp8_e4m3" else 2
+    elt = 1 if wl.kv_dtype.startswith("fp8") else 2
     row = 2 * wl.head_dim * elt
     qo_bytes = 2 * B * wl.q_heads * wl.head_dim * 2      # q read + out written, bf16
 
@@ -478,17 +484,16 @@ def measure(fd, args, wl, dev, local, world, K, W, KE, WE):
         st_b = fd.fdms_cache_stats(cache, stream)
         if st_b["error"]:
             raise RuntimeError(f"device error latched: {fd.status_string(st_b['error'])}")
-        return (a.elapsed_time(b), st_b["slots_decoded"] - st_a["slots_decoded"],
+        return (a.elapsed_time(b), st_b["bytes_decoded"] - st_a["bytes_decoded"],
                 st_b["decode_calls"] - st_a["decode_calls"])
 
     with ClockSampler(local) as clk:
-        elapsed_ms, slots, calls = timed(graph)
+        elapsed_ms, kv_bytes, calls = timed(graph)
     assert calls == K * L, (calls, K * L)
-    kv_bytes = slots * row
-    dec_ms_total, dec_slots, dec_calls = timed(graph_dec)
+    dec_ms_total, dec_bytes, dec_calls = timed(graph_dec)
     assert dec_calls == K * L
     dec_avg_ms = dec_ms_total / dec_calls
-    per_launch_bytes = dec_slots * row / dec_calls + qo_bytes
+    per_launch_bytes = dec_bytes / dec_calls + qo_bytes
 
     # whole-job numbers: max time over ranks, bytes summed over ranks
     t_max, bytes_all = over_ranks(elapsed_ms, kv_bytes, world, dev)
@@ -682,7 +687,7 @@ def run_e2e(fd, cache, wl, stream, dev, s0, warm, steps, row):
         t1.record(stream)
     torch.cuda.synchronize()
     st1 = fd.fdms_cache_stats(cache, stream)
-    return {"ms": t0.elapsed_time(t1), "bytes": (st1["slots_decoded"] - st0["slots_decoded"]) * row,
+    return {"ms": t0.elapsed_time(t1), "bytes": st1["bytes_decoded"] - st0["bytes_decoded"],
             "h2d": step_bytes, "d2h": dout.numel() * dout.element_size()}
 
 

@@ -57,7 +57,8 @@ class fdms_stats(ctypes.Structure):
         ("blocks_free", ctypes.c_longlong), ("bytes_compact", ctypes.c_longlong),
         ("bytes_dense_equiv", ctypes.c_longlong), ("bytes_reserved", ctypes.c_longlong),
         ("fp8_saturations", ctypes.c_longlong), ("slots_decoded", ctypes.c_longlong),
-        ("decode_calls", ctypes.c_longlong), ("error", ctypes.c_int),
+        ("decode_calls", ctypes.c_longlong), ("bytes_decoded", ctypes.c_longlong),
+        ("error", ctypes.c_int),
     ]
 
     def as_dict(self):

@@ -400,6 +400,7 @@ fdms_status fdms_cache_stats(fdms_cache* c, fdms_stats* out, void* stream) {
   out->fp8_saturations = (long long)h.saturations;
   out->slots_decoded = (long long)h.slots_decoded;
   out->decode_calls = (long long)h.decode_calls;
+  out->bytes_decoded = (long long)h.bytes_decoded;
   out->error = h.error;
   return FDMS_OK;
 }

@@ -194,12 +194,6 @@ __device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
   return v;
 }
-__device__ __forceinline__ int4 ld_dsmem_v4(uint32_t addr) {
-  int4 v;
-  asm volatile("ld.shared::cluster.v4.s32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr) : "memory");
-  return v;
-}
 
 // ------------------------------------------------------------- MMA helpers
 template <bool F16>
@@ -789,9 +783,8 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   const int hsel = (int)(blockIdx.x / CS), crank = (int)(blockIdx.x % CS);
   const int v = crank * NCW + warp;
   const long long hi = hi0 + hsel;
-  // cst: [0..3] rank 0's copy of the snapshot, [4..5] rank 0's copy of the
-  // FP8 head scales, [8..10] snapshot planned on, [12..14] lengths now,
-  // [16..17] FP8 head scales (K, V)
+  // cst: [8..10] the lengths the plan is made on (snapshot, or now), [12..14]
+  // the lengths now, floats [16..17] FP8 head scales (K, V)
   int* cst = reinterpret_cast<int*>(smem + T::OFF_HEADS);
   float* hs = reinterpret_cast<float*>(cst) + 16;
   float* mslot = reinterpret_cast<float*>(smem + T::OFF_MERGE);
@@ -832,28 +825,20 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   }
   if (use_snap) {
     // ---- before the wait: the snapshot and the head scales (fixed once the
-    // head holds a token), one copy for the whole cluster
-    if (crank == 0 && tid == 0) {
+    // head holds a token). Every CTA of the cluster reads the same copy: this
+    // call writes the other one
+    if (tid == 0) {
       int4 sv = w.snap_rd[hi];
       const float2 sc = FP8 ? *reinterpret_cast<const float2*>(c.head_scale + hi * 2)
                             : make_float2(1.f, 1.f);
       if (!(sv.x >= 0 && sv.x <= sv.z && sv.z <= sv.y && sv.y <= c.max_seq_len &&
             sv.y - sv.z <= c.R))
         sv = make_int4(0, 0, 0, 0);
-      *reinterpret_cast<int4*>(cst) = sv;
-      reinterpret_cast<float*>(cst)[4] = sc.x;
-      reinterpret_cast<float*>(cst)[5] = sc.y;
-    }
-    cluster_sync_all();
-    if (tid == 0) {
-      const uint32_t r0 = cluster_addr(cst, 0);
-      const int4 sv = ld_dsmem_v4(r0);
-      const float sk = ld_dsmem_f32(r0 + 16), svs = ld_dsmem_f32(r0 + 20);
       cst[8] = sv.x;
       cst[9] = sv.y;
       cst[10] = sv.z;
-      hs[0] = sk;
-      hs[1] = svs;
+      hs[0] = sc.x;
+      hs[1] = sc.y;
     }
     __syncthreads();
     const int len_s = cst[8], n_s = cst[9], r_s = cst[10];
@@ -899,6 +884,7 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
     if (crank == 0) {
       w.snap_wr[hi] = make_int4(len, n, r, 0);
       atomicAdd(&c.ctr->slots_decoded, (unsigned long long)(len + (n - r)));
+      atomicAdd(&c.ctr->bytes_decoded, head_kv_bytes(c, len, n, r));
       if (blockIdx.x == 0) atomicAdd(&c.ctr->decode_calls, 1ull);
     }
   }
@@ -1761,10 +1747,17 @@ k_decode_plan(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
     const int h0 = (int)blockIdx.x * per, h1 = min(NH, h0 + per);
     for (int h = h0 + tid; h < h1; h += NT) w.snap_wr[hi0 + h] = make_int4(cl[h], cn[h], cr[h], 0);
     if (blockIdx.x == 0) {
-      unsigned long long slots = 0;
-      for (int h = tid; h < NH; h += NT) slots += (unsigned long long)(cl[h] + (cn[h] - cr[h]));
-      for (int off = 16; off > 0; off >>= 1) slots += __shfl_xor_sync(0xffffffffu, slots, off);
+      unsigned long long slots = 0, bytes = 0;
+      for (int h = tid; h < NH; h += NT) {
+        slots += (unsigned long long)(cl[h] + (cn[h] - cr[h]));
+        bytes += head_kv_bytes(c, cl[h], cn[h], cr[h]);
+      }
+      for (int off = 16; off > 0; off >>= 1) {
+        slots += __shfl_xor_sync(0xffffffffu, slots, off);
+        bytes += __shfl_xor_sync(0xffffffffu, bytes, off);
+      }
       if (lane == 0 && slots) atomicAdd(&c.ctr->slots_decoded, slots);
+      if (lane == 0 && bytes) atomicAdd(&c.ctr->bytes_decoded, bytes);
       if (tid == 0) atomicAdd(&c.ctr->decode_calls, 1ull);
     }
   }

@@ -20,6 +20,7 @@ struct DevCounters {
   int pad;
   unsigned long long slots_decoded;    // cumulative units scanned by decode calls
   unsigned long long decode_calls;
+  unsigned long long bytes_decoded;    // cumulative K/V bytes those units hold
   // stats scratch (filled by the stats kernel)
   unsigned long long tokens, slots_store, slots_ring, slots_sealed;
 };
@@ -127,6 +128,16 @@ struct AppendWork {
   unsigned* amax;         // [heads][2]: bits of max |x| over the call's K / V (FP8)
   int max_chunks;
 };
+
+// K/V bytes a decode call reads for a head of store length len and ring
+// positions [r, n): one K row and one V row per slot, of D elements (per-block
+// FP8: the sealed blocks' rows in E4M3, the staged block's and the ring's in bf16)
+__device__ inline unsigned long long head_kv_bytes(const CacheView& c, int len, int n, int r) {
+  const unsigned long long row = 2ull * c.RB;
+  if (!c.blk) return (unsigned long long)(len + (n - r)) * row;
+  const int sealed = len / kBlockSlots * kBlockSlots;
+  return (unsigned long long)sealed * row + (unsigned long long)(len - sealed + (n - r)) * 2 * row;
+}
 
 __device__ inline void latch_error(DevCounters* ctr, int code) {
   atomicCAS(&ctr->error, 0, code);

@@ -140,6 +140,8 @@ typedef struct {
   long long slots_decoded;     /* cumulative slots (K row + V row each) read by
                                   decode calls: store slots plus ring slots */
   long long decode_calls;      /* decode calls so far */
+  long long bytes_decoded;     /* cumulative K/V bytes of those slots (per-block FP8:
+                                  sealed slots in E4M3, the others in bf16) */
   int error;                   /* sticky device error (an fdms_status), 0 if none */
 } fdms_stats;
 

@@ -95,6 +95,12 @@ WORKLOADS = {
                               head_dim=128, kv_dtype="fp8_e4m3", window=256, period=1,
                               steps=128, ctx=8192, rate_range=(0.06, 0.20),
                               seed=0xFD45 + 3),
+    # the Qwen3-8B c=8 FP8 workload with the per-block FP8 scale reading (each sealed
+    # 64-slot block's own maxima; the staged block and the ring in bf16)
+    "qwen8b_c8_fp8_block": Workload("qwen8b_c8_fp8_block", batch=8, layers=36, q_heads=32,
+                                    kv_heads=8, head_dim=128, kv_dtype="fp8_e4m3_block",
+                                    window=256, period=1, steps=128, ctx=8192,
+                                    rate_range=(0.06, 0.20), seed=0xFD45 + 3),
     "qwen8b_long_fp8": Workload("qwen8b_long_fp8", batch=32, layers=36, q_heads=32,
                                 kv_heads=8, head_dim=128, kv_dtype="fp8_e4m3", window=256,
                                 period=64, steps=256, ctx_range=(1024, 32768),
