@@ -122,8 +122,10 @@ struct Dec {
   // and one for the CTA
   static constexpr int SLOT = G * D + 2 * G;   // floats
   static constexpr int OFF_MERGE = OFF_HEADS + 128;
-  static size_t smem_bytes_cluster() {
-    return 128 + OFF_MERGE + (size_t)(NCW + 1) * SLOT * 4 + 64;
+  // then the head's block-table row (and FP8 scale pairs), max_blocks entries
+  static constexpr int OFF_BT = (OFF_MERGE + (NCW + 1) * SLOT * 4 + 15) / 16 * 16;
+  static size_t smem_bytes_cluster(int max_blocks) {
+    return 128 + OFF_BT + (size_t)max_blocks * 4 * (FP8 ? 3 : 1) + 64;
   }
   // head dim of P.V accumulator row block i, lane group g, upper half hi:
   // BF16 V^T comes from transposed 8x8 matrix loads (dims in order), FP8 V^T
@@ -274,8 +276,14 @@ __device__ __forceinline__ uint32_t pick16(int role, uint32_t head, uint32_t rem
 template <class T>
 __device__ __forceinline__ TileMeta tile_meta(const CacheView& c, long long hi, int hidx,
                                               int kind, int idx, int len, int n, int r,
-                                              float hs_k, float hs_v) {
+                                              float hs_k, float hs_v,
+                                              const int32_t* bt_row = nullptr,
+                                              const float* bs_row = nullptr) {
   constexpr int TR = T::TR, RB = T::RB;
+  // the head's block-table row and (K, V) scale pairs: given (a copy in shared
+  // memory), or in global memory
+  if (!bt_row) bt_row = c.block_table + hi * c.max_blocks;
+  if (!bs_row) bs_row = c.bt_scale + hi * c.max_blocks * 2;
   TileMeta mt;
   mt.hidx = hidx;
   mt.pad = 0;
@@ -284,10 +292,10 @@ __device__ __forceinline__ TileMeta tile_meta(const CacheView& c, long long hi, 
     const int j = idx * TR / kBlockSlots;
     row0 = 0;
     row1 = min(TR, len - idx * TR);
-    const long long blk = c.block_table[hi * c.max_blocks + j];
+    const long long blk = bt_row[j];
     if (T::FP8) {
-      mt.ks = c.bt_scale[(hi * c.max_blocks + j) * 2];
-      mt.vrel = c.bt_scale[(hi * c.max_blocks + j) * 2 + 1] / hs_v;
+      mt.ks = bs_row[2 * j];
+      mt.vrel = bs_row[2 * j + 1] / hs_v;
     } else {
       mt.ks = mt.vrel = 1.0f;
     }
@@ -788,6 +796,22 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   int* cst = reinterpret_cast<int*>(smem + T::OFF_HEADS);
   float* hs = reinterpret_cast<float*>(cst) + 16;
   float* mslot = reinterpret_cast<float*>(smem + T::OFF_MERGE);
+  // the head's block-table row and scale pairs, copied to shared memory in the
+  // background from the start; entries of blocks the snapshot already held are
+  // final (the store is append-only), later ones are read again after the wait
+  int32_t* s_bt = reinterpret_cast<int32_t*>(smem + T::OFF_BT);
+  float* s_bs = reinterpret_cast<float*>(s_bt + c.max_blocks);
+  {
+    const int32_t* gbt = c.block_table + hi * c.max_blocks;
+    const float* gbs = c.bt_scale + hi * c.max_blocks * 2;
+    for (int j = tid; j < c.max_blocks; j += T::NT) {
+      cp_async4(&s_bt[j], gbt + j);
+      if (FP8) {
+        cp_async4(&s_bs[2 * j], gbs + 2 * j);
+        cp_async4(&s_bs[2 * j + 1], gbs + 2 * j + 1);
+      }
+    }
+  }
   int sp_s = 0, f0_s = 0, a_first = 0, cnt = 0, e0 = 0, E_store = 0, fx0 = 0, nt = 0;
   unsigned pre_mask = 0;
   // warp v's snapshot tiles: a run of the head's tiles, runs differing by at
@@ -840,6 +864,7 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
       hs[0] = sc.x;
       hs[1] = sc.y;
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");   // this thread's block-table copies
     __syncthreads();
     const int len_s = cst[8], n_s = cst[9], r_s = cst[10];
     split(len_s, n_s, r_s);
@@ -848,7 +873,8 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
     if (lane < SPW && lane < cnt) {
       int kind, idx;
       if (!snap_item(lane, kind, idx)) {
-        TileMeta mt = tile_meta<T>(c, hi, hsel, kind, idx, len_s, n_s, r_s, hs[0], hs[1]);
+        TileMeta mt =
+            tile_meta<T>(c, hi, hsel, kind, idx, len_s, n_s, r_s, hs[0], hs[1], s_bt, s_bs);
         mt.rows |= (lane == 0 ? kFirst : 0) << 16;
         ring[lane] = mt;
         stage_tile<T>(c, smem + (warp * SPW + lane) * T::STAGE_BYTES, &full[warp * SPW + lane],
@@ -890,6 +916,23 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   }
   __syncthreads();
   {
+    // block-table entries the copy may have missed: every one without a
+    // snapshot, else those of blocks added since
+    const int nb_ok = use_snap ? (cst[8] + kBlockSlots - 1) / kBlockSlots : 0;
+    const int nb_now = (cst[12] + kBlockSlots - 1) / kBlockSlots;
+    if (!use_snap) asm volatile("cp.async.wait_all;" ::: "memory");
+    if (nb_now > nb_ok) {
+      for (int j = nb_ok + tid; j < nb_now; j += T::NT) {
+        s_bt[j] = c.block_table[hi * c.max_blocks + j];
+        if (FP8) {
+          s_bs[2 * j] = c.bt_scale[(hi * c.max_blocks + j) * 2];
+          s_bs[2 * j + 1] = c.bt_scale[(hi * c.max_blocks + j) * 2 + 1];
+        }
+      }
+    }
+    __syncthreads();
+  }
+  {
     const int len_s = cst[8], n_s = cst[9], r_s = cst[10];
     const int len = cst[12], n = cst[13], r = cst[14];
     if (!use_snap) split(len_s, n_s, r_s);
@@ -921,7 +964,7 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
       kind = e < E_store ? 0 : 1;
       idx = kind == 0 ? sp_s + e : fx0 + (e - E_store);
     }
-    TileMeta mt = tile_meta<T>(c, hi, hsel, kind, idx, len, n, r, hs[0], hs[1]);
+    TileMeta mt = tile_meta<T>(c, hi, hsel, kind, idx, len, n, r, hs[0], hs[1], s_bt, s_bs);
     mt.rows |= ((k == 0 ? kFirst : 0) | (k == nt - 1 ? kLast : 0)) << 16;
     return mt;
   };
@@ -1789,7 +1832,7 @@ cudaError_t launch_cluster_t(fdms_cache* cache, const DecodeWork& w, OutArgs oa,
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(nh * CS));
   cfg.blockDim = dim3(T::NT);
-  cfg.dynamicSmemBytes = T::smem_bytes_cluster();
+  cfg.dynamicSmemBytes = T::smem_bytes_cluster(cache->view.max_blocks);
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1881,11 +1924,11 @@ fdms_status launch_split_t(fdms_cache* cache, const DecodeWork& w_in, OutArgs oa
 }
 
 template <class T, int CS>
-int max_active_clusters() {
+int max_active_clusters(const fdms_cache* cache) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(CS * 64));
   cfg.blockDim = dim3(T::NT);
-  cfg.dynamicSmemBytes = T::smem_bytes_cluster();
+  cfg.dynamicSmemBytes = T::smem_bytes_cluster(cache->view.max_blocks);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = CS;
@@ -1895,7 +1938,7 @@ int max_active_clusters() {
   cfg.numAttrs = 1;
   int n = 0;
   if (cudaFuncSetAttribute(k_decode_split<T, CS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)T::smem_bytes_cluster()) != cudaSuccess ||
+                           (int)T::smem_bytes_cluster(cache->view.max_blocks)) != cudaSuccess ||
       cudaOccupancyMaxActiveClusters(&n, k_decode_split<T, CS>, &cfg) != cudaSuccess)
     n = 0;
   return n;
@@ -1933,11 +1976,11 @@ fdms_status setup_t(fdms_cache* cache) {
   cache->ranges_per_cta = NW;
   // per-head cluster mode: how many clusters of each size fit at once
   cache->max_clusters[0] = 0;
-  cache->max_clusters[1] = max_active_clusters<T, 2>();
-  cache->max_clusters[2] = max_active_clusters<T, 4>();
-  cache->max_clusters[3] = max_active_clusters<T, 8>();
+  cache->max_clusters[1] = max_active_clusters<T, 2>(cache);
+  cache->max_clusters[2] = max_active_clusters<T, 4>(cache);
+  cache->max_clusters[3] = max_active_clusters<T, 8>(cache);
   // (a per-block FP8 cache decodes in the global plan only)
-  cache->cluster_ok = !cache->view.blk && T::smem_bytes_cluster() <= 227 * 1024 &&
+  cache->cluster_ok = !cache->view.blk && T::smem_bytes_cluster(cache->view.max_blocks) <= 227 * 1024 &&
                       cache->max_clusters[3] > 0;
   cudaGetLastError();   // a refused query only turns the cluster mode off
   return FDMS_OK;
