@@ -103,7 +103,7 @@ SMALL = {
 
 # Decode modes: "auto" (decode_ctas = 0) runs these few-head calls as one
 # cluster of CTAs per head; "plan" (an explicit grid) forces the global tile
-# plan with the combine kernel, which calls with many heads use.
+# plan, which calls with many heads use.
 MODES = {"auto": 0, "plan": 148}
 
 
@@ -422,6 +422,73 @@ def test_step_appends_back_to_back(kv_dtype, window, period):
             p.check_heads(layer)
             q = wk.decode_query(wl, layer, 99)
             assert _max_err(p.decode(layer, q), p.oracle_out(layer, q)) <= tol
+        p.check_stats()
+    finally:
+        p.close()
+
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "fp8_e4m3"])
+@pytest.mark.parametrize("mode", list(MODES))
+def test_snapshot_rules(mode, kv_dtype):
+    """Decode plans from the lengths the previous decode of the layer saw (a
+    snapshot) and adds what was appended since. Cases that bend the rules: a
+    smaller then a larger batch than the previous decode, many tokens appended
+    in between (beyond the global plan's spare tiles), two decodes with no
+    append in between, a decode after appends to other layers only, and
+    sequences growing unevenly; every output against the oracle."""
+    wl = wk.scaled(wk.get("llama1b_c8"), layers=2, batch=6, ctx=350, steps=0, kv_dtype=kv_dtype,
+                   head_dim=128 if kv_dtype == "fp8_e4m3" else 64)
+    p = Pair(wl, decode_ctas=MODES[mode], max_seq_len=800)
+    tol = TOL_BF16 if kv_dtype == "bf16" else TOL_FP8_MIRROR
+    g = torch.Generator().manual_seed(11)
+    step = [0]
+
+    def q_of(batch):
+        return torch.randn((batch, wl.q_heads, wl.head_dim), generator=g).to(torch.bfloat16)
+
+    def decode(layer, batch):
+        q = q_of(batch)
+        out = p.decode(layer, q)
+        ref = p.oracle_out(layer, q)
+        assert _max_err(out, ref) <= tol, (layer, batch)
+
+    def append(layer, n_per_seq):
+        base = wk.scaled(wl, ctx=max(n_per_seq), steps=0)
+        inp = wk.prefill_inputs(base, layer)
+        inp = {**inp, "n_new": torch.tensor(n_per_seq, dtype=torch.int32),
+               "max_new": max(n_per_seq)}
+        # fresh values per call: shift the generator's stream by the step
+        step[0] += 1
+        k = inp["k"].float().roll(step[0], dims=1).to(torch.bfloat16)
+        v = inp["v"].float().roll(-step[0], dims=1).to(torch.bfloat16)
+        p.append(layer, {**inp, "k": k, "v": v})
+
+    try:
+        for layer in range(wl.layers):
+            p.append(layer, wk.prefill_inputs(wl, layer))
+        B = wl.batch
+        for layer in range(wl.layers):
+            decode(layer, B)                      # first decode: no snapshot yet
+        for layer in range(wl.layers):
+            append(layer, [1] * B)
+            decode(layer, B // 2)                 # fewer sequences than the snapshot's call
+        for layer in range(wl.layers):
+            append(layer, [1] * B)
+            decode(layer, B)                      # more sequences than the last decode's
+        for layer in range(wl.layers):
+            append(layer, [100] * B)              # beyond the spare tiles
+            decode(layer, B)
+        decode(0, B)                              # nothing appended since
+        decode(0, B)
+        append(1, [3] * B)                        # another layer only
+        decode(0, B)
+        for layer in range(wl.layers):
+            append(layer, [1, 2, 0, 5, 1, 64][:B])   # uneven growth, one sequence idle
+            decode(layer, B)
+            append(layer, [40, 1, 1, 0, 2, 1][:B])
+            decode(layer, B)
+        for layer in range(wl.layers):
+            p.check_heads(layer)
         p.check_stats()
     finally:
         p.close()
