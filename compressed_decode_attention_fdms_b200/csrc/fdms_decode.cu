@@ -771,10 +771,14 @@ __device__ __forceinline__ void init_stages(uint8_t* smem, uint64_t* full, int n
 // dependency wait; the tiles new since then are dealt round-robin after it.
 // The warps' partials are merged in shared memory, the CTAs' through
 // distributed shared memory, and the cluster writes the output.
-template <class T, int CS>
+template <class T, int CS, bool BLK>
 __global__ void __launch_bounds__(T::NT, 1)
 k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
                const uint16_t* __restrict__ q, int use_snap) {
+  // per-block FP8 (BLK): sealed E4M3 tiles with T, the staged block and the
+  // ring in bf16 with T16; planned after the wait (use_snap is 0)
+  using T16 = Dec<T::D, false, T::G>;
+  constexpr int TR16 = T16::TR;
   constexpr int D = T::D, G = T::G, TR = T::TR, SPW = T::SPW, MT = T::MT, NMR = T::NMR,
                 NCW = T::NCW;
   constexpr bool FP8 = T::FP8;
@@ -787,6 +791,10 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   TileMeta* ring = reinterpret_cast<TileMeta*>(smem + T::OFF_META) + warp * NMR;
   (void)batch;
   init_stages<T>(smem, full, T::NSTAGE, T::NT, tid, warp, lane);
+  auto stg = [&](uint8_t* dst, uint64_t* bar, const TileMeta& mt, int phase) {
+    if (BLK && ((mt.rows >> 16) & kBf16)) stage_tile<T16>(c, dst, bar, mt, phase);
+    else stage_tile<T>(c, dst, bar, mt, phase);
+  };
 
   const int hsel = (int)(blockIdx.x / CS), crank = (int)(blockIdx.x % CS);
   const int v = crank * NCW + warp;
@@ -819,7 +827,7 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   auto split = [&](int len_s, int n_s, int r_s) {
     sp_s = (len_s + TR - 1) / TR;
     f0_s = r_s / TR;
-    const int P_s = head_tiles<TR>(len_s, n_s, r_s);
+    const int P_s = BLK ? blk_head_tiles<TR, TR16>(len_s, n_s, r_s) : head_tiles<TR>(len_s, n_s, r_s);
     const int qq = P_s / NW, rem = P_s % NW;
     cnt = qq + (v < rem ? 1 : 0);
     a_first = v * qq + min(v, rem);
@@ -877,7 +885,7 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
             tile_meta<T>(c, hi, hsel, kind, idx, len_s, n_s, r_s, hs[0], hs[1], s_bt, s_bs);
         mt.rows |= (lane == 0 ? kFirst : 0) << 16;
         ring[lane] = mt;
-        stage_tile<T>(c, smem + (warp * SPW + lane) * T::STAGE_BYTES, &full[warp * SPW + lane],
+        stg(smem + (warp * SPW + lane) * T::STAGE_BYTES, &full[warp * SPW + lane],
                       mt, 1);
         pre = true;
       }
@@ -886,19 +894,26 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   }
   WarpTiles<T> wt;
   wt.init(lane, c.softmax_scale);
+  WarpTiles<T16> wt16;   // the bf16 tiles of a per-block FP8 head
+  if (BLK) wt16.init(lane, c.softmax_scale);
   pdl_wait();                 // the previous kernel's writes are visible from here on
   pdl_launch_dependents();
   // q (an input of this call) and the arrivals of the tiles issued early
-  wt.fetch_q(q + ((long long)(hsel / c.Hkv) * c.Hq + (long long)(hsel % c.Hkv) * G) * D, hsel);
+  const uint16_t* qh = q + ((long long)(hsel / c.Hkv) * c.Hq + (long long)(hsel % c.Hkv) * G) * D;
+  wt.fetch_q(qh, hsel);
+  if (BLK) wt16.fetch_q(qh, hsel);
   if ((pre_mask >> lane) & 1)
-    stage_tile<T>(c, smem + (warp * SPW + lane) * T::STAGE_BYTES, &full[warp * SPW + lane],
+    stg(smem + (warp * SPW + lane) * T::STAGE_BYTES, &full[warp * SPW + lane],
                   ring[lane], 2);
   if (tid == 0) {
     const int len = c.store_len[hi], n = c.tok_n[hi], r = c.tok_r[hi];
     cst[12] = len;
     cst[13] = n;
     cst[14] = r;
-    if (!use_snap || cst[9] == 0) {
+    if (BLK) {   // the V unit of the E4M3 tiles: the first sealed block's V scale
+      hs[0] = 1.0f;
+      hs[1] = len >= kBlockSlots ? c.bt_scale[hi * c.max_blocks * 2 + 1] : 1.0f;
+    } else if (!use_snap || cst[9] == 0) {
       hs[0] = FP8 ? c.head_scale[hi * 2] : 1.0f;
       hs[1] = FP8 ? c.head_scale[hi * 2 + 1] : 1.0f;
     }
@@ -943,7 +958,7 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
     const int nfr_s = head_tiles<TR>(0, n_s, r_s);
     fx0 = max(nfr_s > 0 ? f0_s + nfr_s : r / TR, r / TR);
     const int E_ring = n > r ? max(0, (n - 1) / TR - fx0 + 1) : 0;
-    const int E = E_store + E_ring;
+    const int E = BLK ? 0 : E_store + E_ring;   // (per-block FP8 plans from the lengths now)
     nt = cnt + (E > e0 ? (E - e0 + NW - 1) / NW : 0);
   }
   if (lane < G) {   // an empty partial until the warp's last tile replaces it
@@ -955,7 +970,13 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   auto make_meta = [&](int k) -> TileMeta {
     const int len = cst[12], n = cst[13], r = cst[14];
     int kind, idx;
-    if (k < cnt) {
+    if (BLK) {   // sealed tiles, staged tiles (kind 3), ring frames of TR16 positions
+      const int item = a_first + k, n8 = blk_sealed_tiles<TR, TR16>(len);
+      const int nst = (len % kBlockSlots + TR16 - 1) / TR16;
+      if (item < n8) { kind = 0; idx = item; }
+      else if (item < n8 + nst) { kind = 3; idx = item - n8; }
+      else { kind = 1; idx = r / TR16 + (item - n8 - nst); }
+    } else if (k < cnt) {
       const int item = a_first + k;
       kind = item < sp_s ? 0 : 1;
       idx = kind == 0 ? item : f0_s + (item - sp_s);
@@ -964,7 +985,9 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
       kind = e < E_store ? 0 : 1;
       idx = kind == 0 ? sp_s + e : fx0 + (e - E_store);
     }
-    TileMeta mt = tile_meta<T>(c, hi, hsel, kind, idx, len, n, r, hs[0], hs[1], s_bt, s_bs);
+    TileMeta mt = (BLK && kind != 0)
+                      ? tile_meta_b16<T16>(c, hi, hsel, kind, idx, len, n, r)
+                      : tile_meta<T>(c, hi, hsel, kind, idx, len, n, r, hs[0], hs[1], s_bt, s_bs);
     mt.rows |= ((k == 0 ? kFirst : 0) | (k == nt - 1 ? kLast : 0)) << 16;
     return mt;
   };
@@ -976,7 +999,7 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   fill(32);
   __syncwarp();
   if (lane < SPW && lane < nt && !((pre_mask >> lane) & 1))
-    stage_tile<T>(c, smem + (warp * SPW + lane) * T::STAGE_BYTES, &full[warp * SPW + lane],
+    stg(smem + (warp * SPW + lane) * T::STAGE_BYTES, &full[warp * SPW + lane],
                   ring[lane], 0);
 
   // ================= tiles of this warp
@@ -997,7 +1020,10 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
       break;
     }
     const TileMeta tm = ring[k % NMR];
-    wt.tile(smem + s * T::STAGE_BYTES, tm, thresh, keep, c.R, lane);
+    if (BLK && ((tm.rows >> 16) & kBf16))
+      wt16.tile(smem + s * T::STAGE_BYTES, tm, thresh, keep, c.R, lane);
+    else
+      wt.tile(smem + s * T::STAGE_BYTES, tm, thresh, keep, c.R, lane);
     __syncwarp();
     // descriptors come 32 at a time: those of tiles k + 33 .. k + 64 once
     // tile k + 1 starts a new 32
@@ -1007,11 +1033,17 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
     }
     // the stage is free: refill it with tile k + SPW
     if (lane == 0 && k + SPW < nt)
-      stage_tile<T>(c, smem + s * T::STAGE_BYTES, &full[s], ring[(k + SPW) % NMR], 0);
+      stg(smem + s * T::STAGE_BYTES, &full[s], ring[(k + SPW) % NMR], 0);
     if ((tm.rows >> 16) & kLast) {   // the warp's partial, for the CTA's merge
       float o[MT][4], L0, L1;
       wt.finish(o, L0, L1);
-      const float vhead = hs[1];
+      float vhead = hs[1];
+      if constexpr (BLK) {   // the bf16 tiles' partial joins, in the E4M3 layout and V unit 1
+        float o16[MT][4], K0, K1;
+        wt16.finish(o16, K0, K1);
+        merge_kinds<MT>(o, wt.m0, wt.m1, L0, L1, vhead, o16, wt16.m0, wt16.m1, K0, K1, lane);
+        vhead = 1.0f;
+      }
       float* po = mslot + warp * T::SLOT;
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
@@ -1825,7 +1857,7 @@ inline int cluster_size(const fdms_cache* cache, int nh) {
   return 0;
 }
 
-template <class T, int CS>
+template <class T, int CS, bool BLK>
 cudaError_t launch_cluster_t(fdms_cache* cache, const DecodeWork& w, OutArgs oa, int layer,
                              int batch, const void* q, cudaStream_t s, int use_snap) {
   const int nh = batch * cache->view.Hkv;
@@ -1843,7 +1875,7 @@ cudaError_t launch_cluster_t(fdms_cache* cache, const DecodeWork& w, OutArgs oa,
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, k_decode_split<T, CS>, cache->view, w, oa, layer, batch,
+  return cudaLaunchKernelEx(&cfg, k_decode_split<T, CS, BLK>, cache->view, w, oa, layer, batch,
                             static_cast<const uint16_t*>(q), use_snap);
 }
 
@@ -1871,9 +1903,14 @@ fdms_status launch_split_t(fdms_cache* cache, const DecodeWork& w_in, OutArgs oa
   cudaError_t e = cudaErrorUnknown;
   if (cs > 0) {
     const int use_snap = writer_done ? 1 : 0;
-    e = cs == 8   ? launch_cluster_t<T, 8>(cache, w, oa, layer, batch, q, s, use_snap)
-        : cs == 4 ? launch_cluster_t<T, 4>(cache, w, oa, layer, batch, q, s, use_snap)
-                  : launch_cluster_t<T, 2>(cache, w, oa, layer, batch, q, s, use_snap);
+    if (T::FP8 && cache->view.blk)   // per-block FP8: two tile kinds, planned after the wait
+      e = cs == 8   ? launch_cluster_t<T, 8, T::FP8>(cache, w, oa, layer, batch, q, s, 0)
+          : cs == 4 ? launch_cluster_t<T, 4, T::FP8>(cache, w, oa, layer, batch, q, s, 0)
+                    : launch_cluster_t<T, 2, T::FP8>(cache, w, oa, layer, batch, q, s, 0);
+    else
+      e = cs == 8   ? launch_cluster_t<T, 8, false>(cache, w, oa, layer, batch, q, s, use_snap)
+          : cs == 4 ? launch_cluster_t<T, 4, false>(cache, w, oa, layer, batch, q, s, use_snap)
+                    : launch_cluster_t<T, 2, false>(cache, w, oa, layer, batch, q, s, use_snap);
     if (e != cudaSuccess) cudaGetLastError();   // a refused cluster launch falls back to the plan
   }
   if (e != cudaSuccess) {
@@ -1937,9 +1974,13 @@ int max_active_clusters(const fdms_cache* cache) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaFuncSetAttribute(k_decode_split<T, CS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)T::smem_bytes_cluster(cache->view.max_blocks)) != cudaSuccess ||
-      cudaOccupancyMaxActiveClusters(&n, k_decode_split<T, CS>, &cfg) != cudaSuccess)
+  const int smem = (int)T::smem_bytes_cluster(cache->view.max_blocks);
+  if (cudaFuncSetAttribute(k_decode_split<T, CS, false>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+      (T::FP8 && cudaFuncSetAttribute(k_decode_split<T, CS, T::FP8>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      smem) != cudaSuccess) ||
+      cudaOccupancyMaxActiveClusters(&n, k_decode_split<T, CS, false>, &cfg) != cudaSuccess)
     n = 0;
   return n;
 }
@@ -1979,8 +2020,7 @@ fdms_status setup_t(fdms_cache* cache) {
   cache->max_clusters[1] = max_active_clusters<T, 2>(cache);
   cache->max_clusters[2] = max_active_clusters<T, 4>(cache);
   cache->max_clusters[3] = max_active_clusters<T, 8>(cache);
-  // (a per-block FP8 cache decodes in the global plan only)
-  cache->cluster_ok = !cache->view.blk && T::smem_bytes_cluster(cache->view.max_blocks) <= 227 * 1024 &&
+  cache->cluster_ok = T::smem_bytes_cluster(cache->view.max_blocks) <= 227 * 1024 &&
                       cache->max_clusters[3] > 0;
   cudaGetLastError();   // a refused query only turns the cluster mode off
   return FDMS_OK;

@@ -38,7 +38,7 @@ def _expected(oc, layer, batch, wl):
 
 
 @pytest.mark.parametrize("kv_dtype,decode_ctas", [("bf16", 0), ("bf16", 148), ("fp8_e4m3", 0),
-                                                   ("fp8_e4m3_block", 0)])
+                                                   ("fp8_e4m3_block", 0), ("fp8_e4m3_block", 148)])
 def test_layout_and_decode_counters(kv_dtype, decode_ctas):
     wl = wk.scaled(wk.get("llama1b_c8"), layers=2, ctx=300, steps=0, kv_dtype=kv_dtype,
                    head_dim=128 if kv_dtype.startswith("fp8") else 64)
@@ -47,7 +47,7 @@ def test_layout_and_decode_counters(kv_dtype, decode_ctas):
         lay = fd.fdms_decode_layout(p.cache, wl.batch)
         cs, split = lay["cluster_ctas"], lay["split_ctas"]
         nh = wl.batch * wl.kv_heads
-        if decode_ctas > 0 or kv_dtype == "fp8_e4m3_block":
+        if decode_ctas > 0:
             assert cs == 0                       # the global plan
         else:
             assert cs in (2, 4, 8) and nh * cs <= torch.cuda.get_device_properties(0).multi_processor_count

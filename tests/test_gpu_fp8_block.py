@@ -102,17 +102,22 @@ def _append(cache, oc, layer, inp):
               inp["keep"].cpu().numpy())
 
 
-@pytest.mark.parametrize("head_dim,window,period", [(128, 16, 1), (64, 5, 7), (128, 0, 64)])
-def test_block_fp8_appends_match_the_oracle(head_dim, window, period):
+# decode_ctas 0: per-head clusters; 148: the global plan
+@pytest.mark.parametrize("head_dim,window,period,decode_ctas",
+                         [(128, 16, 1, 0), (128, 16, 1, 148), (64, 5, 7, 0), (64, 5, 7, 148),
+                          (128, 0, 64, 0)])
+def test_block_fp8_appends_match_the_oracle(head_dim, window, period, decode_ctas):
     wl = wk.scaled(wk.get("qwen8b_c8_fp8"), layers=2, batch=2, ctx=700, steps=0,
                    head_dim=head_dim, window=window, period=period, rate=0.4)
     cap = wl.ctx + 200
     cfg = fd.make_config(wl.layers, wl.batch, wl.q_heads, wl.kv_heads, wl.head_dim, wl.window,
-                         wl.period, cap, 0, "fp8_e4m3_block")
+                         wl.period, cap, 0, "fp8_e4m3_block", decode_ctas=decode_ctas)
     cache = fd.fdms_cache_create(cfg, 0)
     oc = OracleCache(wl.layers, wl.batch, wl.q_heads, wl.kv_heads, wl.head_dim, wl.window,
                      wl.period, "fp8_e4m3_block", capacity=cap)
     rng = np.random.default_rng(head_dim + window + period)
+    if decode_ctas == 0:   # per-head clusters at this batch
+        assert fd.fdms_decode_layout(cache, wl.batch)["cluster_ctas"] in (2, 4, 8)
     try:
         for layer in range(wl.layers):
             _append(cache, oc, layer, wk.prefill_inputs(wl, layer))
