@@ -99,8 +99,10 @@ typedef enum {
  * block's 64th survivor arrives ("sealing"). Until then the store's partly
  * filled block stays bf16 in a per-head staging block, and the ring holds bf16
  * rows. Decode reads the sealed blocks as E4M3 with their own scales and the
- * staged block and the ring as bf16; it always runs the global plan (four
- * warps per CTA, no per-head clusters). */
+ * staged block and the ring as bf16. Decode runs either mode (see
+ * decode_ctas) with two running states per warp, one per tile kind, planned
+ * from the lengths after the dependency wait (no snapshot: the staged block
+ * changes in place); the global plan uses four warps per CTA. */
 typedef enum { FDMS_KV_BF16 = 0, FDMS_KV_FP8_E4M3 = 1, FDMS_KV_FP8_E4M3_BLOCK = 2 } fdms_kv_dtype;
 
 typedef struct {
