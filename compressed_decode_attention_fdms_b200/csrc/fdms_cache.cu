@@ -11,6 +11,7 @@
 //   - per-(layer, seq, kv head) rings of W + P - 1 slots: the staging area
 //     that holds tokens until their keep decision is applied.
 #include <cmath>
+#include <cstdlib>
 #include <cstdio>
 #include <cstring>
 #include <vector>
@@ -255,6 +256,10 @@ fdms_status fdms_cache_create(const fdms_config* cfg, int device, void* stream,
   v.fp8 = cfg->kv_dtype == FDMS_KV_FP8_E4M3 || v.blk;
   v.RB = v.D * (v.fp8 ? 1 : 2);
   v.RBR = v.blk ? 2 * v.D : v.RB;   // per-block FP8 stages its rows in bf16
+  {
+    const char* stall = std::getenv("FDMS_TEST_STALL_COPIES");
+    v.stall_tx = (stall && stall[0] && std::strcmp(stall, "0") != 0) ? 16u : 0u;
+  }
   v.W = cfg->window;
   v.P = cfg->compact_period;
   // ring capacity: W + P - 1 unresolved tokens at most, rounded up to whole

@@ -739,8 +739,8 @@ __device__ __forceinline__ void stage_tile(const CacheView& c, uint8_t* kdst, ui
   const int row0 = mt.rows & 0xFF, row1 = (mt.rows >> 8) & 0xFF;
   const uint32_t nb = row1 > row0 ? (uint32_t)(row1 - row0) * RB : 0u;
   const long long voff = (long long)((mt.rows >> 16) & kRing ? c.R : kBlockSlots) * RB;
-  if (phase == 0) mbar_arrive_expect_tx(bar, 2u * nb);
-  if (phase == 1) mbar_expect_tx(bar, 2u * nb);
+  if (phase == 0) mbar_arrive_expect_tx(bar, 2u * nb + c.stall_tx);
+  if (phase == 1) mbar_expect_tx(bar, 2u * nb + c.stall_tx);
   if (phase == 2) mbar_arrive_expect_tx(bar, 0u);
   if (phase != 2 && nb > 0) {
     bulk_g2s(kdst + row0 * RB, mt.ksrc + (long long)row0 * RB, nb, bar);

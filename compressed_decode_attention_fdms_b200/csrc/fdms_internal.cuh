@@ -60,6 +60,10 @@ struct CacheView {
   int fp8;
   int blk;                // per-block FP8 scales (FDMS_KV_FP8_E4M3_BLOCK)
   float softmax_scale;
+  // bytes every decode tile stage expects beyond its copies: 0, or 16 when
+  // FDMS_TEST_STALL_COPIES is set at cache creation (failure-detection tests:
+  // the copies land but no stage completes, so every stage wait runs out)
+  uint32_t stall_tx;
 };
 
 // Row layout inside a 64-row page (a store block, or 64 ring slots): the 16-byte

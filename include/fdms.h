@@ -67,7 +67,11 @@
  * sticky word with the first error code and the affected head is left
  * unchanged; fdms_cache_stats reports the word. Device code never traps or
  * waits without a bound (the barriers of one CTA or one cluster aside, which
- * every thread of it reaches).
+ * every thread of it reaches): a decode wait on its tile copies gives up after
+ * 2 s, latches FDMS_ERR_DEVICE and the kernel still finishes. For tests of that
+ * path, a cache created while the environment variable FDMS_TEST_STALL_COPIES
+ * is set (and not "0") has every decode tile stage expect 16 bytes more than
+ * its copies bring, so that its decode waits run out.
  *
  * Layouts: all tensors are dense, row-major, in the order written; "bf16" is
  * the IEEE binary32 upper half. Device pointers must be 16-byte aligned.
