@@ -551,8 +551,10 @@ def decode_kernel_desc(cs):
 
 
 # workloads reported next to the headline one in the default run (their decode
-# call and step at a shorter run): the pages' other single-GPU workloads
-EXTRA_WORKLOADS = ("qwen8b_c8_fp8", "llama1b_c1")
+# call and step at a shorter run): the pages' other single-GPU workloads, the
+# Qwen3-8B one under both FP8 scale readings (one scale pair per head; one per
+# sealed 64-slot block)
+EXTRA_WORKLOADS = ("qwen8b_c8_fp8", "qwen8b_c8_fp8_block", "llama1b_c1")
 
 
 def run_native(args, wl):
@@ -593,7 +595,8 @@ def run_native(args, wl):
                        "timing": "K steps in one CUDA graph; events around each decode call"},
             "roofline": roof,
             "clocks": m["clocks"],
-            "gpu_launches": K * wl.layers * (2 if m["cs"] else 3),
+            # per layer and step: the append kernel and the decode kernel
+            "gpu_launches": K * wl.layers * 2,
             "prefill": m["prefill"],
             "kv_gb_per_step": m["kv_bytes"] / K / 1e9,
             "memory": m["memory"],
