@@ -126,10 +126,10 @@ typedef struct {
                             can all hold a cluster of 8, 4 or 2 CTAs at once on
                             this device runs one cluster (of the largest such
                             size) per pair; other calls run
-                            one plan over SM-count split CTAs (two may share an
-                            SM, so consecutive calls overlap). > 0 -> always
-                            the plan, over this many CTAs, at most as many
-                            as can be resident on the device at once */
+                            one plan over as many split CTAs as can be
+                            resident on the device at once (two per SM for the
+                            shapes here). > 0 -> always the plan, over this
+                            many CTAs, at most that resident count */
 } fdms_config;
 
 typedef struct {

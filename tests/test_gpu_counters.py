@@ -51,7 +51,11 @@ def test_layout_and_decode_counters(kv_dtype, decode_ctas):
             assert cs == 0                       # the global plan
         else:
             assert cs in (2, 4, 8) and nh * cs <= torch.cuda.get_device_properties(0).multi_processor_count
-        assert split == (decode_ctas or torch.cuda.get_device_properties(0).multi_processor_count)
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
+        if decode_ctas > 0:
+            assert split == decode_ctas
+        else:   # every resident slot of the device: a whole number of CTAs per SM
+            assert split >= sms and split % sms == 0
         with pytest.raises(fd.FdmsError):
             fd.fdms_decode_layout(p.cache, wl.batch + 1)
         for layer in range(wl.layers):
