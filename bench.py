@@ -535,7 +535,9 @@ def measure(fd, args, wl, dev, local, world, K, W, KE, WE):
                     "us_per_layer": 1e3 * pre_ms / L, "gb_per_layer": pre_bytes / L / 1e9,
                     "achieved_gbs": pre_bytes / (pre_ms * 1e-3) / 1e9,
                     "frac": pre_bytes / (pre_ms * 1e-3) / 1e9 / peak,
-                    "timing": pre_how + " (4 launches per layer)"},
+                    "timing": pre_how + (" (1 launch per layer: a CTA per head)"
+                                         if wl.kv_dtype == "fp8_e4m3_block"
+                                         else " (4 launches per layer)")},
         "decode_share_of_step": dec_avg_ms * L * K / elapsed_ms,
     }
     del graph, graph_dec

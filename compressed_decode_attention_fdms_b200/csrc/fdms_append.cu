@@ -1225,6 +1225,224 @@ k_append_block(CacheView c, int layer, int batch, const int32_t* __restrict__ n_
   }
 }
 
+
+// The same append for calls of many tokens (prefill): a CTA per (seq, kv head),
+// its warps sharing the work that the warp version does in sequence.
+//   1. each 32-position chunk of the positions resolved now: its survivors'
+//      ballot (shared memory), then a scan of the chunk counts over the CTA;
+//   2. the blocks this call seals, one warp each: its 64 rows are the staged
+//      rows of the open block (store indices below len0) and the survivors of
+//      ranks 0 .. (found by a search over the chunk prefix and the chunk's
+//      ballot); the K and V maxima over the rows, then the rows quantised;
+//   3. (after 2 has read the staging rows) the survivors past the last sealed
+//      block to the staging block;
+//   4. (after every ring row has been read) the unresolved tokens to the ring.
+// Same arithmetic as seal_block: the result is bit-identical.
+constexpr int kBlockCtaThreads = 256;
+constexpr int kBlockCtaWarps = kBlockCtaThreads / 32;
+constexpr int kBlockCtaMinTokens = 64;   // calls with at least this many tokens per sequence
+
+inline size_t block_cta_smem(int max_new, const CacheView& c) {
+  const long long nch = ((long long)max_new + c.W + c.P + 31) / 32 + 2;
+  return (size_t)nch * 2 * sizeof(uint32_t);
+}
+
+__global__ void __launch_bounds__(kBlockCtaThreads)
+k_append_block_cta(CacheView c, int layer, int batch, const int32_t* __restrict__ n_new,
+                   int max_new, const uint16_t* __restrict__ k_in,
+                   const uint16_t* __restrict__ v_in, const uint8_t* __restrict__ keep_in) {
+  pdl_wait();                 // the previous kernel's writes are visible from here on
+  pdl_launch_dependents();
+  extern __shared__ uint32_t s_chunk[];   // [nch] survivor ballots, then [nch] prefixes
+  __shared__ long long s_base;
+  __shared__ int s_fail;
+  __shared__ unsigned s_sat;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int hid = blockIdx.x;
+  if (hid >= batch * c.Hkv) return;
+  const int b = hid / c.Hkv, h = hid % c.Hkv;
+  const long long hi = head_index(c, layer, b, h);
+  const long long in_stride = (long long)c.Hkv * c.D;   // elements between tokens
+  const uint16_t* k_rows = k_in + ((long long)b * max_new * c.Hkv + h) * c.D;
+  const uint16_t* v_rows = v_in + ((long long)b * max_new * c.Hkv + h) * c.D;
+  const uint8_t* keep_rows = keep_in + (long long)b * max_new * c.Hkv + h;
+  uint8_t* rkeep = c.ring_keep + hi * c.Rpad;
+  const int VPR = c.D / 8, SRB = 2 * c.D;
+  constexpr unsigned kAll = 0xffffffffu;
+
+  const int m = n_new[b];
+  const int n0 = c.tok_n[hi], r0 = c.tok_r[hi], len0 = c.store_len[hi];
+  if (m < 0 || m > max_new || (long long)n0 + m > c.max_seq_len) {
+    if (tid == 0) latch_error(c.ctr, FDMS_ERR_DEVICE);
+    return;
+  }
+  if (m == 0) return;
+  const int n1 = n0 + m;
+  const int r1 = (n1 - c.W - r0 >= c.P) ? n1 - c.W : r0;
+  const int nch = (r1 - r0 + 31) / 32;
+  uint32_t* s_ball = s_chunk;
+  uint32_t* s_pre = s_chunk + nch + 1;   // exclusive prefix of the chunk counts; [nch] = total
+  auto keep_of = [&](int p) -> int {
+    return p < n0 ? (rkeep[p % c.R] != 0) : (keep_rows[(long long)(p - n0) * c.Hkv] != 0);
+  };
+
+  // ---- 1. ballots and their prefix
+  for (int ch = warp; ch < nch; ch += kBlockCtaWarps) {
+    const int p = r0 + ch * 32 + lane;
+    const unsigned ball = __ballot_sync(kAll, p < r1 && keep_of(p));
+    if (lane == 0) s_ball[ch] = ball;
+  }
+  if (tid == 0) {
+    s_fail = 0;
+    s_sat = 0;
+  }
+  __syncthreads();
+  if (warp == 0) {   // one warp scans: each lane a contiguous run of chunks
+    const int per = (nch + 31) / 32;
+    const int c0 = min(nch, lane * per), c1 = min(nch, c0 + per);
+    unsigned run = 0;
+    for (int ch = c0; ch < c1; ++ch) run += __popc(s_ball[ch]);
+    unsigned inc = run;
+    for (int off = 1; off < 32; off <<= 1) {
+      const unsigned y = __shfl_up_sync(kAll, inc, off);
+      if (lane >= off) inc += y;
+    }
+    unsigned acc = inc - run;
+    for (int ch = c0; ch < c1; ++ch) {
+      s_pre[ch] = acc;
+      acc += __popc(s_ball[ch]);
+    }
+    if (lane == 31) s_pre[nch] = inc;
+  }
+  __syncthreads();
+  const int total = (int)s_pre[nch];
+  const int len1 = len0 + total;
+  const int jb0 = len0 / kBlockSlots, jb1 = len1 / kBlockSlots;   // blocks sealed: [jb0, jb1)
+  if (tid == 0 && jb1 > jb0) {
+    const long long base = take_blocks(c.ctr, (unsigned long long)(jb1 - jb0), c.num_blocks);
+    if (base < 0) {
+      latch_error(c.ctr, FDMS_ERR_OUT_OF_BLOCKS);
+      s_fail = 1;
+    }
+    s_base = base;
+  }
+  __syncthreads();
+  if (s_fail) return;
+  const long long base_blk = s_base;
+
+  // source position of survivor rank q (0 .. total-1): the chunk whose prefix
+  // holds it (binary search), then the rank inside the chunk's ballot
+  auto src_of = [&](int q) -> int {
+    int lo = 0, hi_c = nch - 1;
+    while (lo < hi_c) {
+      const int mid = (lo + hi_c + 1) >> 1;
+      if ((int)s_pre[mid] <= q) lo = mid;
+      else hi_c = mid - 1;
+    }
+    return r0 + lo * 32 + (int)__fns(s_ball[lo], 0, q - (int)s_pre[lo] + 1);
+  };
+  // bf16 row vector of store index d (>= 64 * jb0): the staged row, or survivor d - len0
+  uint8_t* sk = stage_k(c, hi);
+  uint8_t* sv = stage_v(c, hi);
+  auto row_vec = [&](int d, int vec, uint4& xk, uint4& xv, int& pos) {
+    if (d < len0) {
+      const int row = d % kBlockSlots;
+      xk = *bf16_vec(sk, SRB, false, row, vec);
+      xv = *bf16_vec(sv, SRB, true, row, vec);
+      pos = c.stage_pos[hi * kBlockSlots + row];
+    } else {
+      const int src = src_of(d - len0);
+      pos = src;
+      if (src < n0) {
+        const int slot = src % c.R;
+        xk = *bf16_vec(ring_k(c, hi), SRB, false, slot, vec);
+        xv = *bf16_vec(ring_v(c, hi), SRB, true, slot, vec);
+      } else {
+        const long long t = src - n0;
+        xk = *reinterpret_cast<const uint4*>(k_rows + t * in_stride + vec * 8);
+        xv = *reinterpret_cast<const uint4*>(v_rows + t * in_stride + vec * 8);
+      }
+    }
+  };
+
+  // ---- 2. the sealed blocks, one warp each
+  unsigned sat = 0;
+  for (int jb = jb0 + warp; jb < jb1; jb += kBlockCtaWarps) {
+    float ak = 0.f, av = 0.f;
+    for (int i = lane; i < kBlockSlots * VPR; i += 32) {
+      const int row = i / VPR, vec = i % VPR;
+      uint4 xk, xv;
+      int pos;
+      row_vec(jb * kBlockSlots + row, vec, xk, xv, pos);
+      ak = fmaxf(ak, amax8(xk));
+      av = fmaxf(av, amax8(xv));
+    }
+    for (int off = 16; off > 0; off >>= 1) {
+      ak = fmaxf(ak, __shfl_xor_sync(kAll, ak, off));
+      av = fmaxf(av, __shfl_xor_sync(kAll, av, off));
+    }
+    const float sck = __fdiv_rn(fmaxf(ak, 1.17549435e-38f), 448.0f);
+    const float scv = __fdiv_rn(fmaxf(av, 1.17549435e-38f), 448.0f);
+    const float qk = quant_recip(sck), qv = quant_recip(scv);
+    const long long blk = base_blk + (jb - jb0);
+    uint8_t* dk = block_k(c, blk);
+    uint8_t* dv = block_v(c, blk);
+    for (int i = lane; i < kBlockSlots * VPR; i += 32) {
+      const int row = i / VPR, vec = i % VPR;
+      uint4 xk, xv;
+      int pos;
+      row_vec(jb * kBlockSlots + row, vec, xk, xv, pos);
+      *reinterpret_cast<uint2*>(dk + (long long)row * c.RB + swz_byte(c.RB, false, row, vec * 8)) =
+          quantise8(xk, sck, qk, sat);
+      *reinterpret_cast<uint2*>(dv + (long long)row * c.RB + swz_byte(c.RB, true, row, vec * 8)) =
+          quantise8(xv, scv, qv, sat);
+      if (vec == 0) c.blk_pos[blk * kBlockSlots + row] = pos;
+    }
+    if (lane == 0) {
+      c.block_table[hi * c.max_blocks + jb] = (int32_t)blk;
+      c.bt_scale[(hi * c.max_blocks + jb) * 2] = sck;
+      c.bt_scale[(hi * c.max_blocks + jb) * 2 + 1] = scv;
+    }
+  }
+  __syncthreads();   // the staged rows of the sealed block are read
+
+  // ---- 3. the survivors past the last sealed block to the staging block
+  const int d_lo = max(len0, jb1 * kBlockSlots);
+  for (int i = tid; i < (len1 - d_lo) * VPR; i += kBlockCtaThreads) {
+    const int d = d_lo + i / VPR, vec = i % VPR;
+    uint4 xk, xv;
+    int pos;
+    row_vec(d, vec, xk, xv, pos);
+    const int row = d % kBlockSlots;
+    *bf16_vec(sk, SRB, false, row, vec) = xk;
+    *bf16_vec(sv, SRB, true, row, vec) = xv;
+    if (vec == 0) c.stage_pos[hi * kBlockSlots + row] = pos;
+  }
+  __syncthreads();   // ring slots read above may be overwritten below
+
+  // ---- 4. the call's unresolved tokens to the ring, in bf16
+  const int w0 = r1 > n0 ? r1 : n0;
+  for (int i = tid; i < (n1 - w0) * VPR; i += kBlockCtaThreads) {
+    const int p = w0 + i / VPR, vec = i % VPR;
+    const long long t = p - n0;
+    const int slot = p % c.R;
+    *bf16_vec(ring_k(c, hi), SRB, false, slot, vec) =
+        *reinterpret_cast<const uint4*>(k_rows + t * in_stride + vec * 8);
+    *bf16_vec(ring_v(c, hi), SRB, true, slot, vec) =
+        *reinterpret_cast<const uint4*>(v_rows + t * in_stride + vec * 8);
+    if (vec == 0) rkeep[slot] = keep_rows[t * c.Hkv] ? 1 : 0;
+  }
+  for (int off = 16; off > 0; off >>= 1) sat += __shfl_xor_sync(kAll, sat, off);
+  if (lane == 0 && sat) atomicAdd(&s_sat, sat);
+  __syncthreads();
+  if (tid == 0) {
+    if (s_sat) atomicAdd(&c.ctr->saturations, (unsigned long long)s_sat);
+    c.store_len[hi] = len1;
+    c.tok_n[hi] = n1;
+    c.tok_r[hi] = r1;
+  }
+}
+
 }  // namespace
 }  // namespace fdms
 
@@ -1249,7 +1467,15 @@ fdms_status fdms_launch_append(fdms_cache* cache, int layer, int batch, const in
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e;
-  if (c.blk) {   // per-block FP8: one warp-per-head path for every call size
+  if (c.blk && max_new >= kBlockCtaMinTokens) {   // per-block FP8, many tokens: a CTA per head
+    cfg.gridDim = dim3((unsigned)(batch * c.Hkv));
+    cfg.blockDim = dim3(kBlockCtaThreads);
+    cfg.dynamicSmemBytes = block_cta_smem(max_new, c);
+    if (cfg.dynamicSmemBytes > 48 * 1024) return FDMS_ERR_INVALID_ARG;
+    e = cudaLaunchKernelEx(&cfg, k_append_block_cta, c, layer, batch, n_new, max_new, kk, vv,
+                           keep);
+    last = fdms_log_launch(cache, true);
+  } else if (c.blk) {   // per-block FP8, a few tokens: a warp per head
     cfg.gridDim = dim3((unsigned)((batch * c.Hkv + kSmallWarps - 1) / kSmallWarps));
     cfg.blockDim = dim3(kSmallWarps * 32);
     e = cudaLaunchKernelEx(&cfg, k_append_block, c, layer, batch, n_new, max_new, kk, vv, keep);
