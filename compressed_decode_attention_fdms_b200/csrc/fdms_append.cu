@@ -18,7 +18,9 @@
 // Three paths, one result: decode steps (k_append_step: a warp per head, the
 // loads ordered for latency), calls of up to 16 tokens per sequence
 // (k_append_small: a warp per head) and bulk calls such as prefill (four
-// launches spread over many CTAs per head, below).
+// launches spread over many CTAs per head, below). A per-block FP8 cache has
+// its own two (k_append_block, a warp per head; k_append_block_cta, a CTA per
+// head for calls of 64 tokens or more), at the end of this file.
 //
 // FP8 cache: a sequence's first append fixes each head's K and V scales
 // (max(amax, 2^-126) / 448 of the call's values, or the caller's); every new
