@@ -109,7 +109,7 @@ def _append(cache, oc, layer, inp):
 def test_block_fp8_appends_match_the_oracle(head_dim, window, period, decode_ctas):
     wl = wk.scaled(wk.get("qwen8b_c8_fp8"), layers=2, batch=2, ctx=700, steps=0,
                    head_dim=head_dim, window=window, period=period, rate=0.4)
-    cap = wl.ctx + 200
+    cap = wl.ctx + 500
     cfg = fd.make_config(wl.layers, wl.batch, wl.q_heads, wl.kv_heads, wl.head_dim, wl.window,
                          wl.period, cap, 0, "fp8_e4m3_block", decode_ctas=decode_ctas)
     cache = fd.fdms_cache_create(cfg, 0)
@@ -129,6 +129,9 @@ def test_block_fp8_appends_match_the_oracle(head_dim, window, period, decode_cta
             if step % 7 == 3:   # a few tokens at once, none for one sequence
                 inp = wk.prefill_inputs(wk.scaled(wl, ctx=5), layer)
                 inp = {**inp, "n_new": torch.tensor([5, 0], dtype=torch.int32)}
+            elif step in (21, 30):   # a large call (a CTA per head) over staged and ring rows
+                inp = wk.prefill_inputs(wk.scaled(wl, ctx=150), layer)
+                inp = {**inp, "n_new": torch.tensor([150, 97], dtype=torch.int32)}
             else:
                 inp = wk.decode_inputs(wl, layer, step)
             _append(cache, oc, layer, inp)
