@@ -776,7 +776,9 @@ __global__ void __launch_bounds__(T::NT, 1)
 k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
                const uint16_t* __restrict__ q, int use_snap) {
   // per-block FP8 (BLK): sealed E4M3 tiles with T, the staged block and the
-  // ring in bf16 with T16; planned after the wait (use_snap is 0)
+  // ring in bf16 with T16. A snapshot plans its sealed tiles only (a sealed
+  // block never changes; the staged block does, in place): the staged and
+  // ring tiles, and the blocks sealed since, are dealt after the wait
   using T16 = Dec<T::D, false, T::G>;
   constexpr int TR16 = T16::TR;
   constexpr int D = T::D, G = T::G, TR = T::TR, SPW = T::SPW, MT = T::MT, NMR = T::NMR,
@@ -827,7 +829,9 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   auto split = [&](int len_s, int n_s, int r_s) {
     sp_s = (len_s + TR - 1) / TR;
     f0_s = r_s / TR;
-    const int P_s = BLK ? blk_head_tiles<TR, TR16>(len_s, n_s, r_s) : head_tiles<TR>(len_s, n_s, r_s);
+    const int P_s = !BLK ? head_tiles<TR>(len_s, n_s, r_s)
+                         : (use_snap ? blk_sealed_tiles<TR, TR16>(len_s)
+                                     : blk_head_tiles<TR, TR16>(len_s, n_s, r_s));
     const int qq = P_s / NW, rem = P_s % NW;
     cnt = qq + (v < rem ? 1 : 0);
     a_first = v * qq + min(v, rem);
@@ -838,6 +842,11 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   // filled)
   auto snap_item = [&](int k, int& kind, int& idx) -> bool {
     const int item = a_first + k;
+    if (BLK) {   // a sealed tile: final
+      kind = 0;
+      idx = item;
+      return false;
+    }
     kind = item < sp_s ? 0 : 1;
     idx = kind == 0 ? item : f0_s + (item - sp_s);
     const int len_s = cst[8], n_s = cst[9];
@@ -875,6 +884,10 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
     asm volatile("cp.async.wait_all;" ::: "memory");   // this thread's block-table copies
     __syncthreads();
     const int len_s = cst[8], n_s = cst[9], r_s = cst[10];
+    // BLK: the V unit of the E4M3 tiles is the first sealed block's V scale
+    // (final once sealed)
+    const float hs_k = BLK ? 1.0f : hs[0];
+    const float hs_v = BLK ? (len_s >= kBlockSlots ? s_bs[1] : 1.0f) : hs[1];
     split(len_s, n_s, r_s);
     // copies of the warp's first tiles, unless they can still grow
     bool pre = false;
@@ -882,7 +895,7 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
       int kind, idx;
       if (!snap_item(lane, kind, idx)) {
         TileMeta mt =
-            tile_meta<T>(c, hi, hsel, kind, idx, len_s, n_s, r_s, hs[0], hs[1], s_bt, s_bs);
+            tile_meta<T>(c, hi, hsel, kind, idx, len_s, n_s, r_s, hs_k, hs_v, s_bt, s_bs);
         mt.rows |= (lane == 0 ? kFirst : 0) << 16;
         ring[lane] = mt;
         stg(smem + (warp * SPW + lane) * T::STAGE_BYTES, &full[warp * SPW + lane],
@@ -932,8 +945,11 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
   __syncthreads();
   {
     // block-table entries the copy may have missed: every one without a
-    // snapshot, else those of blocks added since
-    const int nb_ok = use_snap ? (cst[8] + kBlockSlots - 1) / kBlockSlots : 0;
+    // snapshot, else those of blocks added since (BLK: sealed since; the
+    // staged block has no entry until it is sealed)
+    const int nb_ok = !use_snap ? 0
+                      : BLK     ? cst[8] / kBlockSlots
+                                : (cst[8] + kBlockSlots - 1) / kBlockSlots;
     const int nb_now = (cst[12] + kBlockSlots - 1) / kBlockSlots;
     if (!use_snap) asm volatile("cp.async.wait_all;" ::: "memory");
     if (nb_now > nb_ok) {
@@ -958,7 +974,15 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
     const int nfr_s = head_tiles<TR>(0, n_s, r_s);
     fx0 = max(nfr_s > 0 ? f0_s + nfr_s : r / TR, r / TR);
     const int E_ring = n > r ? max(0, (n - 1) / TR - fx0 + 1) : 0;
-    const int E = BLK ? 0 : E_store + E_ring;   // (per-block FP8 plans from the lengths now)
+    int E = E_store + E_ring;
+    if (BLK) {   // without a snapshot the split covers every tile; with one, the
+                 // blocks sealed since, the staged tiles and the ring frames are new
+      const int live = n - r;
+      E = !use_snap ? 0
+                    : (blk_sealed_tiles<TR, TR16>(len) - blk_sealed_tiles<TR, TR16>(len_s)) +
+                          (len % kBlockSlots + TR16 - 1) / TR16 +
+                          (live > 0 ? (live + (r % TR16) + TR16 - 1) / TR16 : 0);
+    }
     nt = cnt + (E > e0 ? (E - e0 + NW - 1) / NW : 0);
   }
   if (lane < G) {   // an empty partial until the warp's last tile replaces it
@@ -971,8 +995,13 @@ k_decode_split(CacheView c, DecodeWork w, OutArgs oa, int layer, int batch,
     const int len = cst[12], n = cst[13], r = cst[14];
     int kind, idx;
     if (BLK) {   // sealed tiles, staged tiles (kind 3), ring frames of TR16 positions
-      const int item = a_first + k, n8 = blk_sealed_tiles<TR, TR16>(len);
+      const int n8 = blk_sealed_tiles<TR, TR16>(len);
       const int nst = (len % kBlockSlots + TR16 - 1) / TR16;
+      // without a snapshot: item a_first + k of the whole list; with one: a
+      // sealed tile of the snapshot, or new tile e of [sealed since, staged, ring]
+      const int n8s = use_snap ? blk_sealed_tiles<TR, TR16>(cst[8]) : 0;
+      int item = a_first + k;
+      if (use_snap && k >= cnt) item = n8s + e0 + (k - cnt) * NW;
       if (item < n8) { kind = 0; idx = item; }
       else if (item < n8 + nst) { kind = 3; idx = item - n8; }
       else { kind = 1; idx = r / TR16 + (item - n8 - nst); }
@@ -1903,10 +1932,10 @@ fdms_status launch_split_t(fdms_cache* cache, const DecodeWork& w_in, OutArgs oa
   cudaError_t e = cudaErrorUnknown;
   if (cs > 0) {
     const int use_snap = writer_done ? 1 : 0;
-    if (T::FP8 && cache->view.blk)   // per-block FP8: two tile kinds, planned after the wait
-      e = cs == 8   ? launch_cluster_t<T, 8, T::FP8>(cache, w, oa, layer, batch, q, s, 0)
-          : cs == 4 ? launch_cluster_t<T, 4, T::FP8>(cache, w, oa, layer, batch, q, s, 0)
-                    : launch_cluster_t<T, 2, T::FP8>(cache, w, oa, layer, batch, q, s, 0);
+    if (T::FP8 && cache->view.blk)   // per-block FP8: two tile kinds
+      e = cs == 8   ? launch_cluster_t<T, 8, T::FP8>(cache, w, oa, layer, batch, q, s, use_snap)
+          : cs == 4 ? launch_cluster_t<T, 4, T::FP8>(cache, w, oa, layer, batch, q, s, use_snap)
+                    : launch_cluster_t<T, 2, T::FP8>(cache, w, oa, layer, batch, q, s, use_snap);
     else
       e = cs == 8   ? launch_cluster_t<T, 8, false>(cache, w, oa, layer, batch, q, s, use_snap)
           : cs == 4 ? launch_cluster_t<T, 4, false>(cache, w, oa, layer, batch, q, s, use_snap)

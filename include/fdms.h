@@ -104,9 +104,11 @@ typedef enum {
  * filled block stays bf16 in a per-head staging block, and the ring holds bf16
  * rows. Decode reads the sealed blocks as E4M3 with their own scales and the
  * staged block and the ring as bf16. Decode runs either mode (see
- * decode_ctas) with two running states per warp, one per tile kind, planned
- * from the lengths after the dependency wait (no snapshot: the staged block
- * changes in place); the global plan uses four warps per CTA. */
+ * decode_ctas) with two running states per warp, one per tile kind. Per-head
+ * clusters plan the sealed tiles the layer's previous decode saw before the
+ * dependency wait (a sealed block never changes) and the staged and ring tiles
+ * after it (the staged block changes in place); the global plan plans every
+ * tile after the wait, with four warps per CTA. */
 typedef enum { FDMS_KV_BF16 = 0, FDMS_KV_FP8_E4M3 = 1, FDMS_KV_FP8_E4M3_BLOCK = 2 } fdms_kv_dtype;
 
 typedef struct {
