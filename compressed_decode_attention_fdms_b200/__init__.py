@@ -179,6 +179,11 @@ def fdms_cache_destroy(cache: Cache):
 
 def _dev_tensor(t, dtype, shape, name, device):
     """Device pointer of a tensor after checking what the C ABI assumes."""
+    # every property at once on the common path (this runs on every call of a
+    # decode step, several times); the checks below name what failed
+    if (isinstance(t, torch.Tensor) and t.dtype is dtype and t.is_cuda and t.shape == shape
+            and t.is_contiguous() and t.get_device() == device):
+        return t.data_ptr()
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name}: expected a torch.Tensor")
     if not t.is_cuda or t.get_device() != device:

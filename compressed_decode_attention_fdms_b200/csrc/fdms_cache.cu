@@ -23,9 +23,11 @@ using namespace fdms;
 namespace {
 
 struct DeviceGuard {
-  int prev = -1;
+  int prev = -1;   // the device to restore, or -1: none (it was already current)
   explicit DeviceGuard(int dev) {
-    if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+    int cur = -1;
+    if (cudaGetDevice(&cur) == cudaSuccess && cur == dev) return;
+    prev = cur;
     cudaSetDevice(dev);
   }
   ~DeviceGuard() {
