@@ -612,7 +612,10 @@ def run_native(args, wl):
                              "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                              "us_per_step": 1e3 * e2e["ms"] / KE, "steps": KE,
                              "path": "Python binding -> C ABI, eager calls per layer; one packed "
-                                     "H2D of the step's inputs and one D2H of all outputs"}
+                                     "H2D of the step's inputs and one D2H of all outputs per "
+                                     "step, on two copy streams with double-buffered device "
+                                     "memory (the next step's inputs go up and the last step's "
+                                     "outputs come down while a step computes)"}
         if not args.no_cpu_baseline and world == 1:
             # decode steps past the workload's own count so that the budget,
             # not the step count, ends the sample
@@ -635,7 +638,10 @@ def run_e2e(fd, cache, wl, stream, dev, s0, warm, steps, row):
     all its inputs (every layer's new token, keep bits and query, packed in
     one pinned buffer) to the device, every layer's fdms_append_evict +
     fdms_decode_attn on views of that buffer, and one copy of every layer's
-    output back to pinned host memory."""
+    output back to pinned host memory. The copies run on two copy streams into
+    double-buffered device memory, so that step s + 1's inputs go up and step
+    s's outputs come down while the compute stream runs a step (events order
+    every buffer's reuse)."""
     L, B = wl.layers, wl.batch
     # packed layout of one step: per layer n_new, k, v, keep, q, 16-byte aligned
     shapes = [("n_new", torch.int32, (B,)),
@@ -662,20 +668,36 @@ def run_e2e(fd, cache, wl, stream, dev, s0, warm, steps, row):
             for name, (o, n, dt, shp) in layout[layer].items():
                 buf[o:o + n].view(dt).view(shp).copy_(src[name])
         host.append(buf)
-    dbuf = torch.empty(step_bytes, dtype=torch.uint8, device=dev)
-    views = [{name: dbuf[o:o + n].view(dt).view(shp) for name, (o, n, dt, shp) in per.items()}
-             for per in layout]
-    dout = torch.empty((L, B, wl.q_heads, wl.head_dim), dtype=torch.bfloat16, device=dev)
-    hout = torch.empty_like(dout, device="cpu").pin_memory()
+    NB = 2   # device input and output buffers in flight
+    dbufs = [torch.empty(step_bytes, dtype=torch.uint8, device=dev) for _ in range(NB)]
+    views = [[{name: dbuf[o:o + n].view(dt).view(shp) for name, (o, n, dt, shp) in per.items()}
+              for per in layout] for dbuf in dbufs]
+    douts = [torch.empty((L, B, wl.q_heads, wl.head_dim), dtype=torch.bfloat16, device=dev)
+             for _ in range(NB)]
+    houts = [torch.empty_like(douts[0], device="cpu").pin_memory() for _ in range(NB)]
+    up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    in_ready = [torch.cuda.Event() for _ in range(NB)]
+    computed = [torch.cuda.Event() for _ in range(NB)]
+    out_read = [torch.cuda.Event() for _ in range(NB)]
 
     def one(s):
-        dbuf.copy_(host[s], non_blocking=True)
+        i = s % NB
+        up.wait_event(computed[i])          # the step that last read dbufs[i] is done
+        with torch.cuda.stream(up):
+            dbufs[i].copy_(host[s], non_blocking=True)
+        in_ready[i].record(up)
+        stream.wait_event(in_ready[i])
+        stream.wait_event(out_read[i])      # douts[i]'s last contents are on the host
         for layer in range(L):
-            d = views[layer]
+            d = views[i][layer]
             fd.fdms_append_evict(cache, layer, B, d["n_new"], 1, d["k"], d["v"], d["keep"],
                                  stream=stream)
-            fd.fdms_decode_attn(cache, layer, B, d["q"], dout[layer], stream=stream)
-        hout.copy_(dout, non_blocking=True)
+            fd.fdms_decode_attn(cache, layer, B, d["q"], douts[i][layer], stream=stream)
+        computed[i].record(stream)
+        down.wait_event(computed[i])
+        with torch.cuda.stream(down):
+            houts[i].copy_(douts[i], non_blocking=True)
+        out_read[i].record(down)
 
     with torch.cuda.stream(stream):
         for s in range(warm):
@@ -687,13 +709,16 @@ def run_e2e(fd, cache, wl, stream, dev, s0, warm, steps, row):
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         t0.record(stream)
+        up.wait_event(t0)
         for s in range(warm, warm + steps):
             one(s)
+        for i in range(NB):
+            stream.wait_event(out_read[i])   # the last outputs are on the host
         t1.record(stream)
     torch.cuda.synchronize()
     st1 = fd.fdms_cache_stats(cache, stream)
     return {"ms": t0.elapsed_time(t1), "bytes": st1["bytes_decoded"] - st0["bytes_decoded"],
-            "h2d": step_bytes, "d2h": dout.numel() * dout.element_size()}
+            "h2d": step_bytes, "d2h": douts[0].numel() * douts[0].element_size()}
 
 
 def main():
