@@ -93,7 +93,7 @@ typedef enum {
   FDMS_ERR_INVALID_ARG = 1,   /* bad argument, found on the host; nothing queued */
   FDMS_ERR_OUT_OF_BLOCKS = 2, /* the shared block pool ran out (device-latched) */
   FDMS_ERR_CUDA = 3,          /* a CUDA runtime call failed */
-  FDMS_ERR_UNSUPPORTED = 4,   /* configuration this build has no kernel for */
+  FDMS_ERR_UNSUPPORTED = 4,   /* configuration the library has no kernel for */
   FDMS_ERR_DEVICE = 5,        /* other device-detected error (sequence longer than
                                  max_seq_len, a bounded wait that ran out) */
 } fdms_status;
