@@ -94,7 +94,6 @@ def code_hash(path):
 def load_traffic(workload):
     """DRAM bytes of one decode call from the committed ncu summary, if it was
     taken on the decode sources as they are now; else None."""
-    import hashlib
     p = os.path.join(ROOT, "profiles", "decode_traffic.txt")
     if not os.path.exists(p):
         return None, "no capture"
@@ -106,8 +105,8 @@ def load_traffic(workload):
             continue
         if f[2:4] == now:
             return float(f[1]), "ncu dram__bytes_read.sum + dram__bytes_write.sum per " \
-                                "decode call, mean over the calls of two full steps " \
-                                f"(profiles/k_decode_split_{workload}.md)"
+                                "decode call, mean over the calls of two full steps of " \
+                                "this workload, one-pass capture on these decode sources"
         return None, "decode kernels changed since the ncu capture"
     return None, "no capture for this workload"
 
