@@ -154,3 +154,33 @@ def test_block_fp8_appends_match_the_oracle(head_dim, window, period, decode_cta
             _check_decode(cache, oc, layer, wl.batch, wl.q_heads, wl.head_dim, 7 + layer)
     finally:
         fd.fdms_cache_destroy(cache)
+
+
+def test_block_fp8_large_append_out_of_blocks_leaves_head_unchanged():
+    """The CTA-per-head append reserves a head's seals before any write: with
+    room for one head's seven sealed blocks of two, exactly one head appends
+    (which one depends on the order the CTAs reach the pool), the other is left
+    unchanged, OUT_OF_BLOCKS is latched and the pool count stays exact."""
+    wl = wk.scaled(wk.get("tiny"), ctx=500, steps=0, window=0, rate=1.0, head_dim=64)
+    cfg = fd.make_config(wl.layers, wl.batch, wl.q_heads, wl.kv_heads, wl.head_dim, wl.window,
+                         wl.period, 640, 8, "fp8_e4m3_block")   # a pool of 8 blocks
+    cache = fd.fdms_cache_create(cfg, 0)
+    oc = OracleCache(wl.layers, wl.batch, wl.q_heads, wl.kv_heads, wl.head_dim, wl.window,
+                     wl.period, "fp8_e4m3_block", capacity=640)
+    dev = "cuda:0"
+    try:
+        inp = wk.prefill_inputs(wl, 0)
+        fd.fdms_append_evict(cache, 0, 1, inp["n_new"].to(dev), inp["max_new"],
+                             inp["k"].to(dev), inp["v"].to(dev), inp["keep"].to(dev))
+        oc.append(0, inp["n_new"].numpy(), bits(inp["k"]), bits(inp["v"]), inp["keep"].numpy())
+        st = fd.fdms_cache_stats(cache)
+        assert st["error"] == fd.FDMS_ERR_OUT_OF_BLOCKS
+        assert st["blocks_used"] == 7 and st["blocks_free"] == 1
+        infos = [fd.fdms_cache_read_head(cache, 0, 0, h) for h in range(wl.kv_heads)]
+        done = [h for h in range(wl.kv_heads) if infos[h]["num_tokens"] == 500]
+        left = [h for h in range(wl.kv_heads) if infos[h]["num_tokens"] == 0]
+        assert len(done) == 1 and len(left) == 1, [i["num_tokens"] for i in infos]
+        assert infos[left[0]]["store_len"] == 0
+        _check_head(cache, oc, 0, 0, done[0])   # the head that fits: bit-exact
+    finally:
+        fd.fdms_cache_destroy(cache)
