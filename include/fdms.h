@@ -61,6 +61,14 @@
  * state, calls on one cache must not run concurrently from several host
  * threads; different caches are independent.
  *
+ * Stream capture: the calls may be captured into a CUDA graph (the host-side
+ * record of the cache is updated when a call is captured). Each launch of such
+ * a graph then stands for the captured calls in their place in the cache's
+ * call order: launch it exactly once, where the captured calls would have run.
+ * A graph launched several times would plan its decode calls from records of
+ * the first time (which snapshot copy to read, how many tokens were appended
+ * since), which later launches no longer match.
+ *
  * Errors: every call validates its arguments on the host and returns a status
  * before queuing any work. Calls that queue kernels are asynchronous; errors
  * found by the device (pool exhausted, sequence too long) are latched into a
