@@ -1259,6 +1259,7 @@ k_append_block_cta(CacheView c, int layer, int batch, const int32_t* __restrict_
   __shared__ long long s_base;
   __shared__ int s_fail;
   __shared__ unsigned s_sat;
+  __shared__ int s_row[kBlockCtaWarps][kBlockSlots];   // a block's rows: position, or -1 - row
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int hid = blockIdx.x;
   if (hid >= batch * c.Hkv) return;
@@ -1343,17 +1344,19 @@ k_append_block_cta(CacheView c, int layer, int batch, const int32_t* __restrict_
     }
     return r0 + lo * 32 + (int)__fns(s_ball[lo], 0, q - (int)s_pre[lo] + 1);
   };
-  // bf16 row vector of store index d (>= 64 * jb0): the staged row, or survivor d - len0
+  // where store index d (>= 64 * jb0) comes from: the staged row (-1 - row)
+  // or survivor d - len0's position; found once per row, by one lane
   uint8_t* sk = stage_k(c, hi);
   uint8_t* sv = stage_v(c, hi);
-  auto row_vec = [&](int d, int vec, uint4& xk, uint4& xv, int& pos) {
-    if (d < len0) {
-      const int row = d % kBlockSlots;
+  auto row_src = [&](int d) -> int { return d < len0 ? -1 - d % kBlockSlots : src_of(d - len0); };
+  // bf16 row vector `vec` of a row found by row_src, and the row's position
+  auto row_vec = [&](int src, int vec, uint4& xk, uint4& xv, int& pos) {
+    if (src < 0) {
+      const int row = -1 - src;
       xk = *bf16_vec(sk, SRB, false, row, vec);
       xv = *bf16_vec(sv, SRB, true, row, vec);
       pos = c.stage_pos[hi * kBlockSlots + row];
     } else {
-      const int src = src_of(d - len0);
       pos = src;
       if (src < n0) {
         const int slot = src % c.R;
@@ -1366,16 +1369,19 @@ k_append_block_cta(CacheView c, int layer, int batch, const int32_t* __restrict_
       }
     }
   };
+  int* rows_w = s_row[warp];
 
   // ---- 2. the sealed blocks, one warp each
   unsigned sat = 0;
   for (int jb = jb0 + warp; jb < jb1; jb += kBlockCtaWarps) {
+    for (int row = lane; row < kBlockSlots; row += 32) rows_w[row] = row_src(jb * kBlockSlots + row);
+    __syncwarp();
     float ak = 0.f, av = 0.f;
     for (int i = lane; i < kBlockSlots * VPR; i += 32) {
       const int row = i / VPR, vec = i % VPR;
       uint4 xk, xv;
       int pos;
-      row_vec(jb * kBlockSlots + row, vec, xk, xv, pos);
+      row_vec(rows_w[row], vec, xk, xv, pos);
       ak = fmaxf(ak, amax8(xk));
       av = fmaxf(av, amax8(xv));
     }
@@ -1393,7 +1399,7 @@ k_append_block_cta(CacheView c, int layer, int batch, const int32_t* __restrict_
       const int row = i / VPR, vec = i % VPR;
       uint4 xk, xv;
       int pos;
-      row_vec(jb * kBlockSlots + row, vec, xk, xv, pos);
+      row_vec(rows_w[row], vec, xk, xv, pos);
       *reinterpret_cast<uint2*>(dk + (long long)row * c.RB + swz_byte(c.RB, false, row, vec * 8)) =
           quantise8(xk, sck, qk, sat);
       *reinterpret_cast<uint2*>(dv + (long long)row * c.RB + swz_byte(c.RB, true, row, vec * 8)) =
@@ -1405,16 +1411,20 @@ k_append_block_cta(CacheView c, int layer, int batch, const int32_t* __restrict_
       c.bt_scale[(hi * c.max_blocks + jb) * 2] = sck;
       c.bt_scale[(hi * c.max_blocks + jb) * 2 + 1] = scv;
     }
+    __syncwarp();   // rows_w is read before the next block's rows are written
   }
   __syncthreads();   // the staged rows of the sealed block are read
 
   // ---- 3. the survivors past the last sealed block to the staging block
-  const int d_lo = max(len0, jb1 * kBlockSlots);
+  const int d_lo = max(len0, jb1 * kBlockSlots);   // (fewer than 64 rows)
+  int* rows_t = s_row[0];
+  for (int k = tid; k < len1 - d_lo; k += kBlockCtaThreads) rows_t[k] = row_src(d_lo + k);
+  __syncthreads();
   for (int i = tid; i < (len1 - d_lo) * VPR; i += kBlockCtaThreads) {
     const int d = d_lo + i / VPR, vec = i % VPR;
     uint4 xk, xv;
     int pos;
-    row_vec(d, vec, xk, xv, pos);
+    row_vec(rows_t[d - d_lo], vec, xk, xv, pos);
     const int row = d % kBlockSlots;
     *bf16_vec(sk, SRB, false, row, vec) = xk;
     *bf16_vec(sv, SRB, true, row, vec) = xv;
