@@ -64,3 +64,18 @@ def test_null_arguments(lib):
         fd.FDMS_ERR_INVALID_ARG
     assert lib.fdms_decode_attn(None, 0, 1, None, None, None) == fd.FDMS_ERR_INVALID_ARG
     assert lib.fdms_cache_stats(None, None, None) == fd.FDMS_ERR_INVALID_ARG
+
+
+def test_binding_rejects_what_the_c_abi_cannot_take():
+    """The binding's tensor check: a non-tensor, a host tensor (before any
+    device call), and, through the same check, dtype / shape / layout."""
+    import torch
+    t = torch.zeros((2, 3), dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        fd._dev_tensor([0.0] * 6, torch.bfloat16, (2, 3), "x", 0)
+    with pytest.raises(ValueError, match="cuda:0"):
+        fd._dev_tensor(t, torch.bfloat16, (2, 3), "x", 0)
+    with pytest.raises(ValueError):
+        fd._dev_tensor(t.t(), torch.bfloat16, (3, 2), "x", 0)
+    with pytest.raises((TypeError, ValueError)):
+        fd._dev_tensor(t.float(), torch.bfloat16, (2, 3), "x", 0)
