@@ -1,8 +1,9 @@
 """Per-block FP8 cache (FDMS_KV_FP8_E4M3_BLOCK) against the oracle's second FP8
 reading (needs a B200).
 
-Appends of every size go through the block-mode kernel; after each call every
-head is read back and compared bit-exactly: positions, lengths, keep bits, the
+Appends go through the block-mode kernels (a warp per head for a few tokens, a
+CTA per head for 64 or more); after each call every head is read back and
+compared bit-exactly: positions, lengths, keep bits, the
 codes and (K, V) scales of every sealed block, the bf16 rows of the staging
 block and of the ring, and the byte and saturation counters. Decode (sealed
 blocks in E4M3 with their own scales, the staged block and the ring in bf16)
